@@ -1,0 +1,419 @@
+"""fp64 CPU oracle for One-Pass to Reason masked attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's
+CPU-baseline leg may import this module.  The CUDA library never calls it, and
+it shares no code, table or helper with the CUDA library.
+
+It is the plain definition of what the one-pass attention layer computes,
+evaluated densely and slowly in float64 with numpy:
+
+* ``build_layout``   token duplication, segment order and position ids
+  (One-Pass to Reason wiki note, sections "Token 复制" and "位置 ID 策略").
+* ``mask_row`` /
+  ``dense_mask``     the visibility rules of the four token types
+  (same note, section "分块稀疏注意力掩码"; English note, "Method").
+* ``block_map``      classification of 128 x 128 tiles as empty / full / partial,
+  counted from the dense mask.
+* ``rope``           rotate-half rotary embedding by position id (the pages'
+  "位置编码等价" argument in "理论保证" relies on it; Qwen-3 uses it).
+* ``attention_fwd`` / ``attention_bwd``
+                     softmax attention under the mask and its analytic gradients.
+* ``npass_rows``     the N-pass baseline: one causal run per turn over
+  [h_1 r_1 ... h_{i-1} r_{i-1} h_i t_i r_i] with contiguous positions
+  ("问题背景" and "理论保证" / Theorem 2.1).
+
+Pins (checked by the tests that do not need a GPU): a hand-derived worked
+example of positions and visibility, closed-form visible-pair counts per turn,
+Theorem 2.1 by brute force (one-pass rows equal N-pass rows to 1e-12),
+PyTorch's float64 causal scaled_dot_product_attention for the single-segment
+case, RoPE invariants, and central finite differences for every gradient.
+
+Readings where the pages are silent (each one listed in the design notes):
+segment order h, t, r_in, r_out inside a turn; each segment causal within
+itself; positions restart at 0 for every packed conversation; conversations
+never see each other; zero-length segments are allowed; softmax scale
+1/sqrt(d); rotate-half RoPE with angle pos * base^(-2j/d); LSE in natural log;
+q head h reads kv head floor(h / (Hq / Hkv)).
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+H, T, RIN, ROUT = 0, 1, 2, 3      # token types
+TILE = 128                          # block-map tile edge
+EMPTY, FULL, PARTIAL = 0, 1, 2      # block-map classes
+
+
+@dataclass
+class Layout:
+    cu_seqlens: np.ndarray   # int64 [n_seqs + 1]
+    token_type: np.ndarray   # int8  [total]
+    turn_idx: np.ndarray     # int32 [total], 0-based within the conversation
+    conv_idx: np.ndarray     # int32 [total], global conversation index
+    pos_id: np.ndarray       # int32 [total]
+    max_seqlen: int
+
+    @property
+    def n_seqs(self) -> int:
+        return len(self.cu_seqlens) - 1
+
+    @property
+    def total(self) -> int:
+        return int(self.cu_seqlens[-1])
+
+
+def build_layout(turn_lens, conv_turn_ptr, seq_conv_ptr) -> Layout:
+    """Lay out every turn as h_i, t_i, r_i^in, r_i^out and assign position ids.
+
+    Position ids follow "位置 ID 策略": t_i and r_i^in both start right after
+    h_i ends, r_i^out starts right after t_i ends, and h_{i+1} starts right
+    after r_i^in ends.  Written with a cursor p (first position of h_i) this is
+    h_i: p..p+h-1, t_i: p+h.., r_i^in: p+h.., r_i^out: p+h+t.., next p = p+h+r,
+    which stays defined when a segment is empty.  p starts at 0 for every
+    conversation.
+    """
+    turn_lens = np.asarray(turn_lens, dtype=np.int64).reshape(-1, 3)
+    conv_turn_ptr = np.asarray(conv_turn_ptr, dtype=np.int64)
+    seq_conv_ptr = np.asarray(seq_conv_ptr, dtype=np.int64)
+    types, turns, convs, poss = [], [], [], []
+    cu = [0]
+    for s in range(len(seq_conv_ptr) - 1):
+        for c in range(seq_conv_ptr[s], seq_conv_ptr[s + 1]):
+            p = 0
+            for i, ti in enumerate(range(conv_turn_ptr[c], conv_turn_ptr[c + 1])):
+                h, t, r = (int(x) for x in turn_lens[ti])
+                for typ, start, n in ((H, p, h), (T, p + h, t), (RIN, p + h, r), (ROUT, p + h + t, r)):
+                    types += [typ] * n
+                    turns += [i] * n
+                    convs += [c] * n
+                    poss += list(range(start, start + n))
+                p = p + h + r
+        cu.append(len(types))
+    cu = np.asarray(cu, dtype=np.int64)
+    max_seqlen = int(np.diff(cu).max()) if len(cu) > 1 else 0
+    return Layout(cu, np.asarray(types, dtype=np.int8), np.asarray(turns, dtype=np.int32),
+                  np.asarray(convs, dtype=np.int32), np.asarray(poss, dtype=np.int32), max_seqlen)
+
+
+def mask_row(lay: Layout, q: int, lo: int, hi: int) -> np.ndarray:
+    """Visibility of keys lo..hi-1 (global token indices) from query token q.
+
+    The four rules of "分块稀疏注意力掩码", with H<i = {h_j, r_j^in : j < i} of
+    the same conversation and every segment causal within itself:
+      h_i      sees H<i and h_i up to itself
+      t_i      sees H<i, h_i and t_i up to itself
+      r_i^in   sees H<i, h_i and r_i^in up to itself
+      r_i^out  sees H<i, h_i, t_i and r_i^out up to itself
+    """
+    idx = np.arange(lo, hi)
+    ty, tu, cv = lay.token_type[lo:hi], lay.turn_idx[lo:hi], lay.conv_idx[lo:hi]
+    c, i, tau = lay.conv_idx[q], lay.turn_idx[q], lay.token_type[q]
+    same_conv = cv == c
+    history = same_conv & (tu < i) & ((ty == H) | (ty == RIN))
+    cur = same_conv & (tu == i)
+    own_prefix = cur & (ty == tau) & (idx <= q)
+    if tau == H:
+        own = own_prefix
+    elif tau == T:
+        own = (cur & (ty == H)) | own_prefix
+    elif tau == RIN:
+        own = (cur & (ty == H)) | own_prefix
+    else:  # ROUT
+        own = (cur & ((ty == H) | (ty == T))) | own_prefix
+    return history | own
+
+
+def dense_mask(lay: Layout, s: int) -> np.ndarray:
+    """Dense bool mask [L, L] of sequence s (row = query, column = key)."""
+    a, b = int(lay.cu_seqlens[s]), int(lay.cu_seqlens[s + 1])
+    m = np.zeros((b - a, b - a), dtype=bool)
+    for q in range(a, b):
+        m[q - a] = mask_row(lay, q, a, b)
+    return m
+
+
+def block_map(lay: Layout, tile: int = TILE, max_seqlen: int | None = None) -> np.ndarray:
+    """uint8 [n_seqs, T, T]: 0 empty, 1 full (tile*tile visible pairs), 2 partial.
+
+    Indices at or past the sequence length count as not visible, so a tail
+    tile is never full.  T = ceil(max_seqlen / tile).
+    """
+    ms = lay.max_seqlen if max_seqlen is None else max_seqlen
+    nt = (ms + tile - 1) // tile
+    out = np.zeros((lay.n_seqs, nt, nt), dtype=np.uint8)
+    for s in range(lay.n_seqs):
+        a, b = int(lay.cu_seqlens[s]), int(lay.cu_seqlens[s + 1])
+        L = b - a
+        counts = np.zeros((nt, nt), dtype=np.int64)
+        edges = np.arange(0, L, tile)
+        for ql in range(L):
+            row = mask_row(lay, a + ql, a, b)
+            counts[ql // tile, :len(edges)] += np.add.reduceat(row.astype(np.int64), edges)
+        cls = np.where(counts == 0, EMPTY, np.where(counts == tile * tile, FULL, PARTIAL))
+        out[s] = cls.astype(np.uint8)
+    return out
+
+
+def rope(x: np.ndarray, pos: np.ndarray, base: float, inverse: bool = False) -> np.ndarray:
+    """Rotate-half rotary embedding, float64.
+
+    x: [tokens, heads, d]; pair (x[j], x[j + d/2]) is rotated by
+    angle = pos * base^(-2j/d) (by -angle when ``inverse``).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    theta = float(base) ** (-(2.0 * np.arange(half, dtype=np.float64)) / d)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * theta[None, :]
+    if inverse:
+        ang = -ang
+    cos = np.cos(ang)[:, None, :]
+    sin = np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
+
+
+def _group(hq: int, hkv: int, h: int) -> int:
+    return h // (hq // hkv)
+
+
+def attention_fwd(q, k, v, lay: Layout, scale: float | None = None):
+    """Masked softmax attention over every sequence.
+
+    q: [total, Hq, d], k/v: [total, Hkv, d] (already rotated).  Returns
+    O [total, Hq, d] and LSE [Hq, total] = ln sum_visible exp(scale * q.k).
+    """
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    total, hq, d = q.shape
+    hkv = k.shape[1]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    o = np.zeros_like(q)
+    lse = np.zeros((hq, total))
+    for s in range(lay.n_seqs):
+        a, b = int(lay.cu_seqlens[s]), int(lay.cu_seqlens[s + 1])
+        if b == a:
+            continue
+        m = dense_mask(lay, s)
+        for h in range(hq):
+            g = _group(hq, hkv, h)
+            S = scale * (q[a:b, h] @ k[a:b, g].T)
+            S = np.where(m, S, -np.inf)
+            mx = S.max(axis=1, keepdims=True)
+            P = np.exp(S - mx)
+            l = P.sum(axis=1, keepdims=True)
+            P = P / l
+            o[a:b, h] = P @ v[a:b, g]
+            lse[h, a:b] = (mx + np.log(l))[:, 0]
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None):
+    """Analytic gradients of O = softmax(scale * q k^T masked) v.
+
+    With P recomputed from LSE: dV = P^T dO, dP = dO V^T, D = rowsum(dO * O),
+    dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q; dK and dV are summed
+    over the q heads that share a kv head.
+    """
+    q, k, v, o, do = (np.asarray(a, dtype=np.float64) for a in (q, k, v, o, do))
+    total, hq, d = q.shape
+    hkv = k.shape[1]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for s in range(lay.n_seqs):
+        a, b = int(lay.cu_seqlens[s]), int(lay.cu_seqlens[s + 1])
+        if b == a:
+            continue
+        m = dense_mask(lay, s)
+        for h in range(hq):
+            g = _group(hq, hkv, h)
+            S = scale * (q[a:b, h] @ k[a:b, g].T)
+            P = np.where(m, np.exp(S - lse[h, a:b][:, None]), 0.0)
+            dP = do[a:b, h] @ v[a:b, g].T
+            D = (do[a:b, h] * o[a:b, h]).sum(axis=1)
+            dS = P * (dP - D[:, None])
+            dq[a:b, h] = scale * (dS @ k[a:b, g])
+            dk[a:b, g] += scale * (dS.T @ q[a:b, h])
+            dv[a:b, g] += P.T @ do[a:b, h]
+    return dq, dk, dv
+
+
+def forward(q_pre, k_pre, v, lay: Layout, base: float, scale: float | None = None):
+    """RoPE by the layout's position ids, then masked attention."""
+    qr = rope(q_pre, lay.pos_id, base)
+    kr = rope(k_pre, lay.pos_id, base)
+    return attention_fwd(qr, kr, v, lay, scale)
+
+
+def backward(q_pre, k_pre, v, o, do, lse, lay: Layout, base: float, scale: float | None = None):
+    """Gradients w.r.t. the pre-RoPE q and k (inverse rotation of dq, dk) and v."""
+    qr = rope(q_pre, lay.pos_id, base)
+    kr = rope(k_pre, lay.pos_id, base)
+    dq, dk, dv = attention_bwd(qr, kr, v, o, do, lse, lay, scale)
+    return rope(dq, lay.pos_id, base, inverse=True), rope(dk, lay.pos_id, base, inverse=True), dv
+
+
+# --------------------------------------------------------------------------
+# Row and column samples, for workloads too large for the dense evaluation.
+# --------------------------------------------------------------------------
+
+def _seq_of(lay: Layout, tok: int) -> int:
+    return int(np.searchsorted(lay.cu_seqlens, tok, side="right") - 1)
+
+
+def attention_rows(q, k, v, lay: Layout, rows, heads, do=None, scale: float | None = None):
+    """O, LSE (and dQ when ``do`` is given) of selected query rows, computed one row at a time.
+
+    q/k already rotated.  Returns dict with o [n, len(heads), d], lse
+    [len(heads), n] and optionally dq [n, len(heads), d] (w.r.t. rotated q).
+    """
+    q, k, v = (np.asarray(a) for a in (q, k, v))
+    hq, d = q.shape[1], q.shape[2]
+    hkv = k.shape[1]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    rows = np.asarray(rows)
+    o = np.zeros((len(rows), len(heads), d))
+    lse = np.zeros((len(heads), len(rows)))
+    dq = np.zeros((len(rows), len(heads), d)) if do is not None else None
+    for n, tok in enumerate(rows):
+        s = _seq_of(lay, int(tok))
+        a = int(lay.cu_seqlens[s])
+        vis = mask_row(lay, int(tok), a, int(tok) + 1)
+        cols = a + np.nonzero(vis)[0]
+        for j, h in enumerate(heads):
+            g = _group(hq, hkv, h)
+            kk = k[cols, g].astype(np.float64)
+            vv = v[cols, g].astype(np.float64)
+            srow = scale * (kk @ q[tok, h].astype(np.float64))
+            mx = srow.max()
+            p = np.exp(srow - mx)
+            l = p.sum()
+            p /= l
+            o[n, j] = p @ vv
+            lse[j, n] = mx + np.log(l)
+            if do is not None:
+                dor = do[tok, h].astype(np.float64)
+                dp = vv @ dor
+                Dq = float(dor @ o[n, j])
+                ds = p * (dp - Dq)
+                dq[n, j] = scale * (ds @ kk)
+    out = dict(o=o, lse=lse)
+    if dq is not None:
+        out["dq"] = dq
+    return out
+
+
+def attention_cols(q, k, v, do, lay: Layout, cols, kv_head: int, scale: float | None = None):
+    """dK and dV (w.r.t. rotated k) of selected key tokens for one kv head.
+
+    Every query row that sees one of the keys is evaluated in full (its own
+    softmax, O and D), then its contributions are summed into the selected keys.
+    """
+    q, k, v, do = (np.asarray(a) for a in (q, k, v, do))
+    hq, d = q.shape[1], q.shape[2]
+    hkv = k.shape[1]
+    group = hq // hkv
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    cols = np.asarray(cols)
+    col_pos = {int(c): n for n, c in enumerate(cols)}
+    dk = np.zeros((len(cols), d))
+    dv = np.zeros((len(cols), d))
+    # candidate rows: same sequence, at or after the earliest selected key
+    cand = set()
+    for c in cols:
+        s = _seq_of(lay, int(c))
+        b = int(lay.cu_seqlens[s + 1])
+        same = np.nonzero(lay.conv_idx[int(c):b] == lay.conv_idx[int(c)])[0] + int(c)
+        cand.update(int(t) for t in same)
+    for tok in sorted(cand):
+        s = _seq_of(lay, tok)
+        a = int(lay.cu_seqlens[s])
+        vis = mask_row(lay, tok, a, tok + 1)
+        vcols = a + np.nonzero(vis)[0]
+        hit = [(j, col_pos[int(c)]) for j, c in enumerate(vcols) if int(c) in col_pos]
+        if not hit:
+            continue
+        kk = k[vcols, kv_head].astype(np.float64)
+        vv = v[vcols, kv_head].astype(np.float64)
+        for h in range(kv_head * group, (kv_head + 1) * group):
+            qr = q[tok, h].astype(np.float64)
+            dor = do[tok, h].astype(np.float64)
+            srow = scale * (kk @ qr)
+            p = np.exp(srow - srow.max())
+            p /= p.sum()
+            orow = p @ vv
+            dp = vv @ dor
+            ds = p * (dp - float(dor @ orow))
+            for j, n in hit:
+                dk[n] += scale * ds[j] * qr
+                dv[n] += p[j] * dor
+    return dk, dv
+
+
+# --------------------------------------------------------------------------
+# N-pass baseline (Theorem 2.1 brute force)
+# --------------------------------------------------------------------------
+
+def npass_token_lists(lay: Layout, turn_lens, conv_turn_ptr):
+    """For each (conversation, turn i): one-pass token indices of the N-pass sequence
+    [h_1 r_1 ... h_{i-1} r_{i-1} h_i t_i r_i], where the context copies r_j are the
+    r_j^in tokens and the current response r_i is the r_i^out tokens."""
+    out = []
+    conv_turn_ptr = np.asarray(conv_turn_ptr)
+    for c in range(len(conv_turn_ptr) - 1):
+        sel = np.nonzero(lay.conv_idx == c)[0]
+        nt = int(conv_turn_ptr[c + 1] - conv_turn_ptr[c])
+        ty, tu = lay.token_type[sel], lay.turn_idx[sel]
+        for i in range(nt):
+            hist = sel[(tu < i) & ((ty == H) | (ty == RIN))]
+            cur = sel[(tu == i) & ((ty == H) | (ty == T) | (ty == ROUT))]
+            out.append((c, i, np.concatenate([hist, cur])))
+    return out
+
+
+def causal_attention(q, k, v, scale: float | None = None):
+    """Plain causal softmax attention of one sequence: q [n, Hq, d], k/v [n, Hkv, d]."""
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    n, hq, d = q.shape
+    hkv = k.shape[1]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    causal = np.tril(np.ones((n, n), dtype=bool))
+    o = np.zeros_like(q)
+    lse = np.zeros((hq, n))
+    for h in range(hq):
+        g = _group(hq, hkv, h)
+        S = np.where(causal, scale * (q[:, h] @ k[:, g].T), -np.inf)
+        mx = S.max(axis=1, keepdims=True)
+        P = np.exp(S - mx)
+        l = P.sum(axis=1, keepdims=True)
+        o[:, h] = (P / l) @ v[:, g]
+        lse[h] = (mx + np.log(l))[:, 0]
+    return o, lse
+
+
+def npass_rows(q_pre, k_pre, v, lay: Layout, turn_lens, conv_turn_ptr, base: float,
+               scale: float | None = None):
+    """Run the N-pass baseline and return, per (conversation, turn), the token
+    indices and the causal run's O and LSE (positions 0..n-1, RoPE applied)."""
+    res = []
+    for c, i, toks in npass_token_lists(lay, turn_lens, conv_turn_ptr):
+        pos = np.arange(len(toks))
+        qr = rope(np.asarray(q_pre)[toks], pos, base)
+        kr = rope(np.asarray(k_pre)[toks], pos, base)
+        o, lse = causal_attention(qr, kr, np.asarray(v)[toks], scale)
+        res.append((c, i, toks, o, lse))
+    return res
+
+
+def visible_pairs(lay: Layout) -> int:
+    """Number of visible (q, k) pairs per head, counted from the mask rows."""
+    n = 0
+    for s in range(lay.n_seqs):
+        a, b = int(lay.cu_seqlens[s]), int(lay.cu_seqlens[s + 1])
+        for q in range(a, b):
+            n += int(mask_row(lay, q, a, q + 1).sum())
+    return n
