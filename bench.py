@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of the one-pass masked attention layer (fwd + bwd) on B200.
+
+One step = the whole hot path over one batch of synthetic conversations:
+opr_build_layout -> opr_rope(q), opr_rope(k) -> opr_attn_fwd -> opr_attn_bwd
+(three kernels) -> opr_rope(inverse) on dq and dk.
+
+Default workload: the Qwen-3-8B-like fwd+bwd configuration (32 q / 8 kv
+heads, head_dim 128, 8 turns per conversation, h~U[32,256], t~U[256,1024],
+r~U[64,512], two sequences packed to 32768 tokens), the first configuration
+on which the fwd+bwd metric is defined.
+
+Metric: useful TFLOP/s = 4 d P Hq (1 + 2.5) / step time, P the visible (q, k)
+pairs per head; plus conversation tokens/s (h + t + r per turn, no
+duplication) against the same kernels run N-pass.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config C]
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "1-pass masked attn fwd+bwd useful TFLOP/s; conv tokens/s vs N-pass"
+UNIT = "TFLOP/s"
+DEFAULT_CONFIG = 2
+L2_FLUSH_BYTES = 512 << 20
+KERNELS_PER_STEP = 7 + 2 + 1 + 3 + 2  # layout, rope x2, fwd, bwd (3), inverse rope x2
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["bf16_tflops"], d.get("bf16_tflops_sustained"), d["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock and throttle samples every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 8:
+                self.samples.append(f)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ our path
+class Runner:
+    """Buffers and calls of one step of the hot path for one workload."""
+
+    def __init__(self, w: synth.Workload, seed: int, device):
+        import torch
+
+        import block_sparse_masked_segment_b200 as opr
+        from block_sparse_masked_segment_b200.pipeline import visible_pairs_closed_form
+
+        self.torch, self.opr, self.w, self.dev = torch, opr, w, device
+        rng = np.random.default_rng(seed)
+        n = w.total_tokens
+        bf = torch.bfloat16
+        host = lambda x: torch.from_numpy(x).to(bf).pin_memory()  # noqa: E731
+        self.h_q = host(synth.gaussian(rng, (n, w.hq, w.d)))
+        self.h_k = host(synth.gaussian(rng, (n, w.hkv, w.d)))
+        self.h_v = host(synth.gaussian(rng, (n, w.hkv, w.d)))
+        self.h_do = host(synth.gaussian(rng, (n, w.hq, w.d)))
+        self.h_lens = [torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).pin_memory()
+                       for a in (w.turn_lens.reshape(-1), w.conv_turn_ptr, w.seq_conv_ptr)]
+        self.q, self.k, self.v, self.do = (t.to(device) for t in (self.h_q, self.h_k, self.h_v, self.h_do))
+        self.lens = [t.to(device) for t in self.h_lens]
+        self.q_rot = torch.empty_like(self.q)
+        self.k_rot = torch.empty_like(self.k)
+        self.grads = (torch.empty((n, w.hq, w.d), dtype=torch.float32, device=device),
+                      torch.empty((n, w.hkv, w.d), dtype=torch.float32, device=device),
+                      torch.empty((n, w.hkv, w.d), dtype=torch.float32, device=device))
+        self.h_grads = tuple(torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in self.grads)
+        self.bwd_ws = torch.empty(max(opr.opr_attn_bwd_workspace_bytes(n, w.hq, w.d), 256), dtype=torch.uint8,
+                                  device=device)
+        self.total, self.max_seqlen = n, w.max_seqlen
+        self.pairs = visible_pairs_closed_form(w.turn_lens, w.conv_turn_ptr)
+        self.conv_tokens = w.conversation_tokens()
+        self.names = ["layout", "rope", "attn_fwd", "bwd_row_terms", "bwd_dq", "bwd_dkdv", "rope_inv"]
+
+    def flops(self):
+        d, hq, P = self.w.d, self.w.hq, self.pairs
+        return {"useful_fwd": 4.0 * d * P * hq, "useful_bwd": 10.0 * d * P * hq,
+                "attn_fwd": 4.0 * d * P * hq, "bwd_dq": 6.0 * d * P * hq, "bwd_dkdv": 8.0 * d * P * hq}
+
+    def step(self, events=None):
+        """One pass of the hot path; `events` = list of CUDA events recorded between calls."""
+        opr, torch = self.opr, self.torch
+        rec = (lambda i: events[i].record()) if events is not None else (lambda i: None)
+        rec(0)
+        lay = opr.opr_build_layout(*self.lens, total_tokens=self.total, max_seqlen=self.max_seqlen, device=self.dev)
+        rec(1)
+        self.q_rot.copy_(self.q)
+        self.k_rot.copy_(self.k)
+        opr.opr_rope(self.q_rot, lay.pos_id, self.w.base)
+        opr.opr_rope(self.k_rot, lay.pos_id, self.w.base)
+        rec(2)
+        o, lse = opr.opr_attn_fwd(self.q_rot, self.k_rot, self.v, lay, out_dtype=torch.bfloat16)
+        rec(3)
+        args = (self.q_rot, self.k_rot, self.v, o, self.do, lse, lay)
+        opr.opr_attn_bwd(*args, workspace=self.bwd_ws, out=self.grads, stages=opr.BWD_ROW_TERMS)
+        rec(4)
+        opr.opr_attn_bwd(*args, workspace=self.bwd_ws, out=self.grads, stages=opr.BWD_DQ)
+        rec(5)
+        opr.opr_attn_bwd(*args, workspace=self.bwd_ws, out=self.grads, stages=opr.BWD_DKDV)
+        rec(6)
+        opr.opr_rope(self.grads[0], lay.pos_id, self.w.base, inverse=True)
+        opr.opr_rope(self.grads[1], lay.pos_id, self.w.base, inverse=True)
+        rec(7)
+        self.layout = lay
+        return lay
+
+    def e2e_step(self):
+        """Same step through host buffers: pinned H2D of inputs, D2H of dq, dk, dv."""
+        for dst, src in zip(self.lens, self.h_lens):
+            dst.copy_(src, non_blocking=True)
+        for dst, src in ((self.q, self.h_q), (self.k, self.h_k), (self.v, self.h_v), (self.do, self.h_do)):
+            dst.copy_(src, non_blocking=True)
+        self.step()
+        for dst, src in zip(self.h_grads, self.grads):
+            dst.copy_(src, non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(t.numel() * t.element_size() for t in (self.h_q, self.h_k, self.h_v, self.h_do, *self.h_lens))
+
+    def d2h_bytes(self):
+        return sum(t.numel() * t.element_size() for t in self.h_grads)
+
+
+def time_runner(r: Runner, steps: int, warmup: int, flush, barrier):
+    torch = r.torch
+    for _ in range(warmup):
+        r.step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush()
+        r.step(ev[i])
+    torch.cuda.synchronize()
+    barrier()
+    per = {name: [] for name in r.names}
+    totals = []
+    for e in ev:
+        t = [e[j].elapsed_time(e[j + 1]) for j in range(7)]
+        for name, x in zip(r.names, t):
+            per[name].append(x)
+        totals.append(e[0].elapsed_time(e[7]))
+    status = r.opr.read_status(r.layout.dev_status)
+    if status:
+        raise RuntimeError(f"device status after timing: {status}")
+    return sum(totals), per
+
+
+def time_e2e(r: Runner, steps: int, warmup: int, flush, barrier):
+    torch = r.torch
+    for _ in range(warmup):
+        r.e2e_step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for a, b in ev:
+        flush()
+        a.record()
+        r.e2e_step()
+        b.record()
+    torch.cuda.synchronize()
+    barrier()
+    return sum(a.elapsed_time(b) for a, b in ev)
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample(w: synth.Workload, target_tokens: int):
+    """The first conversation of the workload, cut after the turn that reaches
+    `target_tokens` one-pass tokens, with one GQA group (Hq/Hkv q heads, 1 kv head)."""
+    t0, t1 = int(w.conv_turn_ptr[0]), int(w.conv_turn_ptr[1])
+    turns, n = [], 0
+    for t in range(t0, t1):
+        h, tt, r = (int(x) for x in w.turn_lens[t])
+        turns.append((h, tt, r))
+        n += h + tt + 2 * r
+        if n >= target_tokens:
+            break
+    g = w.hq // w.hkv
+    sub = synth.make_custom_workload([[turns]], hq=g, hkv=1, d=w.d, base=w.base)
+    return sub
+
+
+def run_oracle_once(sub: synth.Workload, seed: int):
+    from block_sparse_masked_segment_b200.pipeline import visible_pairs_closed_form
+    from oracle import opr_oracle as orc
+
+    rng = np.random.default_rng(seed)
+    n = sub.total_tokens
+    q, k, v, do = (synth.gaussian(rng, (n, h, sub.d)) for h in (sub.hq, sub.hkv, sub.hkv, sub.hq))
+    lay = orc.build_layout(sub.turn_lens, sub.conv_turn_ptr, sub.seq_conv_ptr)
+    t = time.perf_counter()
+    o, lse = orc.forward(q, k, v, lay, sub.base)
+    orc.backward(q, k, v, o, do, lse, lay, sub.base)
+    dt = time.perf_counter() - t
+    pairs = visible_pairs_closed_form(sub.turn_lens, sub.conv_turn_ptr)
+    return dt, 14.0 * sub.d * pairs * sub.hq, sub.conversation_tokens()
+
+
+def cpu_baseline(w: synth.Workload, seed: int, target_tokens=6000):
+    sub = oracle_sample(w, target_tokens)
+    dt, flops, conv_tok = run_oracle_once(sub, seed)
+    cores = len(os.sched_getaffinity(0))
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"fp64 numpy oracle, dense fwd+bwd of the first conversation's first {sub.n_turns} turns "
+                       f"({sub.total_tokens} one-pass tokens), one GQA group ({sub.hq} q heads, 1 kv head), "
+                       f"d={sub.d}; {dt:.1f} s; useful FLOPs as on the GPU"),
+            "seconds": dt, "conv_tokens_per_s": conv_tok / dt}
+
+
+def run_reference(args, cfg_index):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = synth.make_workload(cfg_index)
+    sub = oracle_sample(w, 3000)
+    for i in range(args.warmup):
+        run_oracle_once(sub, 17 + i)
+    t0 = time.perf_counter()
+    flops = tok = 0.0
+    for i in range(args.steps):
+        dt, f, ct = run_oracle_once(sub, 100 + i)
+        flops += f
+        tok += ct
+    total = time.perf_counter() - t0
+    value = flops / total / 1e12
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "sample_tokens": sub.total_tokens, "sample_turns": sub.n_turns,
+                   "heads": f"{sub.hq}q/1kv"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"dense fp64 fwd+bwd, first {sub.n_turns} turns of conversation 0 "
+                                   f"({sub.total_tokens} tokens), one GQA group"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "conv_tokens_per_s": tok / total,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=DEFAULT_CONFIG)
+    ap.add_argument("--turns", type=int, default=None, help="turns per conversation (depth sweep)")
+    ap.add_argument("--no-npass", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        run_reference(args, args.config)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = lambda: flush_buf.zero_()  # noqa: E731
+
+    # every rank runs its own batch of the same shape (weak scaling, no data-path collective)
+    w = synth.make_workload(args.config, seed=1000 + args.config + 7919 * rank, n_turns=args.turns)
+    r = Runner(w, seed=11 + rank, device=device)
+    pairs = r.pairs
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    with ClockSampler(gpu_index) as clocks:
+        total_ms, per = time_runner(r, args.steps, args.warmup, flush, barrier)
+    total_ms = max_over_ranks(total_ms)
+    fl = r.flops()
+    useful = fl["useful_fwd"] + fl["useful_bwd"]
+    all_useful = sum_over_ranks(useful * args.steps)
+    value = all_useful / (total_ms * 1e-3) / 1e12
+    conv_tps = sum_over_ranks(r.conv_tokens * args.steps) / (total_ms * 1e-3)
+    mean = {k: statistics.mean(v) for k, v in per.items()}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms = max_over_ranks(time_e2e(r, args.steps, args.warmup, flush, barrier))
+        e2e = {"value": all_useful / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": r.h2d_bytes(), "d2h_bytes_per_step": r.d2h_bytes(),
+               "ms_per_step": e2e_ms / args.steps}
+
+    npass = None
+    if not args.no_npass:
+        nw, _ = synth.npass_workload(w)
+        del r
+        torch.cuda.empty_cache()
+        rn = Runner(nw, seed=11 + rank, device=device)
+        n_ms, n_per = time_runner(rn, args.steps, args.warmup, flush, barrier)
+        n_ms = max_over_ranks(n_ms)
+        n_conv_tps = sum_over_ranks(w.conversation_tokens() * args.steps) / (n_ms * 1e-3)
+        npass = {"conv_tokens_per_s": n_conv_tps, "ms_per_step": n_ms / args.steps,
+                 "tokens_per_step": nw.total_tokens, "pairs_per_head": rn.pairs,
+                 "kernel_ms": {k: statistics.mean(v) for k, v in n_per.items()},
+                 "one_pass_speedup": conv_tps / n_conv_tps}
+
+    # roofline of the dominant tensor-core kernel, timed live with CUDA events
+    bf16_peak, bf16_sust, hbm, peak_src = peaks()
+    dom = max(("attn_fwd", "bwd_dq", "bwd_dkdv"), key=lambda k: mean[k])
+    achieved = fl[dom] / (mean[dom] * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": achieved / bf16_peak, "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops (burst); sustained {bf16_sust}",
+                "frac_of_sustained": achieved / bf16_sust if bf16_sust else None,
+                "algorithmic_flops": fl[dom]}
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, seed=5)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "config_index": args.config, "sequences": w.n_seqs,
+                   "conversations": w.n_convs, "turns": w.n_turns, "tokens_per_step": w.total_tokens,
+                   "max_seqlen": w.max_seqlen, "conv_tokens_per_step": w.conversation_tokens(),
+                   "hq": w.hq, "hkv": w.hkv, "head_dim": w.d, "pairs_per_head": pairs,
+                   "parallelism": f"dp{world} (independent batches per GPU)",
+                   "l2": "512 MiB buffer zeroed before every step, outside the step's events",
+                   "outputs": "O bf16, LSE fp32, dq/dk/dv fp32"},
+        "useful_tflop_per_step": useful / 1e12,
+        "fraction_of_bf16_peak": value / bf16_peak,
+        "conv_tokens_per_s": conv_tps,
+        "kernel_ms": mean,
+        "roofline": roofline,
+        "e2e": e2e,
+        "npass": npass,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,276 @@
+"""ctypes marshalling for libopr.so: same names as the C entry points.
+
+Each wrapper checks shapes and dtypes, allocates outputs with PyTorch on the
+input's device, passes raw pointers plus the current CUDA stream, and turns a
+non-zero ``opr_status`` into :class:`OprError`.  No arithmetic happens here.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "lib", "libopr.so")
+
+OPR_OK, OPR_INVALID_ARG, OPR_UNSUPPORTED, OPR_CUDA_ERROR, OPR_WORKSPACE_TOO_SMALL = 0, 1, 2, 3, 4
+DEV_BITS = {1: "bad input", 2: "total mismatch", 4: "sequence longer than max_seqlen", 8: "pipeline wait timeout"}
+DTYPE_BF16, DTYPE_FP32 = 0, 1
+TILE = 128
+
+EXPORTED_SYMBOLS = (
+    "opr_version",
+    "opr_layout_workspace_bytes",
+    "opr_build_layout",
+    "opr_rope",
+    "opr_attn_fwd",
+    "opr_attn_bwd_workspace_bytes",
+    "opr_attn_bwd",
+    "opr_attn_bwd_stages",
+)
+
+BWD_ROW_TERMS, BWD_DQ, BWD_DKDV = 1, 2, 4
+
+_STATUS_NAMES = {1: "OPR_INVALID_ARG", 2: "OPR_UNSUPPORTED", 3: "OPR_CUDA_ERROR", 4: "OPR_WORKSPACE_TOO_SMALL"}
+
+
+class OprError(RuntimeError):
+    pass
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libopr.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise OprError(f"{_LIB_PATH} is missing: build it with `python -m block_sparse_masked_segment_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I32, I64, SZ, D, F = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t,
+                             ctypes.c_double, ctypes.c_float)
+    lib.opr_version.restype = ctypes.c_char_p
+    lib.opr_version.argtypes = []
+    lib.opr_layout_workspace_bytes.restype = SZ
+    lib.opr_layout_workspace_bytes.argtypes = [I32, I32, I32, I64, I32]
+    lib.opr_build_layout.restype = I32
+    lib.opr_build_layout.argtypes = [P, P, P, I32, I32, I32, I64, I32, P, P, P, P, P, P, P, SZ, P, P]
+    lib.opr_rope.restype = I32
+    lib.opr_rope.argtypes = [P, I32, P, I64, I32, I32, D, I32, P]
+    lib.opr_attn_fwd.restype = I32
+    lib.opr_attn_fwd.argtypes = [P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F, P, I32, P, P, P]
+    lib.opr_attn_bwd_workspace_bytes.restype = SZ
+    lib.opr_attn_bwd_workspace_bytes.argtypes = [I64, I32, I32]
+    lib.opr_attn_bwd.restype = I32
+    lib.opr_attn_bwd.argtypes = [P, P, P, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F,
+                                 P, P, P, P, SZ, P, P]
+    lib.opr_attn_bwd_stages.restype = I32
+    lib.opr_attn_bwd_stages.argtypes = [P, P, P, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F,
+                                        P, P, P, P, SZ, P, I32, P]
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != OPR_OK:
+        raise OprError(f"{what} returned {_STATUS_NAMES.get(status, status)}")
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need_cuda(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise OprError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise OprError("tensors must be contiguous")
+
+
+def opr_version() -> str:
+    return load_library().opr_version().decode()
+
+
+def opr_layout_workspace_bytes(n_seqs, n_convs, n_turns, total_tokens, max_seqlen) -> int:
+    return int(load_library().opr_layout_workspace_bytes(n_seqs, n_convs, n_turns, total_tokens, max_seqlen))
+
+
+def opr_attn_bwd_workspace_bytes(total_tokens, hq, head_dim) -> int:
+    return int(load_library().opr_attn_bwd_workspace_bytes(total_tokens, hq, head_dim))
+
+
+@dataclass
+class Layout:
+    """Device outputs of opr_build_layout plus the sizes the attention calls need."""
+
+    n_seqs: int
+    n_convs: int
+    n_turns: int
+    total: int
+    max_seqlen: int
+    cu_seqlens: torch.Tensor
+    token_type: torch.Tensor
+    turn_idx: torch.Tensor
+    conv_idx: torch.Tensor
+    pos_id: torch.Tensor
+    block_map: torch.Tensor
+    workspace: torch.Tensor
+    dev_status: torch.Tensor
+
+    @property
+    def T(self) -> int:
+        return (self.max_seqlen + TILE - 1) // TILE
+
+
+def read_status(dev_status: torch.Tensor) -> list[str]:
+    """Synchronise and decode the device status word (empty list = no error)."""
+    v = int(dev_status.item())
+    return [name for bit, name in DEV_BITS.items() if v & bit]
+
+
+def _lens_host(turn_lens, conv_turn_ptr, seq_conv_ptr):
+    tl = np.asarray(turn_lens.cpu() if isinstance(turn_lens, torch.Tensor) else turn_lens, dtype=np.int64)
+    cp = np.asarray(conv_turn_ptr.cpu() if isinstance(conv_turn_ptr, torch.Tensor) else conv_turn_ptr, dtype=np.int64)
+    sp = np.asarray(seq_conv_ptr.cpu() if isinstance(seq_conv_ptr, torch.Tensor) else seq_conv_ptr, dtype=np.int64)
+    return tl.reshape(-1, 3), cp, sp
+
+
+def sizes_from_lengths(turn_lens, conv_turn_ptr, seq_conv_ptr) -> tuple[int, int]:
+    """(total_tokens, max_seqlen) of host length arrays: token counts h + t + 2r."""
+    tl, cp, sp = _lens_host(turn_lens, conv_turn_ptr, seq_conv_ptr)
+    cost = tl[:, 0] + tl[:, 1] + 2 * tl[:, 2]
+    csum = np.concatenate([[0], np.cumsum(cost)])
+    seq_len = csum[cp[sp[1:]]] - csum[cp[sp[:-1]]]
+    return int(cost.sum()), int(seq_len.max()) if seq_len.size else 0
+
+
+def opr_build_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, total_tokens=None, max_seqlen=None,
+                     device="cuda") -> Layout:
+    """Run opr_build_layout.  Length arrays may be host (copied in) or device int32 tensors."""
+    lib = load_library()
+    device = torch.device(device)
+    if total_tokens is None or max_seqlen is None:
+        tot, ms = sizes_from_lengths(turn_lens, conv_turn_ptr, seq_conv_ptr)
+        total_tokens = tot if total_tokens is None else total_tokens
+        max_seqlen = ms if max_seqlen is None else max_seqlen
+
+    def dev_i32(x):
+        t = x if isinstance(x, torch.Tensor) else torch.as_tensor(np.asarray(x, dtype=np.int32))
+        return t.to(device=device, dtype=torch.int32, non_blocking=True).contiguous()
+
+    tl, cp, sp = dev_i32(turn_lens).reshape(-1), dev_i32(conv_turn_ptr), dev_i32(seq_conv_ptr)
+    n_turns, n_convs, n_seqs = tl.numel() // 3, cp.numel() - 1, sp.numel() - 1
+    T = (max_seqlen + TILE - 1) // TILE
+    ws_bytes = opr_layout_workspace_bytes(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)
+    if ws_bytes == 0 and total_tokens > 0:
+        raise OprError("sizes out of range for opr_build_layout")
+    lay = Layout(
+        n_seqs, n_convs, n_turns, int(total_tokens), int(max_seqlen),
+        cu_seqlens=torch.empty(n_seqs + 1, dtype=torch.int32, device=device),
+        token_type=torch.empty(total_tokens, dtype=torch.int8, device=device),
+        turn_idx=torch.empty(total_tokens, dtype=torch.int32, device=device),
+        conv_idx=torch.empty(total_tokens, dtype=torch.int32, device=device),
+        pos_id=torch.empty(total_tokens, dtype=torch.int32, device=device),
+        block_map=torch.empty((n_seqs, T, T), dtype=torch.uint8, device=device),
+        workspace=torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device),
+        dev_status=torch.zeros(1, dtype=torch.int32, device=device),
+    )
+    st = lib.opr_build_layout(
+        _ptr(tl), _ptr(cp), _ptr(sp), n_seqs, n_convs, n_turns, total_tokens, max_seqlen,
+        _ptr(lay.cu_seqlens), _ptr(lay.token_type), _ptr(lay.turn_idx), _ptr(lay.conv_idx), _ptr(lay.pos_id),
+        _ptr(lay.block_map), _ptr(lay.workspace), lay.workspace.numel(), _ptr(lay.dev_status), _stream(device))
+    _check(st, "opr_build_layout")
+    lay._inputs = (tl, cp, sp)  # keep the device copies alive until the stream has used them
+    return lay
+
+
+def opr_rope(x: torch.Tensor, pos_id: torch.Tensor, base: float, inverse: bool = False) -> torch.Tensor:
+    """Rotate x [total, heads, head_dim] (bf16 or fp32) in place by position id."""
+    _need_cuda(x, pos_id)
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise OprError("opr_rope takes bf16 or fp32")
+    total, heads, d = x.shape
+    st = load_library().opr_rope(_ptr(x), DTYPE_BF16 if x.dtype == torch.bfloat16 else DTYPE_FP32, _ptr(pos_id),
+                                 total, heads, d, float(base), int(bool(inverse)), _stream(x.device))
+    _check(st, "opr_rope")
+    return x
+
+
+def _attn_shapes(q, k, v, lay: Layout):
+    _need_cuda(q, k, v)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16:
+            raise OprError("q, k, v must be bf16")
+    total, hq, d = q.shape
+    if k.shape != v.shape or k.shape[0] != total or k.shape[2] != d or total != lay.total:
+        raise OprError("shape mismatch between q, k, v and the layout")
+    return total, hq, k.shape[1], d
+
+
+def opr_attn_fwd(q, k, v, lay: Layout, scale: float | None = None, out_dtype=torch.float32):
+    """O [total, hq, d] (out_dtype) and LSE [hq, total] fp32."""
+    total, hq, hkv, d = _attn_shapes(q, k, v, lay)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty((total, hq, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((hq, total), dtype=torch.float32, device=q.device)
+    st = load_library().opr_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace),
+        lay.n_seqs, lay.n_convs, lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale),
+        _ptr(o), DTYPE_FP32 if out_dtype == torch.float32 else DTYPE_BF16, _ptr(lse), _ptr(lay.dev_status),
+        _stream(q.device))
+    _check(st, "opr_attn_fwd")
+    return o, lse
+
+
+def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, workspace=None, out=None,
+                 stages: int | None = None):
+    """dQ [total, hq, d], dK and dV [total, hkv, d] (fp32), w.r.t. the rotated q, k and v.
+
+    ``out`` = (dq, dk, dv) reuses buffers; ``stages`` (OR of BWD_ROW_TERMS,
+    BWD_DQ, BWD_DKDV) runs only those kernels through opr_attn_bwd_stages, with
+    the row terms kept in ``workspace`` between calls.
+    """
+    total, hq, hkv, d = _attn_shapes(q, k, v, lay)
+    _need_cuda(o, do, lse)
+    if do.dtype != torch.bfloat16 or lse.dtype != torch.float32:
+        raise OprError("dout must be bf16 and lse fp32")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = (torch.empty((total, hq, d), dtype=torch.float32, device=q.device),
+               torch.empty((total, hkv, d), dtype=torch.float32, device=q.device),
+               torch.empty((total, hkv, d), dtype=torch.float32, device=q.device))
+    dq, dk, dv = out
+    wb = opr_attn_bwd_workspace_bytes(total, hq, d)
+    if workspace is None or workspace.numel() < wb:
+        workspace = torch.empty(max(wb, 256), dtype=torch.uint8, device=q.device)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16, _ptr(do),
+            _ptr(lse), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace), lay.n_seqs, lay.n_convs,
+            lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+            _ptr(workspace), workspace.numel(), _ptr(lay.dev_status))
+    lib = load_library()
+    if stages is None:
+        _check(lib.opr_attn_bwd(*args, _stream(q.device)), "opr_attn_bwd")
+    else:
+        _check(lib.opr_attn_bwd_stages(*args, int(stages), _stream(q.device)), "opr_attn_bwd_stages")
+    return dq, dk, dv
+
+
+def opr_attn_bwd_stages(q, k, v, o, do, lse, lay: Layout, stages: int, workspace, out, scale=None):
+    """Run only the backward kernels selected by ``stages`` (see opr_attn_bwd)."""
+    return opr_attn_bwd(q, k, v, o, do, lse, lay, scale, workspace=workspace, out=out, stages=stages)

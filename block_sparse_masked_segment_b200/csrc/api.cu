@@ -1,0 +1,228 @@
+// api.cu - the extern "C" entry points of libopr.so declared in include/opr.h:
+// host-side argument checks, TMA descriptor encoding and kernel dispatch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "attn_common.cuh"
+#include "opr_internal.cuh"
+
+namespace opr {
+cudaError_t launch_attn_fwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_attn_bwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const void* o, int o_fp32, const void* dout,
+                            const AttnParams& pq, const AttnParams& pkv, float* row_d, int stages,
+                            cudaStream_t stream);
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [tokens, heads, head_dim] bf16 tensor as a 3-D TMA map with 128-byte swizzle;
+// a box is 64 head_dim elements x 1 head x 128 tokens (rows past the end read 0).
+bool make_map(CUtensorMap* map, const void* ptr, int64_t total, int32_t heads, int32_t head_dim) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(total)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, static_cast<cuuint64_t>(heads) * head_dim * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kTile)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+opr_status device_check() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return OPR_CUDA_ERROR;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return OPR_CUDA_ERROR;
+  return major == 10 ? OPR_OK : OPR_UNSUPPORTED;
+}
+
+bool sizes_ok(int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total, int32_t max_seqlen) {
+  if (n_seqs < 0 || n_convs < 0 || n_turns < 0 || total < 0 || max_seqlen < 0) return false;
+  if (total >= (int64_t{1} << 31)) return false;  // token offsets are int32
+  if (n_seqs > 65535) return false;
+  const int64_t T = (max_seqlen + kTile - 1) / kTile;
+  if (T > 65535) return false;
+  if (static_cast<int64_t>(n_seqs) * T >= (int64_t{1} << 31)) return false;
+  return true;
+}
+
+AttnParams base_params(const int32_t* cu_seqlens, const int32_t* conv_idx, const void* ws, int32_t n_seqs,
+                       int32_t n_convs, int32_t n_turns, int64_t total, int32_t max_seqlen, int32_t hq, int32_t hkv,
+                       float scale, int32_t* dev_status) {
+  const LayoutWs w = layout_ws_map(n_seqs, n_convs, n_turns, total, max_seqlen);
+  AttnParams p{};
+  p.cu_seqlens = cu_seqlens;
+  p.conv_idx = conv_idx;
+  p.tok_meta = ws_ptr<int32_t>(ws, w.tok_meta);
+  p.row_cnt = ws_ptr<int32_t>(ws, w.row_cnt);
+  p.row_list = ws_ptr<int32_t>(ws, w.row_list);
+  p.col_cnt = ws_ptr<int32_t>(ws, w.col_cnt);
+  p.col_list = ws_ptr<int32_t>(ws, w.col_list);
+  p.sched = ws_ptr<int32_t>(ws, w.q_sched);
+  p.T = w.T;
+  p.n_items = w.n_tiles;
+  p.total = total;
+  p.hq = hq;
+  p.hkv = hkv;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.dev_status = dev_status;
+  return p;
+}
+
+bool attn_args_ok(const void* q, const void* k, const void* v, int32_t hq, int32_t hkv, int32_t head_dim,
+                  float scale) {
+  if (!q || !k || !v) return false;
+  if (hq <= 0 || hkv <= 0 || hq % hkv != 0) return false;
+  if (head_dim != 64 && head_dim != 128) return false;
+  if (!(scale > 0.f)) return false;
+  return aligned16(q) && aligned16(k) && aligned16(v);
+}
+
+}  // namespace
+}  // namespace opr
+
+using namespace opr;
+
+extern "C" {
+
+const char* opr_version(void) { return "opr 0.1.0 sm_100a"; }
+
+size_t opr_layout_workspace_bytes(int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
+                                  int32_t max_seqlen) {
+  if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return 0;
+  return layout_ws_map(n_seqs, n_convs, n_turns, total_tokens, max_seqlen).bytes;
+}
+
+opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* conv_turn_ptr, const int32_t* seq_conv_ptr,
+                            int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
+                            int32_t max_seqlen, int32_t* cu_seqlens, int8_t* token_type, int32_t* turn_idx,
+                            int32_t* conv_idx, int32_t* pos_id, uint8_t* block_map, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return OPR_INVALID_ARG;
+  if (!conv_turn_ptr || !seq_conv_ptr || !cu_seqlens || !workspace || !dev_status) return OPR_INVALID_ARG;
+  if (n_turns > 0 && !turn_lens) return OPR_INVALID_ARG;
+  if (total_tokens > 0 && (!token_type || !turn_idx || !conv_idx || !pos_id)) return OPR_INVALID_ARG;
+  if (max_seqlen > 0 && n_seqs > 0 && !block_map) return OPR_INVALID_ARG;
+  if (workspace_bytes < layout_ws_map(n_seqs, n_convs, n_turns, total_tokens, max_seqlen).bytes)
+    return OPR_WORKSPACE_TOO_SMALL;
+  cudaError_t e = launch_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, n_seqs, n_convs, n_turns, total_tokens,
+                                max_seqlen, cu_seqlens, token_type, turn_idx, conv_idx, pos_id, block_map, workspace,
+                                dev_status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
+}
+
+opr_status opr_rope(void* x, int32_t dtype, const int32_t* pos_id, int64_t total_tokens, int32_t n_heads,
+                    int32_t head_dim, double base, int32_t inverse, void* stream) {
+  if (total_tokens < 0 || n_heads < 0 || head_dim <= 0 || head_dim % 2 != 0 || head_dim > 256) return OPR_INVALID_ARG;
+  if (dtype != OPR_DTYPE_BF16 && dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
+  if (!(base > 1.0)) return OPR_INVALID_ARG;
+  if (total_tokens > 0 && n_heads > 0 && (!x || !pos_id)) return OPR_INVALID_ARG;
+  cudaError_t e = launch_rope(x, dtype, pos_id, total_tokens, n_heads, head_dim, base, inverse,
+                              static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
+}
+
+opr_status opr_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                        const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs, int32_t n_convs,
+                        int32_t n_turns, int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv,
+                        int32_t head_dim, float scale, void* o, int32_t o_dtype, float* lse, int32_t* dev_status,
+                        void* stream) {
+  if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return OPR_INVALID_ARG;
+  if (total_tokens == 0) return OPR_OK;
+  if (!attn_args_ok(q, k, v, hq, hkv, head_dim, scale)) return OPR_INVALID_ARG;
+  if (!cu_seqlens || !conv_idx || !layout_ws || !o || !lse || !dev_status || !aligned16(o)) return OPR_INVALID_ARG;
+  if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
+  opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, total_tokens, hq, head_dim) || !make_map(&tk, k, total_tokens, hkv, head_dim) ||
+      !make_map(&tv, v, total_tokens, hkv, head_dim))
+    return OPR_CUDA_ERROR;
+  AttnParams p = base_params(cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs, n_turns, total_tokens, max_seqlen, hq,
+                             hkv, scale, dev_status);
+  p.o = o;
+  p.o_fp32 = o_dtype == OPR_DTYPE_FP32;
+  p.lse = lse;
+  cudaError_t e = launch_attn_fwd(head_dim, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
+}
+
+size_t opr_attn_bwd_workspace_bytes(int64_t total_tokens, int32_t hq, int32_t head_dim) {
+  (void)head_dim;
+  if (total_tokens < 0 || hq < 0) return 0;
+  return align_up(sizeof(float) * static_cast<size_t>(total_tokens) * static_cast<size_t>(hq), 256);
+}
+
+opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, const void* o, int32_t o_dtype,
+                               const void* dout, const float* lse, const int32_t* cu_seqlens,
+                               const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs, int32_t n_convs,
+                               int32_t n_turns, int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv,
+                               int32_t head_dim, float scale, float* dq, float* dk, float* dv, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, int32_t stages, void* stream) {
+  if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return OPR_INVALID_ARG;
+  if (stages & ~(OPR_BWD_ROW_TERMS | OPR_BWD_DQ | OPR_BWD_DKDV)) return OPR_INVALID_ARG;
+  if (total_tokens == 0 || stages == 0) return OPR_OK;
+  if (!attn_args_ok(q, k, v, hq, hkv, head_dim, scale)) return OPR_INVALID_ARG;
+  if (!o || !dout || !lse || !cu_seqlens || !conv_idx || !layout_ws || !dq || !dk || !dv || !workspace ||
+      !dev_status)
+    return OPR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return OPR_INVALID_ARG;
+  if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
+  if (workspace_bytes < opr_attn_bwd_workspace_bytes(total_tokens, hq, head_dim)) return OPR_WORKSPACE_TOO_SMALL;
+  opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, total_tokens, hq, head_dim) || !make_map(&tk, k, total_tokens, hkv, head_dim) ||
+      !make_map(&tv, v, total_tokens, hkv, head_dim) || !make_map(&tdo, dout, total_tokens, hq, head_dim))
+    return OPR_CUDA_ERROR;
+  const LayoutWs w = layout_ws_map(n_seqs, n_convs, n_turns, total_tokens, max_seqlen);
+  AttnParams pq = base_params(cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs, n_turns, total_tokens, max_seqlen,
+                              hq, hkv, scale, dev_status);
+  pq.lse_in = lse;
+  pq.row_d = static_cast<const float*>(workspace);
+  pq.dq = dq;
+  pq.dk = dk;
+  pq.dv = dv;
+  AttnParams pkv = pq;
+  pkv.sched = ws_ptr<int32_t>(layout_ws, w.k_sched);
+  cudaError_t e = launch_attn_bwd(head_dim, tq, tk, tv, tdo, o, o_dtype == OPR_DTYPE_FP32, dout, pq, pkv,
+                                  static_cast<float*>(workspace), stages, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
+}
+
+opr_status opr_attn_bwd(const void* q, const void* k, const void* v, const void* o, int32_t o_dtype,
+                        const void* dout, const float* lse, const int32_t* cu_seqlens, const int32_t* conv_idx,
+                        const void* layout_ws, int32_t n_seqs, int32_t n_convs, int32_t n_turns,
+                        int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
+                        float scale, float* dq, float* dk, float* dv, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, void* stream) {
+  return opr_attn_bwd_stages(q, k, v, o, o_dtype, dout, lse, cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs,
+                             n_turns, total_tokens, max_seqlen, hq, hkv, head_dim, scale, dq, dk, dv, workspace,
+                             workspace_bytes, dev_status, OPR_BWD_ROW_TERMS | OPR_BWD_DQ | OPR_BWD_DKDV, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,638 @@
+// attn_bwd.cu - block-sparse masked attention backward for sm_100a.
+//
+// Gradients of the One-Pass to Reason attention layer (fine-tuning needs
+// them; the mask is the one of "分块稀疏注意力掩码").  With P recomputed from
+// the forward's log-sum-exp:
+//   D  = rowsum(dO * O)
+//   dV = P^T dO,   dP = dO V^T,   dS = P * (dP - D)
+//   dQ = scale dS K,   dK = scale dS^T Q   (dK, dV summed over a GQA group)
+// Deterministic split into two tcgen05 kernels (no atomics):
+//   dq kernel    one CTA per (query tile, q head), loops over the row's
+//                non-empty key tiles: S, dP -> dS (TMEM) -> dQ += dS K;
+//   dkdv kernel  one CTA per (key tile, kv head), loops over the q heads of
+//                the group and the column's non-empty query tiles:
+//                S^T = K Q^T, dP^T = V dO^T -> P^T, dS^T (TMEM) ->
+//                dV += P^T dO, dK += dS^T Q.
+// Warp roles as in the forward: warp 0 TMA producer (+ metadata lanes),
+// warp 1 TMEM owner and MMA issuer, warps 2..5 one row per thread.
+#include "attn_common.cuh"
+
+namespace opr {
+namespace {
+
+constexpr int kStages = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ----------------------------------------------------------------------------
+// D[h, q] = sum_d dO[q, h, d] * O[q, h, d]; one warp per (token, head).
+template <int D, typename OT>
+__global__ void __launch_bounds__(256) row_d_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                                                    int64_t total, int32_t hq, float* __restrict__ row_d) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= total * hq) return;
+  const int64_t tok = w / hq;
+  const int h = static_cast<int>(w % hq);
+  const size_t base = static_cast<size_t>(w) * D;
+  float acc = 0.f;
+#pragma unroll
+  for (int x = lane; x < D; x += 32) {
+    float ov;
+    if constexpr (sizeof(OT) == 4)
+      ov = o[base + x];
+    else
+      ov = __bfloat162float(o[base + x]);
+    acc = fmaf(ov, __bfloat162float(dout[base + x]), acc);
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
+  if (lane == 0) row_d[static_cast<size_t>(h) * total + tok] = acc;
+}
+
+// ----------------------------------------------------------------------------
+template <int D>
+struct DqSmem {
+  alignas(1024) uint8_t q[TileGeom<D>::kBytes];
+  alignas(1024) uint8_t dout[TileGeom<D>::kBytes];
+  alignas(1024) uint8_t k[kStages][TileGeom<D>::kBytes];
+  alignas(1024) uint8_t v[kStages][TileGeom<D>::kBytes];
+  int32_t kconv[kStages][kTile];
+  int32_t kmeta[kStages][kTile];
+  uint64_t bar_qdo;
+  uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
+  uint64_t bar_sfull, bar_dpfull, bar_dsfull, bar_dqdone, bar_final;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// TMEM columns of the dq kernel: S / dS at 0, dP at 128, dQ accumulator at 256.
+constexpr uint32_t kDqColS = 0, kDqColDP = 128, kDqColAcc = 256;
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const AttnParams p) {
+  constexpr uint32_t kTileBytes = TileGeom<D>::kBytes;
+  extern __shared__ uint8_t smem_raw[];
+  DqSmem<D>& sm = *reinterpret_cast<DqSmem<D>*>(align1024(smem_raw));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int head = blockIdx.x % p.hq;
+  const int item = blockIdx.x / p.hq;
+  if (item >= p.n_items) return;
+  const int tile_id = p.sched[item];
+  const int n = p.row_cnt[tile_id];
+  if (n == 0) return;
+  const int s = tile_id / p.T, I = tile_id % p.T;
+  const int32_t* list = p.row_list + static_cast<size_t>(tile_id) * p.T;
+  const int seq0 = p.cu_seqlens[s];
+  const int seq_len = p.cu_seqlens[s + 1] - seq0;
+  const int q0 = seq0 + I * kTile;
+  const int kvh = head / (p.hq / p.hkv);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_qdo, 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&sm.bar_kfull[st], 1 + 32);  // TMA expect-tx arrival + 32 metadata lanes
+      mbar_init(&sm.bar_kempty[st], 1);
+      mbar_init(&sm.bar_vfull[st], 1);
+      mbar_init(&sm.bar_vempty[st], 1);
+    }
+    mbar_init(&sm.bar_sfull, 1);
+    mbar_init(&sm.bar_dpfull, 1);
+    mbar_init(&sm.bar_dsfull, 128);
+    mbar_init(&sm.bar_dqdone, 1);
+    mbar_init(&sm.bar_final, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.bar_qdo, 2 * kTileBytes);
+      tma_tile<D>(&tm_q, &sm.bar_qdo, sm.q, head, q0);
+      tma_tile<D>(&tm_do, &sm.bar_qdo, sm.dout, head, q0);
+    }
+    int issued_k = 0, issued_v = 0;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % kStages;
+      const uint32_t ph = (j / kStages) & 1;
+      const int e = list[j];
+      const int J = e >> 2;
+      const int k0 = seq0 + J * kTile;
+      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_kempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
+        break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes);
+        tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, k0);
+      }
+      issued_k = j + 1;
+      if ((e & 3) == OPR_TILE_PARTIAL) {
+        for (int x = lane; x < kTile; x += 32) {
+          const bool kv = J * kTile + x < seq_len;
+          sm.kconv[st][x] = kv ? p.conv_idx[k0 + x] : -1;
+          sm.kmeta[st][x] = kv ? p.tok_meta[k0 + x] : 0;
+        }
+      }
+      mbar_arrive(&sm.bar_kfull[st]);
+      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_vempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
+        break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.bar_vfull[st], kTileBytes);
+        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, k0);
+      }
+      issued_v = j + 1;
+    }
+    if (*abort_flag && lane == 0) {
+      mbar_wait(&sm.bar_qdo, 0, nullptr, kWaitLimitNs);
+      for (int j = (issued_k > kStages ? issued_k - kStages : 0); j < issued_k; ++j)
+        mbar_wait(&sm.bar_kfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int j = (issued_v > kStages ? issued_v - kStages : 0); j < issued_v; ++j)
+        mbar_wait(&sm.bar_vfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);  // S = Q K^T, dP = dO V^T
+      constexpr uint32_t idesc_q = idesc_bf16_f32(128, D, 0, 1);    // dQ += dS K (K tile MN-major)
+      const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
+      bool ok = mbar_wait(&sm.bar_qdo, 0, abort_flag, kWaitLimitNs);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        if (!mbar_wait(&sm.bar_kfull[st], ph, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sk = smem_u32(sm.k[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + kDqColS, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.bar_sfull);
+        if (!mbar_wait(&sm.bar_vfull[st], ph, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sv = smem_u32(sm.v[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + kDqColDP, desc_kmajor(sdo, kk), desc_kmajor(sv, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.bar_dpfull);
+        mma_commit(&sm.bar_vempty[st]);
+        if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + kDqColAcc, tmem + kDqColS + kk * 8, desc_mnmajor(sk, kk), idesc_q,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.bar_kempty[st]);
+      }
+      if (ok) mma_commit(&sm.bar_dqdone);
+      mma_commit(&sm.bar_final);
+      mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const bool qv = I * kTile + row < seq_len;
+    const int qg = q0 + row;
+    const int qconv = qv ? p.conv_idx[qg] : -2;
+    const int qmeta = qv ? p.tok_meta[qg] : 0;
+    const float lse2 = qv ? p.lse_in[static_cast<size_t>(head) * p.total + qg] * kLog2e : 0.f;
+    const float dd = qv ? p.row_d[static_cast<size_t>(head) * p.total + qg] : 0.f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % kStages;
+      const int e = list[j];
+      const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+      const int kbase = seq0 + (e >> 2) * kTile;
+      if (partial &&
+          !__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float pv[kTile];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + kDqColS + c * 32, r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) pv[c * 32 + x] = fast_exp2(fmaf(__uint_as_float(r[x]), sl2, -lse2));
+      }
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (!visible(qg, qconv, qmeta, kbase + c, sm.kconv[st][c], sm.kmeta[st][c])) pv[c] = 0.f;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + kDqColDP + c * 32, r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float d0 = pv[c * 32 + 2 * x] * (__uint_as_float(r[2 * x]) - dd);
+          const float d1 = pv[c * 32 + 2 * x + 1] * (__uint_as_float(r[2 * x + 1]) - dd);
+          pk[x] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tl + kDqColS + c * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.bar_dsfull);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_dqdone, 0, abort_flag, kWaitLimitNs))) {
+      tc_fence_after();
+      float* dst = p.dq + (static_cast<size_t>(qg) * p.hq + head) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + kDqColAcc + c * 32, r);
+        if (qv) {
+          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(r[4 * x]) * p.scale, __uint_as_float(r[4 * x + 1]) * p.scale,
+                                __uint_as_float(r[4 * x + 2]) * p.scale, __uint_as_float(r[4 * x + 3]) * p.scale);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && sm.abort_flag) atomicOr(p.dev_status, OPR_DEV_WAIT_TIMEOUT);
+}
+
+// ----------------------------------------------------------------------------
+template <int D>
+struct DkdvSmem {
+  alignas(1024) uint8_t k[TileGeom<D>::kBytes];
+  alignas(1024) uint8_t v[TileGeom<D>::kBytes];
+  alignas(1024) uint8_t q[kStages][TileGeom<D>::kBytes];
+  alignas(1024) uint8_t dout[kStages][TileGeom<D>::kBytes];
+  float qlse2[kStages][kTile];
+  float qd[kStages][kTile];
+  int32_t qconv[kStages][kTile];
+  int32_t qmeta[kStages][kTile];
+  uint64_t bar_kv;
+  uint64_t bar_qfull[kStages], bar_qempty[kStages], bar_dofull[kStages], bar_doempty[kStages];
+  uint64_t bar_sfull, bar_dpfull, bar_pfull, bar_dsfull, bar_accdone, bar_final;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// TMEM columns of the dkdv kernel: S^T / P^T at 0, dP^T / dS^T at 128,
+// dV accumulator at 256, dK accumulator at 256 + D.
+constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvColDV = 256;
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                         const AttnParams p) {
+  constexpr uint32_t kTileBytes = TileGeom<D>::kBytes;
+  constexpr uint32_t kColDK = kKvColDV + D;
+  extern __shared__ uint8_t smem_raw[];
+  DkdvSmem<D>& sm = *reinterpret_cast<DkdvSmem<D>*>(align1024(smem_raw));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kvh = blockIdx.x % p.hkv;
+  const int item = blockIdx.x / p.hkv;
+  if (item >= p.n_items) return;
+  const int tile_id = p.sched[item];
+  const int cnt = p.col_cnt[tile_id];
+  if (cnt == 0) return;
+  const int group = p.hq / p.hkv;
+  const int n = cnt * group;
+  const int s = tile_id / p.T, J = tile_id % p.T;
+  const int32_t* list = p.col_list + static_cast<size_t>(tile_id) * p.T;
+  const int seq0 = p.cu_seqlens[s];
+  const int seq_len = p.cu_seqlens[s + 1] - seq0;
+  const int k0 = seq0 + J * kTile;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_kv, 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&sm.bar_qfull[st], 1 + 32);  // TMA expect-tx arrival + 32 column-data lanes
+      mbar_init(&sm.bar_qempty[st], 1);
+      mbar_init(&sm.bar_dofull[st], 1);
+      mbar_init(&sm.bar_doempty[st], 1);
+    }
+    mbar_init(&sm.bar_sfull, 1);
+    mbar_init(&sm.bar_dpfull, 1);
+    mbar_init(&sm.bar_pfull, 128);
+    mbar_init(&sm.bar_dsfull, 128);
+    mbar_init(&sm.bar_accdone, 1);
+    mbar_init(&sm.bar_final, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
+      tma_tile<D>(&tm_k, &sm.bar_kv, sm.k, kvh, k0);
+      tma_tile<D>(&tm_v, &sm.bar_kv, sm.v, kvh, k0);
+    }
+    int issued_q = 0, issued_do = 0;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % kStages;
+      const uint32_t ph = (j / kStages) & 1;
+      const int g = j / cnt;
+      const int e = list[j % cnt];
+      const int Iq = e >> 2;
+      const int qt0 = seq0 + Iq * kTile;
+      const int h = kvh * group + g;
+      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_qempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
+        break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.bar_qfull[st], kTileBytes);
+        tma_tile<D>(&tm_q, &sm.bar_qfull[st], sm.q[st], h, qt0);
+      }
+      issued_q = j + 1;
+      for (int x = lane; x < kTile; x += 32) {
+        const bool qv = Iq * kTile + x < seq_len;
+        const size_t idx = static_cast<size_t>(h) * p.total + qt0 + x;
+        sm.qlse2[st][x] = qv ? p.lse_in[idx] * kLog2e : INFINITY;
+        sm.qd[st][x] = qv ? p.row_d[idx] : 0.f;
+        if ((e & 3) == OPR_TILE_PARTIAL) {
+          sm.qconv[st][x] = qv ? p.conv_idx[qt0 + x] : -2;
+          sm.qmeta[st][x] = qv ? p.tok_meta[qt0 + x] : 0;
+        }
+      }
+      mbar_arrive(&sm.bar_qfull[st]);
+      if (j >= kStages &&
+          !__all_sync(0xffffffffu, mbar_wait(&sm.bar_doempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
+        break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.bar_dofull[st], kTileBytes);
+        tma_tile<D>(&tm_do, &sm.bar_dofull[st], sm.dout[st], h, qt0);
+      }
+      issued_do = j + 1;
+    }
+    if (*abort_flag && lane == 0) {
+      mbar_wait(&sm.bar_kv, 0, nullptr, kWaitLimitNs);
+      for (int j = (issued_q > kStages ? issued_q - kStages : 0); j < issued_q; ++j)
+        mbar_wait(&sm.bar_qfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int j = (issued_do > kStages ? issued_do - kStages : 0); j < issued_do; ++j)
+        mbar_wait(&sm.bar_dofull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
+      constexpr uint32_t idesc_a = idesc_bf16_f32(128, D, 0, 1);    // dV += P^T dO, dK += dS^T Q
+      const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
+      bool ok = mbar_wait(&sm.bar_kv, 0, abort_flag, kWaitLimitNs);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % kStages;
+        const uint32_t ph = (j / kStages) & 1;
+        if (!mbar_wait(&sm.bar_qfull[st], ph, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sq = smem_u32(sm.q[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + kKvColS, desc_kmajor(sk, kk), desc_kmajor(sq, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.bar_sfull);
+        if (!mbar_wait(&sm.bar_dofull[st], ph, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sdo = smem_u32(sm.dout[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + kKvColDP, desc_kmajor(sv, kk), desc_kmajor(sdo, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.bar_dpfull);
+        if (!mbar_wait(&sm.bar_pfull, j & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + kKvColDV, tmem + kKvColS + kk * 8, desc_mnmajor(sdo, kk), idesc_a,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.bar_doempty[st]);
+        if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + kColDK, tmem + kKvColDP + kk * 8, desc_mnmajor(sq, kk), idesc_a,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.bar_qempty[st]);
+      }
+      if (ok) mma_commit(&sm.bar_accdone);
+      mma_commit(&sm.bar_final);
+      mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const bool kvld = J * kTile + row < seq_len;
+    const int kg = k0 + row;
+    const int kconv = kvld ? p.conv_idx[kg] : -1;
+    const int kmeta = kvld ? p.tok_meta[kg] : 0;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % kStages;
+      const int e = list[j % cnt];
+      const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+      const int qt0 = seq0 + (e >> 2) * kTile;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float pv[kTile];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + kKvColS + c * 32, r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          pv[c * 32 + x] = fast_exp2(fmaf(__uint_as_float(r[x]), sl2, -sm.qlse2[st][c * 32 + x]));
+      }
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (!visible(qt0 + c, sm.qconv[st][c], sm.qmeta[st][c], kg, kconv, kmeta)) pv[c] = 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(pv[c * 32 + 2 * x], pv[c * 32 + 2 * x + 1]);
+        tmem_st16(tl + kKvColS + c * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.bar_pfull);
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + kKvColDP + c * 32, r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float d0 = pv[c * 32 + 2 * x] * (__uint_as_float(r[2 * x]) - sm.qd[st][c * 32 + 2 * x]);
+          const float d1 = pv[c * 32 + 2 * x + 1] * (__uint_as_float(r[2 * x + 1]) - sm.qd[st][c * 32 + 2 * x + 1]);
+          pk[x] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(tl + kKvColDP + c * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.bar_dsfull);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_accdone, 0, abort_flag, kWaitLimitNs))) {
+      tc_fence_after();
+      float* dvp = p.dv + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
+      float* dkp = p.dk + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + kKvColDV + c * 32, r);
+        if (kvld) {
+          float4* d4 = reinterpret_cast<float4*>(dvp + c * 32);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(r[4 * x]), __uint_as_float(r[4 * x + 1]),
+                                __uint_as_float(r[4 * x + 2]), __uint_as_float(r[4 * x + 3]));
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + kColDK + c * 32, r);
+        if (kvld) {
+          float4* d4 = reinterpret_cast<float4*>(dkp + c * 32);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(r[4 * x]) * p.scale, __uint_as_float(r[4 * x + 1]) * p.scale,
+                                __uint_as_float(r[4 * x + 2]) * p.scale, __uint_as_float(r[4 * x + 3]) * p.scale);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && sm.abort_flag) atomicOr(p.dev_status, OPR_DEV_WAIT_TIMEOUT);
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t smem, int* configured) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && configured[dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess && dev < 64) configured[dev] = 1;
+  return e;
+}
+
+template <int D>
+cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                         const void* o, int o_fp32, const void* dout, const AttnParams& pq, const AttnParams& pkv,
+                         float* row_d, int stages, cudaStream_t stream) {
+  static int conf_dq[64] = {0}, conf_kv[64] = {0};
+  cudaError_t e = cudaSuccess;
+  // 1) row terms D
+  const int64_t warps = pq.total * pq.hq;
+  if ((stages & OPR_BWD_ROW_TERMS) && warps > 0) {
+    const int64_t blocks = (warps * 32 + 255) / 256;
+    if (o_fp32)
+      row_d_kernel<D, float><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dout), pq.total, pq.hq, row_d);
+    else
+      row_d_kernel<D, __nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), pq.total, pq.hq, row_d);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // 2) dQ
+  if (stages & OPR_BWD_DQ) {
+    const size_t smem_q = smem_request(sizeof(DqSmem<D>) + 1024);
+    if ((e = set_smem(attn_bwd_dq_kernel<D>, smem_q, conf_dq)) != cudaSuccess) return e;
+    const int64_t bq = static_cast<int64_t>(pq.n_items) * pq.hq;
+    if (bq > 0) attn_bwd_dq_kernel<D><<<static_cast<unsigned>(bq), 192, smem_q, stream>>>(tq, tk, tv, tdo, pq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // 3) dK, dV
+  if (stages & OPR_BWD_DKDV) {
+    const size_t smem_kv = smem_request(sizeof(DkdvSmem<D>) + 1024);
+    if ((e = set_smem(attn_bwd_dkdv_kernel<D>, smem_kv, conf_kv)) != cudaSuccess) return e;
+    const int64_t bkv = static_cast<int64_t>(pkv.n_items) * pkv.hkv;
+    if (bkv > 0)
+      attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(bkv), 192, smem_kv, stream>>>(tq, tk, tv, tdo, pkv);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const void* o, int o_fp32, const void* dout,
+                            const AttnParams& pq, const AttnParams& pkv, float* row_d, int stages,
+                            cudaStream_t stream) {
+  if (head_dim == 128) return launch_bwd_t<128>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream);
+  return launch_bwd_t<64>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream);
+}
+
+}  // namespace opr

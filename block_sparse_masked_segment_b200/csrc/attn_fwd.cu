@@ -1,0 +1,328 @@
+// attn_fwd.cu - block-sparse masked attention forward for sm_100a.
+//
+// One-Pass to Reason, "分块稀疏注意力掩码": attention restricted by the per-type
+// visibility rules, evaluated block-sparsely (the pages use a FlexAttention
+// block mask on H100, "实现细节"; this is a hand-written Blackwell kernel).
+//
+// One CTA per (query tile of 128 rows, q head), 6 warps:
+//   warp 0      loads Q once and the K/V tiles of the row's non-empty tiles
+//               with TMA (2-stage ring); its lanes also stage the key-side
+//               metadata of partial tiles;
+//   warp 1      allocates TMEM and issues tcgen05.mma: S = Q K^T into one of
+//               two TMEM buffers, then O += P V with P read from TMEM;
+//   warps 2..5  one query row per thread: read S from TMEM, apply the
+//               visibility predicate on partial tiles only, online softmax in
+//               base 2, write P (bf16) back over S, rescale O in TMEM only
+//               when the running max grows by more than 2^8; epilogue O / l
+//               and the log-sum-exp.
+// TMEM columns: S/P buffer 0 at 0, buffer 1 at 128, O at 256 (512 allocated).
+#include "attn_common.cuh"
+
+namespace opr {
+namespace {
+
+constexpr int kStages = 2;
+constexpr uint32_t kOCol = 256;
+
+template <int D>
+struct FwdSmem {
+  alignas(1024) uint8_t q[TileGeom<D>::kBytes];
+  alignas(1024) uint8_t k[kStages][TileGeom<D>::kBytes];
+  alignas(1024) uint8_t v[kStages][TileGeom<D>::kBytes];
+  int32_t kconv[kStages][kTile];
+  int32_t kmeta[kStages][kTile];
+  uint64_t bar_q;
+  uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
+  uint64_t bar_sfull[2], bar_pfull[2], bar_odone, bar_final;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  constexpr uint32_t kTileBytes = TileGeom<D>::kBytes;
+  extern __shared__ uint8_t smem_raw[];
+  FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(align1024(smem_raw));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int head = blockIdx.x % p.hq;
+  const int item = blockIdx.x / p.hq;
+  if (item >= p.n_items) return;
+  const int tile_id = p.sched[item];
+  const int n = p.row_cnt[tile_id];
+  if (n == 0) return;  // tile past the end of its sequence
+  const int s = tile_id / p.T, I = tile_id % p.T;
+  const int32_t* list = p.row_list + static_cast<size_t>(tile_id) * p.T;
+  const int seq0 = p.cu_seqlens[s];
+  const int seq_len = p.cu_seqlens[s + 1] - seq0;
+  const int q0 = seq0 + I * kTile;
+  const int kvh = head / (p.hq / p.hkv);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_q, 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&sm.bar_kfull[st], 1);
+      mbar_init(&sm.bar_kempty[st], 1);
+      mbar_init(&sm.bar_vfull[st], 1 + 32);  // TMA expect-tx arrival + 32 metadata lanes
+      mbar_init(&sm.bar_vempty[st], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.bar_sfull[b], 1);
+      mbar_init(&sm.bar_pfull[b], 128);
+    }
+    mbar_init(&sm.bar_odone, 1);
+    mbar_init(&sm.bar_final, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(&sm.bar_q, kTileBytes);
+      tma_tile<D>(&tm_q, &sm.bar_q, sm.q, head, q0);
+    }
+    int issued_k = 0, issued_v = 0;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % kStages;
+      const uint32_t ph = (j / kStages) & 1;
+      const int e = list[j];
+      const int J = e >> 2;
+      const int k0 = seq0 + J * kTile;
+      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_kempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
+        break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes);
+        tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, k0);
+      }
+      issued_k = j + 1;
+      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_vempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
+        break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&sm.bar_vfull[st], kTileBytes);
+        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, k0);
+      }
+      issued_v = j + 1;
+      if ((e & 3) == OPR_TILE_PARTIAL) {
+        for (int x = lane; x < kTile; x += 32) {
+          const bool kv = J * kTile + x < seq_len;
+          sm.kconv[st][x] = kv ? p.conv_idx[k0 + x] : -1;
+          sm.kmeta[st][x] = kv ? p.tok_meta[k0 + x] : 0;
+        }
+      }
+      mbar_arrive(&sm.bar_vfull[st]);
+    }
+    if (*abort_flag && lane == 0) {
+      // Let the copies already in flight land before the CTA exits.
+      for (int j = (issued_k > kStages ? issued_k - kStages : 0); j < issued_k; ++j)
+        mbar_wait(&sm.bar_kfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int j = (issued_v > kStages ? issued_v - kStages : 0); j < issued_v; ++j)
+        mbar_wait(&sm.bar_vfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t sq = smem_u32(sm.q);
+      bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, kWaitLimitNs);
+      auto issue_pv = [&](int jp) -> bool {
+        const int bp = jp & 1, stp = jp % kStages;
+        if (!mbar_wait(&sm.bar_pfull[bp], (jp >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
+        if (!mbar_wait(&sm.bar_vfull[stp], (jp / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
+        tc_fence_after();
+        const uint32_t sv = smem_u32(sm.v[stp]);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + kOCol, tmem + bp * 128 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
+                 (jp > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.bar_vempty[stp]);
+        mma_commit(&sm.bar_odone);
+        return true;
+      };
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % kStages, b = j & 1;
+        if (!mbar_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sk = smem_u32(sm.k[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + b * 128, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.bar_sfull[b]);
+        mma_commit(&sm.bar_kempty[st]);
+        if (j >= 1 && !issue_pv(j - 1)) ok = false;
+      }
+      if (ok) issue_pv(n - 1);
+      // All MMAs issued by this thread must be complete before TMEM is freed.
+      mma_commit(&sm.bar_final);
+      mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int row = quad * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const bool qv = I * kTile + row < seq_len;
+    const int qg = q0 + row;
+    const int qconv = qv ? p.conv_idx[qg] : -2;
+    const int qmeta = qv ? p.tok_meta[qg] : 0;
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int b = j & 1, st = j % kStages;
+      const int e = list[j];
+      const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+      const int kbase = seq0 + (e >> 2) * kTile;
+      if (partial &&
+          !__all_sync(0xffffffffu, mbar_wait(&sm.bar_vfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[b], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[kTile];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + b * 128 + c * 32, r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) sv[c * 32 + x] = __uint_as_float(r[x]);
+      }
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (!visible(qg, qconv, qmeta, kbase + c, sm.kconv[st][c], sm.kmeta[st][c])) sv[c] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, sv[c]);
+      const float m_new = fmaxf(m_run, mx * sl2);
+      const bool need = m_new > m_run + 8.f;  // also true on the first finite max
+      const float m_use = need ? m_new : m_run;
+      const float mb = (m_use == -INFINITY) ? 0.f : m_use;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float p0 = fast_exp2(fmaf(sv[c * 32 + 2 * x], sl2, -mb));
+          const float p1 = fast_exp2(fmaf(sv[c * 32 + 2 * x + 1], sl2, -mb));
+          rs += p0 + p1;
+          pk[x] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tl + b * 128 + c * 16, pk);
+      }
+      tmem_wait_st();
+      // O may be rescaled only once the previous P V product has landed.
+      if (j >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_odone, (j - 1) & 1, abort_flag, kWaitLimitNs))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      const float factor = need ? fast_exp2(m_run - m_new) : 1.f;
+      if (__any_sync(0xffffffffu, need && j >= 1)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tl + kOCol + c * 32, r);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * factor);
+          tmem_st32(tl + kOCol + c * 32, r);
+        }
+        tmem_wait_st();
+      }
+      l_run = l_run * factor + rs;
+      if (need) m_run = m_new;
+      tc_fence_before();
+      mbar_arrive(&sm.bar_pfull[b]);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_odone, (n - 1) & 1, abort_flag, kWaitLimitNs))) {
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+      const size_t orow = (static_cast<size_t>(qg) * p.hq + head) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + kOCol + c * 32, r);
+        if (qv) {
+          if (p.o_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c * 32);
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              dst[x] = make_float4(__uint_as_float(r[4 * x]) * inv, __uint_as_float(r[4 * x + 1]) * inv,
+                                   __uint_as_float(r[4 * x + 2]) * inv, __uint_as_float(r[4 * x + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow + c * 32);
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              dst[x] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * x]) * inv, __uint_as_float(r[8 * x + 1]) * inv),
+                                  pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv, __uint_as_float(r[8 * x + 3]) * inv),
+                                  pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv, __uint_as_float(r[8 * x + 5]) * inv),
+                                  pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv, __uint_as_float(r[8 * x + 7]) * inv));
+          }
+        }
+      }
+      if (qv) p.lse[static_cast<size_t>(head) * p.total + qg] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && sm.abort_flag) atomicOr(p.dev_status, OPR_DEV_WAIT_TIMEOUT);
+}
+
+}  // namespace
+
+template <int D>
+cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const AttnParams& p, cudaStream_t stream) {
+  const size_t smem = smem_request(sizeof(FwdSmem<D>) + 1024);
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  const int64_t blocks = static_cast<int64_t>(p.n_items) * p.hq;
+  if (blocks == 0) return cudaSuccess;
+  attn_fwd_kernel<D><<<static_cast<unsigned>(blocks), 192, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attn_fwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const AttnParams& p, cudaStream_t stream) {
+  if (head_dim == 128) return launch_attn_fwd_t<128>(tq, tk, tv, p, stream);
+  return launch_attn_fwd_t<64>(tq, tk, tv, p, stream);
+}
+
+}  // namespace opr

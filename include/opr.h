@@ -1,0 +1,205 @@
+/*
+ * opr.h - One-Pass to Reason masked attention on NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libopr.so.  The operation is the attention layer of
+ * "One-Pass to Reason: Token Duplication and Block-Sparse Mask for Efficient
+ * Fine-Tuning on Multi-Turn Reasoning" (Goru, Mehta, Jain): every turn i of a
+ * conversation is packed as h_i, t_i, r_i^in, r_i^out (the response r_i is
+ * stored twice), and attention follows per-type visibility rules so that one
+ * pass over the conversation gives the same rows as N causal passes.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Array arguments are DEVICE pointers owned by the caller.  The library
+ *    never allocates, frees or retains device memory; it keeps no state
+ *    between calls except cached kernel attributes and the driver entry point
+ *    used to encode TMA descriptors.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = legacy default stream).  The return value reports host-side
+ *    argument checks and launch errors only.
+ *  - Errors found on the device (inconsistent sizes, a pipeline wait that
+ *    timed out) are OR-ed as OPR_DEV_* bits into the caller's int32
+ *    `dev_status` word, which the caller zeroes before the first call and
+ *    reads after synchronising.  No call aborts, traps or throws.
+ *  - Token-major tensors are [total_tokens, heads, head_dim], contiguous,
+ *    sequences packed back to back (offsets in cu_seqlens).  LSE and the
+ *    backward's row terms are [heads, total_tokens].
+ *  - Token types: 0 = h (human message), 1 = t (reasoning), 2 = r^in (response,
+ *    context copy), 3 = r^out (response, generation copy).
+ */
+#ifndef OPR_H_
+#define OPR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define OPR_API __attribute__((visibility("default")))
+#else
+#define OPR_API
+#endif
+
+typedef int32_t opr_status;
+
+#define OPR_OK 0
+#define OPR_INVALID_ARG 1          /* null pointer, negative size, Hq % Hkv != 0, bad head_dim ... */
+#define OPR_UNSUPPORTED 2          /* dtype or device (needs compute capability 10.0) not supported */
+#define OPR_CUDA_ERROR 3           /* a CUDA runtime/driver call or a kernel launch failed */
+#define OPR_WORKSPACE_TOO_SMALL 4  /* workspace_bytes below what the *_workspace_bytes query returns */
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define OPR_DEV_BAD_INPUT 1        /* negative length or non-monotone turn/conversation pointers */
+#define OPR_DEV_TOTAL_MISMATCH 2   /* sum of h + t + 2r differs from total_tokens */
+#define OPR_DEV_SEQ_TOO_LONG 4     /* a sequence is longer than max_seqlen */
+#define OPR_DEV_WAIT_TIMEOUT 8     /* a pipeline wait exceeded its time limit; outputs are invalid */
+
+#define OPR_DTYPE_BF16 0
+#define OPR_DTYPE_FP32 1
+
+#define OPR_TILE 128               /* edge of a block-map tile, in tokens */
+#define OPR_TILE_EMPTY 0
+#define OPR_TILE_FULL 1
+#define OPR_TILE_PARTIAL 2
+
+/*
+ * Bytes of the layout workspace that opr_build_layout fills and the attention
+ * calls read (per-tile lists of non-empty tiles, packed per-token type/turn,
+ * per-turn offsets and the tile schedule).  Depends only on the sizes.
+ */
+OPR_API size_t opr_layout_workspace_bytes(int32_t n_seqs, int32_t n_convs, int32_t n_turns,
+                                  int64_t total_tokens, int32_t max_seqlen);
+
+/*
+ * opr_build_layout - token duplication, position ids and the block map.
+ *
+ * Defined by the One-Pass to Reason wiki note: "Token 复制" (r_i stored as
+ * r_i^in and r_i^out), "位置 ID 策略" (s_t = s_rin = e_h + 1, s_rout = e_t + 1,
+ * s_h(i+1) = e_rin + 1; the first position of every conversation is 0) and
+ * "分块稀疏注意力掩码" (h_i sees H<i; t_i and r_i^in see H<i and h_i; r_i^out
+ * sees H<i, h_i and t_i; H<i = {h_j, r_j^in : j < i}; every segment causal
+ * within itself; conversations packed in one sequence never see each other).
+ *
+ * Inputs (device):
+ *   turn_lens      int32 [n_turns][3]  (h, t, r) of each turn, each >= 0
+ *   conv_turn_ptr  int32 [n_convs+1]   turns of conversation c are
+ *                                      conv_turn_ptr[c] .. conv_turn_ptr[c+1]-1
+ *   seq_conv_ptr   int32 [n_seqs+1]    conversations of sequence s
+ *   total_tokens   sum over turns of h + t + 2r (host value, checked on device)
+ *   max_seqlen     an upper bound of every sequence's length (host value)
+ * Outputs (device, caller-allocated):
+ *   cu_seqlens     int32 [n_seqs+1]    token offset of each sequence
+ *   token_type     int8  [total]       0 h, 1 t, 2 r^in, 3 r^out
+ *   turn_idx       int32 [total]       turn index within the conversation (0-based)
+ *   conv_idx       int32 [total]       global conversation index
+ *   pos_id         int32 [total]       position id
+ *   block_map      uint8 [n_seqs][T][T], T = ceil(max_seqlen / 128): tile (I, J)
+ *                  of sequence s is 0 empty, 1 full (all 128 x 128 pairs
+ *                  visible), 2 partial; indices past the sequence count as
+ *                  not visible, so tail tiles are never full
+ *   workspace      opr_layout_workspace_bytes(...) bytes, read by the attention calls
+ *   dev_status     int32 word, OPR_DEV_* bits OR-ed in on inconsistent input
+ * Returns OPR_INVALID_ARG for null pointers / negative sizes / n_seqs > n_convs
+ * inconsistencies detectable on the host, OPR_WORKSPACE_TOO_SMALL, OPR_CUDA_ERROR.
+ */
+OPR_API opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* conv_turn_ptr,
+                            const int32_t* seq_conv_ptr, int32_t n_seqs, int32_t n_convs,
+                            int32_t n_turns, int64_t total_tokens, int32_t max_seqlen,
+                            int32_t* cu_seqlens, int8_t* token_type, int32_t* turn_idx,
+                            int32_t* conv_idx, int32_t* pos_id, uint8_t* block_map,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream);
+
+/*
+ * opr_rope - rotary position embedding by position id, in place.
+ *
+ * The pages' position-equivalence argument ("理论保证") is about the rotary
+ * positions of Qwen-3 (rotate-half convention): for j < head_dim/2 the pair
+ * (x[j], x[j + head_dim/2]) is rotated by angle pos_id * base^(-2j/head_dim)
+ * (by -angle when `inverse` != 0, which maps gradients w.r.t. rotated values
+ * back to gradients w.r.t. the unrotated ones).  Angles are formed in fp64.
+ *   x       [total_tokens, n_heads, head_dim], dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32
+ *   pos_id  int32 [total_tokens]
+ * head_dim must be even and <= 256.
+ */
+OPR_API opr_status opr_rope(void* x, int32_t dtype, const int32_t* pos_id, int64_t total_tokens,
+                    int32_t n_heads, int32_t head_dim, double base, int32_t inverse,
+                    void* stream);
+
+/*
+ * opr_attn_fwd - block-sparse masked attention forward (tcgen05 / TMEM / TMA).
+ *
+ * O = softmax(scale * Q K^T restricted to visible keys) V for each q head;
+ * q head h reads kv head h / (hq / hkv).  Tiles marked empty in the block map
+ * are skipped, the visibility predicate is evaluated only on partial tiles.
+ *   q            bf16 [total, hq, head_dim]   (already rotated)
+ *   k, v         bf16 [total, hkv, head_dim]
+ *   cu_seqlens, conv_idx, layout_ws: outputs of opr_build_layout for the same sizes
+ *   o            [total, hq, head_dim], o_dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32
+ *   lse          fp32 [hq, total]: natural-log sum of exp(scale * q.k) over visible keys
+ * head_dim must be 64 or 128; all pointers 16-byte aligned.
+ */
+OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                        const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs,
+                        int32_t n_convs, int32_t n_turns, int64_t total_tokens,
+                        int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
+                        float scale, void* o, int32_t o_dtype, float* lse, int32_t* dev_status,
+                        void* stream);
+
+/* Bytes of scratch that opr_attn_bwd needs (the row terms D = rowsum(dO * O)). */
+OPR_API size_t opr_attn_bwd_workspace_bytes(int64_t total_tokens, int32_t hq, int32_t head_dim);
+
+/*
+ * opr_attn_bwd - gradients of opr_attn_fwd w.r.t. the rotated q, k and v.
+ *
+ * With P recomputed from LSE: D = rowsum(dO * O), dV = P^T dO,
+ * dS = P * (dO V^T - D), dQ = scale dS K, dK = scale dS^T Q; dK and dV sum
+ * over the q heads that share a kv head.  Deterministic (no atomics).
+ *   q, k, v, o, dout  as in opr_attn_fwd (o in o_dtype, dout bf16)
+ *   lse               fp32 [hq, total] from opr_attn_fwd
+ *   dq                fp32 [total, hq, head_dim]
+ *   dk, dv            fp32 [total, hkv, head_dim]
+ *   workspace         opr_attn_bwd_workspace_bytes(...) bytes of device scratch
+ */
+OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        int32_t o_dtype, const void* dout, const float* lse,
+                        const int32_t* cu_seqlens, const int32_t* conv_idx, const void* layout_ws,
+                        int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
+                        int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
+                        float scale, float* dq, float* dk, float* dv, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * opr_attn_bwd_stages - the same computation as opr_attn_bwd, split into its
+ * three kernels so that a caller can order, overlap or time them one by one.
+ * `stages` is an OR of:
+ *   OPR_BWD_ROW_TERMS  D = rowsum(dO * O) into `workspace` (needed by the other two)
+ *   OPR_BWD_DQ         dq   (one CTA per query tile and q head)
+ *   OPR_BWD_DKDV       dk, dv (one CTA per key tile and kv head; GQA group summed in the CTA)
+ * Running all three, in this order on one stream, equals opr_attn_bwd.
+ * Other arguments and error behaviour as for opr_attn_bwd; unknown bits give
+ * OPR_INVALID_ARG.
+ */
+#define OPR_BWD_ROW_TERMS 1
+#define OPR_BWD_DQ 2
+#define OPR_BWD_DKDV 4
+OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, const void* o,
+                                       int32_t o_dtype, const void* dout, const float* lse,
+                                       const int32_t* cu_seqlens, const int32_t* conv_idx,
+                                       const void* layout_ws, int32_t n_seqs, int32_t n_convs,
+                                       int32_t n_turns, int64_t total_tokens, int32_t max_seqlen,
+                                       int32_t hq, int32_t hkv, int32_t head_dim, float scale, float* dq,
+                                       float* dk, float* dv, void* workspace, size_t workspace_bytes,
+                                       int32_t* dev_status, int32_t stages, void* stream);
+
+/* Library version string, e.g. "opr 0.1.0 sm_100a". */
+OPR_API const char* opr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OPR_H_ */

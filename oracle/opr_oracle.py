@@ -319,10 +319,9 @@ def attention_cols(q, k, v, do, lay: Layout, cols, kv_head: int, scale: float | 
     group = hq // hkv
     scale = 1.0 / np.sqrt(d) if scale is None else scale
     cols = np.asarray(cols)
-    col_pos = {int(c): n for n, c in enumerate(cols)}
     dk = np.zeros((len(cols), d))
     dv = np.zeros((len(cols), d))
-    # candidate rows: same sequence, at or after the earliest selected key
+    # candidate rows: same conversation, at or after the earliest selected key
     cand = set()
     for c in cols:
         s = _seq_of(lay, int(c))
@@ -333,10 +332,14 @@ def attention_cols(q, k, v, do, lay: Layout, cols, kv_head: int, scale: float | 
         s = _seq_of(lay, tok)
         a = int(lay.cu_seqlens[s])
         vis = mask_row(lay, tok, a, tok + 1)
-        vcols = a + np.nonzero(vis)[0]
-        hit = [(j, col_pos[int(c)]) for j, c in enumerate(vcols) if int(c) in col_pos]
-        if not hit:
+        sel = cols[(cols >= a) & (cols <= tok)]
+        if not np.any(vis[sel - a]):
             continue
+        vcols = a + np.nonzero(vis)[0]
+        # position of each selected key inside vcols, or -1 when not visible
+        where = np.searchsorted(vcols, cols)
+        hit = [(int(wi), n) for n, (wi, c) in enumerate(zip(where, cols))
+               if wi < len(vcols) and vcols[wi] == c]
         kk = k[vcols, kv_head].astype(np.float64)
         vv = v[vcols, kv_head].astype(np.float64)
         for h in range(kv_head * group, (kv_head + 1) * group):

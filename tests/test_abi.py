@@ -1,0 +1,92 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/opr.h declares, and rejects bad arguments on the host before touching
+the device."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import block_sparse_masked_segment_b200 as opr
+from block_sparse_masked_segment_b200 import build as opr_build
+from block_sparse_masked_segment_b200.pipeline import visible_pairs_closed_form
+import synth
+from oracle import opr_oracle as orc
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "opr.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    opr_build.build()
+    return opr.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"OPR_API\s+[\w\s\*]+?\b(opr_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 8
+    assert set(names) == set(opr.EXPORTED_SYMBOLS)
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_version(lib):
+    assert opr.opr_version().startswith("opr ")
+
+
+def test_workspace_queries(lib):
+    b = opr.opr_layout_workspace_bytes(2, 5, 20, 30000, 16384)
+    assert b > 4 * 30000 and b % 256 == 0
+    assert opr.opr_layout_workspace_bytes(-1, 5, 20, 30000, 16384) == 0
+    assert opr.opr_layout_workspace_bytes(1, 1, 1, 1 << 31, 100) == 0
+    assert opr.opr_attn_bwd_workspace_bytes(1000, 8, 128) >= 4 * 8000
+
+
+def test_host_argument_checks(lib):
+    """Null pointers, bad head counts and dims are refused with OPR_INVALID_ARG
+    (1) before any CUDA call, so this runs without a GPU."""
+    N = None
+    # opr_build_layout with null outputs
+    assert lib.opr_build_layout(N, N, N, 1, 1, 1, 10, 10, N, N, N, N, N, N, N, 0, N, N) == 1
+    # negative sizes
+    assert lib.opr_build_layout(N, N, N, -1, 1, 1, 10, 10, N, N, N, N, N, N, N, 0, N, N) == 1
+    # opr_rope: odd head_dim, bad dtype, null pointer
+    assert lib.opr_rope(N, 0, N, 10, 2, 63, 1e4, 0, N) == 1
+    assert lib.opr_rope(N, 7, N, 10, 2, 64, 1e4, 0, N) == 2
+    assert lib.opr_rope(N, 0, N, 10, 2, 64, 1e4, 0, N) == 1
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    # opr_attn_fwd: null q; hq % hkv != 0; head_dim 96
+    assert lib.opr_attn_fwd(N, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
+                            fake, 0, fake, fake, N) == 1
+    assert lib.opr_attn_fwd(fake, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100, 6, 4, 128, 0.1,
+                            fake, 0, fake, fake, N) == 1
+    assert lib.opr_attn_fwd(fake, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 96, 0.1,
+                            fake, 0, fake, fake, N) == 1
+    # opr_attn_bwd_stages: unknown stage bits
+    assert lib.opr_attn_bwd_stages(fake, fake, fake, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
+                                   4, 2, 128, 0.1, fake, fake, fake, fake, 1 << 20, fake, 8, N) == 1
+    # empty problems are no-ops
+    assert lib.opr_attn_fwd(N, N, N, N, N, N, 0, 0, 0, 0, 0, 4, 2, 128, 0.1, N, 0, N, N, N) == 0
+
+
+def test_closed_form_pair_count_matches_oracle():
+    """The benchmark's useful-work count equals the oracle's mask count."""
+    for seed in range(4):
+        w = synth.random_small_workload(seed)
+        lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+        assert visible_pairs_closed_form(w.turn_lens, w.conv_turn_ptr) == orc.visible_pairs(lay)
+
+
+def test_npass_workload_is_causal_sequences():
+    w = synth.make_workload(3, n_turns=4)
+    nw, origin = synth.npass_workload(w)
+    assert nw.n_seqs == 4 and [i for _, i in origin] == [0, 1, 2, 3]
+    # N-pass sequence of turn i: sum_{j<i}(h+r) + h + t + r = 384 i + 896
+    np.testing.assert_array_equal(nw.seq_lengths(), [896, 1280, 1664, 2048])

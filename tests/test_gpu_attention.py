@@ -1,0 +1,188 @@
+"""GPU parity of the attention forward and backward against the fp64 oracle.
+
+Element by element at sizes the oracle evaluates densely in seconds (several
+128-token tiles, ragged tails, zero-length segments, GQA, head_dim 64 and 128);
+on sampled rows and keys at the full workload sizes, in the launch
+configuration the benchmark times; plus properties that hold at any size.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_masked_segment_b200 as opr
+import synth
+from oracle import opr_oracle as orc
+from parity_helpers import assert_close, inputs, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_gpu(w, q, k, v, do, out_dtype=torch.float32):
+    att = opr.OnePassAttention(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, base=w.base)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    o, lse, qr, kr = att.forward(qd, kd, vd, out_dtype=out_dtype)
+    res = dict(o=o, lse=lse)
+    if do is not None:
+        dq, dk, dv = att.backward(qr, kr, vd, o, to_dev(do), lse)
+        res.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert opr.read_status(att.layout.dev_status) == []
+    return {kk: vv.float().cpu().numpy() for kk, vv in res.items()}, att.layout
+
+
+def _dense_check(w, seed, bwd=True):
+    q, k, v, do = inputs(w, seed, with_do=bwd)
+    got, _ = _run_gpu(w, q, k, v, do)
+    lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    o, lse = orc.forward(q, k, v, lay, w.base)
+    assert_close("O", got["o"], o)
+    assert_close("LSE", got["lse"], lse)
+    if bwd:
+        dq, dk, dv = orc.backward(q, k, v, o, do, lse, lay, w.base)
+        assert_close("dQ", got["dq"], dq)
+        assert_close("dK", got["dk"], dk)
+        assert_close("dV", got["dv"], dv)
+
+
+@pytest.mark.parametrize("seed", range(3))
+@pytest.mark.parametrize("d", [128, 64])
+def test_fwd_bwd_random_ragged(seed, d):
+    w = synth.random_small_workload(seed, n_seqs=2, max_convs=3, max_turns=4, hq=4, hkv=2, d=d, base=1e4)
+    _dense_check(w, 100 + seed)
+
+
+def test_fwd_bwd_tiny_config():
+    """Tiny workload: N = 2 turns of h16 t32 r16, one head of 64, base 1e4 (bf16-rounded inputs)."""
+    _dense_check(synth.make_workload(0), 1000)
+
+
+def test_fwd_bwd_gqa_8_to_1():
+    w = synth.random_small_workload(7, n_seqs=1, max_convs=2, max_turns=3, hq=8, hkv=1, d=128, base=1e6)
+    _dense_check(w, 7)
+
+
+def test_fwd_bwd_segment_edges():
+    """Segments and conversations that start and end on and next to tile edges; a 1-token sequence."""
+    w = synth.make_custom_workload([
+        [[(128, 128, 64)], [(127, 1, 128), (1, 127, 129)]],
+        [[(1, 0, 0)]],
+        [[(0, 0, 1), (3, 0, 0)], [(200, 57, 0)]],
+    ], hq=2, hkv=1, d=128, base=1e4)
+    _dense_check(w, 3)
+
+
+def test_fwd_bf16_output_is_rounded_fp32():
+    w = synth.random_small_workload(11, hq=2, hkv=1, d=128)
+    q, k, v, _ = inputs(w, 11, with_do=False)
+    g32, _ = _run_gpu(w, q, k, v, None, torch.float32)
+    g16, _ = _run_gpu(w, q, k, v, None, torch.bfloat16)
+    np.testing.assert_array_equal(g16["o"], synth.round_bf16(g32["o"]))
+
+
+def test_theorem_2_1_on_gpu_path():
+    """The N-pass runs of the same conversations through the same kernels give the
+    one-pass rows of t_i and r_i^out (and of h_j, r_j^in) within the float standard."""
+    w = synth.random_small_workload(5, n_seqs=1, max_convs=2, max_turns=4, hq=4, hkv=2, d=128, base=1e6)
+    q, k, v, _ = inputs(w, 5, with_do=False)
+    one, _ = _run_gpu(w, q, k, v, None)
+    lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    lists = orc.npass_token_lists(lay, w.turn_lens, w.conv_turn_ptr)
+    idx = np.concatenate([t for _, _, t in lists])
+    nw, origin = synth.npass_workload(w)
+    assert [(c, i) for c, i, _ in lists] == origin
+    many, _ = _run_gpu(nw, q[idx], k[idx], v[idx], None)
+    assert_close("O one-pass vs N-pass", one["o"][idx], many["o"])
+    assert_close("LSE one-pass vs N-pass", one["lse"][:, idx], many["lse"])
+
+
+# ---------------------------------------------------------------- full sizes
+
+def _sample_rows(lay, rng, n):
+    return np.sort(rng.choice(lay.total, size=min(n, lay.total), replace=False))
+
+
+def _tail_keys(lay, rng, n, tail=24):
+    """Keys among the last `tail` tokens of the r^in and r^out segments of each
+    conversation's last turn: only a few rows see them, so the oracle can
+    evaluate their column sums exactly."""
+    keys = []
+    for c in np.unique(lay.conv_idx):
+        sel = np.nonzero(lay.conv_idx == c)[0]
+        last = sel[lay.turn_idx[sel] == lay.turn_idx[sel].max()]
+        for typ in (orc.RIN, orc.ROUT):
+            seg = last[lay.token_type[last] == typ]
+            keys.append(seg[-tail:])
+    keys = np.concatenate(keys)
+    return np.sort(rng.choice(keys, size=min(n, len(keys)), replace=False))
+
+
+def _dk_sum_post_rope(dk_pre, lay, base, kv_head):
+    """Rows of dS sum to zero, so the keys' gradients w.r.t. the rotated k sum to zero."""
+    post = orc.rope(dk_pre[:, kv_head:kv_head + 1, :].astype(np.float64), lay.pos_id, base)[:, 0]
+    return np.abs(post.sum(0)).max() / np.abs(post).sum(0).max()
+
+
+@pytest.mark.parametrize("config", [1, 2, 4])
+def test_full_size_sampled(config):
+    w = synth.make_workload(config)
+    bwd = config != 1
+    q, k, v, do = inputs(w, 1000 + config, with_do=bwd)
+    got, _ = _run_gpu(w, q, k, v, do)
+    lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    qr = orc.rope(q, lay.pos_id, w.base)
+    kr = orc.rope(k, lay.pos_id, w.base)
+    rng = np.random.default_rng(config)
+    rows = _sample_rows(lay, rng, 256)
+    heads = sorted(rng.choice(w.hq, size=4, replace=False).tolist())
+    ref = orc.attention_rows(qr, kr, v, lay, rows, heads, do=do if bwd else None)
+    assert_close("O rows", got["o"][rows][:, heads], ref["o"])
+    assert_close("LSE rows", got["lse"][heads][:, rows], ref["lse"])
+    if not bwd:
+        return
+    # dQ of sampled rows (w.r.t. the unrotated q): rotate the oracle's back
+    dq_rows = orc.rope(ref["dq"], lay.pos_id[rows], w.base, inverse=True)
+    assert_close("dQ rows", got["dq"][rows][:, heads], dq_rows)
+    keys = _tail_keys(lay, rng, 48)
+    g = int(rng.integers(w.hkv))
+    dk, dv = orc.attention_cols(qr, kr, v, do, lay, keys, kv_head=g)
+    dk = orc.rope(dk[:, None, :], lay.pos_id[keys], w.base, inverse=True)[:, 0]
+    assert_close("dK keys", got["dk"][keys, g], dk)
+    assert_close("dV keys", got["dv"][keys, g], dv)
+    # rows of P sum to one: sum over keys of dV equals the sum of dO over the group's rows
+    grp = w.hq // w.hkv
+    for gg in range(w.hkv):
+        want = do[:, gg * grp:(gg + 1) * grp].astype(np.float64).sum((0, 1))
+        np.testing.assert_allclose(got["dv"][:, gg].astype(np.float64).sum(0), want, atol=0.5, rtol=2e-3)
+    assert _dk_sum_post_rope(got["dk"], lay, w.base, g) < 1e-3
+
+
+@pytest.mark.parametrize("n_turns", [2, 8, 16])
+def test_depth_sweep_sampled(n_turns):
+    w = synth.make_workload(3, n_turns=n_turns)
+    q, k, v, do = inputs(w, 3000 + n_turns)
+    got, _ = _run_gpu(w, q, k, v, do)
+    lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    qr = orc.rope(q, lay.pos_id, w.base)
+    kr = orc.rope(k, lay.pos_id, w.base)
+    rng = np.random.default_rng(n_turns)
+    rows = _sample_rows(lay, rng, 192)
+    heads = [0, 13, 31]
+    ref = orc.attention_rows(qr, kr, v, lay, rows, heads, do=do)
+    assert_close("O rows", got["o"][rows][:, heads], ref["o"])
+    assert_close("LSE rows", got["lse"][heads][:, rows], ref["lse"])
+    assert_close("dQ rows", got["dq"][rows][:, heads], orc.rope(ref["dq"], lay.pos_id[rows], w.base, inverse=True))
+    keys = _tail_keys(lay, rng, 32)
+    dk, dv = orc.attention_cols(qr, kr, v, do, lay, keys, kv_head=5)
+    dk = orc.rope(dk[:, None, :], lay.pos_id[keys], w.base, inverse=True)[:, 0]
+    assert_close("dK keys", got["dk"][keys, 5], dk)
+    assert_close("dV keys", got["dv"][keys, 5], dv)
+
+
+def test_deterministic_backward():
+    w = synth.random_small_workload(2, hq=4, hkv=2, d=128)
+    q, k, v, do = inputs(w, 2)
+    a, _ = _run_gpu(w, q, k, v, do)
+    b, _ = _run_gpu(w, q, k, v, do)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        np.testing.assert_array_equal(a[name], b[name])

@@ -1,0 +1,117 @@
+"""GPU parity of opr_build_layout and opr_rope against the oracle.
+
+Layout, position ids and the block map must match bit for bit (One-Pass to
+Reason, "Token 复制", "位置 ID 策略", "分块稀疏注意力掩码").
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_masked_segment_b200 as opr
+import synth
+from oracle import opr_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+
+def _compare_layout(w):
+    lay = opr.opr_build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    ref = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    torch.cuda.synchronize()
+    assert opr.read_status(lay.dev_status) == []
+    np.testing.assert_array_equal(lay.cu_seqlens.cpu().numpy(), ref.cu_seqlens)
+    np.testing.assert_array_equal(lay.token_type.cpu().numpy(), ref.token_type)
+    np.testing.assert_array_equal(lay.turn_idx.cpu().numpy(), ref.turn_idx)
+    np.testing.assert_array_equal(lay.conv_idx.cpu().numpy(), ref.conv_idx)
+    np.testing.assert_array_equal(lay.pos_id.cpu().numpy(), ref.pos_id)
+    bm_ref = orc.block_map(ref, max_seqlen=lay.max_seqlen)
+    np.testing.assert_array_equal(lay.block_map.cpu().numpy(), bm_ref)
+    return lay, ref
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_layout_random_ragged(seed):
+    w = synth.random_small_workload(seed, n_seqs=3, max_convs=4, max_turns=5)
+    _compare_layout(w)
+
+
+def test_layout_zero_lengths_and_tiny_segments():
+    w = synth.make_custom_workload([
+        [[(0, 0, 1), (1, 0, 0), (0, 3, 0)], [(2, 2, 2)]],
+        [[(5, 0, 0)]],
+        [[(130, 0, 0)], [(1, 1, 1), (0, 0, 0), (127, 129, 1)]],
+    ])
+    _compare_layout(w)
+
+
+def test_layout_block_boundaries():
+    """Segments ending exactly on and just off the 128-token tile edges."""
+    w = synth.make_custom_workload([
+        [[(128, 128, 64)], [(127, 1, 128), (1, 127, 129)]],
+        [[(256, 0, 0)], [(128, 0, 0)]],
+    ])
+    _compare_layout(w)
+
+
+@pytest.mark.parametrize("config", [0, 1, 2, 4])
+def test_layout_full_configs(config):
+    w = synth.make_workload(config)
+    _compare_layout(w)
+
+
+@pytest.mark.parametrize("n_turns", synth.DEPTH_SWEEP_TURNS)
+def test_layout_depth_sweep(n_turns):
+    _compare_layout(synth.make_workload(3, n_turns=n_turns))
+
+
+def test_layout_npass_is_causal():
+    w, _ = synth.npass_workload(synth.make_workload(1))
+    lay, ref = _compare_layout(w)
+    bm = lay.block_map.cpu().numpy()
+    for s in range(lay.n_seqs):
+        L = int(ref.cu_seqlens[s + 1] - ref.cu_seqlens[s])
+        nt = (L + 127) // 128
+        for I in range(nt):
+            # causal: everything strictly below the diagonal inside the sequence is full
+            assert all(bm[s, I, J] == 1 for J in range(I))
+            assert all(bm[s, I, J] == 0 for J in range(I + 1, bm.shape[1]))
+
+
+def test_layout_device_status_total_mismatch():
+    w = synth.random_small_workload(3)
+    lay = opr.opr_build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr,
+                               total_tokens=w.total_tokens + 5, max_seqlen=w.max_seqlen)
+    torch.cuda.synchronize()
+    assert "total mismatch" in opr.read_status(lay.dev_status)
+
+
+def test_layout_device_status_seq_too_long():
+    w = synth.random_small_workload(4)
+    lay = opr.opr_build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr,
+                               total_tokens=w.total_tokens, max_seqlen=max(w.max_seqlen - 1, 1))
+    torch.cuda.synchronize()
+    assert "sequence longer than max_seqlen" in opr.read_status(lay.dev_status)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+def test_rope_parity(dtype, d):
+    w = synth.make_workload(4)  # positions up to ~1.4e4
+    ref_lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    lay = opr.opr_build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((lay.total, 2, d)).astype(np.float32)
+    if dtype == torch.bfloat16:
+        x = synth.round_bf16(x)
+    xd = torch.from_numpy(x).to("cuda", dtype)
+    for inverse in (False, True):
+        y = xd.clone()
+        opr.opr_rope(y, lay.pos_id, 1e6, inverse=inverse)
+        ref = orc.rope(x, ref_lay.pos_id, 1e6, inverse=inverse)
+        got = y.float().cpu().numpy()
+        if dtype == torch.float32:
+            np.testing.assert_allclose(got, ref, atol=2e-5, rtol=0)
+        else:
+            # one bf16 rounding of the exact result (8 significant bits)
+            assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
