@@ -123,8 +123,8 @@ class Runner:
                        for a in (w.turn_lens.reshape(-1), w.conv_turn_ptr, w.seq_conv_ptr)]
         self.q, self.k, self.v, self.do = (t.to(device) for t in (self.h_q, self.h_k, self.h_v, self.h_do))
         self.lens = [t.to(device) for t in self.h_lens]
-        self.q_rot = torch.empty_like(self.q)
-        self.k_rot = torch.empty_like(self.k)
+        self.q_rot = torch.empty(self.q.shape, dtype=torch.float16, device=device)
+        self.k_rot = torch.empty(self.k.shape, dtype=torch.float16, device=device)
         self.grads = (torch.empty((n, w.hq, w.d), dtype=torch.float32, device=device),
                       torch.empty((n, w.hkv, w.d), dtype=torch.float32, device=device),
                       torch.empty((n, w.hkv, w.d), dtype=torch.float32, device=device))
@@ -148,10 +148,8 @@ class Runner:
         rec(0)
         lay = opr.opr_build_layout(*self.lens, total_tokens=self.total, max_seqlen=self.max_seqlen, device=self.dev)
         rec(1)
-        self.q_rot.copy_(self.q)
-        self.k_rot.copy_(self.k)
-        opr.opr_rope(self.q_rot, lay.pos_id, self.w.base)
-        opr.opr_rope(self.k_rot, lay.pos_id, self.w.base)
+        opr.opr_rope(self.q, lay.pos_id, self.w.base, out=self.q_rot, dev_status=lay.dev_status)
+        opr.opr_rope(self.k, lay.pos_id, self.w.base, out=self.k_rot, dev_status=lay.dev_status)
         rec(2)
         o, lse = opr.opr_attn_fwd(self.q_rot, self.k_rot, self.v, lay, out_dtype=torch.bfloat16)
         rec(3)

@@ -19,8 +19,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "lib", "libopr.so")
 
 OPR_OK, OPR_INVALID_ARG, OPR_UNSUPPORTED, OPR_CUDA_ERROR, OPR_WORKSPACE_TOO_SMALL = 0, 1, 2, 3, 4
-DEV_BITS = {1: "bad input", 2: "total mismatch", 4: "sequence longer than max_seqlen", 8: "pipeline wait timeout"}
-DTYPE_BF16, DTYPE_FP32 = 0, 1
+DEV_BITS = {1: "bad input", 2: "total mismatch", 4: "sequence longer than max_seqlen", 8: "pipeline wait timeout",
+            16: "fp16 overflow in rope"}
+DTYPE_BF16, DTYPE_FP32, DTYPE_FP16 = 0, 1, 2
 TILE = 128
 
 EXPORTED_SYMBOLS = (
@@ -67,17 +68,17 @@ def load_library() -> ctypes.CDLL:
     lib.opr_build_layout.restype = I32
     lib.opr_build_layout.argtypes = [P, P, P, I32, I32, I32, I64, I32, P, P, P, P, P, P, P, SZ, P, P]
     lib.opr_rope.restype = I32
-    lib.opr_rope.argtypes = [P, I32, P, I64, I32, I32, D, I32, P]
+    lib.opr_rope.argtypes = [P, I32, P, I32, P, I64, I32, I32, D, I32, P, P]
     lib.opr_attn_fwd.restype = I32
-    lib.opr_attn_fwd.argtypes = [P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F, P, I32, P, P, P]
+    lib.opr_attn_fwd.argtypes = [P, P, P, I32, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F, P, I32, P, P, P]
     lib.opr_attn_bwd_workspace_bytes.restype = SZ
     lib.opr_attn_bwd_workspace_bytes.argtypes = [I64, I32, I32]
     lib.opr_attn_bwd.restype = I32
-    lib.opr_attn_bwd.argtypes = [P, P, P, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F,
+    lib.opr_attn_bwd.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F,
                                  P, P, P, P, SZ, P, P]
     lib.opr_attn_bwd_stages.restype = I32
-    lib.opr_attn_bwd_stages.argtypes = [P, P, P, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F,
-                                        P, P, P, P, SZ, P, I32, P]
+    lib.opr_attn_bwd_stages.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32,
+                                        F, P, P, P, P, SZ, P, I32, P]
     _lib = lib
     return lib
 
@@ -200,23 +201,34 @@ def opr_build_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, total_tokens=None, 
     return lay
 
 
-def opr_rope(x: torch.Tensor, pos_id: torch.Tensor, base: float, inverse: bool = False) -> torch.Tensor:
-    """Rotate x [total, heads, head_dim] (bf16 or fp32) in place by position id."""
-    _need_cuda(x, pos_id)
-    if x.dtype not in (torch.bfloat16, torch.float32):
-        raise OprError("opr_rope takes bf16 or fp32")
+_DT = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16, torch.float32: DTYPE_FP32}
+
+
+def opr_rope(x: torch.Tensor, pos_id: torch.Tensor, base: float, inverse: bool = False,
+             out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """Rotate x [total, heads, head_dim] by position id, into ``out`` (default: in place).
+
+    x and out may be bf16, fp16 or fp32 (types may differ when out is not x).
+    """
+    out = x if out is None else out
+    _need_cuda(x, pos_id, out)
+    if x.dtype not in _DT or out.dtype not in _DT:
+        raise OprError("opr_rope takes bf16, fp16 or fp32")
+    if out.shape != x.shape:
+        raise OprError("opr_rope: out must have the shape of x")
     total, heads, d = x.shape
-    st = load_library().opr_rope(_ptr(x), DTYPE_BF16 if x.dtype == torch.bfloat16 else DTYPE_FP32, _ptr(pos_id),
-                                 total, heads, d, float(base), int(bool(inverse)), _stream(x.device))
+    st = load_library().opr_rope(_ptr(x), _DT[x.dtype], _ptr(out), _DT[out.dtype], _ptr(pos_id), total, heads, d,
+                                 float(base), int(bool(inverse)), _ptr(dev_status), _stream(x.device))
     _check(st, "opr_rope")
-    return x
+    return out
 
 
 def _attn_shapes(q, k, v, lay: Layout):
     _need_cuda(q, k, v)
-    for t in (q, k, v):
-        if t.dtype != torch.bfloat16:
-            raise OprError("q, k, v must be bf16")
+    if q.dtype not in (torch.float16, torch.bfloat16) or k.dtype != q.dtype:
+        raise OprError("q and k must both be fp16 or both bf16")
+    if v.dtype != torch.bfloat16:
+        raise OprError("v must be bf16")
     total, hq, d = q.shape
     if k.shape != v.shape or k.shape[0] != total or k.shape[2] != d or total != lay.total:
         raise OprError("shape mismatch between q, k, v and the layout")
@@ -230,7 +242,7 @@ def opr_attn_fwd(q, k, v, lay: Layout, scale: float | None = None, out_dtype=tor
     o = torch.empty((total, hq, d), dtype=out_dtype, device=q.device)
     lse = torch.empty((hq, total), dtype=torch.float32, device=q.device)
     st = load_library().opr_attn_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace),
+        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace),
         lay.n_seqs, lay.n_convs, lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale),
         _ptr(o), DTYPE_FP32 if out_dtype == torch.float32 else DTYPE_BF16, _ptr(lse), _ptr(lay.dev_status),
         _stream(q.device))
@@ -259,7 +271,7 @@ def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, w
     wb = opr_attn_bwd_workspace_bytes(total, hq, d)
     if workspace is None or workspace.numel() < wb:
         workspace = torch.empty(max(wb, 256), dtype=torch.uint8, device=q.device)
-    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16, _ptr(do),
+    args = (_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16, _ptr(do),
             _ptr(lse), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace), lay.n_seqs, lay.n_convs,
             lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
             _ptr(workspace), workspace.numel(), _ptr(lay.dev_status))

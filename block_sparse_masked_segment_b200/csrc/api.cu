@@ -10,10 +10,10 @@
 #include "opr_internal.cuh"
 
 namespace opr {
-cudaError_t launch_attn_fwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const AttnParams& p, cudaStream_t stream);
-cudaError_t launch_attn_bwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const void* o, int o_fp32, const void* dout,
+cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const CUtensorMap& tdo, const void* o, int o_fp32, const void* dout,
                             const AttnParams& pq, const AttnParams& pkv, float* row_d, int stages,
                             cudaStream_t stream);
 
@@ -35,9 +35,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [tokens, heads, head_dim] bf16 tensor as a 3-D TMA map with 128-byte swizzle;
-// a box is 64 head_dim elements x 1 head x 128 tokens (rows past the end read 0).
-bool make_map(CUtensorMap* map, const void* ptr, int64_t total, int32_t heads, int32_t head_dim) {
+// [tokens, heads, head_dim] 16-bit tensor (bf16 or fp16) as a 3-D TMA map with
+// 128-byte swizzle; a box is 64 head_dim elements x 1 head x 128 tokens (rows
+// past the end read 0).
+bool make_map(CUtensorMap* map, const void* ptr, int64_t total, int32_t heads, int32_t head_dim,
+              bool f16 = false) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(heads),
@@ -45,7 +47,7 @@ bool make_map(CUtensorMap* map, const void* ptr, int64_t total, int32_t heads, i
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, static_cast<cuuint64_t>(heads) * head_dim * 2};
   cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kTile)};
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+  return fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -135,18 +137,21 @@ opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* conv_turn_p
   return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
 }
 
-opr_status opr_rope(void* x, int32_t dtype, const int32_t* pos_id, int64_t total_tokens, int32_t n_heads,
-                    int32_t head_dim, double base, int32_t inverse, void* stream) {
+opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, const int32_t* pos_id,
+                    int64_t total_tokens, int32_t n_heads, int32_t head_dim, double base, int32_t inverse,
+                    int32_t* dev_status, void* stream) {
   if (total_tokens < 0 || n_heads < 0 || head_dim <= 0 || head_dim % 2 != 0 || head_dim > 256) return OPR_INVALID_ARG;
-  if (dtype != OPR_DTYPE_BF16 && dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
+  auto known = [](int32_t t) { return t == OPR_DTYPE_BF16 || t == OPR_DTYPE_FP16 || t == OPR_DTYPE_FP32; };
+  if (!known(x_dtype) || !known(y_dtype)) return OPR_UNSUPPORTED;
   if (!(base > 1.0)) return OPR_INVALID_ARG;
-  if (total_tokens > 0 && n_heads > 0 && (!x || !pos_id)) return OPR_INVALID_ARG;
-  cudaError_t e = launch_rope(x, dtype, pos_id, total_tokens, n_heads, head_dim, base, inverse,
-                              static_cast<cudaStream_t>(stream));
+  if (total_tokens > 0 && n_heads > 0 && (!x || !y || !pos_id)) return OPR_INVALID_ARG;
+  if (x == y && x_dtype != y_dtype) return OPR_INVALID_ARG;
+  cudaError_t e = launch_rope(x, x_dtype, y, y_dtype, pos_id, total_tokens, n_heads, head_dim, base, inverse,
+                              dev_status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
 }
 
-opr_status opr_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_dtype, const int32_t* cu_seqlens,
                         const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs, int32_t n_convs,
                         int32_t n_turns, int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv,
                         int32_t head_dim, float scale, void* o, int32_t o_dtype, float* lse, int32_t* dev_status,
@@ -156,10 +161,12 @@ opr_status opr_attn_fwd(const void* q, const void* k, const void* v, const int32
   if (!attn_args_ok(q, k, v, hq, hkv, head_dim, scale)) return OPR_INVALID_ARG;
   if (!cu_seqlens || !conv_idx || !layout_ws || !o || !lse || !dev_status || !aligned16(o)) return OPR_INVALID_ARG;
   if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
+  if (qk_dtype != OPR_DTYPE_BF16 && qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
+  const bool f16 = qk_dtype == OPR_DTYPE_FP16;
   opr_status st = device_check();
   if (st != OPR_OK) return st;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, total_tokens, hq, head_dim) || !make_map(&tk, k, total_tokens, hkv, head_dim) ||
+  if (!make_map(&tq, q, total_tokens, hq, head_dim, f16) || !make_map(&tk, k, total_tokens, hkv, head_dim, f16) ||
       !make_map(&tv, v, total_tokens, hkv, head_dim))
     return OPR_CUDA_ERROR;
   AttnParams p = base_params(cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs, n_turns, total_tokens, max_seqlen, hq,
@@ -167,7 +174,7 @@ opr_status opr_attn_fwd(const void* q, const void* k, const void* v, const int32
   p.o = o;
   p.o_fp32 = o_dtype == OPR_DTYPE_FP32;
   p.lse = lse;
-  cudaError_t e = launch_attn_fwd(head_dim, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_attn_fwd(head_dim, f16, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
 }
 
@@ -177,7 +184,8 @@ size_t opr_attn_bwd_workspace_bytes(int64_t total_tokens, int32_t hq, int32_t he
   return align_up(sizeof(float) * static_cast<size_t>(total_tokens) * static_cast<size_t>(hq), 256);
 }
 
-opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, const void* o, int32_t o_dtype,
+opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int32_t qk_dtype, const void* o,
+                               int32_t o_dtype,
                                const void* dout, const float* lse, const int32_t* cu_seqlens,
                                const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs, int32_t n_convs,
                                int32_t n_turns, int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv,
@@ -192,11 +200,13 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, cons
     return OPR_INVALID_ARG;
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return OPR_INVALID_ARG;
   if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
+  if (qk_dtype != OPR_DTYPE_BF16 && qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
+  const bool f16 = qk_dtype == OPR_DTYPE_FP16;
   if (workspace_bytes < opr_attn_bwd_workspace_bytes(total_tokens, hq, head_dim)) return OPR_WORKSPACE_TOO_SMALL;
   opr_status st = device_check();
   if (st != OPR_OK) return st;
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, total_tokens, hq, head_dim) || !make_map(&tk, k, total_tokens, hkv, head_dim) ||
+  if (!make_map(&tq, q, total_tokens, hq, head_dim, f16) || !make_map(&tk, k, total_tokens, hkv, head_dim, f16) ||
       !make_map(&tv, v, total_tokens, hkv, head_dim) || !make_map(&tdo, dout, total_tokens, hq, head_dim))
     return OPR_CUDA_ERROR;
   const LayoutWs w = layout_ws_map(n_seqs, n_convs, n_turns, total_tokens, max_seqlen);
@@ -209,18 +219,19 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, cons
   pq.dv = dv;
   AttnParams pkv = pq;
   pkv.sched = ws_ptr<int32_t>(layout_ws, w.k_sched);
-  cudaError_t e = launch_attn_bwd(head_dim, tq, tk, tv, tdo, o, o_dtype == OPR_DTYPE_FP32, dout, pq, pkv,
+  cudaError_t e = launch_attn_bwd(head_dim, f16, tq, tk, tv, tdo, o, o_dtype == OPR_DTYPE_FP32, dout, pq, pkv,
                                   static_cast<float*>(workspace), stages, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
 }
 
-opr_status opr_attn_bwd(const void* q, const void* k, const void* v, const void* o, int32_t o_dtype,
+opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int32_t qk_dtype, const void* o,
+                        int32_t o_dtype,
                         const void* dout, const float* lse, const int32_t* cu_seqlens, const int32_t* conv_idx,
                         const void* layout_ws, int32_t n_seqs, int32_t n_convs, int32_t n_turns,
                         int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
                         float scale, float* dq, float* dk, float* dv, void* workspace, size_t workspace_bytes,
                         int32_t* dev_status, void* stream) {
-  return opr_attn_bwd_stages(q, k, v, o, o_dtype, dout, lse, cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs,
+  return opr_attn_bwd_stages(q, k, v, qk_dtype, o, o_dtype, dout, lse, cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs,
                              n_turns, total_tokens, max_seqlen, hq, hkv, head_dim, scale, dq, dk, dv, workspace,
                              workspace_bytes, dev_status, OPR_BWD_ROW_TERMS | OPR_BWD_DQ | OPR_BWD_DKDV, stream);
 }

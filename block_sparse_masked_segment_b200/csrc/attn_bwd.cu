@@ -13,6 +13,8 @@
 //                the group and the column's non-empty query tiles:
 //                S^T = K Q^T, dP^T = V dO^T -> P^T, dS^T (TMEM) ->
 //                dV += P^T dO, dK += dS^T Q.
+// Q/K and the dS operand share one 16-bit type (fp16 when QK16, else bf16);
+// dO, V and P are bf16.
 // Warp roles as in the forward: warp 0 TMA producer (+ metadata lanes),
 // warp 1 TMEM owner and MMA issuer, warps 2..5 one row per thread.
 #include "attn_common.cuh"
@@ -68,7 +70,7 @@ struct DqSmem {
 // TMEM columns of the dq kernel: S / dS at 0, dP at 128, dQ accumulator at 256.
 constexpr uint32_t kDqColS = 0, kDqColDP = 128, kDqColAcc = 256;
 
-template <int D>
+template <int D, bool QK16>
 __global__ void __launch_bounds__(192, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -159,8 +161,9 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);  // S = Q K^T, dP = dO V^T
-      constexpr uint32_t idesc_q = idesc_bf16_f32(128, D, 0, 1);    // dQ += dS K (K tile MN-major)
+      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T (q/k type)
+      constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP = dO V^T (bf16)
+      constexpr uint32_t idesc_q = idesc_f32acc(128, D, QK16, 0, 1);    // dQ += dS K (K tile MN-major)
       const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
       bool ok = mbar_wait(&sm.bar_qdo, 0, abort_flag, kWaitLimitNs);
       for (int j = 0; ok && j < n; ++j) {
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t sv = smem_u32(sm.v[st]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kDqColDP, desc_kmajor(sdo, kk), desc_kmajor(sv, kk), idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kDqColDP, desc_kmajor(sdo, kk), desc_kmajor(sv, kk), idesc_p, kk > 0 ? 1u : 0u);
         mma_commit(&sm.bar_dpfull);
         mma_commit(&sm.bar_vempty[st]);
         if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) {
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int x = 0; x < 16; ++x) {
           const float d0 = pv[c * 32 + 2 * x] * (__uint_as_float(r[2 * x]) - dd);
           const float d1 = pv[c * 32 + 2 * x + 1] * (__uint_as_float(r[2 * x + 1]) - dd);
-          pk[x] = pack_bf16x2(d0, d1);
+          pk[x] = pack_x2<QK16>(d0, d1);
         }
         tmem_st16(tl + kDqColS + c * 16, pk);
       }
@@ -314,7 +317,7 @@ struct DkdvSmem {
 // dV accumulator at 256, dK accumulator at 256 + D.
 constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvColDV = 256;
 
-template <int D>
+template <int D, bool QK16>
 __global__ void __launch_bounds__(192, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -414,8 +417,10 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);  // S^T = K Q^T, dP^T = V dO^T
-      constexpr uint32_t idesc_a = idesc_bf16_f32(128, D, 0, 1);    // dV += P^T dO, dK += dS^T Q
+      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S^T = K Q^T (q/k type)
+      constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP^T = V dO^T (bf16)
+      constexpr uint32_t idesc_v = idesc_bf16_f32(128, D, 0, 1);        // dV += P^T dO (bf16)
+      constexpr uint32_t idesc_k = idesc_f32acc(128, D, QK16, 0, 1);    // dK += dS^T Q (q/k type)
       const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
       bool ok = mbar_wait(&sm.bar_kv, 0, abort_flag, kWaitLimitNs);
       for (int j = 0; ok && j < n; ++j) {
@@ -439,7 +444,7 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t sdo = smem_u32(sm.dout[st]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kKvColDP, desc_kmajor(sv, kk), desc_kmajor(sdo, kk), idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + kKvColDP, desc_kmajor(sv, kk), desc_kmajor(sdo, kk), idesc_p, kk > 0 ? 1u : 0u);
         mma_commit(&sm.bar_dpfull);
         if (!mbar_wait(&sm.bar_pfull, j & 1, abort_flag, kWaitLimitNs)) {
           ok = false;
@@ -448,7 +453,7 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kKvColDV, tmem + kKvColS + kk * 8, desc_mnmajor(sdo, kk), idesc_a,
+          mma_ts(tmem + kKvColDV, tmem + kKvColS + kk * 8, desc_mnmajor(sdo, kk), idesc_v,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar_doempty[st]);
         if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) {
@@ -458,7 +463,7 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kColDK, tmem + kKvColDP + kk * 8, desc_mnmajor(sq, kk), idesc_a,
+          mma_ts(tmem + kColDK, tmem + kKvColDP + kk * 8, desc_mnmajor(sq, kk), idesc_k,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar_qempty[st]);
       }
@@ -528,7 +533,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int x = 0; x < 16; ++x) {
           const float d0 = pv[c * 32 + 2 * x] * (__uint_as_float(r[2 * x]) - sm.qd[st][c * 32 + 2 * x]);
           const float d1 = pv[c * 32 + 2 * x + 1] * (__uint_as_float(r[2 * x + 1]) - sm.qd[st][c * 32 + 2 * x + 1]);
-          pk[x] = pack_bf16x2(d0, d1);
+          pk[x] = pack_x2<QK16>(d0, d1);
         }
         tmem_st16(tl + kKvColDP + c * 16, pk);
       }
@@ -587,7 +592,7 @@ cudaError_t set_smem(K kernel, size_t smem, int* configured) {
   return e;
 }
 
-template <int D>
+template <int D, bool QK16>
 cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                          const void* o, int o_fp32, const void* dout, const AttnParams& pq, const AttnParams& pkv,
                          float* row_d, int stages, cudaStream_t stream) {
@@ -608,18 +613,18 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   // 2) dQ
   if (stages & OPR_BWD_DQ) {
     const size_t smem_q = smem_request(sizeof(DqSmem<D>) + 1024);
-    if ((e = set_smem(attn_bwd_dq_kernel<D>, smem_q, conf_dq)) != cudaSuccess) return e;
+    if ((e = set_smem(attn_bwd_dq_kernel<D, QK16>, smem_q, conf_dq)) != cudaSuccess) return e;
     const int64_t bq = static_cast<int64_t>(pq.n_items) * pq.hq;
-    if (bq > 0) attn_bwd_dq_kernel<D><<<static_cast<unsigned>(bq), 192, smem_q, stream>>>(tq, tk, tv, tdo, pq);
+    if (bq > 0) attn_bwd_dq_kernel<D, QK16><<<static_cast<unsigned>(bq), 192, smem_q, stream>>>(tq, tk, tv, tdo, pq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // 3) dK, dV
   if (stages & OPR_BWD_DKDV) {
     const size_t smem_kv = smem_request(sizeof(DkdvSmem<D>) + 1024);
-    if ((e = set_smem(attn_bwd_dkdv_kernel<D>, smem_kv, conf_kv)) != cudaSuccess) return e;
+    if ((e = set_smem(attn_bwd_dkdv_kernel<D, QK16>, smem_kv, conf_kv)) != cudaSuccess) return e;
     const int64_t bkv = static_cast<int64_t>(pkv.n_items) * pkv.hkv;
     if (bkv > 0)
-      attn_bwd_dkdv_kernel<D><<<static_cast<unsigned>(bkv), 192, smem_kv, stream>>>(tq, tk, tv, tdo, pkv);
+      attn_bwd_dkdv_kernel<D, QK16><<<static_cast<unsigned>(bkv), 192, smem_kv, stream>>>(tq, tk, tv, tdo, pkv);
     e = cudaGetLastError();
   }
   return e;
@@ -627,12 +632,15 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 }  // namespace
 
-cudaError_t launch_attn_bwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const void* o, int o_fp32, const void* dout,
-                            const AttnParams& pq, const AttnParams& pkv, float* row_d, int stages,
+cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const CUtensorMap& tdo, const void* o, int o_fp32,
+                            const void* dout, const AttnParams& pq, const AttnParams& pkv, float* row_d, int stages,
                             cudaStream_t stream) {
-  if (head_dim == 128) return launch_bwd_t<128>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream);
-  return launch_bwd_t<64>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream);
+  if (head_dim == 128)
+    return qk_f16 ? launch_bwd_t<128, true>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream)
+                  : launch_bwd_t<128, false>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream);
+  return qk_f16 ? launch_bwd_t<64, true>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream)
+                : launch_bwd_t<64, false>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream);
 }
 
 }  // namespace opr

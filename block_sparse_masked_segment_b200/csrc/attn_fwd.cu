@@ -16,6 +16,9 @@
 //               when the running max grows by more than 2^8; epilogue O / l
 //               and the log-sum-exp.
 // TMEM columns: S/P buffer 0 at 0, buffer 1 at 128, O at 256 (512 allocated).
+// Q and K may be bf16 or fp16 (QK16: the rotated q, k stored in fp16, whose
+// 11-bit significand keeps the rounding of the rotation 8x smaller); V and P
+// are bf16.
 #include "attn_common.cuh"
 
 namespace opr {
@@ -38,7 +41,7 @@ struct FwdSmem {
   int abort_flag;
 };
 
-template <int D>
+template <int D, bool QK16>
 __global__ void __launch_bounds__(192, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -133,8 +136,8 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);      // O += P V, P and V bf16
       const uint32_t sq = smem_u32(sm.q);
       bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, kWaitLimitNs);
       auto issue_pv = [&](int jp) -> bool {
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(192, 1)
 
 }  // namespace
 
-template <int D>
+template <int D, bool QK16>
 cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const AttnParams& p, cudaStream_t stream) {
   const size_t smem = smem_request(sizeof(FwdSmem<D>) + 1024);
@@ -308,21 +311,24 @@ cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, cons
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, QK16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
   const int64_t blocks = static_cast<int64_t>(p.n_items) * p.hq;
   if (blocks == 0) return cudaSuccess;
-  attn_fwd_kernel<D><<<static_cast<unsigned>(blocks), 192, smem, stream>>>(tq, tk, tv, p);
+  attn_fwd_kernel<D, QK16><<<static_cast<unsigned>(blocks), 192, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_fwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const AttnParams& p, cudaStream_t stream) {
-  if (head_dim == 128) return launch_attn_fwd_t<128>(tq, tk, tv, p, stream);
-  return launch_attn_fwd_t<64>(tq, tk, tv, p, stream);
+cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
+                            const CUtensorMap& tv, const AttnParams& p, cudaStream_t stream) {
+  if (head_dim == 128)
+    return qk_f16 ? launch_attn_fwd_t<128, true>(tq, tk, tv, p, stream)
+                  : launch_attn_fwd_t<128, false>(tq, tk, tv, p, stream);
+  return qk_f16 ? launch_attn_fwd_t<64, true>(tq, tk, tv, p, stream)
+                : launch_attn_fwd_t<64, false>(tq, tk, tv, p, stream);
 }
 
 }  // namespace opr

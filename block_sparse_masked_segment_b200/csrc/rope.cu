@@ -8,9 +8,14 @@
 //
 // One thread per (token, j < d/2): the angle is formed and reduced in fp64 once
 // and applied to every head of the token.  HBM-bound: each element is read and
-// written once.
+// written once.  Input and output types may differ (bf16 in, fp16 out for the
+// rotated q and k; in place when they are the same buffer and type); an fp16
+// output value beyond the fp16 range sets OPR_DEV_FP16_RANGE.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "opr_internal.cuh"
 
@@ -27,6 +32,10 @@ template <>
 __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) {
   return __bfloat162float(v);
 }
+template <>
+__device__ __forceinline__ float to_f<__half>(__half v) {
+  return __half2float(v);
+}
 template <typename T>
 __device__ __forceinline__ T from_f(float v);
 template <>
@@ -37,11 +46,16 @@ template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
 }
+template <>
+__device__ __forceinline__ __half from_f<__half>(float v) {
+  return __float2half_rn(v);
+}
 
-template <typename T>
-__global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ x, const int32_t* __restrict__ pos_id, int64_t total,
-                                                   int32_t n_heads, int32_t half, double neg_log_base_over_half,
-                                                   double sign) {
+template <typename TI, typename TO>
+__global__ void __launch_bounds__(256) rope_kernel(const TI* x, TO* y, const int32_t* __restrict__ pos_id,
+                                                   int64_t total, int32_t n_heads, int32_t half,
+                                                   double neg_log_base_over_half, double sign,
+                                                   int32_t* __restrict__ dev_status) {
   const int tokens_per_block = blockDim.x / half;
   const int64_t tok = static_cast<int64_t>(blockIdx.x) * tokens_per_block + threadIdx.x / half;
   const int j = threadIdx.x % half;
@@ -52,33 +66,56 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ x, const int3
   double sd, cd;
   sincos(ang, &sd, &cd);
   const float c = static_cast<float>(cd), s = static_cast<float>(sd);
-  T* row = x + tok * n_heads * (2 * half);
+  const int64_t row = tok * n_heads * (2 * half);
+  bool out_of_range = false;
   for (int h = 0; h < n_heads; ++h) {
-    T* p = row + static_cast<int64_t>(h) * 2 * half;
-    const float a = to_f(p[j]), b = to_f(p[j + half]);
-    p[j] = from_f<T>(a * c - b * s);
-    p[j + half] = from_f<T>(b * c + a * s);
+    const int64_t o = row + static_cast<int64_t>(h) * 2 * half;
+    const float a = to_f(x[o + j]), b = to_f(x[o + j + half]);
+    const float ya = a * c - b * s, yb = b * c + a * s;
+    if constexpr (sizeof(TO) == 2 && !std::is_same_v<TO, __nv_bfloat16>)
+      out_of_range |= !(fabsf(ya) <= 65504.f) || !(fabsf(yb) <= 65504.f);
+    y[o + j] = from_f<TO>(ya);
+    y[o + j + half] = from_f<TO>(yb);
   }
+  if (out_of_range && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
+}
+
+template <typename TI, typename TO>
+cudaError_t launch_t(const void* x, void* y, const int32_t* pos_id, int64_t total, int32_t n_heads, int32_t half,
+                     double nl, double sign, int32_t* dev_status, cudaStream_t stream) {
+  const int threads = 256 / half * half;
+  const int tpb = threads / half;
+  const int64_t blocks = (total + tpb - 1) / tpb;
+  rope_kernel<TI, TO><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+      static_cast<const TI*>(x), static_cast<TO*>(y), pos_id, total, n_heads, half, nl, sign, dev_status);
+  return cudaGetLastError();
+}
+
+template <typename TI>
+cudaError_t launch_in(const void* x, int32_t y_dtype, void* y, const int32_t* pos_id, int64_t total,
+                      int32_t n_heads, int32_t half, double nl, double sign, int32_t* dev_status,
+                      cudaStream_t stream) {
+  if (y_dtype == OPR_DTYPE_BF16)
+    return launch_t<TI, __nv_bfloat16>(x, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
+  if (y_dtype == OPR_DTYPE_FP16)
+    return launch_t<TI, __half>(x, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
+  return launch_t<TI, float>(x, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_rope(void* x, int32_t dtype, const int32_t* pos_id, int64_t total, int32_t n_heads,
-                        int32_t head_dim, double base, int32_t inverse, cudaStream_t stream) {
+cudaError_t launch_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, const int32_t* pos_id,
+                        int64_t total, int32_t n_heads, int32_t head_dim, double base, int32_t inverse,
+                        int32_t* dev_status, cudaStream_t stream) {
   if (total == 0 || n_heads == 0) return cudaSuccess;
   const int half = head_dim / 2;
-  const int threads = 256 / half * half;
-  const int tpb = threads / half;
-  const int64_t blocks = (total + tpb - 1) / tpb;
   const double nl = -log(base) / static_cast<double>(half);
   const double sign = inverse ? -1.0 : 1.0;
-  if (dtype == OPR_DTYPE_BF16)
-    rope_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        static_cast<__nv_bfloat16*>(x), pos_id, total, n_heads, half, nl, sign);
-  else
-    rope_kernel<float><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(static_cast<float*>(x), pos_id, total,
-                                                                              n_heads, half, nl, sign);
-  return cudaGetLastError();
+  if (x_dtype == OPR_DTYPE_BF16)
+    return launch_in<__nv_bfloat16>(x, y_dtype, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
+  if (x_dtype == OPR_DTYPE_FP16)
+    return launch_in<__half>(x, y_dtype, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
+  return launch_in<float>(x, y_dtype, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
 }
 
 }  // namespace opr

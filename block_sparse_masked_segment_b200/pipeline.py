@@ -1,6 +1,7 @@
 """The one-pass attention layer as a sequence of library calls.
 
-forward:  opr_rope(q), opr_rope(k) by the layout's position ids -> opr_attn_fwd
+forward:  opr_rope(q), opr_rope(k) by the layout's position ids (bf16 in,
+          fp16 out) -> opr_attn_fwd
 backward: opr_attn_bwd -> opr_rope(inverse) on dq and dk
 (One-Pass to Reason: positions from "位置 ID 策略", mask from "分块稀疏注意力掩码").
 Every numerical step runs in libopr's CUDA kernels; this module only orders the
@@ -44,12 +45,13 @@ def useful_flops(pairs: int, hq: int, d: int, backward: bool) -> float:
     return f * 3.5 if backward else f
 
 
-def one_pass_forward(q_pre, k_pre, v, lay: Layout, base: float, scale=None, out_dtype=torch.float32):
-    """RoPE (on copies) then masked attention.  Returns (o, lse, q_rot, k_rot)."""
-    q = q_pre.clone()
-    k = k_pre.clone()
-    opr_rope(q, lay.pos_id, base)
-    opr_rope(k, lay.pos_id, base)
+def one_pass_forward(q_pre, k_pre, v, lay: Layout, base: float, scale=None, out_dtype=torch.float32,
+                     qk_dtype=torch.float16):
+    """RoPE (bf16 in, fp16 out by default) then masked attention.  Returns (o, lse, q_rot, k_rot)."""
+    q = torch.empty(q_pre.shape, dtype=qk_dtype, device=q_pre.device)
+    k = torch.empty(k_pre.shape, dtype=qk_dtype, device=k_pre.device)
+    opr_rope(q_pre, lay.pos_id, base, out=q, dev_status=lay.dev_status)
+    opr_rope(k_pre, lay.pos_id, base, out=k, dev_status=lay.dev_status)
     o, lse = opr_attn_fwd(q, k, v, lay, scale, out_dtype)
     return o, lse, q, k
 
@@ -74,8 +76,8 @@ class OnePassAttention:
         self.layout = opr_build_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, device=device)
         self.base = base
 
-    def forward(self, q_pre, k_pre, v, scale=None, out_dtype=torch.float32):
-        return one_pass_forward(q_pre, k_pre, v, self.layout, self.base, scale, out_dtype)
+    def forward(self, q_pre, k_pre, v, scale=None, out_dtype=torch.float32, qk_dtype=torch.float16):
+        return one_pass_forward(q_pre, k_pre, v, self.layout, self.base, scale, out_dtype, qk_dtype)
 
     def backward(self, q_rot, k_rot, v, o, do, lse, scale=None):
         return one_pass_backward(q_rot, k_rot, v, o, do, lse, self.layout, self.base, scale)

@@ -56,9 +56,11 @@ typedef int32_t opr_status;
 #define OPR_DEV_TOTAL_MISMATCH 2   /* sum of h + t + 2r differs from total_tokens */
 #define OPR_DEV_SEQ_TOO_LONG 4     /* a sequence is longer than max_seqlen */
 #define OPR_DEV_WAIT_TIMEOUT 8     /* a pipeline wait exceeded its time limit; outputs are invalid */
+#define OPR_DEV_FP16_RANGE 16      /* opr_rope wrote an fp16 value beyond +-65504 (inf) */
 
 #define OPR_DTYPE_BF16 0
 #define OPR_DTYPE_FP32 1
+#define OPR_DTYPE_FP16 2
 
 #define OPR_TILE 128               /* edge of a block-map tile, in tokens */
 #define OPR_TILE_EMPTY 0
@@ -114,20 +116,28 @@ OPR_API opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* con
                             void* stream);
 
 /*
- * opr_rope - rotary position embedding by position id, in place.
+ * opr_rope - rotary position embedding by position id.
  *
  * The pages' position-equivalence argument ("理论保证") is about the rotary
  * positions of Qwen-3 (rotate-half convention): for j < head_dim/2 the pair
  * (x[j], x[j + head_dim/2]) is rotated by angle pos_id * base^(-2j/head_dim)
  * (by -angle when `inverse` != 0, which maps gradients w.r.t. rotated values
- * back to gradients w.r.t. the unrotated ones).  Angles are formed in fp64.
- *   x       [total_tokens, n_heads, head_dim], dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32
- *   pos_id  int32 [total_tokens]
- * head_dim must be even and <= 256.
+ * back to gradients w.r.t. the unrotated ones).  Angles are formed in fp64,
+ * the rotation in fp32, the result rounded once to y's type.
+ *   x, y     [total_tokens, n_heads, head_dim]; x_dtype, y_dtype each one of
+ *            OPR_DTYPE_BF16 / OPR_DTYPE_FP16 / OPR_DTYPE_FP32.  y may equal x
+ *            (in place) only when the two types are the same.
+ *   pos_id   int32 [total_tokens]
+ *   dev_status  may be NULL; otherwise OPR_DEV_FP16_RANGE is OR-ed in when an
+ *            fp16 output overflows.
+ * head_dim must be even and <= 256.  The attention calls take the rotated q
+ * and k in fp16 (bf16 in, fp16 out here): same MMA rate as bf16, 8x smaller
+ * rounding of the rotation.
  */
-OPR_API opr_status opr_rope(void* x, int32_t dtype, const int32_t* pos_id, int64_t total_tokens,
-                    int32_t n_heads, int32_t head_dim, double base, int32_t inverse,
-                    void* stream);
+OPR_API opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype,
+                            const int32_t* pos_id, int64_t total_tokens, int32_t n_heads,
+                            int32_t head_dim, double base, int32_t inverse, int32_t* dev_status,
+                            void* stream);
 
 /*
  * opr_attn_fwd - block-sparse masked attention forward (tcgen05 / TMEM / TMA).
@@ -135,14 +145,17 @@ OPR_API opr_status opr_rope(void* x, int32_t dtype, const int32_t* pos_id, int64
  * O = softmax(scale * Q K^T restricted to visible keys) V for each q head;
  * q head h reads kv head h / (hq / hkv).  Tiles marked empty in the block map
  * are skipped, the visibility predicate is evaluated only on partial tiles.
- *   q            bf16 [total, hq, head_dim]   (already rotated)
- *   k, v         bf16 [total, hkv, head_dim]
+ *   q            [total, hq, head_dim]   (already rotated), qk_dtype
+ *   k            [total, hkv, head_dim]  (already rotated), qk_dtype
+ *   qk_dtype     OPR_DTYPE_FP16 or OPR_DTYPE_BF16 (the type of the S = Q K^T MMA)
+ *   v            bf16 [total, hkv, head_dim]
  *   cu_seqlens, conv_idx, layout_ws: outputs of opr_build_layout for the same sizes
  *   o            [total, hq, head_dim], o_dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32
  *   lse          fp32 [hq, total]: natural-log sum of exp(scale * q.k) over visible keys
  * head_dim must be 64 or 128; all pointers 16-byte aligned.
  */
-OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_dtype,
+                        const int32_t* cu_seqlens,
                         const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs,
                         int32_t n_convs, int32_t n_turns, int64_t total_tokens,
                         int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
@@ -158,14 +171,15 @@ OPR_API size_t opr_attn_bwd_workspace_bytes(int64_t total_tokens, int32_t hq, in
  * With P recomputed from LSE: D = rowsum(dO * O), dV = P^T dO,
  * dS = P * (dO V^T - D), dQ = scale dS K, dK = scale dS^T Q; dK and dV sum
  * over the q heads that share a kv head.  Deterministic (no atomics).
- *   q, k, v, o, dout  as in opr_attn_fwd (o in o_dtype, dout bf16)
+ *   q, k, v, o, dout  as in opr_attn_fwd (o in o_dtype, dout bf16); dS is formed
+ *                     in qk_dtype for the dQ and dK products
  *   lse               fp32 [hq, total] from opr_attn_fwd
  *   dq                fp32 [total, hq, head_dim]
  *   dk, dv            fp32 [total, hkv, head_dim]
  *   workspace         opr_attn_bwd_workspace_bytes(...) bytes of device scratch
  */
-OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, const void* o,
-                        int32_t o_dtype, const void* dout, const float* lse,
+OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int32_t qk_dtype,
+                        const void* o, int32_t o_dtype, const void* dout, const float* lse,
                         const int32_t* cu_seqlens, const int32_t* conv_idx, const void* layout_ws,
                         int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
                         int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
@@ -186,8 +200,8 @@ OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, con
 #define OPR_BWD_ROW_TERMS 1
 #define OPR_BWD_DQ 2
 #define OPR_BWD_DKDV 4
-OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, const void* o,
-                                       int32_t o_dtype, const void* dout, const float* lse,
+OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v,
+                                       int32_t qk_dtype, const void* o, int32_t o_dtype, const void* dout, const float* lse,
                                        const int32_t* cu_seqlens, const int32_t* conv_idx,
                                        const void* layout_ws, int32_t n_seqs, int32_t n_convs,
                                        int32_t n_turns, int64_t total_tokens, int32_t max_seqlen,

@@ -57,23 +57,27 @@ def test_host_argument_checks(lib):
     assert lib.opr_build_layout(N, N, N, 1, 1, 1, 10, 10, N, N, N, N, N, N, N, 0, N, N) == 1
     # negative sizes
     assert lib.opr_build_layout(N, N, N, -1, 1, 1, 10, 10, N, N, N, N, N, N, N, 0, N, N) == 1
-    # opr_rope: odd head_dim, bad dtype, null pointer
-    assert lib.opr_rope(N, 0, N, 10, 2, 63, 1e4, 0, N) == 1
-    assert lib.opr_rope(N, 7, N, 10, 2, 64, 1e4, 0, N) == 2
-    assert lib.opr_rope(N, 0, N, 10, 2, 64, 1e4, 0, N) == 1
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
+    # opr_rope: odd head_dim, bad dtype, null pointer, in place with two types
+    assert lib.opr_rope(N, 0, N, 0, N, 10, 2, 63, 1e4, 0, N, N) == 1
+    assert lib.opr_rope(N, 7, N, 0, N, 10, 2, 64, 1e4, 0, N, N) == 2
+    assert lib.opr_rope(N, 0, N, 0, N, 10, 2, 64, 1e4, 0, N, N) == 1
+    assert lib.opr_rope(fake, 0, fake, 2, fake, 10, 2, 64, 1e4, 0, N, N) == 1
     # opr_attn_fwd: null q; hq % hkv != 0; head_dim 96
-    assert lib.opr_attn_fwd(N, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
+    assert lib.opr_attn_fwd(N, fake, fake, 2, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
                             fake, 0, fake, fake, N) == 1
-    assert lib.opr_attn_fwd(fake, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100, 6, 4, 128, 0.1,
+    assert lib.opr_attn_fwd(fake, fake, fake, 2, fake, fake, fake, 1, 1, 1, 100, 100, 6, 4, 128, 0.1,
                             fake, 0, fake, fake, N) == 1
-    assert lib.opr_attn_fwd(fake, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 96, 0.1,
+    assert lib.opr_attn_fwd(fake, fake, fake, 2, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 96, 0.1,
                             fake, 0, fake, fake, N) == 1
+    # q/k of fp32 are not an MMA type
+    assert lib.opr_attn_fwd(fake, fake, fake, 1, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
+                            fake, 0, fake, fake, N) == 2
     # opr_attn_bwd_stages: unknown stage bits
-    assert lib.opr_attn_bwd_stages(fake, fake, fake, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
+    assert lib.opr_attn_bwd_stages(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
                                    4, 2, 128, 0.1, fake, fake, fake, fake, 1 << 20, fake, 8, N) == 1
     # empty problems are no-ops
-    assert lib.opr_attn_fwd(N, N, N, N, N, N, 0, 0, 0, 0, 0, 4, 2, 128, 0.1, N, 0, N, N, N) == 0
+    assert lib.opr_attn_fwd(N, N, N, 2, N, N, N, 0, 0, 0, 0, 0, 4, 2, 128, 0.1, N, 0, N, N, N) == 0
 
 
 def test_closed_form_pair_count_matches_oracle():

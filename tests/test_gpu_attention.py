@@ -18,10 +18,10 @@ from parity_helpers import assert_close, inputs, to_dev
 pytestmark = pytest.mark.gpu
 
 
-def _run_gpu(w, q, k, v, do, out_dtype=torch.float32):
+def _run_gpu(w, q, k, v, do, out_dtype=torch.float32, qk_dtype=torch.float16):
     att = opr.OnePassAttention(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, base=w.base)
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
-    o, lse, qr, kr = att.forward(qd, kd, vd, out_dtype=out_dtype)
+    o, lse, qr, kr = att.forward(qd, kd, vd, out_dtype=out_dtype, qk_dtype=qk_dtype)
     res = dict(o=o, lse=lse)
     if do is not None:
         dq, dk, dv = att.backward(qr, kr, vd, o, to_dev(do), lse)
@@ -31,18 +31,18 @@ def _run_gpu(w, q, k, v, do, out_dtype=torch.float32):
     return {kk: vv.float().cpu().numpy() for kk, vv in res.items()}, att.layout
 
 
-def _dense_check(w, seed, bwd=True):
+def _dense_check(w, seed, bwd=True, qk_dtype=torch.float16, max_abs=1e-2):
     q, k, v, do = inputs(w, seed, with_do=bwd)
-    got, _ = _run_gpu(w, q, k, v, do)
+    got, _ = _run_gpu(w, q, k, v, do, qk_dtype=qk_dtype)
     lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
     o, lse = orc.forward(q, k, v, lay, w.base)
-    assert_close("O", got["o"], o)
-    assert_close("LSE", got["lse"], lse)
+    assert_close("O", got["o"], o, max_abs=max_abs)
+    assert_close("LSE", got["lse"], lse, max_abs=max_abs)
     if bwd:
         dq, dk, dv = orc.backward(q, k, v, o, do, lse, lay, w.base)
-        assert_close("dQ", got["dq"], dq)
-        assert_close("dK", got["dk"], dk)
-        assert_close("dV", got["dv"], dv)
+        assert_close("dQ", got["dq"], dq, max_abs=max_abs)
+        assert_close("dK", got["dk"], dk, max_abs=max_abs)
+        assert_close("dV", got["dv"], dv, max_abs=max_abs)
 
 
 @pytest.mark.parametrize("seed", range(3))
@@ -55,6 +55,13 @@ def test_fwd_bwd_random_ragged(seed, d):
 def test_fwd_bwd_tiny_config():
     """Tiny workload: N = 2 turns of h16 t32 r16, one head of 64, base 1e4 (bf16-rounded inputs)."""
     _dense_check(synth.make_workload(0), 1000)
+
+
+def test_bf16_qk_variant():
+    """Rotated q and k kept in bf16 (S, dS in bf16): the relative standard holds; the
+    absolute one is relaxed to 2e-2 because the bf16 rounding of the rotation alone
+    moves dK by up to ~8e-3 on this workload (the default path stores them in fp16)."""
+    _dense_check(synth.make_workload(0), 1000, qk_dtype=torch.bfloat16, max_abs=2e-2)
 
 
 def test_fwd_bwd_gqa_8_to_1():

@@ -94,24 +94,41 @@ def test_layout_device_status_seq_too_long():
     assert "sequence longer than max_seqlen" in opr.read_status(lay.dev_status)
 
 
-@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("in_dtype,out_dtype", [(torch.float32, torch.float32), (torch.bfloat16, torch.bfloat16),
+                                                (torch.bfloat16, torch.float16), (torch.float16, torch.float16)])
 @pytest.mark.parametrize("d", [64, 128])
-def test_rope_parity(dtype, d):
+def test_rope_parity(in_dtype, out_dtype, d):
     w = synth.make_workload(4)  # positions up to ~1.4e4
     ref_lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
     lay = opr.opr_build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
     rng = np.random.default_rng(0)
     x = rng.standard_normal((lay.total, 2, d)).astype(np.float32)
-    if dtype == torch.bfloat16:
+    if in_dtype == torch.bfloat16:
         x = synth.round_bf16(x)
-    xd = torch.from_numpy(x).to("cuda", dtype)
+    elif in_dtype == torch.float16:
+        x = x.astype(np.float16).astype(np.float32)
+    xd = torch.from_numpy(x).to("cuda", in_dtype)
+    # significand bits of the output type: one rounding of the exact rotation
+    ulp_half = {torch.float32: 2.0 ** -24, torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11}[out_dtype]
     for inverse in (False, True):
-        y = xd.clone()
-        opr.opr_rope(y, lay.pos_id, 1e6, inverse=inverse)
+        if out_dtype == in_dtype:
+            y = xd.clone()
+            opr.opr_rope(y, lay.pos_id, 1e6, inverse=inverse)
+        else:
+            y = torch.empty(xd.shape, dtype=out_dtype, device="cuda")
+            opr.opr_rope(xd, lay.pos_id, 1e6, inverse=inverse, out=y, dev_status=lay.dev_status)
         ref = orc.rope(x, ref_lay.pos_id, 1e6, inverse=inverse)
         got = y.float().cpu().numpy()
-        if dtype == torch.float32:
-            np.testing.assert_allclose(got, ref, atol=2e-5, rtol=0)
-        else:
-            # one bf16 rounding of the exact result (8 significant bits)
-            assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
+        # fp32 arithmetic of the rotation adds a few 1e-7 on top of the final rounding
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * ulp_half + 2e-6)
+    torch.cuda.synchronize()
+    assert opr.read_status(lay.dev_status) == []
+
+
+def test_rope_fp16_overflow_is_flagged():
+    lay = opr.opr_build_layout([[4, 0, 0]], [0, 1], [0, 1])
+    x = torch.full((4, 1, 64), 1e5, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(x.shape, dtype=torch.float16, device="cuda")
+    opr.opr_rope(x, lay.pos_id, 1e4, out=y, dev_status=lay.dev_status)
+    torch.cuda.synchronize()
+    assert "fp16 overflow in rope" in opr.read_status(lay.dev_status)
