@@ -60,6 +60,7 @@ struct DqSmem {
   alignas(1024) uint8_t v[kStages][TileGeom<D>::kBytes];
   int32_t kconv[kStages][kTile];
   int32_t kmeta[kStages][kTile];
+  uint32_t kstarts[kStages][4];
   uint64_t bar_qdo;
   uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
   uint64_t bar_sfull, bar_dpfull, bar_dsfull, bar_dqdone, bar_final;
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(192, 1)
           sm.kconv[st][x] = kv ? p.conv_idx[k0 + x] : -1;
           sm.kmeta[st][x] = kv ? p.tok_meta[k0 + x] : 0;
         }
+        build_run_starts(sm.kconv[st], sm.kmeta[st], sm.kstarts[st], lane);
       }
       mbar_arrive(&sm.bar_kfull[st]);
       if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_vempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
@@ -233,17 +235,18 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       float pv[kTile];
+      {
+        uint32_t sr[kTile];
+        tmem_ld128(tl + kDqColS, sr);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tl + kDqColS + c * 32, r);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) pv[c * 32 + x] = fast_exp2(fmaf(__uint_as_float(r[x]), sl2, -lse2));
+        for (int c = 0; c < kTile; ++c) pv[c] = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
       }
       if (partial) {
+        uint32_t m[4];
+        query_row_mask(sm.kstarts[st], sm.kconv[st], sm.kmeta[st], kbase, qg, qconv, qmeta, m);
 #pragma unroll
         for (int c = 0; c < kTile; ++c)
-          if (!visible(qg, qconv, qmeta, kbase + c, sm.kconv[st][c], sm.kmeta[st][c])) pv[c] = 0.f;
+          if (!mask_bit(m, c)) pv[c] = 0.f;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
@@ -306,6 +309,7 @@ struct DkdvSmem {
   float qd[kStages][kTile];
   int32_t qconv[kStages][kTile];
   int32_t qmeta[kStages][kTile];
+  uint32_t qstarts[kStages][4];
   uint64_t bar_kv;
   uint64_t bar_qfull[kStages], bar_qempty[kStages], bar_dofull[kStages], bar_doempty[kStages];
   uint64_t bar_sfull, bar_dpfull, bar_pfull, bar_dsfull, bar_accdone, bar_final;
@@ -398,6 +402,7 @@ __global__ void __launch_bounds__(192, 1)
           sm.qmeta[st][x] = qv ? p.tok_meta[qt0 + x] : 0;
         }
       }
+      if ((e & 3) == OPR_TILE_PARTIAL) build_run_starts(sm.qconv[st], sm.qmeta[st], sm.qstarts[st], lane);
       mbar_arrive(&sm.bar_qfull[st]);
       if (j >= kStages &&
           !__all_sync(0xffffffffu, mbar_wait(&sm.bar_doempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
@@ -455,6 +460,9 @@ __global__ void __launch_bounds__(192, 1)
         for (int kk = 0; kk < kTile / 16; ++kk)
           mma_ts(tmem + kKvColDV, tmem + kKvColS + kk * 8, desc_mnmajor(sdo, kk), idesc_v,
                  (j > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + kKvColDV, tmem + kKvColS + 64 + kk * 8, desc_mnmajor(sdo, kk), idesc_v, 1u);
         mma_commit(&sm.bar_doempty[st]);
         if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) {
           ok = false;
@@ -496,25 +504,33 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       float pv[kTile];
+      {
+        uint32_t sr[kTile];
+        tmem_ld128(tl + kKvColS, sr);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tl + kKvColS + c * 32, r);
-#pragma unroll
-        for (int x = 0; x < 32; ++x)
-          pv[c * 32 + x] = fast_exp2(fmaf(__uint_as_float(r[x]), sl2, -sm.qlse2[st][c * 32 + x]));
+        for (int c = 0; c < kTile; ++c) pv[c] = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -sm.qlse2[st][c]));
       }
       if (partial) {
+        uint32_t m[4];
+        key_row_mask(sm.qstarts[st], sm.qconv[st], sm.qmeta[st], qt0, kg, kconv, kmeta, m);
 #pragma unroll
         for (int c = 0; c < kTile; ++c)
-          if (!visible(qt0 + c, sm.qconv[st][c], sm.qmeta[st][c], kg, kconv, kmeta)) pv[c] = 0.f;
+          if (!mask_bit(m, c)) pv[c] = 0.f;
       }
+      // P^T for dV = P^T dO as bf16 hi + lo parts (columns 0..63 and 64..127 of
+      // the S^T region): the lo part carries the rounding error of the hi part.
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(pv[c * 32 + 2 * x], pv[c * 32 + 2 * x + 1]);
-        tmem_st16(tl + kKvColS + c * 16, pk);
+        for (int x = 0; x < 16; ++x) {
+          const float a = pv[c * 32 + 2 * x], b = pv[c * 32 + 2 * x + 1];
+          const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+          hi[x] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[x] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
+        }
+        tmem_st16(tl + kKvColS + c * 16, hi);
+        tmem_st16(tl + kKvColS + 64 + c * 16, lo);
       }
       tmem_wait_st();
       tc_fence_before();

@@ -34,6 +34,7 @@ struct FwdSmem {
   alignas(1024) uint8_t v[kStages][TileGeom<D>::kBytes];
   int32_t kconv[kStages][kTile];
   int32_t kmeta[kStages][kTile];
+  uint32_t kstarts[kStages][4];  // column-run starts of a partial tile
   uint64_t bar_q;
   uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
   uint64_t bar_sfull[2], bar_pfull[2], bar_odone, bar_final;
@@ -123,6 +124,7 @@ __global__ void __launch_bounds__(192, 1)
           sm.kconv[st][x] = kv ? p.conv_idx[k0 + x] : -1;
           sm.kmeta[st][x] = kv ? p.tok_meta[k0 + x] : 0;
         }
+        build_run_starts(sm.kconv[st], sm.kmeta[st], sm.kstarts[st], lane);
       }
       mbar_arrive(&sm.bar_vfull[st]);
     }
@@ -201,27 +203,31 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
+      uint32_t sr[kTile];
+      tmem_ld128(tl + b * 128, sr);
       float sv[kTile];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tl + b * 128 + c * 32, r);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) sv[c * 32 + x] = __uint_as_float(r[x]);
-      }
+      for (int c = 0; c < kTile; ++c) sv[c] = __uint_as_float(sr[c]);
       if (partial) {
+        uint32_t m[4];
+        query_row_mask(sm.kstarts[st], sm.kconv[st], sm.kmeta[st], kbase, qg, qconv, qmeta, m);
 #pragma unroll
         for (int c = 0; c < kTile; ++c)
-          if (!visible(qg, qconv, qmeta, kbase + c, sm.kconv[st][c], sm.kmeta[st][c])) sv[c] = -INFINITY;
+          if (!mask_bit(m, c)) sv[c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max as a tree (8 independent chains)
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) mx = fmaxf(mx, sv[c]);
+      for (int x = 0; x < 8; ++x) mx8[x] = sv[x];
+#pragma unroll
+      for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m_run, mx * sl2);
       const bool need = m_new > m_run + 8.f;  // also true on the first finite max
       const float m_use = need ? m_new : m_run;
       const float mb = (m_use == -INFINITY) ? 0.f : m_use;
-      float rs = 0.f;
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -229,11 +235,12 @@ __global__ void __launch_bounds__(192, 1)
         for (int x = 0; x < 16; ++x) {
           const float p0 = fast_exp2(fmaf(sv[c * 32 + 2 * x], sl2, -mb));
           const float p1 = fast_exp2(fmaf(sv[c * 32 + 2 * x + 1], sl2, -mb));
-          rs += p0 + p1;
+          rs8[x & 7] += p0 + p1;
           pk[x] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tl + b * 128 + c * 16, pk);
       }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       tmem_wait_st();
       // O may be rescaled only once the previous P V product has landed.
       if (j >= 1) {

@@ -135,7 +135,7 @@ def test_full_size_sampled(config):
     w = synth.make_workload(config)
     bwd = config != 1
     q, k, v, do = inputs(w, 1000 + config, with_do=bwd)
-    got, _ = _run_gpu(w, q, k, v, do)
+    got, _ = _run_gpu(w, q, k, v, do, out_dtype=torch.bfloat16)  # O stored as the benchmark stores it
     lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
     qr = orc.rope(q, lay.pos_id, w.base)
     kr = orc.rope(k, lay.pos_id, w.base)
@@ -168,7 +168,7 @@ def test_full_size_sampled(config):
 def test_depth_sweep_sampled(n_turns):
     w = synth.make_workload(3, n_turns=n_turns)
     q, k, v, do = inputs(w, 3000 + n_turns)
-    got, _ = _run_gpu(w, q, k, v, do)
+    got, _ = _run_gpu(w, q, k, v, do, out_dtype=torch.bfloat16)
     lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
     qr = orc.rope(q, lay.pos_id, w.base)
     kr = orc.rope(k, lay.pos_id, w.base)

@@ -73,8 +73,11 @@ def test_layout_npass_is_causal():
         L = int(ref.cu_seqlens[s + 1] - ref.cu_seqlens[s])
         nt = (L + 127) // 128
         for I in range(nt):
-            # causal: everything strictly below the diagonal inside the sequence is full
-            assert all(bm[s, I, J] == 1 for J in range(I))
+            # causal: strictly below the diagonal is full, except in a tail tile row
+            # (rows past the end count as not visible), which is partial
+            below = 1 if (I + 1) * 128 <= L else 2
+            assert all(bm[s, I, J] == below for J in range(I))
+            assert bm[s, I, I] == 2
             assert all(bm[s, I, J] == 0 for J in range(I + 1, bm.shape[1]))
 
 
