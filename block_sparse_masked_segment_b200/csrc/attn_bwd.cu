@@ -16,7 +16,8 @@
 // Q/K and the dS operand share one 16-bit type (fp16 when QK16, else bf16);
 // dO, V and P are bf16.
 // Warp roles as in the forward: warp 0 TMA producer (+ metadata lanes),
-// warp 1 TMEM owner and MMA issuer, warps 2..5 one row per thread.
+// warp 1 TMEM owner and MMA issuer, warps 2..9 two threads per TMEM lane
+// (row), each owning 64 of the tile's 128 columns.
 #include "attn_common.cuh"
 
 namespace opr {
@@ -63,16 +64,17 @@ struct DqSmem {
   uint32_t kstarts[kStages][4];
   uint64_t bar_qdo;
   uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
-  uint64_t bar_sfull, bar_dpfull, bar_dsfull, bar_dqdone, bar_final;
+  uint64_t bar_sfull, bar_sfree, bar_dpfull, bar_dsfull, bar_dqdone, bar_final;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// TMEM columns of the dq kernel: S / dS at 0, dP at 128, dQ accumulator at 256.
-constexpr uint32_t kDqColS = 0, kDqColDP = 128, kDqColAcc = 256;
+// TMEM columns of the dq kernel: S at 0, dP at 128, dQ accumulator at 256,
+// dS (16-bit, 64 columns) at 384.
+constexpr uint32_t kDqColS = 0, kDqColDP = 128, kDqColAcc = 256, kDqColDS = 384;
 
 template <int D, bool QK16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                        const AttnParams p) {
@@ -103,8 +105,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&sm.bar_vempty[st], 1);
     }
     mbar_init(&sm.bar_sfull, 1);
+    mbar_init(&sm.bar_sfree, kComputeThreads);
     mbar_init(&sm.bar_dpfull, 1);
-    mbar_init(&sm.bar_dsfull, 128);
+    mbar_init(&sm.bar_dsfull, kComputeThreads);
     mbar_init(&sm.bar_dqdone, 1);
     mbar_init(&sm.bar_final, 1);
     sm.abort_flag = 0;
@@ -167,24 +170,22 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP = dO V^T (bf16)
       constexpr uint32_t idesc_q = idesc_f32acc(128, D, QK16, 0, 1);    // dQ += dS K (K tile MN-major)
       const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
-      bool ok = mbar_wait(&sm.bar_qdo, 0, abort_flag, kWaitLimitNs);
-      for (int j = 0; ok && j < n; ++j) {
+      // S(j) = Q K(j)^T
+      auto issue_s = [&](int j) -> bool {
         const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (!mbar_wait(&sm.bar_kfull[st], ph, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t sk = smem_u32(sm.k[st]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + kDqColS, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
         mma_commit(&sm.bar_sfull);
-        if (!mbar_wait(&sm.bar_vfull[st], ph, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
+        return true;
+      };
+      // dP(j) = dO V(j)^T; releases V(j)
+      auto issue_dp = [&](int j) -> bool {
+        const int st = j % kStages;
+        if (!mbar_wait(&sm.bar_vfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t sv = smem_u32(sm.v[st]);
 #pragma unroll
@@ -192,23 +193,40 @@ __global__ void __launch_bounds__(192, 1)
           mma_ss(tmem + kDqColDP, desc_kmajor(sdo, kk), desc_kmajor(sv, kk), idesc_p, kk > 0 ? 1u : 0u);
         mma_commit(&sm.bar_dpfull);
         mma_commit(&sm.bar_vempty[st]);
-        if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
+        return true;
+      };
+      // dQ += dS(j) K(j); releases K(j) and its metadata
+      auto issue_dq = [&](int j) -> bool {
+        const int st = j % kStages;
+        if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
+        const uint32_t sk = smem_u32(sm.k[st]);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kDqColAcc, tmem + kDqColS + kk * 8, desc_mnmajor(sk, kk), idesc_q,
+          mma_ts(tmem + kDqColAcc, tmem + kDqColDS + kk * 8, desc_mnmajor(sk, kk), idesc_q,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar_kempty[st]);
+        return true;
+      };
+      // Issue order S(0) dP(0) | S(1) dQ(0) dP(1) | S(2) dQ(1) dP(2) | ...: S(j+1) starts as
+      // soon as the compute warps have read S(j), while they still form P(j) and dS(j).
+      bool ok = mbar_wait(&sm.bar_qdo, 0, abort_flag, kWaitLimitNs) && issue_s(0) && issue_dp(0);
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 1 < n) {
+          ok = mbar_wait(&sm.bar_sfree, j & 1, abort_flag, kWaitLimitNs) && issue_s(j + 1);
+          if (!ok) break;
+        }
+        ok = issue_dq(j);
+        if (ok && j + 1 < n) ok = issue_dp(j + 1);
       }
       if (ok) mma_commit(&sm.bar_dqdone);
       mma_commit(&sm.bar_final);
       mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
     }
   } else {
+    // two threads per query row: `half` selects key columns [64 half, 64 half + 64)
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const bool qv = I * kTile + row < seq_len;
@@ -229,42 +247,50 @@ __global__ void __launch_bounds__(192, 1)
         ok = false;
         break;
       }
+      // visibility of this thread's 64 key columns (all set on full tiles)
+      uint32_t mm[2] = {0xffffffffu, 0xffffffffu};
+      if (partial) {
+        uint32_t m[4];
+        query_row_mask(sm.kstarts[st], sm.kconv[st], sm.kmeta[st], kbase, qg, qconv, qmeta, m);
+        mm[0] = half ? m[2] : m[0];
+        mm[1] = half ? m[3] : m[1];
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float pv[kTile];
+      float pv[64];
       {
-        uint32_t sr[kTile];
-        tmem_ld128(tl + kDqColS, sr);
+        uint32_t sr[64];
+        tmem_ld64(tl + kDqColS + half * 64, sr);
+        tc_fence_before();
+        mbar_arrive(&sm.bar_sfree);  // S may be overwritten by the next Q K^T
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) pv[c] = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
+        for (int c = 0; c < 64; ++c) pv[c] = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
       }
-      if (partial) {
-        uint32_t m[4];
-        query_row_mask(sm.kstarts[st], sm.kconv[st], sm.kmeta[st], kbase, qg, qconv, qmeta, m);
 #pragma unroll
-        for (int c = 0; c < kTile; ++c)
-          if (!mask_bit(m, c)) pv[c] = 0.f;
-      }
+      for (int c = 0; c < 64; ++c)
+        if (!((mm[c >> 5] >> (c & 31)) & 1u)) pv[c] = 0.f;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      {
+        uint32_t r[64];
+        tmem_ld64(tl + kDqColDP + half * 64, r);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tl + kDqColDP + c * 32, r);
-        uint32_t pk[16];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const float d0 = pv[c * 32 + 2 * x] * (__uint_as_float(r[2 * x]) - dd);
-          const float d1 = pv[c * 32 + 2 * x + 1] * (__uint_as_float(r[2 * x + 1]) - dd);
-          pk[x] = pack_x2<QK16>(d0, d1);
+          for (int x = 0; x < 16; ++x) {
+            const float d0 = pv[c * 32 + 2 * x] * (__uint_as_float(r[c * 32 + 2 * x]) - dd);
+            const float d1 = pv[c * 32 + 2 * x + 1] * (__uint_as_float(r[c * 32 + 2 * x + 1]) - dd);
+            pk[x] = pack_x2<QK16>(d0, d1);
+          }
+          tmem_st16(tl + kDqColDS + half * 32 + c * 16, pk);
         }
-        tmem_st16(tl + kDqColS + c * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -274,11 +300,12 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       float* dst = p.dq + (static_cast<size_t>(qg) * p.hq + head) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
-        tmem_ld32(tl + kDqColAcc + c * 32, r);
+        const int oc = half * (D / 2) + c * 32;
+        tmem_ld32(tl + kDqColAcc + oc, r);
         if (qv) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+          float4* d4 = reinterpret_cast<float4*>(dst + oc);
 #pragma unroll
           for (int x = 0; x < 8; ++x)
             d4[x] = make_float4(__uint_as_float(r[4 * x]) * p.scale, __uint_as_float(r[4 * x + 1]) * p.scale,
@@ -322,7 +349,7 @@ struct DkdvSmem {
 constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvColDV = 256;
 
 template <int D, bool QK16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                          const AttnParams p) {
@@ -356,8 +383,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(&sm.bar_sfull, 1);
     mbar_init(&sm.bar_dpfull, 1);
-    mbar_init(&sm.bar_pfull, 128);
-    mbar_init(&sm.bar_dsfull, 128);
+    mbar_init(&sm.bar_pfull, kComputeThreads);
+    mbar_init(&sm.bar_dsfull, kComputeThreads);
     mbar_init(&sm.bar_accdone, 1);
     mbar_init(&sm.bar_final, 1);
     sm.abort_flag = 0;
@@ -427,35 +454,36 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idesc_v = idesc_bf16_f32(128, D, 0, 1);        // dV += P^T dO (bf16)
       constexpr uint32_t idesc_k = idesc_f32acc(128, D, QK16, 0, 1);    // dK += dS^T Q (q/k type)
       const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
-      bool ok = mbar_wait(&sm.bar_kv, 0, abort_flag, kWaitLimitNs);
-      for (int j = 0; ok && j < n; ++j) {
+      // S^T(j) = K Q(j)^T into the S region
+      auto issue_s = [&](int j) -> bool {
         const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (!mbar_wait(&sm.bar_qfull[st], ph, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
+        if (!mbar_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t sq = smem_u32(sm.q[st]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + kKvColS, desc_kmajor(sk, kk), desc_kmajor(sq, kk), idesc_s, kk > 0 ? 1u : 0u);
         mma_commit(&sm.bar_sfull);
-        if (!mbar_wait(&sm.bar_dofull[st], ph, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
+        return true;
+      };
+      // dP^T(j) = V dO(j)^T into the dP region
+      auto issue_dp = [&](int j) -> bool {
+        const int st = j % kStages;
+        if (!mbar_wait(&sm.bar_dofull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t sdo = smem_u32(sm.dout[st]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           mma_ss(tmem + kKvColDP, desc_kmajor(sv, kk), desc_kmajor(sdo, kk), idesc_p, kk > 0 ? 1u : 0u);
         mma_commit(&sm.bar_dpfull);
-        if (!mbar_wait(&sm.bar_pfull, j & 1, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
+        return true;
+      };
+      // dV += P^T(j) dO(j), P^T as bf16 hi + lo parts; releases dO(j)
+      auto issue_dv = [&](int j) -> bool {
+        const int st = j % kStages;
+        if (!mbar_wait(&sm.bar_pfull, j & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
+        const uint32_t sdo = smem_u32(sm.dout[st]);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
           mma_ts(tmem + kKvColDV, tmem + kKvColS + kk * 8, desc_mnmajor(sdo, kk), idesc_v,
@@ -464,23 +492,39 @@ __global__ void __launch_bounds__(192, 1)
         for (int kk = 0; kk < kTile / 16; ++kk)
           mma_ts(tmem + kKvColDV, tmem + kKvColS + 64 + kk * 8, desc_mnmajor(sdo, kk), idesc_v, 1u);
         mma_commit(&sm.bar_doempty[st]);
-        if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
+        return true;
+      };
+      // dK += dS^T(j) Q(j); releases Q(j) and its column data
+      auto issue_dk = [&](int j) -> bool {
+        const int st = j % kStages;
+        if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
+        const uint32_t sq = smem_u32(sm.q[st]);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
           mma_ts(tmem + kColDK, tmem + kKvColDP + kk * 8, desc_mnmajor(sq, kk), idesc_k,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar_qempty[st]);
+        return true;
+      };
+      // Issue order S(0) dP(0) | dV(0) S(1) dK(0) dP(1) | dV(1) S(2) dK(1) dP(2) | ...
+      // so that the next S^T is formed while the compute warps turn dP^T into dS^T,
+      // and the next dP^T while they turn S^T into P^T.
+      bool ok = mbar_wait(&sm.bar_kv, 0, abort_flag, kWaitLimitNs) && issue_s(0) && issue_dp(0);
+      for (int j = 0; ok && j < n; ++j) {
+        ok = issue_dv(j);
+        if (ok && j + 1 < n) ok = issue_s(j + 1);
+        if (ok) ok = issue_dk(j);
+        if (ok && j + 1 < n) ok = issue_dp(j + 1);
       }
       if (ok) mma_commit(&sm.bar_accdone);
       mma_commit(&sm.bar_final);
       mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
     }
   } else {
+    // two threads per key row: `half` selects query columns [64 half, 64 half + 64)
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const bool kvld = J * kTile + row < seq_len;
@@ -488,6 +532,7 @@ __global__ void __launch_bounds__(192, 1)
     const int kconv = kvld ? p.conv_idx[kg] : -1;
     const int kmeta = kvld ? p.tok_meta[kg] : 0;
     const float sl2 = p.scale_log2;
+    const int c0 = half * 64;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j % kStages;
@@ -498,29 +543,41 @@ __global__ void __launch_bounds__(192, 1)
         ok = false;
         break;
       }
+      // visibility of this thread's 64 query columns (all set on full tiles)
+      uint32_t mm[2] = {0xffffffffu, 0xffffffffu};
+      if (partial) {
+        uint32_t m[4];
+        key_row_mask(sm.qstarts[st], sm.qconv[st], sm.qmeta[st], qt0, kg, kconv, kmeta, m);
+        mm[0] = half ? m[2] : m[0];
+        mm[1] = half ? m[3] : m[1];
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float pv[kTile];
-      {
-        uint32_t sr[kTile];
-        tmem_ld128(tl + kKvColS, sr);
+      float pv[64];
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) pv[c] = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -sm.qlse2[st][c]));
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sr[32];
+        tmem_ld32(tl + kKvColS + c0 + cc * 32, sr);
+        const float4* l4 = reinterpret_cast<const float4*>(&sm.qlse2[st][c0 + cc * 32]);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const float4 l = l4[x];
+          pv[cc * 32 + 4 * x] = fast_exp2(fmaf(__uint_as_float(sr[4 * x]), sl2, -l.x));
+          pv[cc * 32 + 4 * x + 1] = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 1]), sl2, -l.y));
+          pv[cc * 32 + 4 * x + 2] = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 2]), sl2, -l.z));
+          pv[cc * 32 + 4 * x + 3] = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 3]), sl2, -l.w));
+        }
       }
-      if (partial) {
-        uint32_t m[4];
-        key_row_mask(sm.qstarts[st], sm.qconv[st], sm.qmeta[st], qt0, kg, kconv, kmeta, m);
 #pragma unroll
-        for (int c = 0; c < kTile; ++c)
-          if (!mask_bit(m, c)) pv[c] = 0.f;
-      }
-      // P^T for dV = P^T dO as bf16 hi + lo parts (columns 0..63 and 64..127 of
-      // the S^T region): the lo part carries the rounding error of the hi part.
+      for (int c = 0; c < 64; ++c)
+        if (!((mm[c >> 5] >> (c & 31)) & 1u)) pv[c] = 0.f;
+      // P^T for dV = P^T dO as bf16 hi + lo parts (TMEM columns 0..63 and 64..127 of
+      // the S^T region, two values per column): lo carries the rounding error of hi.
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
@@ -529,8 +586,8 @@ __global__ void __launch_bounds__(192, 1)
           hi[x] = *reinterpret_cast<const uint32_t*>(&h);
           lo[x] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
         }
-        tmem_st16(tl + kKvColS + c * 16, hi);
-        tmem_st16(tl + kKvColS + 64 + c * 16, lo);
+        tmem_st16(tl + kKvColS + half * 32 + c * 16, hi);
+        tmem_st16(tl + kKvColS + 64 + half * 32 + c * 16, lo);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -541,17 +598,18 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
-        tmem_ld32(tl + kKvColDP + c * 32, r);
+        tmem_ld32(tl + kKvColDP + c0 + c * 32, r);
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          const float d0 = pv[c * 32 + 2 * x] * (__uint_as_float(r[2 * x]) - sm.qd[st][c * 32 + 2 * x]);
-          const float d1 = pv[c * 32 + 2 * x + 1] * (__uint_as_float(r[2 * x + 1]) - sm.qd[st][c * 32 + 2 * x + 1]);
+          const int q = c * 32 + 2 * x;
+          const float d0 = pv[q] * (__uint_as_float(r[2 * x]) - sm.qd[st][c0 + q]);
+          const float d1 = pv[q + 1] * (__uint_as_float(r[2 * x + 1]) - sm.qd[st][c0 + q + 1]);
           pk[x] = pack_x2<QK16>(d0, d1);
         }
-        tmem_st16(tl + kKvColDP + c * 16, pk);
+        tmem_st16(tl + kKvColDP + half * 32 + c * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -562,11 +620,12 @@ __global__ void __launch_bounds__(192, 1)
       float* dvp = p.dv + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
       float* dkp = p.dk + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
-        tmem_ld32(tl + kKvColDV + c * 32, r);
+        const int oc = half * (D / 2) + c * 32;
+        tmem_ld32(tl + kKvColDV + oc, r);
         if (kvld) {
-          float4* d4 = reinterpret_cast<float4*>(dvp + c * 32);
+          float4* d4 = reinterpret_cast<float4*>(dvp + oc);
 #pragma unroll
           for (int x = 0; x < 8; ++x)
             d4[x] = make_float4(__uint_as_float(r[4 * x]), __uint_as_float(r[4 * x + 1]),
@@ -574,11 +633,12 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
-        tmem_ld32(tl + kColDK + c * 32, r);
+        const int oc = half * (D / 2) + c * 32;
+        tmem_ld32(tl + kColDK + oc, r);
         if (kvld) {
-          float4* d4 = reinterpret_cast<float4*>(dkp + c * 32);
+          float4* d4 = reinterpret_cast<float4*>(dkp + oc);
 #pragma unroll
           for (int x = 0; x < 8; ++x)
             d4[x] = make_float4(__uint_as_float(r[4 * x]) * p.scale, __uint_as_float(r[4 * x + 1]) * p.scale,
@@ -631,7 +691,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     const size_t smem_q = smem_request(sizeof(DqSmem<D>) + 1024);
     if ((e = set_smem(attn_bwd_dq_kernel<D, QK16>, smem_q, conf_dq)) != cudaSuccess) return e;
     const int64_t bq = static_cast<int64_t>(pq.n_items) * pq.hq;
-    if (bq > 0) attn_bwd_dq_kernel<D, QK16><<<static_cast<unsigned>(bq), 192, smem_q, stream>>>(tq, tk, tv, tdo, pq);
+    if (bq > 0) attn_bwd_dq_kernel<D, QK16><<<static_cast<unsigned>(bq), kThreads, smem_q, stream>>>(tq, tk, tv, tdo, pq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // 3) dK, dV
@@ -640,7 +700,7 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     if ((e = set_smem(attn_bwd_dkdv_kernel<D, QK16>, smem_kv, conf_kv)) != cudaSuccess) return e;
     const int64_t bkv = static_cast<int64_t>(pkv.n_items) * pkv.hkv;
     if (bkv > 0)
-      attn_bwd_dkdv_kernel<D, QK16><<<static_cast<unsigned>(bkv), 192, smem_kv, stream>>>(tq, tk, tv, tdo, pkv);
+      attn_bwd_dkdv_kernel<D, QK16><<<static_cast<unsigned>(bkv), kThreads, smem_kv, stream>>>(tq, tk, tv, tdo, pkv);
     e = cudaGetLastError();
   }
   return e;

@@ -13,6 +13,13 @@ namespace opr {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: any pipeline wait longer than this is a hang
 
+// CTA shape shared by the attention kernels: warp 0 TMA producer, warp 1 TMEM
+// owner / MMA issuer, warps 2..9 compute.  Two compute warps share each TMEM
+// lane quadrant (warp % 4): warps 2..5 own columns 0..63 of their rows, warps
+// 6..9 columns 64..127.
+constexpr int kThreads = 320;
+constexpr int kComputeThreads = 256;
+
 // A 128-row tile of head_dim D bf16 values is stored as D/64 "chunks", each
 // 128 rows x 128 bytes with the 128-byte swizzle TMA writes (box {64, 1, 128}).
 constexpr int kChunkBytes = kTile * 128;  // 16 KiB

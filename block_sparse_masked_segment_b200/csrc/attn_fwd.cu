@@ -10,11 +10,13 @@
 //               metadata of partial tiles;
 //   warp 1      allocates TMEM and issues tcgen05.mma: S = Q K^T into one of
 //               two TMEM buffers, then O += P V with P read from TMEM;
-//   warps 2..5  one query row per thread: read S from TMEM, apply the
-//               visibility predicate on partial tiles only, online softmax in
-//               base 2, write P (bf16) back over S, rescale O in TMEM only
-//               when the running max grows by more than 2^8; epilogue O / l
-//               and the log-sum-exp.
+//   warps 2..9  two threads per query row, each owning 64 of the tile's 128
+//               key columns: read S from TMEM, apply the visibility mask on
+//               partial tiles only, online softmax in base 2 (the row max is
+//               taken over all 128 columns by both threads, so no exchange is
+//               needed), write their half of P (bf16) back over S, rescale
+//               their half of O in TMEM only when the running max grows by
+//               more than 2^8; epilogue O / l and the log-sum-exp.
 // TMEM columns: S/P buffer 0 at 0, buffer 1 at 128, O at 256 (512 allocated).
 // Q and K may be bf16 or fp16 (QK16: the rotated q, k stored in fp16, whose
 // 11-bit significand keeps the rounding of the rotation 8x smaller); V and P
@@ -35,6 +37,7 @@ struct FwdSmem {
   int32_t kconv[kStages][kTile];
   int32_t kmeta[kStages][kTile];
   uint32_t kstarts[kStages][4];  // column-run starts of a partial tile
+  float lsum[2][kTile];           // row-sum halves, combined in the epilogue
   uint64_t bar_q;
   uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
   uint64_t bar_sfull[2], bar_pfull[2], bar_odone, bar_final;
@@ -43,7 +46,7 @@ struct FwdSmem {
 };
 
 template <int D, bool QK16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   constexpr uint32_t kTileBytes = TileGeom<D>::kBytes;
@@ -74,7 +77,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.bar_sfull[b], 1);
-      mbar_init(&sm.bar_pfull[b], 128);
+      mbar_init(&sm.bar_pfull[b], kComputeThreads);
     }
     mbar_init(&sm.bar_odone, 1);
     mbar_init(&sm.bar_final, 1);
@@ -178,7 +181,8 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int quad = warp & 3;        // TMEM lane quadrant this warp may access
+    const int half = (warp - 2) >> 2;  // key columns [64 half, 64 half + 64)
     const int row = quad * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const bool qv = I * kTile + row < seq_len;
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(192, 1)
     const int qconv = qv ? p.conv_idx[qg] : -2;
     const int qmeta = qv ? p.tok_meta[qg] : 0;
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int b = j & 1, st = j % kStages;
@@ -198,24 +202,36 @@ __global__ void __launch_bounds__(192, 1)
         ok = false;
         break;
       }
+      // visibility: own 64 columns in words 0..1, the partner's in 2..3 (all set on full tiles)
+      uint32_t mm[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      if (partial) {
+        uint32_t m[4];
+        query_row_mask(sm.kstarts[st], sm.kconv[st], sm.kmeta[st], kbase, qg, qconv, qmeta, m);
+        mm[0] = half ? m[2] : m[0];
+        mm[1] = half ? m[3] : m[1];
+        mm[2] = half ? m[0] : m[2];
+        mm[3] = half ? m[1] : m[3];
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[b], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[kTile];
-      tmem_ld128(tl + b * 128, sr);
+      // own 64 columns in sv[0..63], the partner thread's 64 in sv[64..127] (max only)
       float sv[kTile];
+      {
+        uint32_t sr[kTile];
+        const uint32_t own = tl + b * 128 + half * 64, oth = tl + b * 128 + (half ^ 1) * 64;
+        tmem_ld32x4(own, own + 32, oth, oth + 32, sr);
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) sv[c] = __uint_as_float(sr[c]);
+        for (int c = 0; c < kTile; ++c) sv[c] = __uint_as_float(sr[c]);
+      }
       if (partial) {
-        uint32_t m[4];
-        query_row_mask(sm.kstarts[st], sm.kconv[st], sm.kmeta[st], kbase, qg, qconv, qmeta, m);
 #pragma unroll
         for (int c = 0; c < kTile; ++c)
-          if (!mask_bit(m, c)) sv[c] = -INFINITY;
+          if (!mask_bit(mm, c)) sv[c] = -INFINITY;
       }
-      // row max as a tree (8 independent chains)
+      // row max over all 128 columns (8 independent chains)
       float mx8[8];
 #pragma unroll
       for (int x = 0; x < 8; ++x) mx8[x] = sv[x];
@@ -227,9 +243,10 @@ __global__ void __launch_bounds__(192, 1)
       const bool need = m_new > m_run + 8.f;  // also true on the first finite max
       const float m_use = need ? m_new : m_run;
       const float mb = (m_use == -INFINITY) ? 0.f : m_use;
+      // this thread's 64 columns of P, packed two per TMEM column over S
       float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
@@ -238,7 +255,7 @@ __global__ void __launch_bounds__(192, 1)
           rs8[x & 7] += p0 + p1;
           pk[x] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tl + b * 128 + c * 16, pk);
+        tmem_st16(tl + b * 128 + half * 32 + c * 16, pk);
       }
       const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       tmem_wait_st();
@@ -253,12 +270,13 @@ __global__ void __launch_bounds__(192, 1)
       const float factor = need ? fast_exp2(m_run - m_new) : 1.f;
       if (__any_sync(0xffffffffu, need && j >= 1)) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t r[32];
-          tmem_ld32(tl + kOCol + c * 32, r);
+          const uint32_t oc = kOCol + half * (D / 2) + c * 32;
+          tmem_ld32(tl + oc, r);
 #pragma unroll
           for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * factor);
-          tmem_st32(tl + kOCol + c * 32, r);
+          tmem_st32(tl + oc, r);
         }
         tmem_wait_st();
       }
@@ -268,23 +286,28 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(&sm.bar_pfull[b]);
     }
     // ------------------------------------------------------------ epilogue
+    // Every compute thread reaches this barrier exactly once (also after an abort).
+    sm.lsum[half][row] = l_run;
+    named_bar_sync(1, kComputeThreads);
     if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_odone, (n - 1) & 1, abort_flag, kWaitLimitNs))) {
       tc_fence_after();
-      const float inv = 1.f / l_run;
+      const float l_tot = sm.lsum[0][row] + sm.lsum[1][row];
+      const float inv = 1.f / l_tot;
       const size_t orow = (static_cast<size_t>(qg) * p.hq + head) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
-        tmem_ld32(tl + kOCol + c * 32, r);
+        const int oc = half * (D / 2) + c * 32;
+        tmem_ld32(tl + kOCol + oc, r);
         if (qv) {
           if (p.o_fp32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c * 32);
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + oc);
 #pragma unroll
             for (int x = 0; x < 8; ++x)
               dst[x] = make_float4(__uint_as_float(r[4 * x]) * inv, __uint_as_float(r[4 * x + 1]) * inv,
                                    __uint_as_float(r[4 * x + 2]) * inv, __uint_as_float(r[4 * x + 3]) * inv);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow + c * 32);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow + oc);
 #pragma unroll
             for (int x = 0; x < 4; ++x)
               dst[x] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * x]) * inv, __uint_as_float(r[8 * x + 1]) * inv),
@@ -294,7 +317,8 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
-      if (qv) p.lse[static_cast<size_t>(head) * p.total + qg] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (qv && half == 0)
+        p.lse[static_cast<size_t>(head) * p.total + qg] = (m_run + __log2f(l_tot)) * 0.69314718055994531f;
     }
   }
 
@@ -325,7 +349,7 @@ cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, cons
   }
   const int64_t blocks = static_cast<int64_t>(p.n_items) * p.hq;
   if (blocks == 0) return cudaSuccess;
-  attn_fwd_kernel<D, QK16><<<static_cast<unsigned>(blocks), 192, smem, stream>>>(tq, tk, tv, p);
+  attn_fwd_kernel<D, QK16><<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
