@@ -345,8 +345,14 @@ struct DkdvSmem {
 };
 
 // TMEM columns of the dkdv kernel: S^T / P^T at 0, dP^T / dS^T at 128,
-// dV accumulator at 256, dK accumulator at 256 + D.
+// dV accumulator at 256, dK accumulator at 256 + D.  Each compute thread
+// overwrites only the 64 columns it has itself read: the packed 16-bit values
+// of query columns 0..63 go to region columns 0..31 (P^T hi; P^T lo at
+// 32..63) and those of query columns 64..127 to 64..95 (lo at 96..127), so the
+// MMA's K step kk reads region column split_col(kk).
 constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvColDV = 256;
+
+__device__ __forceinline__ uint32_t split_col(int kk) { return (kk & 3) * 8 + (kk >> 2) * 64; }
 
 template <int D, bool QK16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -486,11 +492,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sdo = smem_u32(sm.dout[st]);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kKvColDV, tmem + kKvColS + kk * 8, desc_mnmajor(sdo, kk), idesc_v,
+          mma_ts(tmem + kKvColDV, tmem + kKvColS + split_col(kk), desc_mnmajor(sdo, kk), idesc_v,
                  (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kKvColDV, tmem + kKvColS + 64 + kk * 8, desc_mnmajor(sdo, kk), idesc_v, 1u);
+          mma_ts(tmem + kKvColDV, tmem + kKvColS + 32 + split_col(kk), desc_mnmajor(sdo, kk), idesc_v, 1u);
         mma_commit(&sm.bar_doempty[st]);
         return true;
       };
@@ -502,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sq = smem_u32(sm.q[st]);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kColDK, tmem + kKvColDP + kk * 8, desc_mnmajor(sq, kk), idesc_k,
+          mma_ts(tmem + kColDK, tmem + kKvColDP + split_col(kk), desc_mnmajor(sq, kk), idesc_k,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar_qempty[st]);
         return true;
@@ -574,8 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 64; ++c)
         if (!((mm[c >> 5] >> (c & 31)) & 1u)) pv[c] = 0.f;
-      // P^T for dV = P^T dO as bf16 hi + lo parts (TMEM columns 0..63 and 64..127 of
-      // the S^T region, two values per column): lo carries the rounding error of hi.
+      // P^T for dV = P^T dO as bf16 hi + lo parts, two values per TMEM column, in this
+      // thread's own 64 columns of the S^T region: lo carries the rounding error of hi.
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t hi[16], lo[16];
@@ -586,8 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           hi[x] = *reinterpret_cast<const uint32_t*>(&h);
           lo[x] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
         }
-        tmem_st16(tl + kKvColS + half * 32 + c * 16, hi);
-        tmem_st16(tl + kKvColS + 64 + half * 32 + c * 16, lo);
+        tmem_st16(tl + kKvColS + c0 + c * 16, hi);
+        tmem_st16(tl + kKvColS + c0 + 32 + c * 16, lo);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -609,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float d1 = pv[q + 1] * (__uint_as_float(r[2 * x + 1]) - sm.qd[st][c0 + q + 1]);
           pk[x] = pack_x2<QK16>(d0, d1);
         }
-        tmem_st16(tl + kKvColDP + half * 32 + c * 16, pk);
+        tmem_st16(tl + kKvColDP + c0 + c * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();

@@ -14,10 +14,11 @@
 //               key columns: read S from TMEM, apply the visibility mask on
 //               partial tiles only, online softmax in base 2 (the row max is
 //               taken over all 128 columns by both threads, so no exchange is
-//               needed), write their half of P (bf16) back over S, rescale
+//               needed), write their half of P (bf16) to TMEM, rescale
 //               their half of O in TMEM only when the running max grows by
 //               more than 2^8; epilogue O / l and the log-sum-exp.
-// TMEM columns: S/P buffer 0 at 0, buffer 1 at 128, O at 256 (512 allocated).
+// TMEM columns: S buffer 0 at 0, buffer 1 at 128, O at 256, P buffers at 384
+// and 448 (512 allocated).
 // Q and K may be bf16 or fp16 (QK16: the rotated q, k stored in fp16, whose
 // 11-bit significand keeps the rounding of the rotation 8x smaller); V and P
 // are bf16.
@@ -28,6 +29,8 @@ namespace {
 
 constexpr int kStages = 2;
 constexpr uint32_t kOCol = 256;
+constexpr uint32_t kPCol = 384;  // P buffers (bf16, 64 columns each): never alias S, which both
+                                 // threads of a row read for the row max
 
 template <int D>
 struct FwdSmem {
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sv = smem_u32(sm.v[stp]);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kOCol, tmem + bp * 128 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
+          mma_ts(tmem + kOCol, tmem + kPCol + bp * 64 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
                  (jp > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&sm.bar_vempty[stp]);
         mma_commit(&sm.bar_odone);
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           rs8[x & 7] += p0 + p1;
           pk[x] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tl + b * 128 + half * 32 + c * 16, pk);
+        tmem_st16(tl + kPCol + b * 64 + half * 32 + c * 16, pk);
       }
       const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       tmem_wait_st();
