@@ -129,8 +129,8 @@ class Runner:
                       torch.empty((n, w.hkv, w.d), dtype=torch.float32, device=device),
                       torch.empty((n, w.hkv, w.d), dtype=torch.float32, device=device))
         self.h_grads = tuple(torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in self.grads)
-        self.bwd_ws = torch.empty(max(opr.opr_attn_bwd_workspace_bytes(n, w.hq, w.d), 256), dtype=torch.uint8,
-                                  device=device)
+        self.bwd_ws = torch.empty(max(opr.opr_attn_bwd_workspace_bytes(w.n_seqs, w.max_seqlen, w.hq, w.d), 256),
+                                  dtype=torch.uint8, device=device)
         self.total, self.max_seqlen = n, w.max_seqlen
         self.pairs = visible_pairs_closed_form(w.turn_lens, w.conv_turn_ptr)
         self.conv_tokens = w.conversation_tokens()

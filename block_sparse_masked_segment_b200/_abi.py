@@ -72,7 +72,7 @@ def load_library() -> ctypes.CDLL:
     lib.opr_attn_fwd.restype = I32
     lib.opr_attn_fwd.argtypes = [P, P, P, I32, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F, P, I32, P, P, P]
     lib.opr_attn_bwd_workspace_bytes.restype = SZ
-    lib.opr_attn_bwd_workspace_bytes.argtypes = [I64, I32, I32]
+    lib.opr_attn_bwd_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.opr_attn_bwd.restype = I32
     lib.opr_attn_bwd.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F,
                                  P, P, P, P, SZ, P, P]
@@ -112,8 +112,8 @@ def opr_layout_workspace_bytes(n_seqs, n_convs, n_turns, total_tokens, max_seqle
     return int(load_library().opr_layout_workspace_bytes(n_seqs, n_convs, n_turns, total_tokens, max_seqlen))
 
 
-def opr_attn_bwd_workspace_bytes(total_tokens, hq, head_dim) -> int:
-    return int(load_library().opr_attn_bwd_workspace_bytes(total_tokens, hq, head_dim))
+def opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) -> int:
+    return int(load_library().opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim))
 
 
 @dataclass
@@ -268,7 +268,7 @@ def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, w
                torch.empty((total, hkv, d), dtype=torch.float32, device=q.device),
                torch.empty((total, hkv, d), dtype=torch.float32, device=q.device))
     dq, dk, dv = out
-    wb = opr_attn_bwd_workspace_bytes(total, hq, d)
+    wb = opr_attn_bwd_workspace_bytes(lay.n_seqs, lay.max_seqlen, hq, d)
     if workspace is None or workspace.numel() < wb:
         workspace = torch.empty(max(wb, 256), dtype=torch.uint8, device=q.device)
     args = (_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16, _ptr(do),

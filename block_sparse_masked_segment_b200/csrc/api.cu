@@ -84,6 +84,7 @@ AttnParams base_params(const int32_t* cu_seqlens, const int32_t* conv_idx, const
   p.col_cnt = ws_ptr<int32_t>(ws, w.col_cnt);
   p.col_list = ws_ptr<int32_t>(ws, w.col_list);
   p.sched = ws_ptr<int32_t>(ws, w.q_sched);
+  p.tile_meta = ws_ptr<TileMeta>(ws, w.tile_meta);
   p.T = w.T;
   p.n_items = w.n_tiles;
   p.total = total;
@@ -178,10 +179,12 @@ opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_
   return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
 }
 
-size_t opr_attn_bwd_workspace_bytes(int64_t total_tokens, int32_t hq, int32_t head_dim) {
+size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
   (void)head_dim;
-  if (total_tokens < 0 || hq < 0) return 0;
-  return align_up(sizeof(float) * static_cast<size_t>(total_tokens) * static_cast<size_t>(hq), 256);
+  if (n_seqs < 0 || max_seqlen < 0 || hq < 0) return 0;
+  const size_t T = (static_cast<size_t>(max_seqlen) + kTile - 1) / kTile;
+  // D and LSE * log2(e) per (head, tile, token of the tile)
+  return align_up(2 * sizeof(float) * static_cast<size_t>(hq) * static_cast<size_t>(n_seqs) * T * kTile, 256);
 }
 
 opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int32_t qk_dtype, const void* o,
@@ -202,7 +205,8 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
   if (qk_dtype != OPR_DTYPE_BF16 && qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
   const bool f16 = qk_dtype == OPR_DTYPE_FP16;
-  if (workspace_bytes < opr_attn_bwd_workspace_bytes(total_tokens, hq, head_dim)) return OPR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim))
+    return OPR_WORKSPACE_TOO_SMALL;
   opr_status st = device_check();
   if (st != OPR_OK) return st;
   CUtensorMap tq, tk, tv, tdo;
@@ -213,7 +217,8 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   AttnParams pq = base_params(cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs, n_turns, total_tokens, max_seqlen,
                               hq, hkv, scale, dev_status);
   pq.lse_in = lse;
-  pq.row_d = static_cast<const float*>(workspace);
+  pq.d_tiles = static_cast<const float*>(workspace);
+  pq.lse2_tiles = pq.d_tiles + static_cast<size_t>(hq) * pq.n_items * kTile;
   pq.dq = dq;
   pq.dk = dk;
   pq.dv = dv;

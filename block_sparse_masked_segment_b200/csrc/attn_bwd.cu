@@ -24,32 +24,59 @@ namespace opr {
 namespace {
 
 constexpr int kStages = 2;
+constexpr int kListSmem = 1024;  // entries of a tile list kept in shared memory
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ----------------------------------------------------------------------------
-// D[h, q] = sum_d dO[q, h, d] * O[q, h, d]; one warp per (token, head).
+// Row terms, stored per 128-token tile so the kernels can bulk-copy them:
+// d_tiles[h][tile][c] = sum_d dO * O and lse2_tiles[h][tile][c] = LSE * log2(e)
+// of token c of tile (s, J); 0 and +inf past the end of the sequence.
+// One block of 128 threads per (tile, head), one token per thread.
 template <int D, typename OT>
-__global__ void __launch_bounds__(256) row_d_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                                                    int64_t total, int32_t hq, float* __restrict__ row_d) {
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= total * hq) return;
-  const int64_t tok = w / hq;
-  const int h = static_cast<int>(w % hq);
-  const size_t base = static_cast<size_t>(w) * D;
-  float acc = 0.f;
-#pragma unroll
-  for (int x = lane; x < D; x += 32) {
-    float ov;
-    if constexpr (sizeof(OT) == 4)
-      ov = o[base + x];
-    else
-      ov = __bfloat162float(o[base + x]);
-    acc = fmaf(ov, __bfloat162float(dout[base + x]), acc);
+__global__ void __launch_bounds__(128) row_terms_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                                                        const float* __restrict__ lse, const int32_t* __restrict__ cu_seqlens,
+                                                        int64_t total, int32_t hq, int32_t T, float* __restrict__ d_tiles,
+                                                        float* __restrict__ lse2_tiles) {
+  const int tile = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
+  const int s = tile / T, J = tile % T;
+  const int seq0 = cu_seqlens[s];
+  const int L = cu_seqlens[s + 1] - seq0;
+  const size_t out = (static_cast<size_t>(h) * gridDim.x + tile) * kTile + c;
+  if (J * kTile + c >= L) {
+    d_tiles[out] = 0.f;
+    lse2_tiles[out] = INFINITY;
+    return;
   }
+  const int64_t tok = seq0 + J * kTile + c;
+  const size_t base = (static_cast<size_t>(tok) * hq + h) * D;
+  const uint4* dp = reinterpret_cast<const uint4*>(dout + base);
+  float acc = 0.f;
+#pragma unroll 4
+  for (int x = 0; x < D / 8; ++x) {
+    const uint4 dv = dp[x];
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+    float ov[8];
+    if constexpr (sizeof(OT) == 4) {
+      const float4* op = reinterpret_cast<const float4*>(o + base) + 2 * x;
+      const float4 a = op[0], b = op[1];
+      ov[0] = a.x; ov[1] = a.y; ov[2] = a.z; ov[3] = a.w; ov[4] = b.x; ov[5] = b.y; ov[6] = b.z; ov[7] = b.w;
+    } else {
+      const uint4 ou = reinterpret_cast<const uint4*>(o + base)[x];
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ou);
 #pragma unroll
-  for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
-  if (lane == 0) row_d[static_cast<size_t>(h) * total + tok] = acc;
+      for (int y = 0; y < 4; ++y) {
+        ov[2 * y] = __low2float(o2[y]);
+        ov[2 * y + 1] = __high2float(o2[y]);
+      }
+    }
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      acc = fmaf(ov[2 * y], __low2float(d2[y]), acc);
+      acc = fmaf(ov[2 * y + 1], __high2float(d2[y]), acc);
+    }
+  }
+  d_tiles[out] = acc;
+  lse2_tiles[out] = lse[static_cast<size_t>(h) * total + tok] * kLog2e;
 }
 
 // ----------------------------------------------------------------------------
@@ -59,9 +86,8 @@ struct DqSmem {
   alignas(1024) uint8_t dout[TileGeom<D>::kBytes];
   alignas(1024) uint8_t k[kStages][TileGeom<D>::kBytes];
   alignas(1024) uint8_t v[kStages][TileGeom<D>::kBytes];
-  int32_t kconv[kStages][kTile];
-  int32_t kmeta[kStages][kTile];
-  uint32_t kstarts[kStages][4];
+  alignas(16) TileMeta kmeta[kStages];  // key metadata of a partial tile, rides with its K tile
+  int32_t list[kListSmem];
   uint64_t bar_qdo;
   uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
   uint64_t bar_sfull, bar_sfree, bar_dpfull, bar_dsfull, bar_dqdone, bar_final;
@@ -96,10 +122,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = seq0 + I * kTile;
   const int kvh = head / (p.hq / p.hkv);
 
+  for (int x = threadIdx.x; x < n && x < kListSmem; x += blockDim.x) sm.list[x] = list[x];
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_qdo, 1);
     for (int st = 0; st < kStages; ++st) {
-      mbar_init(&sm.bar_kfull[st], 1 + 32);  // TMA expect-tx arrival + 32 metadata lanes
+      mbar_init(&sm.bar_kfull[st], 1);
       mbar_init(&sm.bar_kempty[st], 1);
       mbar_init(&sm.bar_vfull[st], 1);
       mbar_init(&sm.bar_vempty[st], 1);
@@ -120,49 +147,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
+  const int32_t* lst = sm.list;
+  auto entry = [&](int j) { return j < kListSmem ? lst[j] : list[j]; };
+
   if (warp == 0) {
+    // lane 0: Q and dO once, then the K ring (+ key metadata of partial tiles); lane 1: the V ring
     if (lane == 0) {
+      const TileMeta* tmeta = p.tile_meta + static_cast<size_t>(s) * p.T;
       mbar_arrive_expect_tx(&sm.bar_qdo, 2 * kTileBytes);
       tma_tile<D>(&tm_q, &sm.bar_qdo, sm.q, head, q0);
       tma_tile<D>(&tm_do, &sm.bar_qdo, sm.dout, head, q0);
-    }
-    int issued_k = 0, issued_v = 0;
-    for (int j = 0; j < n; ++j) {
-      const int st = j % kStages;
-      const uint32_t ph = (j / kStages) & 1;
-      const int e = list[j];
-      const int J = e >> 2;
-      const int k0 = seq0 + J * kTile;
-      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_kempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
-        break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes);
-        tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, k0);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStages;
+        const int e = entry(j);
+        const int J = e >> 2;
+        if (j >= kStages && !mbar_wait(&sm.bar_kempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
+          break;
+        const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+        mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes + (partial ? sizeof(TileMeta) : 0));
+        tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, seq0 + J * kTile);
+        if (partial) bulk_load(&sm.kmeta[st], tmeta + J, sizeof(TileMeta), &sm.bar_kfull[st]);
+        issued = j + 1;
       }
-      issued_k = j + 1;
-      if ((e & 3) == OPR_TILE_PARTIAL) {
-        for (int x = lane; x < kTile; x += 32) {
-          const bool kv = J * kTile + x < seq_len;
-          sm.kconv[st][x] = kv ? p.conv_idx[k0 + x] : -1;
-          sm.kmeta[st][x] = kv ? p.tok_meta[k0 + x] : 0;
-        }
-        build_run_starts(sm.kconv[st], sm.kmeta[st], sm.kstarts[st], lane);
+      if (*abort_flag) {
+        mbar_wait(&sm.bar_qdo, 0, nullptr, kWaitLimitNs);
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_wait(&sm.bar_kfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
       }
-      mbar_arrive(&sm.bar_kfull[st]);
-      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_vempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
-        break;
-      if (lane == 0) {
+    } else if (lane == 1) {
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStages;
+        if (j >= kStages && !mbar_wait(&sm.bar_vempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
+          break;
         mbar_arrive_expect_tx(&sm.bar_vfull[st], kTileBytes);
-        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, k0);
+        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + (entry(j) >> 2) * kTile);
+        issued = j + 1;
       }
-      issued_v = j + 1;
-    }
-    if (*abort_flag && lane == 0) {
-      mbar_wait(&sm.bar_qdo, 0, nullptr, kWaitLimitNs);
-      for (int j = (issued_k > kStages ? issued_k - kStages : 0); j < issued_k; ++j)
-        mbar_wait(&sm.bar_kfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
-      for (int j = (issued_v > kStages ? issued_v - kStages : 0); j < issued_v; ++j)
-        mbar_wait(&sm.bar_vfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      if (*abort_flag)
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_wait(&sm.bar_vfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -233,13 +258,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qg = q0 + row;
     const int qconv = qv ? p.conv_idx[qg] : -2;
     const int qmeta = qv ? p.tok_meta[qg] : 0;
-    const float lse2 = qv ? p.lse_in[static_cast<size_t>(head) * p.total + qg] * kLog2e : 0.f;
-    const float dd = qv ? p.row_d[static_cast<size_t>(head) * p.total + qg] : 0.f;
+    const size_t rt = (static_cast<size_t>(head) * p.n_items + tile_id) * kTile + row;
+    const float lse2 = qv ? p.lse2_tiles[rt] : 0.f;
+    const float dd = qv ? p.d_tiles[rt] : 0.f;
     const float sl2 = p.scale_log2;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j % kStages;
-      const int e = list[j];
+      const int e = entry(j);
       const bool partial = (e & 3) == OPR_TILE_PARTIAL;
       const int kbase = seq0 + (e >> 2) * kTile;
       if (partial &&
@@ -251,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t mm[2] = {0xffffffffu, 0xffffffffu};
       if (partial) {
         uint32_t m[4];
-        query_row_mask(sm.kstarts[st], sm.kconv[st], sm.kmeta[st], kbase, qg, qconv, qmeta, m);
+        query_row_mask(sm.kmeta[st].starts, sm.kmeta[st].conv, sm.kmeta[st].meta, kbase, qg, qconv, qmeta, m);
         mm[0] = half ? m[2] : m[0];
         mm[1] = half ? m[3] : m[1];
       }
@@ -332,11 +358,12 @@ struct DkdvSmem {
   alignas(1024) uint8_t v[TileGeom<D>::kBytes];
   alignas(1024) uint8_t q[kStages][TileGeom<D>::kBytes];
   alignas(1024) uint8_t dout[kStages][TileGeom<D>::kBytes];
-  float qlse2[kStages][kTile];
-  float qd[kStages][kTile];
-  int32_t qconv[kStages][kTile];
-  int32_t qmeta[kStages][kTile];
-  uint32_t qstarts[kStages][4];
+  // column data of a query tile, bulk-copied with its Q tile: LSE * log2(e), D and
+  // (for partial tiles) the query metadata
+  alignas(16) float qlse2[kStages][kTile];
+  alignas(16) float qd[kStages][kTile];
+  alignas(16) TileMeta qmeta[kStages];
+  int32_t list[kListSmem];
   uint64_t bar_kv;
   uint64_t bar_qfull[kStages], bar_qempty[kStages], bar_dofull[kStages], bar_doempty[kStages];
   uint64_t bar_sfull, bar_dpfull, bar_pfull, bar_dsfull, bar_accdone, bar_final;
@@ -379,10 +406,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int seq_len = p.cu_seqlens[s + 1] - seq0;
   const int k0 = seq0 + J * kTile;
 
+  for (int x = threadIdx.x; x < cnt && x < kListSmem; x += blockDim.x) sm.list[x] = list[x];
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_kv, 1);
     for (int st = 0; st < kStages; ++st) {
-      mbar_init(&sm.bar_qfull[st], 1 + 32);  // TMA expect-tx arrival + 32 column-data lanes
+      mbar_init(&sm.bar_qfull[st], 1);
       mbar_init(&sm.bar_qempty[st], 1);
       mbar_init(&sm.bar_dofull[st], 1);
       mbar_init(&sm.bar_doempty[st], 1);
@@ -403,55 +431,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
+  const int32_t* lst = sm.list;
+  auto entry = [&](int j) { return j < kListSmem ? lst[j] : list[j]; };
+
   if (warp == 0) {
+    // lane 0: K and V once, then the Q ring with each query tile's column data;
+    // lane 1: the dO ring.  Iteration j covers q head kvh * group + j / cnt and
+    // query tile entry(j % cnt).
     if (lane == 0) {
+      const TileMeta* tmeta = p.tile_meta + static_cast<size_t>(s) * p.T;
       mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
       tma_tile<D>(&tm_k, &sm.bar_kv, sm.k, kvh, k0);
       tma_tile<D>(&tm_v, &sm.bar_kv, sm.v, kvh, k0);
-    }
-    int issued_q = 0, issued_do = 0;
-    for (int j = 0; j < n; ++j) {
-      const int st = j % kStages;
-      const uint32_t ph = (j / kStages) & 1;
-      const int g = j / cnt;
-      const int e = list[j % cnt];
-      const int Iq = e >> 2;
-      const int qt0 = seq0 + Iq * kTile;
-      const int h = kvh * group + g;
-      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_qempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
-        break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.bar_qfull[st], kTileBytes);
-        tma_tile<D>(&tm_q, &sm.bar_qfull[st], sm.q[st], h, qt0);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStages;
+        const int e = entry(j % cnt);
+        const int Iq = e >> 2;
+        const int h = kvh * group + j / cnt;
+        if (j >= kStages && !mbar_wait(&sm.bar_qempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
+          break;
+        const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+        mbar_arrive_expect_tx(&sm.bar_qfull[st],
+                              kTileBytes + 2 * kTile * sizeof(float) + (partial ? sizeof(TileMeta) : 0));
+        tma_tile<D>(&tm_q, &sm.bar_qfull[st], sm.q[st], h, seq0 + Iq * kTile);
+        const size_t rt = (static_cast<size_t>(h) * p.n_items + s * p.T + Iq) * kTile;
+        bulk_load(sm.qlse2[st], p.lse2_tiles + rt, kTile * sizeof(float), &sm.bar_qfull[st]);
+        bulk_load(sm.qd[st], p.d_tiles + rt, kTile * sizeof(float), &sm.bar_qfull[st]);
+        if (partial) bulk_load(&sm.qmeta[st], tmeta + Iq, sizeof(TileMeta), &sm.bar_qfull[st]);
+        issued = j + 1;
       }
-      issued_q = j + 1;
-      for (int x = lane; x < kTile; x += 32) {
-        const bool qv = Iq * kTile + x < seq_len;
-        const size_t idx = static_cast<size_t>(h) * p.total + qt0 + x;
-        sm.qlse2[st][x] = qv ? p.lse_in[idx] * kLog2e : INFINITY;
-        sm.qd[st][x] = qv ? p.row_d[idx] : 0.f;
-        if ((e & 3) == OPR_TILE_PARTIAL) {
-          sm.qconv[st][x] = qv ? p.conv_idx[qt0 + x] : -2;
-          sm.qmeta[st][x] = qv ? p.tok_meta[qt0 + x] : 0;
-        }
+      if (*abort_flag) {
+        mbar_wait(&sm.bar_kv, 0, nullptr, kWaitLimitNs);
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_wait(&sm.bar_qfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
       }
-      if ((e & 3) == OPR_TILE_PARTIAL) build_run_starts(sm.qconv[st], sm.qmeta[st], sm.qstarts[st], lane);
-      mbar_arrive(&sm.bar_qfull[st]);
-      if (j >= kStages &&
-          !__all_sync(0xffffffffu, mbar_wait(&sm.bar_doempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
-        break;
-      if (lane == 0) {
+    } else if (lane == 1) {
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStages;
+        const int h = kvh * group + j / cnt;
+        if (j >= kStages && !mbar_wait(&sm.bar_doempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
+          break;
         mbar_arrive_expect_tx(&sm.bar_dofull[st], kTileBytes);
-        tma_tile<D>(&tm_do, &sm.bar_dofull[st], sm.dout[st], h, qt0);
+        tma_tile<D>(&tm_do, &sm.bar_dofull[st], sm.dout[st], h, seq0 + (entry(j % cnt) >> 2) * kTile);
+        issued = j + 1;
       }
-      issued_do = j + 1;
-    }
-    if (*abort_flag && lane == 0) {
-      mbar_wait(&sm.bar_kv, 0, nullptr, kWaitLimitNs);
-      for (int j = (issued_q > kStages ? issued_q - kStages : 0); j < issued_q; ++j)
-        mbar_wait(&sm.bar_qfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
-      for (int j = (issued_do > kStages ? issued_do - kStages : 0); j < issued_do; ++j)
-        mbar_wait(&sm.bar_dofull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      if (*abort_flag)
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_wait(&sm.bar_dofull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -542,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j % kStages;
-      const int e = list[j % cnt];
+      const int e = entry(j % cnt);
       const bool partial = (e & 3) == OPR_TILE_PARTIAL;
       const int qt0 = seq0 + (e >> 2) * kTile;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs))) {
@@ -553,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t mm[2] = {0xffffffffu, 0xffffffffu};
       if (partial) {
         uint32_t m[4];
-        key_row_mask(sm.qstarts[st], sm.qconv[st], sm.qmeta[st], qt0, kg, kconv, kmeta, m);
+        key_row_mask(sm.qmeta[st].starts, sm.qmeta[st].conv, sm.qmeta[st].meta, qt0, kg, kconv, kmeta, m);
         mm[0] = half ? m[2] : m[0];
         mm[1] = half ? m[3] : m[1];
       }
@@ -680,16 +708,17 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
                          float* row_d, int stages, cudaStream_t stream) {
   static int conf_dq[64] = {0}, conf_kv[64] = {0};
   cudaError_t e = cudaSuccess;
-  // 1) row terms D
-  const int64_t warps = pq.total * pq.hq;
-  if ((stages & OPR_BWD_ROW_TERMS) && warps > 0) {
-    const int64_t blocks = (warps * 32 + 255) / 256;
+  // 1) row terms D and LSE * log2(e), per 128-token tile
+  if ((stages & OPR_BWD_ROW_TERMS) && pq.n_items > 0) {
+    const dim3 grid(pq.n_items, pq.hq);
     if (o_fp32)
-      row_d_kernel<D, float><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-          static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dout), pq.total, pq.hq, row_d);
+      row_terms_kernel<D, float><<<grid, kTile, 0, stream>>>(
+          static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dout), pq.lse_in, pq.cu_seqlens, pq.total,
+          pq.hq, pq.T, row_d, row_d + static_cast<size_t>(pq.hq) * pq.n_items * kTile);
     else
-      row_d_kernel<D, __nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), pq.total, pq.hq, row_d);
+      row_terms_kernel<D, __nv_bfloat16><<<grid, kTile, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), pq.lse_in, pq.cu_seqlens,
+          pq.total, pq.hq, pq.T, row_d, row_d + static_cast<size_t>(pq.hq) * pq.n_items * kTile);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // 2) dQ

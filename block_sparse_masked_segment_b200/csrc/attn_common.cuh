@@ -156,6 +156,7 @@ struct AttnParams {
   const int32_t* col_cnt;
   const int32_t* col_list;
   const int32_t* sched;
+  const TileMeta* tile_meta;
   int32_t T;
   int32_t n_items;
   int64_t total;
@@ -167,8 +168,9 @@ struct AttnParams {
   int32_t o_fp32;
   float* lse;
   // backward
-  const float* lse_in;
-  const float* row_d;  // D = rowsum(dO * O), [hq, total]
+  const float* lse_in;      // [hq, total]
+  const float* d_tiles;     // D = rowsum(dO * O), [hq][n_items][128]
+  const float* lse2_tiles;  // LSE * log2(e), [hq][n_items][128]
   float* dq;
   float* dk;
   float* dv;

@@ -5,9 +5,10 @@
 // block mask on H100, "实现细节"; this is a hand-written Blackwell kernel).
 //
 // One CTA per (query tile of 128 rows, q head), 6 warps:
-//   warp 0      loads Q once and the K/V tiles of the row's non-empty tiles
-//               with TMA (2-stage ring); its lanes also stage the key-side
-//               metadata of partial tiles;
+//   warp 0      lane 0 loads Q once, then the K tiles of the row's non-empty
+//               tiles (3-stage ring) with TMA, plus, for partial tiles, the
+//               tile's precomputed key metadata (one bulk copy); lane 1
+//               loads the V tiles (2-stage ring);
 //   warp 1      allocates TMEM and issues tcgen05.mma: S = Q K^T into one of
 //               two TMEM buffers, then O += P V with P read from TMEM;
 //   warps 2..9  two threads per query row, each owning 64 of the tile's 128
@@ -27,7 +28,8 @@
 namespace opr {
 namespace {
 
-constexpr int kStages = 2;
+constexpr int kStagesK = 3, kStagesV = 2;
+constexpr int kListSmem = 1024;  // entries of the row's tile list kept in shared memory
 constexpr uint32_t kOCol = 256;
 constexpr uint32_t kPCol = 384;  // P buffers (bf16, 64 columns each): never alias S, which both
                                  // threads of a row read for the row max
@@ -35,14 +37,13 @@ constexpr uint32_t kPCol = 384;  // P buffers (bf16, 64 columns each): never ali
 template <int D>
 struct FwdSmem {
   alignas(1024) uint8_t q[TileGeom<D>::kBytes];
-  alignas(1024) uint8_t k[kStages][TileGeom<D>::kBytes];
-  alignas(1024) uint8_t v[kStages][TileGeom<D>::kBytes];
-  int32_t kconv[kStages][kTile];
-  int32_t kmeta[kStages][kTile];
-  uint32_t kstarts[kStages][4];  // column-run starts of a partial tile
-  float lsum[2][kTile];           // row-sum halves, combined in the epilogue
+  alignas(1024) uint8_t k[kStagesK][TileGeom<D>::kBytes];
+  alignas(1024) uint8_t v[kStagesV][TileGeom<D>::kBytes];
+  alignas(16) TileMeta kmeta[kStagesK];  // key metadata of a partial tile, rides with its K tile
+  int32_t list[kListSmem];
+  float lsum[2][kTile];  // row-sum halves, combined in the epilogue
   uint64_t bar_q;
-  uint64_t bar_kfull[kStages], bar_kempty[kStages], bar_vfull[kStages], bar_vempty[kStages];
+  uint64_t bar_kfull[kStagesK], bar_kempty[kStagesK], bar_vfull[kStagesV], bar_vempty[kStagesV];
   uint64_t bar_sfull[2], bar_pfull[2], bar_odone, bar_final;
   uint32_t tmem_base;
   int abort_flag;
@@ -70,12 +71,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = seq0 + I * kTile;
   const int kvh = head / (p.hq / p.hkv);
 
+  for (int x = threadIdx.x; x < n && x < kListSmem; x += blockDim.x) sm.list[x] = list[x];
   if (threadIdx.x == 0) {
     mbar_init(&sm.bar_q, 1);
-    for (int st = 0; st < kStages; ++st) {
+    for (int st = 0; st < kStagesK; ++st) {
       mbar_init(&sm.bar_kfull[st], 1);
-      mbar_init(&sm.bar_kempty[st], 1);
-      mbar_init(&sm.bar_vfull[st], 1 + 32);  // TMA expect-tx arrival + 32 metadata lanes
+      // released when S = Q K^T has completed and every compute thread has read the metadata
+      mbar_init(&sm.bar_kempty[st], 1 + kComputeThreads);
+    }
+    for (int st = 0; st < kStagesV; ++st) {
+      mbar_init(&sm.bar_vfull[st], 1);
       mbar_init(&sm.bar_vempty[st], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -94,52 +99,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
+  const int32_t* lst = sm.list;
+  auto entry = [&](int j) { return j < kListSmem ? lst[j] : list[j]; };
+  const TileMeta* tmeta = p.tile_meta + static_cast<size_t>(s) * p.T;
+
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producers
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(&sm.bar_q, kTileBytes);
       tma_tile<D>(&tm_q, &sm.bar_q, sm.q, head, q0);
-    }
-    int issued_k = 0, issued_v = 0;
-    for (int j = 0; j < n; ++j) {
-      const int st = j % kStages;
-      const uint32_t ph = (j / kStages) & 1;
-      const int e = list[j];
-      const int J = e >> 2;
-      const int k0 = seq0 + J * kTile;
-      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_kempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
-        break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes);
-        tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, k0);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStagesK;
+        const int e = entry(j);
+        const int J = e >> 2;
+        if (j >= kStagesK && !mbar_wait(&sm.bar_kempty[st], ((j / kStagesK) + 1) & 1, abort_flag, kWaitLimitNs))
+          break;
+        const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+        mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes + (partial ? sizeof(TileMeta) : 0));
+        tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, seq0 + J * kTile);
+        if (partial) bulk_load(&sm.kmeta[st], tmeta + J, sizeof(TileMeta), &sm.bar_kfull[st]);
+        issued = j + 1;
       }
-      issued_k = j + 1;
-      if (j >= kStages && !__all_sync(0xffffffffu, mbar_wait(&sm.bar_vempty[st], ph ^ 1, abort_flag, kWaitLimitNs)))
-        break;
-      if (lane == 0) {
+      if (*abort_flag)  // let the copies already in flight land before the CTA exits
+        for (int j = (issued > kStagesK ? issued - kStagesK : 0); j < issued; ++j)
+          mbar_wait(&sm.bar_kfull[j % kStagesK], (j / kStagesK) & 1, nullptr, kWaitLimitNs);
+    } else if (lane == 1) {
+      tma_prefetch_desc(&tm_v);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % kStagesV;
+        if (j >= kStagesV && !mbar_wait(&sm.bar_vempty[st], ((j / kStagesV) + 1) & 1, abort_flag, kWaitLimitNs))
+          break;
         mbar_arrive_expect_tx(&sm.bar_vfull[st], kTileBytes);
-        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, k0);
+        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + (entry(j) >> 2) * kTile);
+        issued = j + 1;
       }
-      issued_v = j + 1;
-      if ((e & 3) == OPR_TILE_PARTIAL) {
-        for (int x = lane; x < kTile; x += 32) {
-          const bool kv = J * kTile + x < seq_len;
-          sm.kconv[st][x] = kv ? p.conv_idx[k0 + x] : -1;
-          sm.kmeta[st][x] = kv ? p.tok_meta[k0 + x] : 0;
-        }
-        build_run_starts(sm.kconv[st], sm.kmeta[st], sm.kstarts[st], lane);
-      }
-      mbar_arrive(&sm.bar_vfull[st]);
-    }
-    if (*abort_flag && lane == 0) {
-      // Let the copies already in flight land before the CTA exits.
-      for (int j = (issued_k > kStages ? issued_k - kStages : 0); j < issued_k; ++j)
-        mbar_wait(&sm.bar_kfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
-      for (int j = (issued_v > kStages ? issued_v - kStages : 0); j < issued_v; ++j)
-        mbar_wait(&sm.bar_vfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      if (*abort_flag)
+        for (int j = (issued > kStagesV ? issued - kStagesV : 0); j < issued; ++j)
+          mbar_wait(&sm.bar_vfull[j % kStagesV], (j / kStagesV) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -149,9 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sq = smem_u32(sm.q);
       bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, kWaitLimitNs);
       auto issue_pv = [&](int jp) -> bool {
-        const int bp = jp & 1, stp = jp % kStages;
+        const int bp = jp & 1, stp = jp % kStagesV;
         if (!mbar_wait(&sm.bar_pfull[bp], (jp >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
-        if (!mbar_wait(&sm.bar_vfull[stp], (jp / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
+        if (!mbar_wait(&sm.bar_vfull[stp], (jp / kStagesV) & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
         const uint32_t sv = smem_u32(sm.v[stp]);
 #pragma unroll
@@ -163,8 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       for (int j = 0; ok && j < n; ++j) {
-        const int st = j % kStages, b = j & 1;
-        if (!mbar_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) {
+        const int st = j % kStagesK, b = j & 1;
+        if (!mbar_wait(&sm.bar_kfull[st], (j / kStagesK) & 1, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
         }
@@ -196,12 +196,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      const int b = j & 1, st = j % kStages;
-      const int e = list[j];
+      const int b = j & 1, st = j % kStagesK;
+      const int e = entry(j);
       const bool partial = (e & 3) == OPR_TILE_PARTIAL;
       const int kbase = seq0 + (e >> 2) * kTile;
-      if (partial &&
-          !__all_sync(0xffffffffu, mbar_wait(&sm.bar_vfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs))) {
+      // the K stage carries the tile's key metadata; it is released after this read
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / kStagesK) & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
@@ -209,12 +209,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t mm[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
       if (partial) {
         uint32_t m[4];
-        query_row_mask(sm.kstarts[st], sm.kconv[st], sm.kmeta[st], kbase, qg, qconv, qmeta, m);
+        query_row_mask(sm.kmeta[st].starts, sm.kmeta[st].conv, sm.kmeta[st].meta, kbase, qg, qconv, qmeta, m);
         mm[0] = half ? m[2] : m[0];
         mm[1] = half ? m[3] : m[1];
         mm[2] = half ? m[0] : m[2];
         mm[3] = half ? m[1] : m[3];
       }
+      mbar_arrive(&sm.bar_kempty[st]);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[b], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
         break;

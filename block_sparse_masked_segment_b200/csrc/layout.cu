@@ -219,6 +219,30 @@ __global__ void tile_lists_kernel(const uint8_t* __restrict__ block_map, int32_t
   if (lane == 0) (rows ? row_cnt : col_cnt)[line] = n;
 }
 
+// One block of 128 threads per tile (s, J): the tile's TileMeta record.
+__global__ void __launch_bounds__(128) tile_meta_kernel(const int32_t* __restrict__ cu_seqlens,
+                                                        const int32_t* __restrict__ conv_idx,
+                                                        const int32_t* __restrict__ tok_meta, int32_t T,
+                                                        TileMeta* __restrict__ out) {
+  __shared__ int32_t sconv[kTile], smeta[kTile];
+  const int tile = blockIdx.x;
+  const int s = tile / T, J = tile % T;
+  const int c = threadIdx.x;
+  const int seq0 = cu_seqlens[s];
+  const int L = cu_seqlens[s + 1] - seq0;
+  const bool v = J * kTile + c < L;
+  const int cv = v ? conv_idx[seq0 + J * kTile + c] : -1;
+  const int mt = v ? tok_meta[seq0 + J * kTile + c] : 0;
+  sconv[c] = cv;
+  smeta[c] = mt;
+  out[tile].conv[c] = cv;
+  out[tile].meta[c] = mt;
+  __syncthreads();
+  const bool st = (c == 0) || sconv[c] != sconv[c - 1] || smeta[c] != smeta[c - 1];
+  const uint32_t b = __ballot_sync(0xffffffffu, st);
+  if ((c & 31) == 0) out[tile].starts[c >> 5] = b;
+}
+
 // Single block: order tiles by descending number of non-empty tiles in their
 // row (q_sched) or column (k_sched), ties by index, so the longest work
 // items start first.  Bitonic sort in shared memory; above kMaxSort items the
@@ -288,6 +312,8 @@ cudaError_t launch_layout(const int32_t* turn_lens, const int32_t* conv_turn_ptr
   if (w.n_tiles > 0) {
     dim3 grid(w.T, w.T, n_seqs);
     block_map_kernel<<<grid, 128, 0, stream>>>(cu_seqlens, conv_idx, tok_meta, w.T, block_map);
+    tile_meta_kernel<<<w.n_tiles, 128, 0, stream>>>(cu_seqlens, conv_idx, tok_meta, w.T,
+                                                    ws_ptr<TileMeta>(ws, w.tile_meta));
     tile_lists_kernel<<<dim3(w.n_tiles, 2), 32, 0, stream>>>(
         block_map, w.T, ws_ptr<int32_t>(ws, w.row_cnt), ws_ptr<int32_t>(ws, w.row_list),
         ws_ptr<int32_t>(ws, w.col_cnt), ws_ptr<int32_t>(ws, w.col_list));

@@ -38,6 +38,17 @@ __host__ __device__ __forceinline__ bool visible(int32_t qg, int32_t qconv, int3
 
 __host__ __device__ __forceinline__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Key/query metadata of one 128-token tile of a sequence, precomputed by the
+// layout so that the attention kernels fetch it with one bulk copy: run
+// starts (bit c set when token c starts a new (conversation, turn, type)
+// run), conversation index (-1 past the sequence end) and (turn << 2 | type).
+struct TileMeta {
+  uint32_t starts[4];
+  int32_t conv[kTile];
+  int32_t meta[kTile];
+};
+static_assert(sizeof(TileMeta) % 16 == 0, "bulk copies move multiples of 16 bytes");
+
 // Byte offsets of the arrays inside the layout workspace.
 struct LayoutWs {
   int32_t T;          // tiles per sequence edge
@@ -53,6 +64,7 @@ struct LayoutWs {
   size_t turn_off;    // int64 [n_turns]        token offset of each turn inside its conversation
   size_t turn_pos0;   // int32 [n_turns]        first position id of h_i
   size_t turn_conv;   // int32 [n_turns]        conversation of each turn
+  size_t tile_meta;   // TileMeta [n_tiles]     per 128-token tile: run starts, conversations, metas
   size_t bytes;       // total
 };
 
@@ -80,6 +92,7 @@ __host__ __device__ inline LayoutWs layout_ws_map(int32_t n_seqs, int32_t n_conv
   w.turn_off = take(sizeof(int64_t) * static_cast<size_t>(n_turns));
   w.turn_pos0 = take(sizeof(int32_t) * static_cast<size_t>(n_turns));
   w.turn_conv = take(sizeof(int32_t) * static_cast<size_t>(n_turns));
+  w.tile_meta = take(sizeof(TileMeta) * nt);
   w.bytes = off;
   return w;
 }

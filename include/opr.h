@@ -162,8 +162,13 @@ OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int
                         float scale, void* o, int32_t o_dtype, float* lse, int32_t* dev_status,
                         void* stream);
 
-/* Bytes of scratch that opr_attn_bwd needs (the row terms D = rowsum(dO * O)). */
-OPR_API size_t opr_attn_bwd_workspace_bytes(int64_t total_tokens, int32_t hq, int32_t head_dim);
+/*
+ * Bytes of device scratch that opr_attn_bwd needs: the row terms
+ * D = rowsum(dO * O) and LSE * log2(e), stored per 128-token tile
+ * (2 * 4 * hq * n_seqs * ceil(max_seqlen / 128) * 128 bytes, rounded up to 256).
+ */
+OPR_API size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq,
+                                            int32_t head_dim);
 
 /*
  * opr_attn_bwd - gradients of opr_attn_fwd w.r.t. the rotated q, k and v.

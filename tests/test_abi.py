@@ -46,7 +46,7 @@ def test_workspace_queries(lib):
     assert b > 4 * 30000 and b % 256 == 0
     assert opr.opr_layout_workspace_bytes(-1, 5, 20, 30000, 16384) == 0
     assert opr.opr_layout_workspace_bytes(1, 1, 1, 1 << 31, 100) == 0
-    assert opr.opr_attn_bwd_workspace_bytes(1000, 8, 128) >= 4 * 8000
+    assert opr.opr_attn_bwd_workspace_bytes(2, 1000, 8, 128) >= 2 * 4 * 8 * 2 * 8 * 128
 
 
 def test_host_argument_checks(lib):
