@@ -336,24 +336,345 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && sm.abort_flag) atomicOr(p.dev_status, OPR_DEV_WAIT_TIMEOUT);
 }
 
+
+// ----------------------------------------------------------------------------
+// Head-pair forward: one CTA per (query tile, two q heads of one GQA group).
+// Both heads read the same K/V tiles and the same mask, so the two heads are
+// two independent softmax streams on one K/V pipeline: while the tensor core
+// forms head B's S (or P V) the compute warps of head A work, and vice versa.
+//   warp 0      lane 0: both Q tiles, then the K ring (+ key metadata of
+//               partial tiles); lane 1: the V ring
+//   warp 1      TMEM owner, MMA issuer: S_A(0) S_B(0) | P_A V, S_A(j+1),
+//               P_B V, S_B(j+1) | ...
+//   warps 2..5  head A, warps 6..9 head B: one query row per thread, P (bf16)
+//               written over the first 64 columns of the thread's own row of S
+// TMEM columns: S_A 0, S_B 128, O_A 256, O_B 384.
+template <int D>
+struct FwdPairSmem {
+  alignas(1024) uint8_t q[2][TileGeom<D>::kBytes];
+  alignas(1024) uint8_t k[kStagesV][TileGeom<D>::kBytes];
+  alignas(1024) uint8_t v[kStagesV][TileGeom<D>::kBytes];
+  alignas(16) TileMeta kmeta[kStagesV];
+  int32_t list[kListSmem];
+  uint64_t bar_q;
+  uint64_t bar_kfull[kStagesV], bar_kempty[kStagesV], bar_vfull[kStagesV], bar_vempty[kStagesV];
+  uint64_t bar_sfull[2], bar_pfull[2], bar_odone[2], bar_final;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D, bool QK16>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  constexpr int NS = kStagesV;  // K and V rings share a depth here (two Q tiles resident)
+  constexpr uint32_t kTileBytes = TileGeom<D>::kBytes;
+  extern __shared__ uint8_t smem_raw[];
+  FwdPairSmem<D>& sm = *reinterpret_cast<FwdPairSmem<D>*>(align1024(smem_raw));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int npairs = p.hq / 2;
+  const int pair = blockIdx.x % npairs;
+  const int item = blockIdx.x / npairs;
+  if (item >= p.n_items) return;
+  const int tile_id = p.sched[item];
+  const int n = p.row_cnt[tile_id];
+  if (n == 0) return;
+  const int s = tile_id / p.T, I = tile_id % p.T;
+  const int32_t* list = p.row_list + static_cast<size_t>(tile_id) * p.T;
+  const int seq0 = p.cu_seqlens[s];
+  const int seq_len = p.cu_seqlens[s + 1] - seq0;
+  const int q0 = seq0 + I * kTile;
+  const int head0 = 2 * pair;
+  const int kvh = head0 / (p.hq / p.hkv);  // both heads of the pair share it (even group size)
+
+  for (int x = threadIdx.x; x < n && x < kListSmem; x += blockDim.x) sm.list[x] = list[x];
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_q, 1);
+    for (int st = 0; st < NS; ++st) {
+      mbar_init(&sm.bar_kfull[st], 1);
+      // released when both S = Q K^T have completed and every compute thread has read the metadata
+      mbar_init(&sm.bar_kempty[st], 1 + kComputeThreads);
+      mbar_init(&sm.bar_vfull[st], 1);
+      mbar_init(&sm.bar_vempty[st], 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&sm.bar_sfull[h], 1);
+      mbar_init(&sm.bar_pfull[h], 128);
+      mbar_init(&sm.bar_odone[h], 1);
+    }
+    mbar_init(&sm.bar_final, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+  const int32_t* lst = sm.list;
+  auto entry = [&](int j) { return j < kListSmem ? lst[j] : list[j]; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const TileMeta* tmeta = p.tile_meta + static_cast<size_t>(s) * p.T;
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      mbar_arrive_expect_tx(&sm.bar_q, 2 * kTileBytes);
+      tma_tile<D>(&tm_q, &sm.bar_q, sm.q[0], head0, q0);
+      tma_tile<D>(&tm_q, &sm.bar_q, sm.q[1], head0 + 1, q0);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % NS;
+        const int e = entry(j);
+        const int J = e >> 2;
+        if (j >= NS && !mbar_wait(&sm.bar_kempty[st], ((j / NS) + 1) & 1, abort_flag, kWaitLimitNs)) break;
+        const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+        mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes + (partial ? sizeof(TileMeta) : 0));
+        tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, seq0 + J * kTile);
+        if (partial) bulk_load(&sm.kmeta[st], tmeta + J, sizeof(TileMeta), &sm.bar_kfull[st]);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait(&sm.bar_q, 0, nullptr, kWaitLimitNs);
+        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+          mbar_wait(&sm.bar_kfull[j % NS], (j / NS) & 1, nullptr, kWaitLimitNs);
+      }
+    } else if (lane == 1) {
+      tma_prefetch_desc(&tm_v);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % NS;
+        if (j >= NS && !mbar_wait(&sm.bar_vempty[st], ((j / NS) + 1) & 1, abort_flag, kWaitLimitNs)) break;
+        mbar_arrive_expect_tx(&sm.bar_vfull[st], kTileBytes);
+        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + (entry(j) >> 2) * kTile);
+        issued = j + 1;
+      }
+      if (*abort_flag)
+        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+          mbar_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);        // O += P V, P and V bf16
+      const uint32_t sq[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+      auto issue_s = [&](int h, int j) {
+        const uint32_t sk = smem_u32(sm.k[j % NS]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + h * 128, desc_kmajor(sq[h], kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.bar_sfull[h]);
+      };
+      auto issue_pv = [&](int h, int j) -> bool {
+        if (!mbar_wait(&sm.bar_pfull[h], j & 1, abort_flag, kWaitLimitNs)) return false;
+        tc_fence_after();
+        const uint32_t sv = smem_u32(sm.v[j % NS]);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sm.bar_odone[h]);
+        return true;
+      };
+      bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, kWaitLimitNs) &&
+                mbar_wait(&sm.bar_kfull[0], 0, abort_flag, kWaitLimitNs);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        mma_commit(&sm.bar_kempty[0]);
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const bool more = j + 1 < n;
+        if (!mbar_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        if (!(ok = issue_pv(0, j))) break;
+        if (more) {
+          if (!mbar_wait(&sm.bar_kfull[(j + 1) % NS], ((j + 1) / NS) & 1, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!(ok = issue_pv(1, j))) break;
+        mma_commit(&sm.bar_vempty[j % NS]);
+        if (more) {
+          issue_s(1, j + 1);
+          mma_commit(&sm.bar_kempty[(j + 1) % NS]);
+        }
+      }
+      mma_commit(&sm.bar_final);
+      mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
+    }
+  } else {
+    const int hx = (warp - 2) >> 2;  // 0: head A (warps 2..5), 1: head B (warps 6..9)
+    const int head = head0 + hx;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t scol = hx * 128, ocol = 256 + hx * 128;
+    const bool qv = I * kTile + row < seq_len;
+    const int qg = q0 + row;
+    const int qconv = qv ? p.conv_idx[qg] : -2;
+    const int qmeta = qv ? p.tok_meta[qg] : 0;
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int st = j % NS;
+      const int e = entry(j);
+      const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+      const int kbase = seq0 + (e >> 2) * kTile;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / NS) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      uint32_t mm[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      if (partial)
+        query_row_mask(sm.kmeta[st].starts, sm.kmeta[st].conv, sm.kmeta[st].meta, kbase, qg, qconv, qmeta, mm);
+      mbar_arrive(&sm.bar_kempty[st]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[hx], j & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float sv[kTile];
+      {
+        uint32_t sr[kTile];
+        tmem_ld128(tl + scol, sr);
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) sv[c] = __uint_as_float(sr[c]);
+      }
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (!mask_bit(mm, c)) sv[c] = -INFINITY;
+      }
+      float mx8[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) mx8[x] = sv[x];
+#pragma unroll
+      for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_new = fmaxf(m_run, mx * sl2);
+      const bool need = m_new > m_run + 8.f;  // also true on the first finite max
+      const float m_use = need ? m_new : m_run;
+      const float mb = (m_use == -INFINITY) ? 0.f : m_use;
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const float p0 = fast_exp2(fmaf(sv[c * 32 + 2 * x], sl2, -mb));
+          const float p1 = fast_exp2(fmaf(sv[c * 32 + 2 * x + 1], sl2, -mb));
+          rs8[x & 7] += p0 + p1;
+          pk[x] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tl + scol + c * 16, pk);  // own row, columns already read
+      }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      tmem_wait_st();
+      if (j >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (j - 1) & 1, abort_flag, kWaitLimitNs))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      const float factor = need ? fast_exp2(m_run - m_new) : 1.f;
+      if (__any_sync(0xffffffffu, need && j >= 1)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tl + ocol + c * 32, r);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * factor);
+          tmem_st32(tl + ocol + c * 32, r);
+        }
+        tmem_wait_st();
+      }
+      l_run = l_run * factor + rs;
+      if (need) m_run = m_new;
+      tc_fence_before();
+      mbar_arrive(&sm.bar_pfull[hx]);
+    }
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (n - 1) & 1, abort_flag, kWaitLimitNs))) {
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+      const size_t orow = (static_cast<size_t>(qg) * p.hq + head) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tl + ocol + c * 32, r);
+        if (qv) {
+          if (p.o_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c * 32);
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              dst[x] = make_float4(__uint_as_float(r[4 * x]) * inv, __uint_as_float(r[4 * x + 1]) * inv,
+                                   __uint_as_float(r[4 * x + 2]) * inv, __uint_as_float(r[4 * x + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow + c * 32);
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              dst[x] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * x]) * inv, __uint_as_float(r[8 * x + 1]) * inv),
+                                  pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv, __uint_as_float(r[8 * x + 3]) * inv),
+                                  pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv, __uint_as_float(r[8 * x + 5]) * inv),
+                                  pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv, __uint_as_float(r[8 * x + 7]) * inv));
+          }
+        }
+      }
+      if (qv) p.lse[static_cast<size_t>(head) * p.total + qg] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && sm.abort_flag) atomicOr(p.dev_status, OPR_DEV_WAIT_TIMEOUT);
+}
+
 }  // namespace
 
 template <int D, bool QK16>
 cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const AttnParams& p, cudaStream_t stream) {
-  const size_t smem = smem_request(sizeof(FwdSmem<D>) + 1024);
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
+  const bool pairs = (p.hq / p.hkv) % 2 == 0;
+  const size_t smem_single = smem_request(sizeof(FwdSmem<D>) + 1024);
+  const size_t smem_pair = smem_request(sizeof(FwdPairSmem<D>) + 1024);
   if (dev < 64 && !configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, QK16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+                                         static_cast<int>(smem_single));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_fwd_pair_kernel<D, QK16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_pair));
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  const int64_t blocks = static_cast<int64_t>(p.n_items) * p.hq;
-  if (blocks == 0) return cudaSuccess;
-  attn_fwd_kernel<D, QK16><<<static_cast<unsigned>(blocks), kThreads, smem, stream>>>(tq, tk, tv, p);
+  if (pairs) {
+    // two q heads of one GQA group per CTA
+    const int64_t blocks = static_cast<int64_t>(p.n_items) * (p.hq / 2);
+    if (blocks == 0) return cudaSuccess;
+    attn_fwd_pair_kernel<D, QK16><<<static_cast<unsigned>(blocks), kThreads, smem_pair, stream>>>(tq, tk, tv, p);
+  } else {
+    const int64_t blocks = static_cast<int64_t>(p.n_items) * p.hq;
+    if (blocks == 0) return cudaSuccess;
+    attn_fwd_kernel<D, QK16><<<static_cast<unsigned>(blocks), kThreads, smem_single, stream>>>(tq, tk, tv, p);
+  }
   return cudaGetLastError();
 }
 
