@@ -190,64 +190,63 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&sm.bar_vfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T (q/k type)
-      constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP = dO V^T (bf16)
-      constexpr uint32_t idesc_q = idesc_f32acc(128, D, QK16, 0, 1);    // dQ += dS K (K tile MN-major)
-      const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
-      // S(j) = Q K(j)^T
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sk = smem_u32(sm.k[st]);
+    // the whole warp runs this loop; elect.sync picks the issuing lane
+    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T (q/k type)
+    constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP = dO V^T (bf16)
+    constexpr uint32_t idesc_q = idesc_f32acc(128, D, QK16, 0, 1);    // dQ += dS K (K tile MN-major)
+    const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
+    // S(j) = Q K(j)^T
+    auto issue_s = [&](int j) -> bool {
+      const int st = j % kStages;
+      if (!warp_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sk = smem_u32(sm.k[st]);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kDqColS, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.bar_sfull);
-        return true;
-      };
-      // dP(j) = dO V(j)^T; releases V(j)
-      auto issue_dp = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(&sm.bar_vfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sv = smem_u32(sm.v[st]);
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tmem + kDqColS, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+      mma_commit(&sm.bar_sfull);
+      return true;
+    };
+    // dP(j) = dO V(j)^T; releases V(j)
+    auto issue_dp = [&](int j) -> bool {
+      const int st = j % kStages;
+      if (!warp_wait(&sm.bar_vfull[st], (j / kStages) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sv = smem_u32(sm.v[st]);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kDqColDP, desc_kmajor(sdo, kk), desc_kmajor(sv, kk), idesc_p, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.bar_dpfull);
-        mma_commit(&sm.bar_vempty[st]);
-        return true;
-      };
-      // dQ += dS(j) K(j); releases K(j) and its metadata
-      auto issue_dq = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sk = smem_u32(sm.k[st]);
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tmem + kDqColDP, desc_kmajor(sdo, kk), desc_kmajor(sv, kk), idesc_p, kk > 0 ? 1u : 0u);
+      mma_commit(&sm.bar_dpfull);
+      mma_commit(&sm.bar_vempty[st]);
+      return true;
+    };
+    // dQ += dS(j) K(j); releases K(j) and its metadata
+    auto issue_dq = [&](int j) -> bool {
+      const int st = j % kStages;
+      if (!warp_wait(&sm.bar_dsfull, j & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sk = smem_u32(sm.k[st]);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kDqColAcc, tmem + kDqColDS + kk * 8, desc_mnmajor(sk, kk), idesc_q,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&sm.bar_kempty[st]);
-        return true;
-      };
-      // Issue order S(0) dP(0) | S(1) dQ(0) dP(1) | S(2) dQ(1) dP(2) | ...: S(j+1) starts as
-      // soon as the compute warps have read S(j), while they still form P(j) and dS(j).
-      bool ok = mbar_wait(&sm.bar_qdo, 0, abort_flag, kWaitLimitNs) && issue_s(0) && issue_dp(0);
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n) {
-          ok = mbar_wait(&sm.bar_sfree, j & 1, abort_flag, kWaitLimitNs) && issue_s(j + 1);
-          if (!ok) break;
-        }
-        ok = issue_dq(j);
-        if (ok && j + 1 < n) ok = issue_dp(j + 1);
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_ts(tmem + kDqColAcc, tmem + kDqColDS + kk * 8, desc_mnmajor(sk, kk), idesc_q,
+               (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&sm.bar_kempty[st]);
+      return true;
+    };
+    // Issue order S(0) dP(0) | S(1) dQ(0) dP(1) | S(2) dQ(1) dP(2) | ...: S(j+1) starts as
+    // soon as the compute warps have read S(j), while they still form P(j) and dS(j).
+    bool ok = warp_wait(&sm.bar_qdo, 0, abort_flag) && issue_s(0) && issue_dp(0);
+    for (int j = 0; ok && j < n; ++j) {
+      if (j + 1 < n) {
+        ok = warp_wait(&sm.bar_sfree, j & 1, abort_flag) && issue_s(j + 1);
+        if (!ok) break;
       }
-      if (ok) mma_commit(&sm.bar_dqdone);
-      mma_commit(&sm.bar_final);
-      mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
+      ok = issue_dq(j);
+      if (ok && j + 1 < n) ok = issue_dp(j + 1);
     }
+    if (ok) mma_commit(&sm.bar_dqdone);
+    mma_commit(&sm.bar_final);
+    __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs));
   } else {
     // two threads per query row: `half` selects key columns [64 half, 64 half + 64)
     const int quad = warp & 3;
@@ -277,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t mm[2] = {0xffffffffu, 0xffffffffu};
       if (partial) {
         uint32_t m[4];
-        query_row_mask(sm.kmeta[st].starts, sm.kmeta[st].conv, sm.kmeta[st].meta, kbase, qg, qconv, qmeta, m);
+        query_row_mask(sm.kmeta[st], kbase, qg, qconv, qmeta, m);
         mm[0] = half ? m[2] : m[0];
         mm[1] = half ? m[3] : m[1];
       }
@@ -482,79 +481,78 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&sm.bar_dofull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S^T = K Q^T (q/k type)
-      constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP^T = V dO^T (bf16)
-      constexpr uint32_t idesc_v = idesc_bf16_f32(128, D, 0, 1);        // dV += P^T dO (bf16)
-      constexpr uint32_t idesc_k = idesc_f32acc(128, D, QK16, 0, 1);    // dK += dS^T Q (q/k type)
-      const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
-      // S^T(j) = K Q(j)^T into the S region
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sq = smem_u32(sm.q[st]);
+    // the whole warp runs this loop; elect.sync picks the issuing lane
+    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S^T = K Q^T (q/k type)
+    constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP^T = V dO^T (bf16)
+    constexpr uint32_t idesc_v = idesc_bf16_f32(128, D, 0, 1);        // dV += P^T dO (bf16)
+    constexpr uint32_t idesc_k = idesc_f32acc(128, D, QK16, 0, 1);    // dK += dS^T Q (q/k type)
+    const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
+    // S^T(j) = K Q(j)^T into the S region
+    auto issue_s = [&](int j) -> bool {
+      const int st = j % kStages;
+      if (!warp_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sq = smem_u32(sm.q[st]);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kKvColS, desc_kmajor(sk, kk), desc_kmajor(sq, kk), idesc_s, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.bar_sfull);
-        return true;
-      };
-      // dP^T(j) = V dO(j)^T into the dP region
-      auto issue_dp = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(&sm.bar_dofull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sdo = smem_u32(sm.dout[st]);
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tmem + kKvColS, desc_kmajor(sk, kk), desc_kmajor(sq, kk), idesc_s, kk > 0 ? 1u : 0u);
+      mma_commit(&sm.bar_sfull);
+      return true;
+    };
+    // dP^T(j) = V dO(j)^T into the dP region
+    auto issue_dp = [&](int j) -> bool {
+      const int st = j % kStages;
+      if (!warp_wait(&sm.bar_dofull[st], (j / kStages) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sdo = smem_u32(sm.dout[st]);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kKvColDP, desc_kmajor(sv, kk), desc_kmajor(sdo, kk), idesc_p, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.bar_dpfull);
-        return true;
-      };
-      // dV += P^T(j) dO(j), P^T as bf16 hi + lo parts; releases dO(j)
-      auto issue_dv = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(&sm.bar_pfull, j & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sdo = smem_u32(sm.dout[st]);
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tmem + kKvColDP, desc_kmajor(sv, kk), desc_kmajor(sdo, kk), idesc_p, kk > 0 ? 1u : 0u);
+      mma_commit(&sm.bar_dpfull);
+      return true;
+    };
+    // dV += P^T(j) dO(j), P^T as bf16 hi + lo parts; releases dO(j)
+    auto issue_dv = [&](int j) -> bool {
+      const int st = j % kStages;
+      if (!warp_wait(&sm.bar_pfull, j & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sdo = smem_u32(sm.dout[st]);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kKvColDV, tmem + kKvColS + split_col(kk), desc_mnmajor(sdo, kk), idesc_v,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_ts(tmem + kKvColDV, tmem + kKvColS + split_col(kk), desc_mnmajor(sdo, kk), idesc_v,
+               (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kKvColDV, tmem + kKvColS + 32 + split_col(kk), desc_mnmajor(sdo, kk), idesc_v, 1u);
-        mma_commit(&sm.bar_doempty[st]);
-        return true;
-      };
-      // dK += dS^T(j) Q(j); releases Q(j) and its column data
-      auto issue_dk = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(&sm.bar_dsfull, j & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sq = smem_u32(sm.q[st]);
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_ts(tmem + kKvColDV, tmem + kKvColS + 32 + split_col(kk), desc_mnmajor(sdo, kk), idesc_v, 1u);
+      mma_commit(&sm.bar_doempty[st]);
+      return true;
+    };
+    // dK += dS^T(j) Q(j); releases Q(j) and its column data
+    auto issue_dk = [&](int j) -> bool {
+      const int st = j % kStages;
+      if (!warp_wait(&sm.bar_dsfull, j & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sq = smem_u32(sm.q[st]);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kColDK, tmem + kKvColDP + split_col(kk), desc_mnmajor(sq, kk), idesc_k,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&sm.bar_qempty[st]);
-        return true;
-      };
-      // Issue order S(0) dP(0) | dV(0) S(1) dK(0) dP(1) | dV(1) S(2) dK(1) dP(2) | ...
-      // so that the next S^T is formed while the compute warps turn dP^T into dS^T,
-      // and the next dP^T while they turn S^T into P^T.
-      bool ok = mbar_wait(&sm.bar_kv, 0, abort_flag, kWaitLimitNs) && issue_s(0) && issue_dp(0);
-      for (int j = 0; ok && j < n; ++j) {
-        ok = issue_dv(j);
-        if (ok && j + 1 < n) ok = issue_s(j + 1);
-        if (ok) ok = issue_dk(j);
-        if (ok && j + 1 < n) ok = issue_dp(j + 1);
-      }
-      if (ok) mma_commit(&sm.bar_accdone);
-      mma_commit(&sm.bar_final);
-      mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_ts(tmem + kColDK, tmem + kKvColDP + split_col(kk), desc_mnmajor(sq, kk), idesc_k,
+               (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&sm.bar_qempty[st]);
+      return true;
+    };
+    // Issue order S(0) dP(0) | dV(0) S(1) dK(0) dP(1) | dV(1) S(2) dK(1) dP(2) | ...
+    // so that the next S^T is formed while the compute warps turn dP^T into dS^T,
+    // and the next dP^T while they turn S^T into P^T.
+    bool ok = warp_wait(&sm.bar_kv, 0, abort_flag) && issue_s(0) && issue_dp(0);
+    for (int j = 0; ok && j < n; ++j) {
+      ok = issue_dv(j);
+      if (ok && j + 1 < n) ok = issue_s(j + 1);
+      if (ok) ok = issue_dk(j);
+      if (ok && j + 1 < n) ok = issue_dp(j + 1);
     }
+    if (ok) mma_commit(&sm.bar_accdone);
+    mma_commit(&sm.bar_final);
+    __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs));
   } else {
     // two threads per key row: `half` selects query columns [64 half, 64 half + 64)
     const int quad = warp & 3;
@@ -581,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t mm[2] = {0xffffffffu, 0xffffffffu};
       if (partial) {
         uint32_t m[4];
-        key_row_mask(sm.qmeta[st].starts, sm.qmeta[st].conv, sm.qmeta[st].meta, qt0, kg, kconv, kmeta, m);
+        key_row_mask(sm.qmeta[st], qt0, kg, kconv, kmeta, m);
         mm[0] = half ? m[2] : m[0];
         mm[1] = half ? m[3] : m[1];
       }

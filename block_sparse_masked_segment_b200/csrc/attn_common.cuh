@@ -20,6 +20,11 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: any pipeline wait long
 constexpr int kThreads = 320;
 constexpr int kComputeThreads = 256;
 
+// Bounded mbarrier wait taken by a whole warp; the result is warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kWaitLimitNs));
+}
+
 // A 128-row tile of head_dim D bf16 values is stored as D/64 "chunks", each
 // 128 rows x 128 bytes with the 128-byte swizzle TMA writes (box {64, 1, 128}).
 constexpr int kChunkBytes = kTile * 128;  // 16 KiB
@@ -67,45 +72,14 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ---------------------------------------------------------------- partial tiles
-// The 128 columns of a partial tile split into runs of equal (conversation,
-// turn, type).  Warp-wide: lanes have written conv[]/meta[] of the tile; the
-// run starts are returned as a 128-bit mask (bit c of starts[c / 32]).
-__device__ __forceinline__ void build_run_starts(const int32_t* conv, const int32_t* meta, uint32_t* starts,
-                                                 int lane) {
-  __syncwarp();
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const int c = w * 32 + lane;
-    const bool st = (c == 0) || conv[c] != conv[c - 1] || meta[c] != meta[c - 1];
-    const uint32_t b = __ballot_sync(0xffffffffu, st);
-    if (lane == 0) starts[w] = b;
-  }
-}
-
-// First run start at or after column x (128 if none).
-__device__ __forceinline__ int next_run_start(const uint32_t (&st)[4], int x) {
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    if (x < 32 * (w + 1)) {
-      const int sh = x - 32 * w;
-      const uint32_t m = sh <= 0 ? st[w] : (st[w] & (0xffffffffu << sh));
-      if (m) return 32 * w + __ffs(m) - 1;
-    }
-  }
-  return 128;
-}
-
-// Set bits [a, b) of a 128-bit mask.
-__device__ __forceinline__ void set_bit_range(uint32_t (&m)[4], int a, int b) {
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const int lo = max(a, 32 * w), hi = min(b, 32 * w + 32);
-    if (lo < hi) {
-      const int n = hi - lo;
-      const uint32_t bits = n == 32 ? 0xffffffffu : ((1u << n) - 1u);
-      m[w] |= bits << (lo - 32 * w);
-    }
-  }
+// Set bits [a, b) (0 <= a <= b <= 128) of a 128-bit mask held as two 64-bit words.
+__device__ __forceinline__ void set_range128(uint64_t& lo, uint64_t& hi, int a, int b) {
+  const int la = min(a, 64), lb = min(b, 64);
+  const int ha = max(a, 64) - 64, hb = max(b, 64) - 64;
+  const uint64_t lmask = (lb == 64 ? ~0ull : ((1ull << lb) - 1ull)) & ~((la == 64) ? ~0ull : ((1ull << la) - 1ull));
+  const uint64_t hmask = (hb == 64 ? ~0ull : ((1ull << hb) - 1ull)) & ~((ha == 64) ? ~0ull : ((1ull << ha) - 1ull));
+  if (la < lb) lo |= lmask;
+  if (ha < hb) hi |= hmask;
 }
 
 // Does a query of meta qmeta see a key of meta kmeta (same conversation, key not after the query)?
@@ -115,34 +89,38 @@ __device__ __forceinline__ bool type_rule(int32_t qmeta, int32_t kmeta) {
 }
 
 // Mask of the keys kbase + c (c < 128) visible from query qg: one rule test per
-// column run, with the causal limit k <= qg.
-__device__ __forceinline__ void query_row_mask(const uint32_t* starts_smem, const int32_t* kconv, const int32_t* kmeta,
-                                               int kbase, int qg, int qconv, int qmeta, uint32_t (&m)[4]) {
-  m[0] = m[1] = m[2] = m[3] = 0u;
-  const int lim = min(qg - kbase + 1, 128);
-  if (lim <= 0) return;
-  const uint32_t st[4] = {starts_smem[0], starts_smem[1], starts_smem[2], starts_smem[3]};
-  int a = 0;
-  while (a < lim) {
-    const int b = next_run_start(st, a + 1);
-    if (kconv[a] == qconv && type_rule(qmeta, kmeta[a])) set_bit_range(m, a, min(b, lim));
-    a = b;
+// run of the key tile, with the causal limit k <= qg.  m[w] holds columns 32w..32w+31.
+__device__ __forceinline__ void query_row_mask(const TileMeta& t, int kbase, int qg, int qconv, int qmeta,
+                                               uint32_t (&m)[4]) {
+  uint64_t lo = 0ull, hi = 0ull;
+  const int lim = min(max(qg - kbase + 1, 0), 128);
+  const int nr = t.nruns;
+#pragma unroll 4
+  for (int r = 0; r < nr; ++r) {
+    const int a = t.bound[r], b = min(t.bound[r + 1], lim);
+    if (a < b && t.conv[r] == qconv && type_rule(qmeta, t.meta[r])) set_range128(lo, hi, a, b);
   }
+  m[0] = static_cast<uint32_t>(lo);
+  m[1] = static_cast<uint32_t>(lo >> 32);
+  m[2] = static_cast<uint32_t>(hi);
+  m[3] = static_cast<uint32_t>(hi >> 32);
 }
 
-// Mask of the queries qbase + c (c < 128) that see key kg (roles of query_row_mask swapped).
-__device__ __forceinline__ void key_row_mask(const uint32_t* starts_smem, const int32_t* qconv, const int32_t* qmeta,
-                                             int qbase, int kg, int kconv, int kmeta, uint32_t (&m)[4]) {
-  m[0] = m[1] = m[2] = m[3] = 0u;
-  const int first = max(kg - qbase, 0);
-  if (first >= 128) return;
-  const uint32_t st[4] = {starts_smem[0], starts_smem[1], starts_smem[2], starts_smem[3]};
-  int a = 0;
-  while (a < 128) {
-    const int b = next_run_start(st, a + 1);
-    if (b > first && qconv[a] == kconv && type_rule(qmeta[a], kmeta)) set_bit_range(m, max(a, first), b);
-    a = b;
+// Mask of the queries qbase + c (c < 128) that see key kg (roles swapped: runs of the query tile).
+__device__ __forceinline__ void key_row_mask(const TileMeta& t, int qbase, int kg, int kconv, int kmeta,
+                                             uint32_t (&m)[4]) {
+  uint64_t lo = 0ull, hi = 0ull;
+  const int first = min(max(kg - qbase, 0), 128);
+  const int nr = t.nruns;
+#pragma unroll 4
+  for (int r = 0; r < nr; ++r) {
+    const int a = max(t.bound[r], first), b = t.bound[r + 1];
+    if (a < b && t.conv[r] == kconv && type_rule(t.meta[r], kmeta)) set_range128(lo, hi, a, b);
   }
+  m[0] = static_cast<uint32_t>(lo);
+  m[1] = static_cast<uint32_t>(lo >> 32);
+  m[2] = static_cast<uint32_t>(hi);
+  m[3] = static_cast<uint32_t>(hi >> 32);
 }
 
 __device__ __forceinline__ bool mask_bit(const uint32_t (&m)[4], int c) { return (m[c >> 5] >> (c & 31)) & 1u; }

@@ -142,46 +142,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&sm.bar_vfull[j % kStagesV], (j / kStagesV) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
+    // the whole warp runs this loop; elect.sync picks the issuing lane
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);      // O += P V, P and V bf16
-      const uint32_t sq = smem_u32(sm.q);
-      bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, kWaitLimitNs);
-      auto issue_pv = [&](int jp) -> bool {
-        const int bp = jp & 1, stp = jp % kStagesV;
-        if (!mbar_wait(&sm.bar_pfull[bp], (jp >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
-        if (!mbar_wait(&sm.bar_vfull[stp], (jp / kStagesV) & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sv = smem_u32(sm.v[stp]);
+    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);      // O += P V, P and V bf16
+    const uint32_t sq = smem_u32(sm.q);
+    bool ok = warp_wait(&sm.bar_q, 0, abort_flag);
+    auto issue_pv = [&](int jp) -> bool {
+      const int bp = jp & 1, stp = jp % kStagesV;
+      if (!warp_wait(&sm.bar_pfull[bp], (jp >> 1) & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_vfull[stp], (jp / kStagesV) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sv = smem_u32(sm.v[stp]);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + kOCol, tmem + kPCol + bp * 64 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
-                 (jp > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&sm.bar_vempty[stp]);
-        mma_commit(&sm.bar_odone);
-        return true;
-      };
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j % kStagesK, b = j & 1;
-        if (!mbar_wait(&sm.bar_kfull[st], (j / kStagesK) & 1, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t sk = smem_u32(sm.k[st]);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + b * 128, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.bar_sfull[b]);
-        mma_commit(&sm.bar_kempty[st]);
-        if (j >= 1 && !issue_pv(j - 1)) ok = false;
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_ts(tmem + kOCol, tmem + kPCol + bp * 64 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
+               (jp > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&sm.bar_vempty[stp]);
+      mma_commit(&sm.bar_odone);
+      return true;
+    };
+    for (int j = 0; ok && j < n; ++j) {
+      const int st = j % kStagesK, b = j & 1;
+      if (!warp_wait(&sm.bar_kfull[st], (j / kStagesK) & 1, abort_flag)) {
+        ok = false;
+        break;
       }
-      if (ok) issue_pv(n - 1);
-      // All MMAs issued by this thread must be complete before TMEM is freed.
-      mma_commit(&sm.bar_final);
-      mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
+      tc_fence_after();
+      const uint32_t sk = smem_u32(sm.k[st]);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tmem + b * 128, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+      mma_commit(&sm.bar_sfull[b]);
+      mma_commit(&sm.bar_kempty[st]);
+      if (j >= 1 && !issue_pv(j - 1)) ok = false;
     }
+    if (ok) issue_pv(n - 1);
+    // All MMAs issued by this thread must be complete before TMEM is freed.
+    mma_commit(&sm.bar_final);
+    __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs));
   } else {
     // ------------------------------------------------------------ softmax
     const int quad = warp & 3;        // TMEM lane quadrant this warp may access
@@ -209,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t mm[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
       if (partial) {
         uint32_t m[4];
-        query_row_mask(sm.kmeta[st].starts, sm.kmeta[st].conv, sm.kmeta[st].meta, kbase, qg, qconv, qmeta, m);
+        query_row_mask(sm.kmeta[st], kbase, qg, qconv, qmeta, m);
         mm[0] = half ? m[2] : m[0];
         mm[1] = half ? m[3] : m[1];
         mm[2] = half ? m[0] : m[2];
@@ -456,61 +455,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);        // O += P V, P and V bf16
-      const uint32_t sq[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
-      auto issue_s = [&](int h, int j) {
-        const uint32_t sk = smem_u32(sm.k[j % NS]);
+    // the whole warp runs this loop; elect.sync picks the issuing lane
+    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);        // O += P V, P and V bf16
+    const uint32_t sq[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+    auto issue_s = [&](int h, int j) {
+      const uint32_t sk = smem_u32(sm.k[j % NS]);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + h * 128, desc_kmajor(sq[h], kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.bar_sfull[h]);
-      };
-      auto issue_pv = [&](int h, int j) -> bool {
-        if (!mbar_wait(&sm.bar_pfull[h], j & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t sv = smem_u32(sm.v[j % NS]);
+      for (int kk = 0; kk < D / 16; ++kk)
+        mma_ss(tmem + h * 128, desc_kmajor(sq[h], kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+      mma_commit(&sm.bar_sfull[h]);
+    };
+    auto issue_pv = [&](int h, int j) -> bool {
+      if (!warp_wait(&sm.bar_pfull[h], j & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sv = smem_u32(sm.v[j % NS]);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&sm.bar_odone[h]);
-        return true;
-      };
-      bool ok = mbar_wait(&sm.bar_q, 0, abort_flag, kWaitLimitNs) &&
-                mbar_wait(&sm.bar_kfull[0], 0, abort_flag, kWaitLimitNs);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        mma_commit(&sm.bar_kempty[0]);
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
+               (j > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(&sm.bar_odone[h]);
+      return true;
+    };
+    bool ok = warp_wait(&sm.bar_q, 0, abort_flag) &&
+              warp_wait(&sm.bar_kfull[0], 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0, 0);
+      issue_s(1, 0);
+      mma_commit(&sm.bar_kempty[0]);
+    }
+    for (int j = 0; ok && j < n; ++j) {
+      const bool more = j + 1 < n;
+      if (!warp_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, abort_flag)) {
+        ok = false;
+        break;
       }
-      for (int j = 0; ok && j < n; ++j) {
-        const bool more = j + 1 < n;
-        if (!mbar_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, abort_flag, kWaitLimitNs)) {
+      if (!(ok = issue_pv(0, j))) break;
+      if (more) {
+        if (!warp_wait(&sm.bar_kfull[(j + 1) % NS], ((j + 1) / NS) & 1, abort_flag)) {
           ok = false;
           break;
         }
-        if (!(ok = issue_pv(0, j))) break;
-        if (more) {
-          if (!mbar_wait(&sm.bar_kfull[(j + 1) % NS], ((j + 1) / NS) & 1, abort_flag, kWaitLimitNs)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_s(0, j + 1);
-        }
-        if (!(ok = issue_pv(1, j))) break;
-        mma_commit(&sm.bar_vempty[j % NS]);
-        if (more) {
-          issue_s(1, j + 1);
-          mma_commit(&sm.bar_kempty[(j + 1) % NS]);
-        }
+        tc_fence_after();
+        issue_s(0, j + 1);
       }
-      mma_commit(&sm.bar_final);
-      mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs);
+      if (!(ok = issue_pv(1, j))) break;
+      mma_commit(&sm.bar_vempty[j % NS]);
+      if (more) {
+        issue_s(1, j + 1);
+        mma_commit(&sm.bar_kempty[(j + 1) % NS]);
+      }
     }
+    mma_commit(&sm.bar_final);
+    __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs));
   } else {
     const int hx = (warp - 2) >> 2;  // 0: head A (warps 2..5), 1: head B (warps 6..9)
     const int head = head0 + hx;
@@ -536,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t mm[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
       if (partial)
-        query_row_mask(sm.kmeta[st].starts, sm.kmeta[st].conv, sm.kmeta[st].meta, kbase, qg, qconv, qmeta, mm);
+        query_row_mask(sm.kmeta[st], kbase, qg, qconv, qmeta, mm);
       mbar_arrive(&sm.bar_kempty[st]);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[hx], j & 1, abort_flag, kWaitLimitNs))) {
         ok = false;

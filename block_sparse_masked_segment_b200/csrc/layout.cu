@@ -219,28 +219,40 @@ __global__ void tile_lists_kernel(const uint8_t* __restrict__ block_map, int32_t
   if (lane == 0) (rows ? row_cnt : col_cnt)[line] = n;
 }
 
-// One block of 128 threads per tile (s, J): the tile's TileMeta record.
+// One block of 128 threads per tile (s, J): the tile's TileMeta record (runs of
+// equal conversation and meta, in token order).
 __global__ void __launch_bounds__(128) tile_meta_kernel(const int32_t* __restrict__ cu_seqlens,
                                                         const int32_t* __restrict__ conv_idx,
                                                         const int32_t* __restrict__ tok_meta, int32_t T,
                                                         TileMeta* __restrict__ out) {
   __shared__ int32_t sconv[kTile], smeta[kTile];
+  __shared__ int32_t wcount[4];
   const int tile = blockIdx.x;
   const int s = tile / T, J = tile % T;
-  const int c = threadIdx.x;
+  const int c = threadIdx.x, lane = c & 31, w = c >> 5;
   const int seq0 = cu_seqlens[s];
   const int L = cu_seqlens[s + 1] - seq0;
   const bool v = J * kTile + c < L;
-  const int cv = v ? conv_idx[seq0 + J * kTile + c] : -1;
-  const int mt = v ? tok_meta[seq0 + J * kTile + c] : 0;
-  sconv[c] = cv;
-  smeta[c] = mt;
-  out[tile].conv[c] = cv;
-  out[tile].meta[c] = mt;
+  sconv[c] = v ? conv_idx[seq0 + J * kTile + c] : -1;
+  smeta[c] = v ? tok_meta[seq0 + J * kTile + c] : 0;
   __syncthreads();
   const bool st = (c == 0) || sconv[c] != sconv[c - 1] || smeta[c] != smeta[c - 1];
   const uint32_t b = __ballot_sync(0xffffffffu, st);
-  if ((c & 31) == 0) out[tile].starts[c >> 5] = b;
+  if (lane == 0) wcount[w] = __popc(b);
+  __syncthreads();
+  int base = 0;
+  for (int x = 0; x < w; ++x) base += wcount[x];
+  if (st) {
+    const int r = base + __popc(b & ((1u << lane) - 1u));
+    out[tile].bound[r] = c;
+    out[tile].conv[r] = sconv[c];
+    out[tile].meta[r] = smeta[c];
+  }
+  if (c == 0) {
+    const int nr = wcount[0] + wcount[1] + wcount[2] + wcount[3];
+    out[tile].nruns = nr;
+    out[tile].bound[nr] = kTile;
+  }
 }
 
 // Single block: order tiles by descending number of non-empty tiles in their

@@ -39,11 +39,14 @@ __host__ __device__ __forceinline__ bool visible(int32_t qg, int32_t qconv, int3
 __host__ __device__ __forceinline__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Key/query metadata of one 128-token tile of a sequence, precomputed by the
-// layout so that the attention kernels fetch it with one bulk copy: run
-// starts (bit c set when token c starts a new (conversation, turn, type)
-// run), conversation index (-1 past the sequence end) and (turn << 2 | type).
+// layout so that the attention kernels fetch it with one bulk copy: the tile's
+// tokens split into runs of equal (conversation, turn, type); run r covers
+// tokens bound[r] .. bound[r + 1] - 1 of the tile and has conversation conv[r]
+// (-1 past the sequence end) and meta[r] = (turn << 2) | type.
 struct TileMeta {
-  uint32_t starts[4];
+  int32_t nruns;
+  int32_t pad_[3];
+  int32_t bound[kTile + 4];  // bound[nruns] = 128
   int32_t conv[kTile];
   int32_t meta[kTile];
 };
