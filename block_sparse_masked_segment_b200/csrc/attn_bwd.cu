@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sk = smem_u32(sm.k[st]);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + kDqColS, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kDqColS, (desc_kmajor(sq, 0) + kmajor_step(kk)), (desc_kmajor(sk, 0) + kmajor_step(kk)), idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_sfull);
       return true;
     };
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sv = smem_u32(sm.v[st]);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + kDqColDP, desc_kmajor(sdo, kk), desc_kmajor(sv, kk), idesc_p, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kDqColDP, (desc_kmajor(sdo, 0) + kmajor_step(kk)), (desc_kmajor(sv, 0) + kmajor_step(kk)), idesc_p, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_dpfull);
       mma_commit(&sm.bar_vempty[st]);
       return true;
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sk = smem_u32(sm.k[st]);
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kDqColAcc, tmem + kDqColDS + kk * 8, desc_mnmajor(sk, kk), idesc_q,
+        mma_ts(tmem + kDqColAcc, tmem + kDqColDS + kk * 8, (desc_mnmajor(sk, 0) + mnmajor_step(kk)), idesc_q,
                (j > 0 || kk > 0) ? 1u : 0u);
       mma_commit(&sm.bar_kempty[st]);
       return true;
@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sq = smem_u32(sm.q[st]);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + kKvColS, desc_kmajor(sk, kk), desc_kmajor(sq, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kKvColS, (desc_kmajor(sk, 0) + kmajor_step(kk)), (desc_kmajor(sq, 0) + kmajor_step(kk)), idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_sfull);
       return true;
     };
@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sdo = smem_u32(sm.dout[st]);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + kKvColDP, desc_kmajor(sv, kk), desc_kmajor(sdo, kk), idesc_p, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kKvColDP, (desc_kmajor(sv, 0) + kmajor_step(kk)), (desc_kmajor(sdo, 0) + kmajor_step(kk)), idesc_p, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_dpfull);
       return true;
     };
@@ -519,11 +519,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sdo = smem_u32(sm.dout[st]);
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kKvColDV, tmem + kKvColS + split_col(kk), desc_mnmajor(sdo, kk), idesc_v,
+        mma_ts(tmem + kKvColDV, tmem + kKvColS + split_col(kk), (desc_mnmajor(sdo, 0) + mnmajor_step(kk)), idesc_v,
                (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kKvColDV, tmem + kKvColS + 32 + split_col(kk), desc_mnmajor(sdo, kk), idesc_v, 1u);
+        mma_ts(tmem + kKvColDV, tmem + kKvColS + 32 + split_col(kk), (desc_mnmajor(sdo, 0) + mnmajor_step(kk)), idesc_v, 1u);
       mma_commit(&sm.bar_doempty[st]);
       return true;
     };
@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sq = smem_u32(sm.q[st]);
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kColDK, tmem + kKvColDP + split_col(kk), desc_mnmajor(sq, kk), idesc_k,
+        mma_ts(tmem + kColDK, tmem + kKvColDP + split_col(kk), (desc_mnmajor(sq, 0) + mnmajor_step(kk)), idesc_k,
                (j > 0 || kk > 0) ? 1u : 0u);
       mma_commit(&sm.bar_qempty[st]);
       return true;

@@ -51,6 +51,16 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_saddr, int kk) {
   return smem_desc_sw128(tile_saddr + kk * 2048, kChunkBytes, 1024);
 }
 
+// The same descriptors as a base (K step 0) plus a per-step increment of the
+// start-address field: the MMA issue loops build the base once per tile and
+// add a compile-time constant per step, so each MMA costs one 64-bit add.
+// (Shared-memory addresses stay below 2^18 bytes, so the 14-bit start field
+// never carries into the next field.)
+__device__ __forceinline__ constexpr uint64_t kmajor_step(int kk) {
+  return static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+}
+__device__ __forceinline__ constexpr uint64_t mnmajor_step(int kk) { return static_cast<uint64_t>((kk * 2048) >> 4); }
+
 // Loads a [128 tokens][D] tile of one head with TMA (D/64 boxes).
 template <int D>
 __device__ __forceinline__ void tma_tile(const CUtensorMap* map, uint64_t* bar, void* dst, int head, int tok0) {

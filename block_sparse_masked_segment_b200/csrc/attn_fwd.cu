@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sv = smem_u32(sm.v[stp]);
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kOCol, tmem + kPCol + bp * 64 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
+        mma_ts(tmem + kOCol, tmem + kPCol + bp * 64 + kk * 8, (desc_mnmajor(sv, 0) + mnmajor_step(kk)), idesc_o,
                (jp > 0 || kk > 0) ? 1u : 0u);
       mma_commit(&sm.bar_vempty[stp]);
       mma_commit(&sm.bar_odone);
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sk = smem_u32(sm.k[st]);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + b * 128, desc_kmajor(sq, kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + b * 128, (desc_kmajor(sq, 0) + kmajor_step(kk)), (desc_kmajor(sk, 0) + kmajor_step(kk)), idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_sfull[b]);
       mma_commit(&sm.bar_kempty[st]);
       if (j >= 1 && !issue_pv(j - 1)) ok = false;
@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sk = smem_u32(sm.k[j % NS]);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + h * 128, desc_kmajor(sq[h], kk), desc_kmajor(sk, kk), idesc_s, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + h * 128, (desc_kmajor(sq[h], 0) + kmajor_step(kk)), (desc_kmajor(sk, 0) + kmajor_step(kk)), idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_sfull[h]);
     };
     auto issue_pv = [&](int h, int j) -> bool {
@@ -472,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sv = smem_u32(sm.v[j % NS]);
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, desc_mnmajor(sv, kk), idesc_o,
+        mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, (desc_mnmajor(sv, 0) + mnmajor_step(kk)), idesc_o,
                (j > 0 || kk > 0) ? 1u : 0u);
       mma_commit(&sm.bar_odone[h]);
       return true;
