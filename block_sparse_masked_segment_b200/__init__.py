@@ -17,6 +17,7 @@ from ._abi import (  # noqa: F401
     opr_attn_fwd,
     opr_attn_bwd,
     opr_attn_bwd_stages,
+    opr_attn_bwd_noalloc,
     BWD_ROW_TERMS,
     BWD_DQ,
     BWD_DKDV,

@@ -33,11 +33,15 @@ EXPORTED_SYMBOLS = (
     "opr_attn_bwd_workspace_bytes",
     "opr_attn_bwd",
     "opr_attn_bwd_stages",
+    "opr_attn_bwd_noalloc",
 )
 
 BWD_ROW_TERMS, BWD_DQ, BWD_DKDV = 1, 2, 4
 
-_STATUS_NAMES = {1: "OPR_INVALID_ARG", 2: "OPR_UNSUPPORTED", 3: "OPR_CUDA_ERROR", 4: "OPR_WORKSPACE_TOO_SMALL"}
+_STATUS_NAMES = {1: "OPR_INVALID_ARG", 2: "OPR_UNSUPPORTED", 3: "OPR_CUDA_ERROR", 4: "OPR_WORKSPACE_TOO_SMALL",
+                 5: "OPR_SCRATCH_TOO_LARGE"}
+OPR_SCRATCH_TOO_LARGE = 5
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class OprError(RuntimeError):
@@ -79,6 +83,9 @@ def load_library() -> ctypes.CDLL:
     lib.opr_attn_bwd_stages.restype = I32
     lib.opr_attn_bwd_stages.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32,
                                         F, P, P, P, P, SZ, P, I32, P]
+    lib.opr_attn_bwd_noalloc.restype = I32
+    lib.opr_attn_bwd_noalloc.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32,
+                                         F, P, P, P, P, P]
     _lib = lib
     return lib
 
@@ -286,3 +293,29 @@ def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, w
 def opr_attn_bwd_stages(q, k, v, o, do, lse, lay: Layout, stages: int, workspace, out, scale=None):
     """Run only the backward kernels selected by ``stages`` (see opr_attn_bwd)."""
     return opr_attn_bwd(q, k, v, o, do, lse, lay, scale, workspace=workspace, out=out, stages=stages)
+
+
+def opr_attn_bwd_noalloc(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, out=None):
+    """opr_attn_bwd with the scratch in the library's fixed device array (no workspace argument).
+
+    For callers that cannot allocate device memory at the call; see the C
+    header for the size limit and the sharing rules of the array.  ``out`` =
+    (dq, dk, dv) lets the caller provide the output buffers too.
+    """
+    total, hq, hkv, d = _attn_shapes(q, k, v, lay)
+    _need_cuda(o, do, lse)
+    if do.dtype != torch.bfloat16 or lse.dtype != torch.float32:
+        raise OprError("dout must be bf16 and lse fp32")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = (torch.empty((total, hq, d), dtype=torch.float32, device=q.device),
+               torch.empty((total, hkv, d), dtype=torch.float32, device=q.device),
+               torch.empty((total, hkv, d), dtype=torch.float32, device=q.device))
+    dq, dk, dv = out
+    st = load_library().opr_attn_bwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16,
+        _ptr(do), _ptr(lse), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace), lay.n_seqs, lay.n_convs,
+        lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(lay.dev_status), _stream(q.device))
+    _check(st, "opr_attn_bwd_noalloc")
+    return dq, dk, dv

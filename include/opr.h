@@ -50,6 +50,7 @@ typedef int32_t opr_status;
 #define OPR_UNSUPPORTED 2          /* dtype or device (needs compute capability 10.0) not supported */
 #define OPR_CUDA_ERROR 3           /* a CUDA runtime/driver call or a kernel launch failed */
 #define OPR_WORKSPACE_TOO_SMALL 4  /* workspace_bytes below what the *_workspace_bytes query returns */
+#define OPR_SCRATCH_TOO_LARGE 5    /* opr_attn_bwd_noalloc: scratch needed exceeds OPR_NOALLOC_SCRATCH_BYTES */
 
 /* Bits OR-ed into *dev_status by the kernels. */
 #define OPR_DEV_BAD_INPUT 1        /* negative length or non-monotone turn/conversation pointers */
@@ -213,6 +214,39 @@ OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void*
                                        int32_t hq, int32_t hkv, int32_t head_dim, float scale, float* dq,
                                        float* dk, float* dv, void* workspace, size_t workspace_bytes,
                                        int32_t* dev_status, int32_t stages, void* stream);
+
+/*
+ * opr_attn_bwd_noalloc - opr_attn_bwd for callers that cannot allocate device
+ * memory at the call (no counterpart in the paper; a convenience of this
+ * library).  Examples: a host framework that owns every device allocation and
+ * offers extensions no allocator hook, or a latency-critical path that must
+ * not call cudaMalloc, which can block and synchronize the device.
+ *
+ * Same inputs, outputs and error behaviour as opr_attn_bwd, without the
+ * workspace arguments: the scratch (the row terms) lives in one fixed
+ * library-owned device array of OPR_NOALLOC_SCRATCH_BYTES, allocated by the
+ * CUDA loader on every GPU that loads the library and held until the process
+ * exits.  The call allocates and frees nothing.
+ *   - Returns OPR_SCRATCH_TOO_LARGE, before touching the device, when
+ *     opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) exceeds
+ *     OPR_NOALLOC_SCRATCH_BYTES.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents in
+ *     it; nothing needs clearing because each call rewrites every entry it
+ *     reads.  Calls whose work overlaps on the GPU (other streams, other host
+ *     threads) race on the array: order them on one stream.
+ */
+#define OPR_NOALLOC_SCRATCH_BYTES (32u << 20)
+OPR_API opr_status opr_attn_bwd_noalloc(const void* q, const void* k, const void* v, int32_t qk_dtype,
+                                        const void* o, int32_t o_dtype, const void* dout,
+                                        const float* lse, const int32_t* cu_seqlens,
+                                        const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs,
+                                        int32_t n_convs, int32_t n_turns, int64_t total_tokens,
+                                        int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
+                                        float scale, float* dq, float* dk, float* dv,
+                                        int32_t* dev_status, void* stream);
 
 /* Library version string, e.g. "opr 0.1.0 sm_100a". */
 OPR_API const char* opr_version(void);

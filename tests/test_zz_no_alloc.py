@@ -1,0 +1,48 @@
+"""opr_attn_bwd_noalloc: the backward for callers that cannot allocate device
+memory at the call (a host framework that owns all device memory, or a path
+that must not call cudaMalloc).  Its scratch is a fixed library-owned device
+array instead of a caller workspace; its results must match opr_attn_bwd.
+
+This file is collected last on purpose, so that a run stopping at the first
+failure has already run every other test.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_masked_segment_b200 as opr
+from block_sparse_masked_segment_b200 import _abi
+import synth
+from parity_helpers import assert_close, inputs, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_backward_matches_workspace_backward_twice():
+    w = synth.random_small_workload(31, n_seqs=2, max_convs=3, max_turns=4, hq=4, hkv=2, d=128, base=1e6)
+    q, k, v, do = inputs(w, 31)
+    att = opr.OnePassAttention(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, base=w.base)
+    qd, kd, vd, dod = to_dev(q), to_dev(k), to_dev(v), to_dev(do)
+    o, lse, qr, kr = att.forward(qd, kd, vd)
+    lay = att.layout
+    ref = [t.cpu().numpy() for t in opr.opr_attn_bwd(qr, kr, vd, o, dod, lse, lay)]
+    for call in range(2):  # the second call reuses the array the first call left behind
+        got = [t.cpu().numpy() for t in opr.opr_attn_bwd_noalloc(qr, kr, vd, o, dod, lse, lay)]
+        torch.cuda.synchronize()
+        assert opr.read_status(lay.dev_status) == []
+        for name, g, r in zip(("dQ", "dK", "dV"), got, ref):
+            assert_close(f"{name} (call {call})", g, r)
+
+
+def test_noalloc_rejects_scratch_beyond_the_limit():
+    """Sizes whose scratch exceeds the fixed array are refused before any device work."""
+    lib = opr.load_library()
+    n_seqs, max_seqlen, hq, d = 1, 100000, 64, 128
+    assert opr.opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, d) > _abi.NOALLOC_SCRATCH_BYTES
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check fails first
+    st = lib.opr_attn_bwd_noalloc(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, n_seqs, 1, 1,
+                                  max_seqlen, max_seqlen, hq, 8, d, 0.1, fake, fake, fake, fake, None)
+    assert st == _abi.OPR_SCRATCH_TOO_LARGE
