@@ -40,7 +40,7 @@ METRIC = "1-pass masked attn fwd+bwd useful TFLOP/s; conv tokens/s vs N-pass"
 UNIT = "TFLOP/s"
 DEFAULT_CONFIG = 2
 L2_FLUSH_BYTES = 512 << 20
-KERNELS_PER_STEP = 7 + 2 + 1 + 3 + 2  # layout, rope x2, fwd, bwd (3), inverse rope x2
+KERNELS_PER_STEP = 8 + 2 + 1 + 3 + 2  # layout (8), rope x2, fwd, bwd (3), inverse rope x2
 
 
 def peaks():
@@ -181,6 +181,44 @@ class Runner:
 
     def d2h_bytes(self):
         return sum(t.numel() * t.element_size() for t in self.h_grads)
+
+
+# ------------------------------------------------------------------ ranks
+class Ranks:
+    """Rank plumbing of a weak-scaling run (one process per GPU).
+
+    Every rank times its own batch between barriers; the job's time is the
+    maximum over ranks and its work the sum over ranks.  The two reductions
+    run on timing scalars only: the data path has no collective.
+    """
+
+    def __init__(self, world: int, device):
+        import torch
+        import torch.distributed as dist
+
+        self.world, self.device, self._torch, self._dist = world, device, torch, dist
+
+    def barrier(self):
+        if self.world > 1:
+            self._dist.barrier()
+
+    def _reduce(self, x: float, op) -> float:
+        if self.world == 1:
+            return x
+        t = self._torch.tensor([x], dtype=self._torch.float64, device=self.device)
+        self._dist.all_reduce(t, op=op)
+        return float(t.item())
+
+    def max(self, x: float) -> float:
+        return self._reduce(x, self._dist.ReduceOp.MAX)
+
+    def sum(self, x: float) -> float:
+        return self._reduce(x, self._dist.ReduceOp.SUM)
+
+
+def rank_workload(config: int, rank: int, turns: int | None = None) -> synth.Workload:
+    """This rank's batch: the configuration's shape and length mix, drawn from a rank-specific seed."""
+    return synth.make_workload(config, seed=1000 + config + 7919 * rank, n_turns=turns)
 
 
 def time_runner(r: Runner, steps: int, warmup: int, flush, barrier):
@@ -335,30 +373,14 @@ def main():
         from datetime import timedelta
 
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+    ranks = Ranks(world, device)
+    barrier, max_over_ranks, sum_over_ranks = ranks.barrier, ranks.max, ranks.sum
 
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     flush = lambda: flush_buf.zero_()  # noqa: E731
 
     # every rank runs its own batch of the same shape (weak scaling, no data-path collective)
-    w = synth.make_workload(args.config, seed=1000 + args.config + 7919 * rank, n_turns=args.turns)
+    w = rank_workload(args.config, rank, args.turns)
     r = Runner(w, seed=11 + rank, device=device)
     pairs = r.pairs
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
@@ -405,6 +427,8 @@ def main():
                 "algorithmic_flops": fl[dom]}
 
     if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:

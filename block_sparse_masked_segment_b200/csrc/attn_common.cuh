@@ -104,7 +104,7 @@ __device__ __forceinline__ void query_row_mask(const TileMeta& t, int kbase, int
                                                uint32_t (&m)[4]) {
   uint64_t lo = 0ull, hi = 0ull;
   const int lim = min(max(qg - kbase + 1, 0), 128);
-  const int nr = t.nruns;
+  const int nr = min(t.nruns, kTile);  // a record always has 1..128 runs
 #pragma unroll 4
   for (int r = 0; r < nr; ++r) {
     const int a = t.bound[r], b = min(t.bound[r + 1], lim);
@@ -121,7 +121,7 @@ __device__ __forceinline__ void key_row_mask(const TileMeta& t, int qbase, int k
                                              uint32_t (&m)[4]) {
   uint64_t lo = 0ull, hi = 0ull;
   const int first = min(max(kg - qbase, 0), 128);
-  const int nr = t.nruns;
+  const int nr = min(t.nruns, kTile);  // a record always has 1..128 runs
 #pragma unroll 4
   for (int r = 0; r < nr; ++r) {
     const int a = max(t.bound[r], first), b = t.bound[r + 1];
