@@ -20,12 +20,13 @@ _LIB_PATH = os.path.join(_HERE, "lib", "libopr.so")
 
 OPR_OK, OPR_INVALID_ARG, OPR_UNSUPPORTED, OPR_CUDA_ERROR, OPR_WORKSPACE_TOO_SMALL = 0, 1, 2, 3, 4
 DEV_BITS = {1: "bad input", 2: "total mismatch", 4: "sequence longer than max_seqlen", 8: "pipeline wait timeout",
-            16: "fp16 overflow in rope"}
+            16: "fp16 range exceeded (rope output or backward fp16 copy)"}
 DTYPE_BF16, DTYPE_FP32, DTYPE_FP16 = 0, 1, 2
 TILE = 128
 
 EXPORTED_SYMBOLS = (
     "opr_version",
+    "opr_last_error",
     "opr_layout_workspace_bytes",
     "opr_build_layout",
     "opr_rope",
@@ -67,6 +68,8 @@ def load_library() -> ctypes.CDLL:
                              ctypes.c_double, ctypes.c_float)
     lib.opr_version.restype = ctypes.c_char_p
     lib.opr_version.argtypes = []
+    lib.opr_last_error.restype = ctypes.c_char_p
+    lib.opr_last_error.argtypes = []
     lib.opr_layout_workspace_bytes.restype = SZ
     lib.opr_layout_workspace_bytes.argtypes = [I32, I32, I32, I64, I32]
     lib.opr_build_layout.restype = I32
@@ -92,7 +95,8 @@ def load_library() -> ctypes.CDLL:
 
 def _check(status: int, what: str) -> None:
     if status != OPR_OK:
-        raise OprError(f"{what} returned {_STATUS_NAMES.get(status, status)}")
+        detail = f" ({load_library().opr_last_error().decode()})" if status == 3 else ""
+        raise OprError(f"{what} returned {_STATUS_NAMES.get(status, status)}{detail}")
 
 
 def _ptr(t: torch.Tensor | None) -> int | None:

@@ -12,10 +12,8 @@
 namespace opr {
 cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const AttnParams& p, cudaStream_t stream);
-cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
-                            const CUtensorMap& tv, const CUtensorMap& tdo, const void* o, int o_fp32, const void* dout,
-                            const AttnParams& pq, const AttnParams& pkv, float* row_d, int stages,
-                            cudaStream_t stream);
+cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const BwdMaps& m, const BwdBuffers& b, const AttnParams& pq,
+                            const AttnParams& pkv, int stages, cudaStream_t stream);
 
 namespace {
 
@@ -33,6 +31,21 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   }
   return fn;
+}
+
+// Text of the last OPR_CUDA_ERROR returned on this host thread (opr_last_error).
+thread_local const char* g_last_error = "no error";
+
+opr_status cuda_fail(cudaError_t e) {
+  g_last_error = cudaGetErrorString(e);
+  return OPR_CUDA_ERROR;
+}
+
+opr_status status_of(cudaError_t e) { return e == cudaSuccess ? OPR_OK : cuda_fail(e); }
+
+opr_status map_fail() {
+  g_last_error = "TMA tensor map encoding failed (cuTensorMapEncodeTiled)";
+  return OPR_CUDA_ERROR;
 }
 
 // [tokens, heads, head_dim] 16-bit tensor (bf16 or fp16) as a 3-D TMA map with
@@ -56,8 +69,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 opr_status device_check() {
   int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return OPR_CUDA_ERROR;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return OPR_CUDA_ERROR;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
   return major == 10 ? OPR_OK : OPR_UNSUPPORTED;
 }
 
@@ -114,6 +128,8 @@ extern "C" {
 
 const char* opr_version(void) { return "opr 0.1.0 sm_100a"; }
 
+const char* opr_last_error(void) { return g_last_error; }
+
 size_t opr_layout_workspace_bytes(int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
                                   int32_t max_seqlen) {
   if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return 0;
@@ -135,7 +151,7 @@ opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* conv_turn_p
   cudaError_t e = launch_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, n_seqs, n_convs, n_turns, total_tokens,
                                 max_seqlen, cu_seqlens, token_type, turn_idx, conv_idx, pos_id, block_map, workspace,
                                 dev_status, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
+  return status_of(e);
 }
 
 opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, const int32_t* pos_id,
@@ -149,7 +165,7 @@ opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, co
   if (x == y && x_dtype != y_dtype) return OPR_INVALID_ARG;
   cudaError_t e = launch_rope(x, x_dtype, y, y_dtype, pos_id, total_tokens, n_heads, head_dim, base, inverse,
                               dev_status, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
+  return status_of(e);
 }
 
 opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_dtype, const int32_t* cu_seqlens,
@@ -169,22 +185,39 @@ opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, total_tokens, hq, head_dim, f16) || !make_map(&tk, k, total_tokens, hkv, head_dim, f16) ||
       !make_map(&tv, v, total_tokens, hkv, head_dim))
-    return OPR_CUDA_ERROR;
+    return map_fail();
   AttnParams p = base_params(cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs, n_turns, total_tokens, max_seqlen, hq,
                              hkv, scale, dev_status);
   p.o = o;
   p.o_fp32 = o_dtype == OPR_DTYPE_FP32;
   p.lse = lse;
   cudaError_t e = launch_attn_fwd(head_dim, f16, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
+  return status_of(e);
 }
 
-size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
-  (void)head_dim;
-  if (n_seqs < 0 || max_seqlen < 0 || hq < 0) return 0;
+namespace {
+// Backward scratch: the row terms, then fp16 copies of dO and V.  Token counts
+// are bounded by n_seqs * ceil(max_seqlen / 128) * 128 and the kv heads by hq.
+struct BwdWs {
+  size_t row_terms, dout16, v16, bytes;
+};
+
+BwdWs bwd_ws_map(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
   const size_t T = (static_cast<size_t>(max_seqlen) + kTile - 1) / kTile;
-  // D and LSE * log2(e) per (head, tile, token of the tile)
-  return align_up(2 * sizeof(float) * static_cast<size_t>(hq) * static_cast<size_t>(n_seqs) * T * kTile, 256);
+  const size_t tokens = static_cast<size_t>(n_seqs) * T * kTile;
+  BwdWs w;
+  w.row_terms = 0;
+  w.dout16 = align_up(2 * sizeof(float) * static_cast<size_t>(hq) * tokens, 256);
+  const size_t copy = align_up(sizeof(uint16_t) * tokens * static_cast<size_t>(hq) * static_cast<size_t>(head_dim), 256);
+  w.v16 = w.dout16 + copy;
+  w.bytes = w.v16 + copy;
+  return w;
+}
+}  // namespace
+
+size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
+  if (n_seqs < 0 || max_seqlen < 0 || hq < 0 || head_dim < 0) return 0;
+  return bwd_ws_map(n_seqs, max_seqlen, hq, head_dim).bytes;
 }
 
 opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int32_t qk_dtype, const void* o,
@@ -201,7 +234,8 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   if (!o || !dout || !lse || !cu_seqlens || !conv_idx || !layout_ws || !dq || !dk || !dv || !workspace ||
       !dev_status)
     return OPR_INVALID_ARG;
-  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return OPR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return OPR_INVALID_ARG;
   if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
   if (qk_dtype != OPR_DTYPE_BF16 && qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
   const bool f16 = qk_dtype == OPR_DTYPE_FP16;
@@ -209,24 +243,34 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
     return OPR_WORKSPACE_TOO_SMALL;
   opr_status st = device_check();
   if (st != OPR_OK) return st;
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, total_tokens, hq, head_dim, f16) || !make_map(&tk, k, total_tokens, hkv, head_dim, f16) ||
-      !make_map(&tv, v, total_tokens, hkv, head_dim) || !make_map(&tdo, dout, total_tokens, hq, head_dim))
-    return OPR_CUDA_ERROR;
+  const BwdWs bw = bwd_ws_map(n_seqs, max_seqlen, hq, head_dim);
+  BwdBuffers buf;
+  buf.o = o;
+  buf.o_fp32 = o_dtype == OPR_DTYPE_FP32;
+  buf.dout = static_cast<const __nv_bfloat16*>(dout);
+  buf.v = static_cast<const __nv_bfloat16*>(v);
+  buf.row_terms = reinterpret_cast<float*>(static_cast<char*>(workspace) + bw.row_terms);
+  buf.dout16 = reinterpret_cast<__half*>(static_cast<char*>(workspace) + bw.dout16);
+  buf.v16 = reinterpret_cast<__half*>(static_cast<char*>(workspace) + bw.v16);
+  BwdMaps maps;
+  if (!make_map(&maps.q, q, total_tokens, hq, head_dim, f16) || !make_map(&maps.k, k, total_tokens, hkv, head_dim, f16) ||
+      !make_map(&maps.v, v, total_tokens, hkv, head_dim) || !make_map(&maps.dout, dout, total_tokens, hq, head_dim) ||
+      !make_map(&maps.v16, buf.v16, total_tokens, hkv, head_dim, true) ||
+      !make_map(&maps.dout16, buf.dout16, total_tokens, hq, head_dim, true))
+    return map_fail();
   const LayoutWs w = layout_ws_map(n_seqs, n_convs, n_turns, total_tokens, max_seqlen);
   AttnParams pq = base_params(cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs, n_turns, total_tokens, max_seqlen,
                               hq, hkv, scale, dev_status);
   pq.lse_in = lse;
-  pq.d_tiles = static_cast<const float*>(workspace);
+  pq.d_tiles = buf.row_terms;
   pq.lse2_tiles = pq.d_tiles + static_cast<size_t>(hq) * pq.n_items * kTile;
   pq.dq = dq;
   pq.dk = dk;
   pq.dv = dv;
   AttnParams pkv = pq;
   pkv.sched = ws_ptr<int32_t>(layout_ws, w.k_sched);
-  cudaError_t e = launch_attn_bwd(head_dim, f16, tq, tk, tv, tdo, o, o_dtype == OPR_DTYPE_FP32, dout, pq, pkv,
-                                  static_cast<float*>(workspace), stages, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? OPR_OK : OPR_CUDA_ERROR;
+  cudaError_t e = launch_attn_bwd(head_dim, f16, maps, buf, pq, pkv, stages, static_cast<cudaStream_t>(stream));
+  return status_of(e);
 }
 
 opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int32_t qk_dtype, const void* o,

@@ -13,11 +13,17 @@
 //                the group and the column's non-empty query tiles:
 //                S^T = K Q^T, dP^T = V dO^T -> P^T, dS^T (TMEM) ->
 //                dV += P^T dO, dK += dS^T Q.
-// Q/K and the dS operand share one 16-bit type (fp16 when QK16, else bf16);
-// dO, V and P are bf16.
+// Q/K and the dS operand share one 16-bit type (fp16 when QK16, else bf16).
+// The dq kernel forms dP from the bf16 dO and V; the dkdv kernel works on
+// fp16 copies of dO and V (written by the row-terms stage), so that P^T is
+// an fp16 operand of dV = P^T dO (bf16 P^T loses too much there).
 // Warp roles as in the forward: warp 0 TMA producer (+ metadata lanes),
 // warp 1 TMEM owner and MMA issuer, warps 2..9 two threads per TMEM lane
 // (row), each owning 64 of the tile's 128 columns.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
 #include "attn_common.cuh"
 
 namespace opr {
@@ -30,13 +36,19 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ----------------------------------------------------------------------------
 // Row terms, stored per 128-token tile so the kernels can bulk-copy them:
 // d_tiles[h][tile][c] = sum_d dO * O and lse2_tiles[h][tile][c] = LSE * log2(e)
-// of token c of tile (s, J); 0 and +inf past the end of the sequence.
+// of token c of tile (s, J); 0 and +inf past the end of the sequence.  The
+// kernel also writes dout16, the fp16 copy of dO that the dkdv kernel reads
+// (bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]; a larger one sets
+// OPR_DEV_FP16_RANGE).
 // One block of 128 threads per (tile, head), one token per thread.
+__device__ __forceinline__ bool fp16_range_ok(float x) { return fabsf(x) <= 65504.f; }
+
 template <int D, typename OT>
 __global__ void __launch_bounds__(128) row_terms_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                                                         const float* __restrict__ lse, const int32_t* __restrict__ cu_seqlens,
                                                         int64_t total, int32_t hq, int32_t T, float* __restrict__ d_tiles,
-                                                        float* __restrict__ lse2_tiles) {
+                                                        float* __restrict__ lse2_tiles, __half* __restrict__ dout16,
+                                                        int32_t* __restrict__ dev_status) {
   const int tile = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
   const int s = tile / T, J = tile % T;
   const int seq0 = cu_seqlens[s];
@@ -50,12 +62,19 @@ __global__ void __launch_bounds__(128) row_terms_kernel(const OT* __restrict__ o
   const int64_t tok = seq0 + J * kTile + c;
   const size_t base = (static_cast<size_t>(tok) * hq + h) * D;
   const uint4* dp = reinterpret_cast<const uint4*>(dout + base);
+  uint4* d16 = reinterpret_cast<uint4*>(dout16 + base);
   float acc = 0.f;
+  bool in_range = true;
 #pragma unroll 4
   for (int x = 0; x < D / 8; ++x) {
     const uint4 dv = dp[x];
     const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
-    float ov[8];
+    float ov[8], df[8];
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      df[2 * y] = __low2float(d2[y]);
+      df[2 * y + 1] = __high2float(d2[y]);
+    }
     if constexpr (sizeof(OT) == 4) {
       const float4* op = reinterpret_cast<const float4*>(o + base) + 2 * x;
       const float4 a = op[0], b = op[1];
@@ -70,13 +89,38 @@ __global__ void __launch_bounds__(128) row_terms_kernel(const OT* __restrict__ o
       }
     }
 #pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      acc = fmaf(ov[2 * y], __low2float(d2[y]), acc);
-      acc = fmaf(ov[2 * y + 1], __high2float(d2[y]), acc);
+    for (int y = 0; y < 8; ++y) {
+      acc = fmaf(ov[y], df[y], acc);
+      in_range &= fp16_range_ok(df[y]);
     }
+    d16[x] = make_uint4(pack_f16x2(df[0], df[1]), pack_f16x2(df[2], df[3]), pack_f16x2(df[4], df[5]),
+                        pack_f16x2(df[6], df[7]));
   }
   d_tiles[out] = acc;
   lse2_tiles[out] = lse[static_cast<size_t>(h) * total + tok] * kLog2e;
+  if (!in_range) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
+}
+
+// fp16 copy of V for the dkdv kernel, eight values per thread (same range rule).
+__global__ void __launch_bounds__(256) cast_f16_kernel(const __nv_bfloat16* __restrict__ x, __half* __restrict__ y,
+                                                       int64_t n8, int32_t* __restrict__ dev_status) {
+  bool in_range = true;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    float f[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __low2float(b2[k]);
+      f[2 * k + 1] = __high2float(b2[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) in_range &= fp16_range_ok(f[k]);
+    reinterpret_cast<uint4*>(y)[i] =
+        make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]), pack_f16x2(f[4], f[5]), pack_f16x2(f[6], f[7]));
+  }
+  if (!in_range) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
 // ----------------------------------------------------------------------------
@@ -354,9 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 struct DkdvSmem {
   alignas(1024) uint8_t k[TileGeom<D>::kBytes];
-  alignas(1024) uint8_t v[TileGeom<D>::kBytes];
+  alignas(1024) uint8_t v[TileGeom<D>::kBytes];              // fp16 copy of V
   alignas(1024) uint8_t q[kStages][TileGeom<D>::kBytes];
-  alignas(1024) uint8_t dout[kStages][TileGeom<D>::kBytes];
+  alignas(1024) uint8_t dout[kStages][TileGeom<D>::kBytes];  // fp16 copy of dO
   // column data of a query tile, bulk-copied with its Q tile: LSE * log2(e), D and
   // (for partial tiles) the query metadata
   alignas(16) float qlse2[kStages][kTile];
@@ -365,25 +409,24 @@ struct DkdvSmem {
   int32_t list[kListSmem];
   uint64_t bar_kv;
   uint64_t bar_qfull[kStages], bar_qempty[kStages], bar_dofull[kStages], bar_doempty[kStages];
-  uint64_t bar_sfull, bar_dpfull, bar_pfull, bar_dsfull, bar_accdone, bar_final;
+  uint64_t bar_sfull, bar_dpfull;
+  uint64_t bar_pfull[2], bar_dsfull[2];  // one per query half
+  uint64_t bar_accdone, bar_final;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// TMEM columns of the dkdv kernel: S^T / P^T at 0, dP^T / dS^T at 128,
-// dV accumulator at 256, dK accumulator at 256 + D.  Each compute thread
-// overwrites only the 64 columns it has itself read: the packed 16-bit values
-// of query columns 0..63 go to region columns 0..31 (P^T hi; P^T lo at
-// 32..63) and those of query columns 64..127 to 64..95 (lo at 96..127), so the
-// MMA's K step kk reads region column split_col(kk).
+// TMEM columns of the dkdv kernel: S^T at 0..127 and dP^T at 128..255 (one
+// column per query of the tile), dV accumulator at 256, dK at 256 + D.  The
+// compute warps of query half h (columns 64h..64h+63 of each region) write
+// the packed fp16 P^T and dS^T of their half over the first 32 of those
+// columns, which the dV and dK products read as their A operand.
 constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvColDV = 256;
-
-__device__ __forceinline__ uint32_t split_col(int kk) { return (kk & 3) * 8 + (kk >> 2) * 64; }
 
 template <int D, bool QK16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ CUtensorMap tm_v16, const __grid_constant__ CUtensorMap tm_do16,
                          const AttnParams p) {
   constexpr uint32_t kTileBytes = TileGeom<D>::kBytes;
   constexpr uint32_t kColDK = kKvColDV + D;
@@ -416,8 +459,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sm.bar_sfull, 1);
     mbar_init(&sm.bar_dpfull, 1);
-    mbar_init(&sm.bar_pfull, kComputeThreads);
-    mbar_init(&sm.bar_dsfull, kComputeThreads);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&sm.bar_pfull[h], kComputeThreads / 2);
+      mbar_init(&sm.bar_dsfull[h], kComputeThreads / 2);
+    }
     mbar_init(&sm.bar_accdone, 1);
     mbar_init(&sm.bar_final, 1);
     sm.abort_flag = 0;
@@ -441,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileMeta* tmeta = p.tile_meta + static_cast<size_t>(s) * p.T;
       mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
       tma_tile<D>(&tm_k, &sm.bar_kv, sm.k, kvh, k0);
-      tma_tile<D>(&tm_v, &sm.bar_kv, sm.v, kvh, k0);
+      tma_tile<D>(&tm_v16, &sm.bar_kv, sm.v, kvh, k0);
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
@@ -473,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= kStages && !mbar_wait(&sm.bar_doempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
           break;
         mbar_arrive_expect_tx(&sm.bar_dofull[st], kTileBytes);
-        tma_tile<D>(&tm_do, &sm.bar_dofull[st], sm.dout[st], h, seq0 + (entry(j % cnt) >> 2) * kTile);
+        tma_tile<D>(&tm_do16, &sm.bar_dofull[st], sm.dout[st], h, seq0 + (entry(j % cnt) >> 2) * kTile);
         issued = j + 1;
       }
       if (*abort_flag)
@@ -483,82 +528,84 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // the whole warp runs this loop; elect.sync picks the issuing lane
     constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S^T = K Q^T (q/k type)
-    constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP^T = V dO^T (bf16)
-    constexpr uint32_t idesc_v = idesc_bf16_f32(128, D, 0, 1);        // dV += P^T dO (bf16)
-    constexpr uint32_t idesc_k = idesc_f32acc(128, D, QK16, 0, 1);    // dK += dS^T Q (q/k type)
-    const uint32_t sk = smem_u32(sm.k), sv = smem_u32(sm.v);
-    // S^T(j) = K Q(j)^T into the S region
+    constexpr uint32_t idesc_p = idesc_f32acc(128, 128, true, 0, 0);  // dP^T = V dO^T (fp16)
+    constexpr uint32_t idesc_v = idesc_f32acc(128, D, true, 0, 1);    // dV += P_h^T dO_h (fp16)
+    constexpr uint32_t idesc_k = idesc_f32acc(128, D, QK16, 0, 1);    // dK += dS_h^T Q_h (q/k type)
+    const uint64_t dk_base = desc_kmajor(smem_u32(sm.k), 0), dv_base = desc_kmajor(smem_u32(sm.v), 0);
+    // S^T(j) = K Q(j)^T.  Full 128-query products: both operands come from shared
+    // memory, whose bandwidth a narrower N would spend faster than the tensor core.
     auto issue_s = [&](int j) -> bool {
       const int st = j % kStages;
       if (!warp_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t sq = smem_u32(sm.q[st]);
+      const uint64_t qb = desc_kmajor(smem_u32(sm.q[st]), 0);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + kKvColS, (desc_kmajor(sk, 0) + kmajor_step(kk)), (desc_kmajor(sq, 0) + kmajor_step(kk)), idesc_s, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kKvColS, dk_base + kmajor_step(kk), qb + kmajor_step(kk), idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_sfull);
       return true;
     };
-    // dP^T(j) = V dO(j)^T into the dP region
+    // dP^T(j) = V dO(j)^T
     auto issue_dp = [&](int j) -> bool {
       const int st = j % kStages;
       if (!warp_wait(&sm.bar_dofull[st], (j / kStages) & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t sdo = smem_u32(sm.dout[st]);
+      const uint64_t ob = desc_kmajor(smem_u32(sm.dout[st]), 0);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + kKvColDP, (desc_kmajor(sv, 0) + kmajor_step(kk)), (desc_kmajor(sdo, 0) + kmajor_step(kk)), idesc_p, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kKvColDP, dv_base + kmajor_step(kk), ob + kmajor_step(kk), idesc_p, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_dpfull);
       return true;
     };
-    // dV += P^T(j) dO(j), P^T as bf16 hi + lo parts; releases dO(j)
-    auto issue_dv = [&](int j) -> bool {
+    // dV += P^T(j)[:, half h] dO(j)[half h]; the second half releases dO(j)
+    auto issue_dv = [&](int h, int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_pfull, j & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_pfull[h], j & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t sdo = smem_u32(sm.dout[st]);
+      const uint64_t ob = desc_mnmajor(smem_u32(sm.dout[st]), 4 * h);
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kKvColDV, tmem + kKvColS + split_col(kk), (desc_mnmajor(sdo, 0) + mnmajor_step(kk)), idesc_v,
-               (j > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kKvColDV, tmem + kKvColS + 32 + split_col(kk), (desc_mnmajor(sdo, 0) + mnmajor_step(kk)), idesc_v, 1u);
-      mma_commit(&sm.bar_doempty[st]);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(tmem + kKvColDV, tmem + kKvColS + 64 * h + kk * 8, ob + mnmajor_step(kk), idesc_v,
+               (j > 0 || h > 0 || kk > 0) ? 1u : 0u);
+      if (h == 1) mma_commit(&sm.bar_doempty[st]);
       return true;
     };
-    // dK += dS^T(j) Q(j); releases Q(j) and its column data
-    auto issue_dk = [&](int j) -> bool {
+    // dK += dS^T(j)[:, half h] Q(j)[half h]; the second half releases Q(j) and its column data
+    auto issue_dk = [&](int h, int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_dsfull, j & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_dsfull[h], j & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t sq = smem_u32(sm.q[st]);
+      const uint64_t qb = desc_mnmajor(smem_u32(sm.q[st]), 4 * h);
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kColDK, tmem + kKvColDP + split_col(kk), (desc_mnmajor(sq, 0) + mnmajor_step(kk)), idesc_k,
-               (j > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(&sm.bar_qempty[st]);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(tmem + kColDK, tmem + kKvColDP + 64 * h + kk * 8, qb + mnmajor_step(kk), idesc_k,
+               (j > 0 || h > 0 || kk > 0) ? 1u : 0u);
+      if (h == 1) mma_commit(&sm.bar_qempty[st]);
       return true;
     };
-    // Issue order S(0) dP(0) | dV(0) S(1) dK(0) dP(1) | dV(1) S(2) dK(1) dP(2) | ...
-    // so that the next S^T is formed while the compute warps turn dP^T into dS^T,
-    // and the next dP^T while they turn S^T into P^T.
+    // Issue order S(0) dP(0) | dV_0(j) dV_1(j) S(j+1) dK_0(j) dK_1(j) dP(j+1) | ...:
+    // the next S^T is formed while the compute warps turn dP^T into dS^T, and
+    // the next dP^T while they turn S^T into P^T; each half's dV (dK) product
+    // starts as soon as that half's P^T (dS^T) is in place.
     bool ok = warp_wait(&sm.bar_kv, 0, abort_flag) && issue_s(0) && issue_dp(0);
     for (int j = 0; ok && j < n; ++j) {
-      ok = issue_dv(j);
-      if (ok && j + 1 < n) ok = issue_s(j + 1);
-      if (ok) ok = issue_dk(j);
-      if (ok && j + 1 < n) ok = issue_dp(j + 1);
+      const bool more = j + 1 < n;
+      ok = issue_dv(0, j) && issue_dv(1, j);
+      if (ok && more) ok = issue_s(j + 1);
+      if (ok) ok = issue_dk(0, j) && issue_dk(1, j);
+      if (ok && more) ok = issue_dp(j + 1);
     }
     if (ok) mma_commit(&sm.bar_accdone);
     mma_commit(&sm.bar_final);
     __all_sync(0xffffffffu, mbar_wait(&sm.bar_final, 0, nullptr, kWaitLimitNs));
   } else {
-    // two threads per key row: `half` selects query columns [64 half, 64 half + 64)
+    // query half `half`: warps 2..5 own query columns 0..63, warps 6..9 columns
+    // 64..127; one key row per thread
     const int quad = warp & 3;
     const int half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t cs = kKvColS + 64 * half, cdp = kKvColDP + 64 * half;
     const bool kvld = J * kTile + row < seq_len;
     const int kg = k0 + row;
     const int kconv = kvld ? p.conv_idx[kg] : -1;
@@ -575,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
-      // visibility of this thread's 64 query columns (all set on full tiles)
+      // visibility of this stream's 64 query columns (all set on full tiles)
       uint32_t mm[2] = {0xffffffffu, 0xffffffffu};
       if (partial) {
         uint32_t m[4];
@@ -588,64 +635,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float pv[64];
+      // P^T as fp16, two query columns per TMEM column, over this half's own S^T
+      // columns; the packed values also serve the dS step below
+      uint32_t pp[32];
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t sr[32];
-        tmem_ld32(tl + kKvColS + c0 + cc * 32, sr);
+        tmem_ld32(tl + cs + cc * 32, sr);
         const float4* l4 = reinterpret_cast<const float4*>(&sm.qlse2[st][c0 + cc * 32]);
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
           const float4 l = l4[x];
-          pv[cc * 32 + 4 * x] = fast_exp2(fmaf(__uint_as_float(sr[4 * x]), sl2, -l.x));
-          pv[cc * 32 + 4 * x + 1] = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 1]), sl2, -l.y));
-          pv[cc * 32 + 4 * x + 2] = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 2]), sl2, -l.z));
-          pv[cc * 32 + 4 * x + 3] = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 3]), sl2, -l.w));
+          const int c = cc * 32 + 4 * x;
+          float p0 = fast_exp2(fmaf(__uint_as_float(sr[4 * x]), sl2, -l.x));
+          float p1 = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 1]), sl2, -l.y));
+          float p2 = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 2]), sl2, -l.z));
+          float p3 = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 3]), sl2, -l.w));
+          if (partial) {
+            const uint32_t b = mm[c >> 5] >> (c & 31);
+            p0 = (b & 1u) ? p0 : 0.f;
+            p1 = (b & 2u) ? p1 : 0.f;
+            p2 = (b & 4u) ? p2 : 0.f;
+            p3 = (b & 8u) ? p3 : 0.f;
+          }
+          pp[cc * 16 + 2 * x] = pack_f16x2(p0, p1);
+          pp[cc * 16 + 2 * x + 1] = pack_f16x2(p2, p3);
         }
       }
-#pragma unroll
-      for (int c = 0; c < 64; ++c)
-        if (!((mm[c >> 5] >> (c & 31)) & 1u)) pv[c] = 0.f;
-      // P^T for dV = P^T dO as bf16 hi + lo parts, two values per TMEM column, in this
-      // thread's own 64 columns of the S^T region: lo carries the rounding error of hi.
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const float a = pv[c * 32 + 2 * x], b = pv[c * 32 + 2 * x + 1];
-          const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-          hi[x] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[x] = pack_bf16x2(a - __low2float(h), b - __high2float(h));
-        }
-        tmem_st16(tl + kKvColS + c0 + c * 16, hi);
-        tmem_st16(tl + kKvColS + c0 + 32 + c * 16, lo);
-      }
+      tmem_st16(tl + cs, reinterpret_cast<const uint32_t(&)[16]>(pp[0]));
+      tmem_st16(tl + cs + 16, reinterpret_cast<const uint32_t(&)[16]>(pp[16]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.bar_pfull);
+      mbar_arrive(&sm.bar_pfull[half]);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, kWaitLimitNs))) {
         ok = false;
         break;
       }
       tc_fence_after();
+      // dS^T = P^T (dP^T - D) in the q/k type, over this half's own dP^T columns
+      {
+        const float4* d4 = reinterpret_cast<const float4*>(&sm.qd[st][c0]);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tl + kKvColDP + c0 + c * 32, r);
-        uint32_t pk[16];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tl + cdp + c * 32, r);
+          uint32_t pk[16];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int q = c * 32 + 2 * x;
-          const float d0 = pv[q] * (__uint_as_float(r[2 * x]) - sm.qd[st][c0 + q]);
-          const float d1 = pv[q + 1] * (__uint_as_float(r[2 * x + 1]) - sm.qd[st][c0 + q + 1]);
-          pk[x] = pack_x2<QK16>(d0, d1);
+          for (int x = 0; x < 8; ++x) {
+            const float4 dd = d4[c * 8 + x];
+            const float2 pa = __half22float2(*reinterpret_cast<const __half2*>(&pp[c * 16 + 2 * x]));
+            const float2 pb = __half22float2(*reinterpret_cast<const __half2*>(&pp[c * 16 + 2 * x + 1]));
+            const float d0 = pa.x * (__uint_as_float(r[4 * x]) - dd.x);
+            const float d1 = pa.y * (__uint_as_float(r[4 * x + 1]) - dd.y);
+            const float d2 = pb.x * (__uint_as_float(r[4 * x + 2]) - dd.z);
+            const float d3 = pb.y * (__uint_as_float(r[4 * x + 3]) - dd.w);
+            pk[2 * x] = pack_x2<QK16>(d0, d1);
+            pk[2 * x + 1] = pack_x2<QK16>(d2, d3);
+          }
+          tmem_st16(tl + cdp + c * 16, pk);
         }
-        tmem_st16(tl + kKvColDP + c0 + c * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.bar_dsfull);
+      mbar_arrive(&sm.bar_dsfull[half]);
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_accdone, 0, abort_flag, kWaitLimitNs))) {
       tc_fence_after();
@@ -701,30 +753,38 @@ cudaError_t set_smem(K kernel, size_t smem, int* configured) {
 }
 
 template <int D, bool QK16>
-cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
-                         const void* o, int o_fp32, const void* dout, const AttnParams& pq, const AttnParams& pkv,
-                         float* row_d, int stages, cudaStream_t stream) {
+cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams& pq, const AttnParams& pkv,
+                         int stages, cudaStream_t stream) {
   static int conf_dq[64] = {0}, conf_kv[64] = {0};
   cudaError_t e = cudaSuccess;
-  // 1) row terms D and LSE * log2(e), per 128-token tile
+  // 1) row terms D and LSE * log2(e) per 128-token tile, and the fp16 copies of dO and V
   if ((stages & OPR_BWD_ROW_TERMS) && pq.n_items > 0) {
     const dim3 grid(pq.n_items, pq.hq);
-    if (o_fp32)
-      row_terms_kernel<D, float><<<grid, kTile, 0, stream>>>(
-          static_cast<const float*>(o), static_cast<const __nv_bfloat16*>(dout), pq.lse_in, pq.cu_seqlens, pq.total,
-          pq.hq, pq.T, row_d, row_d + static_cast<size_t>(pq.hq) * pq.n_items * kTile);
+    float* row_d = b.row_terms;
+    float* row_l = b.row_terms + static_cast<size_t>(pq.hq) * pq.n_items * kTile;
+    if (b.o_fp32)
+      row_terms_kernel<D, float><<<grid, kTile, 0, stream>>>(static_cast<const float*>(b.o), b.dout, pq.lse_in,
+                                                               pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d, row_l,
+                                                               b.dout16, pq.dev_status);
     else
       row_terms_kernel<D, __nv_bfloat16><<<grid, kTile, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), pq.lse_in, pq.cu_seqlens,
-          pq.total, pq.hq, pq.T, row_d, row_d + static_cast<size_t>(pq.hq) * pq.n_items * kTile);
+          static_cast<const __nv_bfloat16*>(b.o), b.dout, pq.lse_in, pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d,
+          row_l, b.dout16, pq.dev_status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int64_t n8 = pq.total * pq.hkv * D / 8;
+    if (n8 > 0) {
+      const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, 148 * 16);
+      cast_f16_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(b.v, b.v16, n8, pq.dev_status);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
   }
   // 2) dQ
   if (stages & OPR_BWD_DQ) {
     const size_t smem_q = smem_request(sizeof(DqSmem<D>) + 1024);
     if ((e = set_smem(attn_bwd_dq_kernel<D, QK16>, smem_q, conf_dq)) != cudaSuccess) return e;
     const int64_t bq = static_cast<int64_t>(pq.n_items) * pq.hq;
-    if (bq > 0) attn_bwd_dq_kernel<D, QK16><<<static_cast<unsigned>(bq), kThreads, smem_q, stream>>>(tq, tk, tv, tdo, pq);
+    if (bq > 0)
+      attn_bwd_dq_kernel<D, QK16><<<static_cast<unsigned>(bq), kThreads, smem_q, stream>>>(m.q, m.k, m.v, m.dout, pq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // 3) dK, dV
@@ -733,7 +793,8 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
     if ((e = set_smem(attn_bwd_dkdv_kernel<D, QK16>, smem_kv, conf_kv)) != cudaSuccess) return e;
     const int64_t bkv = static_cast<int64_t>(pkv.n_items) * pkv.hkv;
     if (bkv > 0)
-      attn_bwd_dkdv_kernel<D, QK16><<<static_cast<unsigned>(bkv), kThreads, smem_kv, stream>>>(tq, tk, tv, tdo, pkv);
+      attn_bwd_dkdv_kernel<D, QK16>
+          <<<static_cast<unsigned>(bkv), kThreads, smem_kv, stream>>>(m.q, m.k, m.v16, m.dout16, pkv);
     e = cudaGetLastError();
   }
   return e;
@@ -741,15 +802,13 @@ cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 }  // namespace
 
-cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
-                            const CUtensorMap& tv, const CUtensorMap& tdo, const void* o, int o_fp32,
-                            const void* dout, const AttnParams& pq, const AttnParams& pkv, float* row_d, int stages,
-                            cudaStream_t stream) {
+cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const BwdMaps& m, const BwdBuffers& b, const AttnParams& pq,
+                            const AttnParams& pkv, int stages, cudaStream_t stream) {
   if (head_dim == 128)
-    return qk_f16 ? launch_bwd_t<128, true>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream)
-                  : launch_bwd_t<128, false>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream);
-  return qk_f16 ? launch_bwd_t<64, true>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream)
-                : launch_bwd_t<64, false>(tq, tk, tv, tdo, o, o_fp32, dout, pq, pkv, row_d, stages, stream);
+    return qk_f16 ? launch_bwd_t<128, true>(m, b, pq, pkv, stages, stream)
+                  : launch_bwd_t<128, false>(m, b, pq, pkv, stages, stream);
+  return qk_f16 ? launch_bwd_t<64, true>(m, b, pq, pkv, stages, stream)
+                : launch_bwd_t<64, false>(m, b, pq, pkv, stages, stream);
 }
 
 }  // namespace opr

@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "opr_internal.cuh"
@@ -134,6 +135,22 @@ __device__ __forceinline__ void key_row_mask(const TileMeta& t, int qbase, int k
 }
 
 __device__ __forceinline__ bool mask_bit(const uint32_t (&m)[4], int c) { return (m[c >> 5] >> (c & 31)) & 1u; }
+
+// Tensor maps and buffers of one backward call (built by the entry point).
+struct BwdMaps {
+  CUtensorMap q, k, v, dout;  // the call's operands (q/k type, bf16 v and dO)
+  CUtensorMap v16, dout16;    // fp16 copies of v and dO in the workspace
+};
+
+struct BwdBuffers {
+  const void* o;
+  int o_fp32;
+  const __nv_bfloat16* dout;
+  const __nv_bfloat16* v;
+  float* row_terms;  // D tiles, then LSE * log2(e) tiles
+  __half* dout16;
+  __half* v16;
+};
 
 struct AttnParams {
   const int32_t* cu_seqlens;

@@ -57,7 +57,8 @@ typedef int32_t opr_status;
 #define OPR_DEV_TOTAL_MISMATCH 2   /* sum of h + t + 2r differs from total_tokens */
 #define OPR_DEV_SEQ_TOO_LONG 4     /* a sequence is longer than max_seqlen */
 #define OPR_DEV_WAIT_TIMEOUT 8     /* a pipeline wait exceeded its time limit; outputs are invalid */
-#define OPR_DEV_FP16_RANGE 16      /* opr_rope wrote an fp16 value beyond +-65504 (inf) */
+#define OPR_DEV_FP16_RANGE 16      /* an fp16 value beyond +-65504 was written (opr_rope output, or the
+                                      backward's fp16 copies of dO and v) */
 
 #define OPR_DTYPE_BF16 0
 #define OPR_DTYPE_FP32 1
@@ -164,9 +165,13 @@ OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int
                         void* stream);
 
 /*
- * Bytes of device scratch that opr_attn_bwd needs: the row terms
- * D = rowsum(dO * O) and LSE * log2(e), stored per 128-token tile
- * (2 * 4 * hq * n_seqs * ceil(max_seqlen / 128) * 128 bytes, rounded up to 256).
+ * Bytes of device scratch that opr_attn_bwd needs.  With
+ * N = n_seqs * ceil(max_seqlen / 128) * 128 (a bound on the token count):
+ *   the row terms D = rowsum(dO * O) and LSE * log2(e), stored per 128-token
+ *   tile: 2 * 4 * hq * N bytes;
+ *   an fp16 copy of dO: 2 * N * hq * head_dim bytes;
+ *   an fp16 copy of v (kv heads bounded by hq): 2 * N * hq * head_dim bytes;
+ * each part rounded up to 256 bytes.  Returns 0 for negative arguments.
  */
 OPR_API size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq,
                                             int32_t head_dim);
@@ -182,7 +187,13 @@ OPR_API size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, 
  *   lse               fp32 [hq, total] from opr_attn_fwd
  *   dq                fp32 [total, hq, head_dim]
  *   dk, dv            fp32 [total, hkv, head_dim]
- *   workspace         opr_attn_bwd_workspace_bytes(...) bytes of device scratch
+ *   workspace         opr_attn_bwd_workspace_bytes(...) bytes of device scratch,
+ *                     16-byte aligned, owned by the caller; the call overwrites it
+ * The dK/dV products use fp16 copies of dO and v (dV = P^T dO needs P^T with
+ * more mantissa than bf16 has, and the two operands of one tensor-core product
+ * share a type).  bf16 -> fp16 is exact for magnitudes in [2^-14, 65504];
+ * smaller ones lose low bits and a larger one sets OPR_DEV_FP16_RANGE in
+ * *dev_status (the results are then invalid).
  */
 OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int32_t qk_dtype,
                         const void* o, int32_t o_dtype, const void* dout, const float* lse,
@@ -196,7 +207,8 @@ OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int
  * opr_attn_bwd_stages - the same computation as opr_attn_bwd, split into its
  * three kernels so that a caller can order, overlap or time them one by one.
  * `stages` is an OR of:
- *   OPR_BWD_ROW_TERMS  D = rowsum(dO * O) into `workspace` (needed by the other two)
+ *   OPR_BWD_ROW_TERMS  D = rowsum(dO * O) and the fp16 copies of dO and v into
+ *                      `workspace` (needed by the other two)
  *   OPR_BWD_DQ         dq   (one CTA per query tile and q head)
  *   OPR_BWD_DKDV       dk, dv (one CTA per key tile and kv head; GQA group summed in the CTA)
  * Running all three, in this order on one stream, equals opr_attn_bwd.
@@ -223,7 +235,8 @@ OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void*
  * not call cudaMalloc, which can block and synchronize the device.
  *
  * Same inputs, outputs and error behaviour as opr_attn_bwd, without the
- * workspace arguments: the scratch (the row terms) lives in one fixed
+ * workspace arguments: the scratch (the row terms and the fp16 copies of dO
+ * and v) lives in one fixed
  * library-owned device array of OPR_NOALLOC_SCRATCH_BYTES, allocated by the
  * CUDA loader on every GPU that loads the library and held until the process
  * exits.  The call allocates and frees nothing.
@@ -250,6 +263,13 @@ OPR_API opr_status opr_attn_bwd_noalloc(const void* q, const void* k, const void
 
 /* Library version string, e.g. "opr 0.1.0 sm_100a". */
 OPR_API const char* opr_version(void);
+
+/*
+ * Text of the CUDA error behind the last OPR_CUDA_ERROR that an entry point
+ * returned on the calling host thread ("no error" before any).  The string
+ * is static; the caller does not free it.
+ */
+OPR_API const char* opr_last_error(void);
 
 #ifdef __cplusplus
 }

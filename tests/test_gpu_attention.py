@@ -193,3 +193,32 @@ def test_deterministic_backward():
     b, _ = _run_gpu(w, q, k, v, do)
     for name in ("o", "lse", "dq", "dk", "dv"):
         np.testing.assert_array_equal(a[name], b[name])
+
+
+def test_backward_flags_do_beyond_fp16_range():
+    """The dK/dV products read an fp16 copy of dO: a value beyond 65504 is reported, not silently clipped."""
+    from block_sparse_masked_segment_b200 import _abi
+
+    w = synth.random_small_workload(4, hq=4, hkv=2, d=128)
+    q, k, v, do = inputs(w, 4)
+    do = do.copy()
+    do[w.total_tokens // 2, 1, 7] = 1.0e5
+    att = opr.OnePassAttention(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, base=w.base)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    o, lse, qr, kr = att.forward(qd, kd, vd)
+    att.backward(qr, kr, vd, o, to_dev(do), lse)
+    torch.cuda.synchronize()
+    assert opr.read_status(att.layout.dev_status) == [_abi.DEV_BITS[16]]
+
+
+def test_backward_in_range_values_leave_status_clear():
+    """Large but representable dO and v (|x| up to 6e4) pass the fp16 copy without a flag."""
+    w = synth.random_small_workload(5, hq=4, hkv=2, d=64)
+    q, k, v, do = inputs(w, 5)
+    do = do * 0 + np.float32(6.0e4) * np.sign(do)
+    att = opr.OnePassAttention(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, base=w.base)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    o, lse, qr, kr = att.forward(qd, kd, vd)
+    att.backward(qr, kr, vd, o, to_dev(do), lse)
+    torch.cuda.synchronize()
+    assert opr.read_status(att.layout.dev_status) == []

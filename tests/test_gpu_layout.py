@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import block_sparse_masked_segment_b200 as opr
+from block_sparse_masked_segment_b200 import _abi
 import synth
 from oracle import opr_oracle as orc
 
@@ -134,4 +135,4 @@ def test_rope_fp16_overflow_is_flagged():
     y = torch.empty(x.shape, dtype=torch.float16, device="cuda")
     opr.opr_rope(x, lay.pos_id, 1e4, out=y, dev_status=lay.dev_status)
     torch.cuda.synchronize()
-    assert "fp16 overflow in rope" in opr.read_status(lay.dev_status)
+    assert _abi.DEV_BITS[16] in opr.read_status(lay.dev_status)
