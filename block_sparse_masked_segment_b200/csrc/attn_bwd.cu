@@ -34,9 +34,10 @@ constexpr int kListSmem = 1024;  // entries of a tile list kept in shared memory
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ----------------------------------------------------------------------------
-// Row terms, stored per 128-token tile so the kernels can bulk-copy them:
-// d_tiles[h][tile][c] = sum_d dO * O and lse2_tiles[h][tile][c] = LSE * log2(e)
-// of token c of tile (s, J); 0 and +inf past the end of the sequence.  The
+// Row terms, stored negated and per 128-token tile so the kernels can
+// bulk-copy them and fold each into one fused multiply-add:
+// d_tiles[h][tile][c] = -sum_d dO * O and lse2_tiles[h][tile][c] = -LSE * log2(e)
+// of token c of tile (s, J); 0 and -inf past the end of the sequence.  The
 // kernel also writes dout16, the fp16 copy of dO that the dkdv kernel reads
 // (bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]; a larger one sets
 // OPR_DEV_FP16_RANGE).
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(128) row_terms_kernel(const OT* __restrict__ o
   const size_t out = (static_cast<size_t>(h) * gridDim.x + tile) * kTile + c;
   if (J * kTile + c >= L) {
     d_tiles[out] = 0.f;
-    lse2_tiles[out] = INFINITY;
+    lse2_tiles[out] = -INFINITY;
     return;
   }
   const int64_t tok = seq0 + J * kTile + c;
@@ -96,8 +97,8 @@ __global__ void __launch_bounds__(128) row_terms_kernel(const OT* __restrict__ o
     d16[x] = make_uint4(pack_f16x2(df[0], df[1]), pack_f16x2(df[2], df[3]), pack_f16x2(df[4], df[5]),
                         pack_f16x2(df[6], df[7]));
   }
-  d_tiles[out] = acc;
-  lse2_tiles[out] = lse[static_cast<size_t>(h) * total + tok] * kLog2e;
+  d_tiles[out] = -acc;
+  lse2_tiles[out] = -lse[static_cast<size_t>(h) * total + tok] * kLog2e;
   if (!in_range) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
@@ -302,9 +303,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qconv = qv ? p.conv_idx[qg] : -2;
     const int qmeta = qv ? p.tok_meta[qg] : 0;
     const size_t rt = (static_cast<size_t>(head) * p.n_items + tile_id) * kTile + row;
-    const float lse2 = qv ? p.lse2_tiles[rt] : 0.f;
-    const float dd = qv ? p.d_tiles[rt] : 0.f;
-    const float sl2 = p.scale_log2;
+    const float nlse2 = qv ? p.lse2_tiles[rt] : 0.f;  // -LSE * log2(e)
+    const float nd = qv ? p.d_tiles[rt] : 0.f;        // -D
+    const uint64_t sl2x2 = f2(p.scale_log2, p.scale_log2), nlse2x2 = f2(nlse2, nlse2), ndx2 = f2(nd, nd);
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j % kStages;
@@ -336,7 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&sm.bar_sfree);  // S may be overwritten by the next Q K^T
 #pragma unroll
-        for (int c = 0; c < 64; ++c) pv[c] = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, -lse2));
+        for (int c = 0; c < 64; c += 2) {
+          float a0, a1;
+          f2_split(ffma2(f2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, nlse2x2), a0, a1);
+          pv[c] = fast_exp2(a0);
+          pv[c + 1] = fast_exp2(a1);
+        }
       }
 #pragma unroll
       for (int c = 0; c < 64; ++c)
@@ -354,8 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            const float d0 = pv[c * 32 + 2 * x] * (__uint_as_float(r[c * 32 + 2 * x]) - dd);
-            const float d1 = pv[c * 32 + 2 * x + 1] * (__uint_as_float(r[c * 32 + 2 * x + 1]) - dd);
+            const uint64_t t = fadd2(f2(__uint_as_float(r[c * 32 + 2 * x]), __uint_as_float(r[c * 32 + 2 * x + 1])), ndx2);
+            float d0, d1;
+            f2_split(fmul2(f2(pv[c * 32 + 2 * x], pv[c * 32 + 2 * x + 1]), t), d0, d1);
             pk[x] = pack_x2<QK16>(d0, d1);
           }
           tmem_st16(tl + kDqColDS + half * 32 + c * 16, pk);
@@ -610,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kg = k0 + row;
     const int kconv = kvld ? p.conv_idx[kg] : -1;
     const int kmeta = kvld ? p.tok_meta[kg] : 0;
-    const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2(p.scale_log2, p.scale_log2);
     const int c0 = half * 64;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -645,12 +652,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4* l4 = reinterpret_cast<const float4*>(&sm.qlse2[st][c0 + cc * 32]);
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-          const float4 l = l4[x];
+          const float4 l = l4[x];  // -LSE * log2(e) of four query columns
           const int c = cc * 32 + 4 * x;
-          float p0 = fast_exp2(fmaf(__uint_as_float(sr[4 * x]), sl2, -l.x));
-          float p1 = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 1]), sl2, -l.y));
-          float p2 = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 2]), sl2, -l.z));
-          float p3 = fast_exp2(fmaf(__uint_as_float(sr[4 * x + 3]), sl2, -l.w));
+          float a0, a1, a2, a3;
+          f2_split(ffma2(f2(__uint_as_float(sr[4 * x]), __uint_as_float(sr[4 * x + 1])), sl2x2, f2(l.x, l.y)), a0, a1);
+          f2_split(ffma2(f2(__uint_as_float(sr[4 * x + 2]), __uint_as_float(sr[4 * x + 3])), sl2x2, f2(l.z, l.w)), a2,
+                   a3);
+          float p0 = fast_exp2(a0);
+          float p1 = fast_exp2(a1);
+          float p2 = fast_exp2(a2);
+          float p3 = fast_exp2(a3);
           if (partial) {
             const uint32_t b = mm[c >> 5] >> (c & 31);
             p0 = (b & 1u) ? p0 : 0.f;
@@ -682,13 +693,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
-            const float4 dd = d4[c * 8 + x];
+            const float4 nd = d4[c * 8 + x];  // -D of four query columns
             const float2 pa = __half22float2(*reinterpret_cast<const __half2*>(&pp[c * 16 + 2 * x]));
             const float2 pb = __half22float2(*reinterpret_cast<const __half2*>(&pp[c * 16 + 2 * x + 1]));
-            const float d0 = pa.x * (__uint_as_float(r[4 * x]) - dd.x);
-            const float d1 = pa.y * (__uint_as_float(r[4 * x + 1]) - dd.y);
-            const float d2 = pb.x * (__uint_as_float(r[4 * x + 2]) - dd.z);
-            const float d3 = pb.y * (__uint_as_float(r[4 * x + 3]) - dd.w);
+            float d0, d1, d2, d3;
+            f2_split(fmul2(f2(pa.x, pa.y), fadd2(f2(__uint_as_float(r[4 * x]), __uint_as_float(r[4 * x + 1])),
+                                                 f2(nd.x, nd.y))),
+                     d0, d1);
+            f2_split(fmul2(f2(pb.x, pb.y), fadd2(f2(__uint_as_float(r[4 * x + 2]), __uint_as_float(r[4 * x + 3])),
+                                                 f2(nd.z, nd.w))),
+                     d2, d3);
             pk[2 * x] = pack_x2<QK16>(d0, d1);
             pk[2 * x + 1] = pack_x2<QK16>(d2, d3);
           }

@@ -174,8 +174,8 @@ struct AttnParams {
   float* lse;
   // backward
   const float* lse_in;      // [hq, total]
-  const float* d_tiles;     // D = rowsum(dO * O), [hq][n_items][128]
-  const float* lse2_tiles;  // LSE * log2(e), [hq][n_items][128]
+  const float* d_tiles;     // -D = -rowsum(dO * O), [hq][n_items][128]
+  const float* lse2_tiles;  // -LSE * log2(e), [hq][n_items][128]
   float* dq;
   float* dk;
   float* dv;

@@ -553,25 +553,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kTile; ++c)
           if (!mask_bit(mm, c)) sv[c] = -INFINITY;
       }
+      // row max: eight three-input chains
       float mx8[8];
 #pragma unroll
       for (int x = 0; x < 8; ++x) mx8[x] = sv[x];
 #pragma unroll
-      for (int c = 8; c < kTile; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], sv[c]);
+      for (int c = 8; c < kTile; c += 16)
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx8[x] = fmax3(mx8[x], sv[c + x], sv[c + 8 + x]);
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m_run, mx * sl2);
       const bool need = m_new > m_run + 8.f;  // also true on the first finite max
       const float m_use = need ? m_new : m_run;
       const float mb = (m_use == -INFINITY) ? 0.f : m_use;
+      // P = 2^(S scale log2(e) - m), the scale-and-shift on fp32 pairs
+      const uint64_t sl2x2 = f2(sl2, sl2), nmb2 = f2(-mb, -mb);
       float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          const float p0 = fast_exp2(fmaf(sv[c * 32 + 2 * x], sl2, -mb));
-          const float p1 = fast_exp2(fmaf(sv[c * 32 + 2 * x + 1], sl2, -mb));
+          float a0, a1;
+          f2_split(ffma2(f2(sv[c * 32 + 2 * x], sv[c * 32 + 2 * x + 1]), sl2x2, nmb2), a0, a1);
+          const float p0 = fast_exp2(a0);
+          const float p1 = fast_exp2(a1);
           rs8[x & 7] += p0 + p1;
           pk[x] = pack_bf16x2(p0, p1);
         }
