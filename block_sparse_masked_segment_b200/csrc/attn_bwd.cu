@@ -154,10 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   DqSmem<D>& sm = *reinterpret_cast<DqSmem<D>*>(align1024(smem_raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int head = blockIdx.x % p.hq;
-  const int item = blockIdx.x / p.hq;
-  if (item >= p.n_items) return;
-  const int tile_id = p.sched[item];
+  // head-major grid: the CTAs that run together share one kv head's K/V tiles in L2
+  const int head = blockIdx.x / p.n_items;
+  const int tile_id = p.sched[blockIdx.x % p.n_items];
+  if (head >= p.hq) return;
   const int n = p.row_cnt[tile_id];
   if (n == 0) return;
   const int s = tile_id / p.T, I = tile_id % p.T;
@@ -441,10 +441,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   DkdvSmem<D>& sm = *reinterpret_cast<DkdvSmem<D>*>(align1024(smem_raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x % p.hkv;
-  const int item = blockIdx.x / p.hkv;
-  if (item >= p.n_items) return;
-  const int tile_id = p.sched[item];
+  // kv-head-major grid over a schedule grouped by sequence: the CTAs that run
+  // together stream the Q and dO tiles of one kv head group and sequence,
+  // which stay in L2
+  const int kvh = blockIdx.x / p.n_items;
+  const int tile_id = p.sched[blockIdx.x % p.n_items];
+  if (kvh >= p.hkv) return;
   const int cnt = p.col_cnt[tile_id];
   if (cnt == 0) return;
   const int group = p.hq / p.hkv;

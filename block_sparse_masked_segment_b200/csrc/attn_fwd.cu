@@ -58,10 +58,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   FwdSmem<D>& sm = *reinterpret_cast<FwdSmem<D>*>(align1024(smem_raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int head = blockIdx.x % p.hq;
-  const int item = blockIdx.x / p.hq;
-  if (item >= p.n_items) return;
-  const int tile_id = p.sched[item];
+  // head-major grid: the CTAs that run together share one kv head's K/V tiles in L2
+  const int head = blockIdx.x / p.n_items;
+  const int tile_id = p.sched[blockIdx.x % p.n_items];
+  if (head >= p.hq) return;
   const int n = p.row_cnt[tile_id];
   if (n == 0) return;  // tile past the end of its sequence
   const int s = tile_id / p.T, I = tile_id % p.T;
@@ -372,11 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   FwdPairSmem<D>& sm = *reinterpret_cast<FwdPairSmem<D>*>(align1024(smem_raw));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int npairs = p.hq / 2;
-  const int pair = blockIdx.x % npairs;
-  const int item = blockIdx.x / npairs;
-  if (item >= p.n_items) return;
-  const int tile_id = p.sched[item];
+  // pair-major grid: the CTAs that run together share one kv head's K/V tiles in L2
+  const int pair = blockIdx.x / p.n_items;
+  const int tile_id = p.sched[blockIdx.x % p.n_items];
+  if (pair >= p.hq / 2) return;
   const int n = p.row_cnt[tile_id];
   if (n == 0) return;
   const int s = tile_id / p.T, I = tile_id % p.T;

@@ -257,11 +257,14 @@ __global__ void __launch_bounds__(128) tile_meta_kernel(const int32_t* __restric
 
 // Single block: order tiles by descending number of non-empty tiles in their
 // row (q_sched) or column (k_sched), ties by index, so the longest work
-// items start first.  Bitonic sort in shared memory; above kMaxSort items the
-// natural order is kept.
+// items start first.  With by_seq the tiles are first grouped by sequence
+// (k_sched): the dkdv CTAs that run at the same time then stream the query
+// tiles of one sequence, which stay in L2.  Bitonic sort in shared memory;
+// above kMaxSort items the natural order is kept.
 constexpr int kMaxSort = 8192;
 
-__global__ void __launch_bounds__(1024) sched_kernel(const int32_t* __restrict__ cnt, int32_t n, int32_t* __restrict__ order) {
+__global__ void __launch_bounds__(1024) sched_kernel(const int32_t* __restrict__ cnt, int32_t n, int32_t T,
+                                                    int32_t by_seq, int32_t* __restrict__ order) {
   extern __shared__ unsigned long long keys[];
   if (n > kMaxSort) {
     for (int i = threadIdx.x; i < n; i += blockDim.x) order[i] = i;
@@ -270,7 +273,8 @@ __global__ void __launch_bounds__(1024) sched_kernel(const int32_t* __restrict__
   int np = 1;
   while (np < n) np <<= 1;
   for (int i = threadIdx.x; i < np; i += blockDim.x)
-    keys[i] = (i < n) ? ((static_cast<unsigned long long>(cnt[i]) << 32) | (0xFFFFFFFFull - static_cast<unsigned>(i)))
+    keys[i] = (i < n) ? ((by_seq ? static_cast<unsigned long long>(0xFFFFu - static_cast<unsigned>(i / T)) << 48 : 0ull) |
+                         (static_cast<unsigned long long>(cnt[i]) << 32) | (0xFFFFFFFFull - static_cast<unsigned>(i)))
                       : 0ull;
   __syncthreads();
   for (int k = 2; k <= np; k <<= 1) {
@@ -338,9 +342,9 @@ cudaError_t launch_layout(const int32_t* turn_lens, const int32_t* conv_turn_ptr
                            static_cast<int>(sizeof(unsigned long long) * kMaxSort));
       attr_set = true;
     }
-    sched_kernel<<<1, 1024, smem, stream>>>(ws_ptr<int32_t>(ws, w.row_cnt), w.n_tiles,
+    sched_kernel<<<1, 1024, smem, stream>>>(ws_ptr<int32_t>(ws, w.row_cnt), w.n_tiles, w.T, 0,
                                             ws_ptr<int32_t>(ws, w.q_sched));
-    sched_kernel<<<1, 1024, smem, stream>>>(ws_ptr<int32_t>(ws, w.col_cnt), w.n_tiles,
+    sched_kernel<<<1, 1024, smem, stream>>>(ws_ptr<int32_t>(ws, w.col_cnt), w.n_tiles, w.T, 1,
                                             ws_ptr<int32_t>(ws, w.k_sched));
   }
   return cudaGetLastError();
