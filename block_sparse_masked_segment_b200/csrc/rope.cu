@@ -7,7 +7,8 @@
 // pair (x[j], x[j + d/2]) rotated by pos * base^(-2j/d).
 //
 // One thread per (token, j < d/2): the angle is formed and reduced in fp64 once
-// and applied to every head of the token.  HBM-bound: each element is read and
+// and applied to every head of the token (general form; aligned tensors with
+// d/2 a multiple of 8 take the vectorised form below).  HBM-bound: each element is read and
 // written once.  Input and output types may differ (bf16 in, fp16 out for the
 // rotated q and k; in place when they are the same buffer and type); an fp16
 // output value beyond the fp16 range sets OPR_DEV_FP16_RANGE.
@@ -15,6 +16,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <cstdint>
 #include <type_traits>
 
 #include "opr_internal.cuh"
@@ -80,9 +82,95 @@ __global__ void __launch_bounds__(256) rope_kernel(const TI* x, TO* y, const int
   if (out_of_range && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
+// Eight consecutive elements as floats, with 16-byte accesses (the element
+// offset is a multiple of 8 and the tensor 16-byte aligned).
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]) {
+  if constexpr (std::is_same_v<T, float>) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = to_f(e[k]);
+  }
+}
+template <typename T>
+__device__ __forceinline__ void store8(T* p, const float (&v)[8]) {
+  if constexpr (std::is_same_v<T, float>) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint4 u;
+    T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) e[k] = from_f<T>(v[k]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+}
+
+// Vectorised form for 16-byte aligned tensors with d/2 a multiple of 8: a block
+// takes kRopeTok tokens, forms their cos/sin once in shared memory (fp64 angle
+// as above), and each thread rotates eight consecutive pairs (j .. j+7 with
+// j+d/2 .. j+d/2+7) of one head; consecutive threads take consecutive chunks,
+// so a warp reads and writes whole 128-byte lines.
+constexpr int kRopeTok = 8;
+
+template <typename TI, typename TO>
+__global__ void __launch_bounds__(256) rope_vec_kernel(const TI* x, TO* y, const int32_t* __restrict__ pos_id,
+                                                       int64_t total, int32_t n_heads, int32_t half,
+                                                       double neg_log_base_over_half, double sign,
+                                                       int32_t* __restrict__ dev_status) {
+  extern __shared__ float2 cs[];  // [kRopeTok][half]: (cos, sin)
+  const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRopeTok;
+  const int ntok = static_cast<int>(total - tok0 < kRopeTok ? total - tok0 : kRopeTok);
+  for (int i = threadIdx.x; i < ntok * half; i += blockDim.x) {
+    const int t = i / half, j = i % half;
+    const double theta = exp(static_cast<double>(j) * neg_log_base_over_half);
+    const double ang = sign * static_cast<double>(pos_id[tok0 + t]) * theta;
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    cs[i] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
+  }
+  __syncthreads();
+  const int chunks = half / 8;
+  const int items = ntok * n_heads * chunks;
+  bool out_of_range = false;
+  for (int it = threadIdx.x; it < items; it += blockDim.x) {
+    const int c = it % chunks, th = it / chunks;
+    const int h = th % n_heads, t = th / n_heads;
+    const int64_t o = ((tok0 + t) * n_heads + h) * static_cast<int64_t>(2 * half) + 8 * c;
+    float a[8], b[8], ya[8], yb[8];
+    load8(x + o, a);
+    load8(x + o + half, b);
+    const float2* w = cs + t * half + 8 * c;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 cw = w[k];
+      ya[k] = a[k] * cw.x - b[k] * cw.y;
+      yb[k] = b[k] * cw.x + a[k] * cw.y;
+      if constexpr (sizeof(TO) == 2 && !std::is_same_v<TO, __nv_bfloat16>)
+        out_of_range |= !(fabsf(ya[k]) <= 65504.f) || !(fabsf(yb[k]) <= 65504.f);
+    }
+    store8(y + o, ya);
+    store8(y + o + half, yb);
+  }
+  if (out_of_range && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
+}
+
 template <typename TI, typename TO>
 cudaError_t launch_t(const void* x, void* y, const int32_t* pos_id, int64_t total, int32_t n_heads, int32_t half,
                      double nl, double sign, int32_t* dev_status, cudaStream_t stream) {
+  const bool vec = half % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(y) & 15u) == 0;
+  if (vec) {
+    const int64_t blocks = (total + kRopeTok - 1) / kRopeTok;
+    const size_t smem = sizeof(float2) * kRopeTok * half;
+    rope_vec_kernel<TI, TO><<<static_cast<unsigned>(blocks), 256, smem, stream>>>(
+        static_cast<const TI*>(x), static_cast<TO*>(y), pos_id, total, n_heads, half, nl, sign, dev_status);
+    return cudaGetLastError();
+  }
   const int threads = 256 / half * half;
   const int tpb = threads / half;
   const int64_t blocks = (total + tpb - 1) / tpb;

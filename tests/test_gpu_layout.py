@@ -129,6 +129,24 @@ def test_rope_parity(in_dtype, out_dtype, d):
     assert opr.read_status(lay.dev_status) == []
 
 
+@pytest.mark.parametrize("d,offset", [(40, 0), (128, 1)])
+def test_rope_general_form(d, offset):
+    """Shapes the vectorised kernel does not take: d/2 not a multiple of 8, or a tensor off 16-byte alignment."""
+    w = synth.make_workload(1)
+    ref_lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    lay = opr.opr_build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    rng = np.random.default_rng(1)
+    x = synth.round_bf16(rng.standard_normal((lay.total, 3, d)).astype(np.float32))
+    buf = torch.empty(x.size + offset, dtype=torch.bfloat16, device="cuda")
+    xd = buf[offset:].view(x.shape)
+    xd.copy_(torch.from_numpy(x).to("cuda", torch.bfloat16))
+    assert (xd.data_ptr() % 16 != 0) == (offset != 0)
+    opr.opr_rope(xd, lay.pos_id, 1e6)
+    ref = orc.rope(x, ref_lay.pos_id, 1e6)
+    got = xd.float().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 2e-6)
+
+
 def test_rope_fp16_overflow_is_flagged():
     lay = opr.opr_build_layout([[4, 0, 0]], [0, 1], [0, 1])
     x = torch.full((4, 1, 64), 1e5, dtype=torch.bfloat16, device="cuda")
