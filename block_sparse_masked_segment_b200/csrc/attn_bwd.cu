@@ -41,64 +41,68 @@ constexpr float kLog2e = 1.4426950408889634f;
 // kernel also writes dout16, the fp16 copy of dO that the dkdv kernel reads
 // (bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]; a larger one sets
 // OPR_DEV_FP16_RANGE).
-// One block of 128 threads per (tile, head), one token per thread.
 __device__ __forceinline__ bool fp16_range_ok(float x) { return fabsf(x) <= 65504.f; }
 
+// One block of 256 threads per (tile, head); each warp walks 16 of the tile's
+// tokens, one token row per step with the whole warp (lane l holds elements
+// [l D/32, (l+1) D/32) of the row), so every access is a full coalesced row.
 template <int D, typename OT>
-__global__ void __launch_bounds__(128) row_terms_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+__global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                                                         const float* __restrict__ lse, const int32_t* __restrict__ cu_seqlens,
                                                         int64_t total, int32_t hq, int32_t T, float* __restrict__ d_tiles,
                                                         float* __restrict__ lse2_tiles, __half* __restrict__ dout16,
                                                         int32_t* __restrict__ dev_status) {
-  const int tile = blockIdx.x, h = blockIdx.y, c = threadIdx.x;
+  constexpr int kE = D / 32;  // elements per lane: 4 (D = 128) or 2 (D = 64)
+  const int tile = blockIdx.x, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = tile / T, J = tile % T;
   const int seq0 = cu_seqlens[s];
   const int L = cu_seqlens[s + 1] - seq0;
-  const size_t out = (static_cast<size_t>(h) * gridDim.x + tile) * kTile + c;
-  if (J * kTile + c >= L) {
-    d_tiles[out] = 0.f;
-    lse2_tiles[out] = -INFINITY;
-    return;
-  }
-  const int64_t tok = seq0 + J * kTile + c;
-  const size_t base = (static_cast<size_t>(tok) * hq + h) * D;
-  const uint4* dp = reinterpret_cast<const uint4*>(dout + base);
-  uint4* d16 = reinterpret_cast<uint4*>(dout16 + base);
-  float acc = 0.f;
   bool in_range = true;
-#pragma unroll 4
-  for (int x = 0; x < D / 8; ++x) {
-    const uint4 dv = dp[x];
-    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
-    float ov[8], df[8];
-#pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      df[2 * y] = __low2float(d2[y]);
-      df[2 * y + 1] = __high2float(d2[y]);
+  for (int i = 0; i < kTile / 8; ++i) {
+    const int c = warp * (kTile / 8) + i;
+    const size_t out = (static_cast<size_t>(h) * gridDim.x + tile) * kTile + c;
+    if (J * kTile + c >= L) {
+      if (lane == 0) {
+        d_tiles[out] = 0.f;
+        lse2_tiles[out] = -INFINITY;
+      }
+      continue;
+    }
+    const int64_t tok = seq0 + J * kTile + c;
+    const size_t base = (static_cast<size_t>(tok) * hq + h) * D + lane * kE;
+    float df[kE], ov[kE];
+    if constexpr (kE == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(dout + base);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+      df[0] = __low2float(d2[0]); df[1] = __high2float(d2[0]); df[2] = __low2float(d2[1]); df[3] = __high2float(d2[1]);
+      *reinterpret_cast<uint2*>(dout16 + base) = make_uint2(pack_f16x2(df[0], df[1]), pack_f16x2(df[2], df[3]));
+    } else {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(dout + base);
+      const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(&u);
+      df[0] = __low2float(d2); df[1] = __high2float(d2);
+      *reinterpret_cast<uint32_t*>(dout16 + base) = pack_f16x2(df[0], df[1]);
     }
     if constexpr (sizeof(OT) == 4) {
-      const float4* op = reinterpret_cast<const float4*>(o + base) + 2 * x;
-      const float4 a = op[0], b = op[1];
-      ov[0] = a.x; ov[1] = a.y; ov[2] = a.z; ov[3] = a.w; ov[4] = b.x; ov[5] = b.y; ov[6] = b.z; ov[7] = b.w;
+#pragma unroll
+      for (int k = 0; k < kE; ++k) ov[k] = static_cast<const float*>(o)[base + k];
     } else {
-      const uint4 ou = reinterpret_cast<const uint4*>(o + base)[x];
-      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ou);
 #pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        ov[2 * y] = __low2float(o2[y]);
-        ov[2 * y + 1] = __high2float(o2[y]);
-      }
+      for (int k = 0; k < kE; ++k) ov[k] = __bfloat162float(o[base + k]);
+    }
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < kE; ++k) {
+      acc = fmaf(ov[k], df[k], acc);
+      in_range &= fp16_range_ok(df[k]);
     }
 #pragma unroll
-    for (int y = 0; y < 8; ++y) {
-      acc = fmaf(ov[y], df[y], acc);
-      in_range &= fp16_range_ok(df[y]);
+    for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (lane == 0) {
+      d_tiles[out] = -acc;
+      lse2_tiles[out] = -lse[static_cast<size_t>(h) * total + tok] * kLog2e;
     }
-    d16[x] = make_uint4(pack_f16x2(df[0], df[1]), pack_f16x2(df[2], df[3]), pack_f16x2(df[4], df[5]),
-                        pack_f16x2(df[6], df[7]));
   }
-  d_tiles[out] = -acc;
-  lse2_tiles[out] = -lse[static_cast<size_t>(h) * total + tok] * kLog2e;
   if (!in_range) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
@@ -779,11 +783,11 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
     float* row_d = b.row_terms;
     float* row_l = b.row_terms + static_cast<size_t>(pq.hq) * pq.n_items * kTile;
     if (b.o_fp32)
-      row_terms_kernel<D, float><<<grid, kTile, 0, stream>>>(static_cast<const float*>(b.o), b.dout, pq.lse_in,
+      row_terms_kernel<D, float><<<grid, 256, 0, stream>>>(static_cast<const float*>(b.o), b.dout, pq.lse_in,
                                                                pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d, row_l,
                                                                b.dout16, pq.dev_status);
     else
-      row_terms_kernel<D, __nv_bfloat16><<<grid, kTile, 0, stream>>>(
+      row_terms_kernel<D, __nv_bfloat16><<<grid, 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(b.o), b.dout, pq.lse_in, pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d,
           row_l, b.dout16, pq.dev_status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
