@@ -21,9 +21,14 @@ evaluated densely and slowly in float64 with numpy:
 * ``npass_rows``     the N-pass baseline: one causal run per turn over
   [h_1 r_1 ... h_{i-1} r_{i-1} h_i t_i r_i] with contiguous positions
   ("问题背景" and "理论保证" / Theorem 2.1).
+* ``duplication_index`` / ``gather_rows`` / ``fold_rows``
+                     the step before the attention layer: the one-pass token
+                     stream as copies of the original (h, t, r per turn) stream,
+                     and the gradient of that copy, which sums the gradients of
+                     r^in and r^out into their original token ("Token 复制").
 
 Pins (checked by the tests that do not need a GPU): a hand-derived worked
-example of positions and visibility, closed-form visible-pair counts per turn,
+example of positions, visibility and the duplication map, closed-form visible-pair counts per turn,
 Theorem 2.1 by brute force (one-pass rows equal N-pass rows to 1e-12),
 PyTorch's float64 causal scaled_dot_product_attention for the single-segment
 case, RoPE invariants, and central finite differences for every gradient.
@@ -420,3 +425,48 @@ def visible_pairs(lay: Layout) -> int:
         for q in range(a, b):
             n += int(mask_row(lay, q, a, q + 1).sum())
     return n
+
+
+# --------------------------------------------------------------------------
+# Token duplication ("Token 复制"): the step before the attention layer.
+#
+# The original stream holds each conversation's turns once, h_i t_i r_i, and
+# conversations back to back in index order; the one-pass stream holds
+# h_i t_i r_i^in r_i^out.  Every one-pass token is a copy of one original token.
+
+def duplication_index(turn_lens, conv_turn_ptr):
+    """(src, copies): src[i] = original index of one-pass token i; copies[o] = the
+    one-pass positions of original token o as [first, second], second = -1 for
+    h and t tokens (one copy) and the r^out position for r tokens (two copies)."""
+    turn_lens = np.asarray(turn_lens, dtype=np.int64).reshape(-1, 3)
+    conv_turn_ptr = np.asarray(conv_turn_ptr, dtype=np.int64)
+    src, copies = [], []
+    one_pass = 0
+    orig = 0
+    for c in range(len(conv_turn_ptr) - 1):
+        for t in range(conv_turn_ptr[c], conv_turn_ptr[c + 1]):
+            h, tt, r = (int(x) for x in turn_lens[t])
+            h_orig, t_orig, r_orig = orig, orig + h, orig + h + tt
+            h_one, t_one, rin_one, rout_one = one_pass, one_pass + h, one_pass + h + tt, one_pass + h + tt + r
+            src += list(range(h_orig, h_orig + h)) + list(range(t_orig, t_orig + tt))
+            src += list(range(r_orig, r_orig + r)) + list(range(r_orig, r_orig + r))
+            copies += [[h_one + x, -1] for x in range(h)] + [[t_one + x, -1] for x in range(tt)]
+            copies += [[rin_one + x, rout_one + x] for x in range(r)]
+            one_pass += h + tt + 2 * r
+            orig += h + tt + r
+    return np.asarray(src, dtype=np.int32), np.asarray(copies, dtype=np.int32).reshape(-1, 2)
+
+
+def gather_rows(x: np.ndarray, src: np.ndarray) -> np.ndarray:
+    """The one-pass stream's rows: row i is a copy of original row src[i]."""
+    return np.stack([x[int(o)] for o in src]) if len(src) else x[:0]
+
+
+def fold_rows(dy: np.ndarray, copies: np.ndarray) -> np.ndarray:
+    """Gradient of gather_rows w.r.t. x, in float32: each original row sums the
+    rows of its copies, first copy plus second copy (r tokens), in that order."""
+    dy = np.asarray(dy, dtype=np.float32)
+    out = np.zeros((len(copies),) + dy.shape[1:], dtype=np.float32)
+    for o, (a, b) in enumerate(copies):
+        out[o] = dy[a] if b < 0 else dy[a] + dy[b]
+    return out
