@@ -360,6 +360,53 @@ def time_e2e(r: Runner, steps: int, warmup: int, barrier):
     return a.elapsed_time(b)
 
 
+# ------------------------------------------------------------------ token duplication
+def time_duplication(w: synth.Workload, device, hbm_gbs: float, hidden: int = 4096, reps: int = 5):
+    """The step before the attention layer at this workload's size: the one-pass map, a gather of
+    bf16 hidden rows (width `hidden`) into the one-pass stream and the fp32 fold of their gradient.
+    HBM-bound; bytes are each launch's algorithmic reads plus writes."""
+    import torch
+
+    import block_sparse_masked_segment_b200 as opr
+
+    src, copies = opr.opr_duplication_index(w.turn_lens, w.conv_turn_ptr, device=device)
+    total, n_orig = src.numel(), copies.shape[0]
+    x = torch.randn(n_orig, hidden, device=device).to(torch.bfloat16)
+    y = torch.empty(total, hidden, device=device, dtype=torch.bfloat16)
+    dy = torch.randn(total, hidden, device=device)
+    dx = torch.empty(n_orig, hidden, device=device)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    t_map = timed(lambda: opr.opr_duplication_index(w.turn_lens, w.conv_turn_ptr, total, n_orig, device=device))
+    t_gather = timed(lambda: opr.opr_gather_rows(x, src, out=y))
+    t_fold = timed(lambda: opr.opr_fold_rows(dy, copies, out=dx))
+    gather_bytes = 2 * total * hidden * 2
+    fold_bytes = total * hidden * 4 + n_orig * hidden * 4
+    status = opr.read_status(src._inputs[2])
+    if status:
+        raise RuntimeError(f"device status after duplication timing: {status}")
+    return {
+        "tokens": {"one_pass": total, "original": n_orig, "hidden": hidden},
+        "index_ms": t_map,
+        "gather_ms": t_gather, "gather_gbs": gather_bytes / (t_gather * 1e-3) / 1e9,
+        "gather_frac_hbm": gather_bytes / (t_gather * 1e-3) / 1e9 / hbm_gbs,
+        "fold_ms": t_fold, "fold_gbs": fold_bytes / (t_fold * 1e-3) / 1e9,
+        "fold_frac_hbm": fold_bytes / (t_fold * 1e-3) / 1e9 / hbm_gbs,
+    }
+
+
 # ------------------------------------------------------------------ oracle timing
 def oracle_sample(w: synth.Workload, target_tokens: int):
     """The first conversation of the workload, cut after the turn that reaches
@@ -505,6 +552,9 @@ def main():
                "mode": "pinned host buffers; copies of steps i-1, i+1 overlap step i on separate streams; "
                        "inputs larger than L2, no flush"}
 
+    _, _, hbm, _ = peaks()
+    duplication = time_duplication(w, device, hbm)
+
     npass = None
     if not args.no_npass:
         nw, _ = synth.npass_workload(w)
@@ -555,6 +605,7 @@ def main():
         "roofline": roofline,
         "e2e": e2e,
         "npass": npass,
+        "next_rows": {"token_duplication": duplication},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": dict(clocks.summary(), remeasured=remeasured),
         "cpu_baseline": cpu,

@@ -18,6 +18,9 @@ from ._abi import (  # noqa: F401
     opr_attn_bwd,
     opr_attn_bwd_stages,
     opr_attn_bwd_noalloc,
+    opr_duplication_index,
+    opr_gather_rows,
+    opr_fold_rows,
     BWD_ROW_TERMS,
     BWD_DQ,
     BWD_DKDV,

@@ -35,6 +35,9 @@ EXPORTED_SYMBOLS = (
     "opr_attn_bwd",
     "opr_attn_bwd_stages",
     "opr_attn_bwd_noalloc",
+    "opr_duplication_index",
+    "opr_gather_rows",
+    "opr_fold_rows",
 )
 
 BWD_ROW_TERMS, BWD_DQ, BWD_DKDV = 1, 2, 4
@@ -70,6 +73,12 @@ def load_library() -> ctypes.CDLL:
     lib.opr_version.argtypes = []
     lib.opr_last_error.restype = ctypes.c_char_p
     lib.opr_last_error.argtypes = []
+    lib.opr_duplication_index.restype = ctypes.c_int
+    lib.opr_duplication_index.argtypes = [P, P, I32, I32, I64, I64, P, P, P, P]
+    lib.opr_gather_rows.restype = ctypes.c_int
+    lib.opr_gather_rows.argtypes = [P, I64, I64, P, I64, P, P, P]
+    lib.opr_fold_rows.restype = ctypes.c_int
+    lib.opr_fold_rows.argtypes = [P, I64, I64, P, I64, P, P, P]
     lib.opr_layout_workspace_bytes.restype = SZ
     lib.opr_layout_workspace_bytes.argtypes = [I32, I32, I32, I64, I32]
     lib.opr_build_layout.restype = I32
@@ -323,3 +332,69 @@ def opr_attn_bwd_noalloc(q, k, v, o, do, lse, lay: Layout, scale: float | None =
         _ptr(lay.dev_status), _stream(q.device))
     _check(st, "opr_attn_bwd_noalloc")
     return dq, dk, dv
+
+
+# ------------------------------------------------------------------ token duplication
+def opr_duplication_index(turn_lens, conv_turn_ptr, total_tokens=None, orig_tokens=None, device="cuda",
+                          dev_status: torch.Tensor | None = None):
+    """(src_index [total], copy_index [orig, 2]) int32 device tensors: the one-pass stream
+    (h, t, r^in, r^out per turn) as copies of the original stream (h, t, r per turn)."""
+    lib = load_library()
+    device = torch.device(device)
+
+    def dev_i32(x):
+        t = x if isinstance(x, torch.Tensor) else torch.as_tensor(np.asarray(x, dtype=np.int32))
+        return t.to(device=device, dtype=torch.int32).contiguous()
+
+    tl, cp = dev_i32(turn_lens).reshape(-1), dev_i32(conv_turn_ptr)
+    if total_tokens is None or orig_tokens is None:
+        lens = np.asarray(turn_lens.cpu() if isinstance(turn_lens, torch.Tensor) else turn_lens,
+                          dtype=np.int64).reshape(-1, 3)
+        lens = np.maximum(lens, 0)
+        total_tokens = int(lens[:, 0].sum() + lens[:, 1].sum() + 2 * lens[:, 2].sum()) \
+            if total_tokens is None else total_tokens
+        orig_tokens = int(lens.sum()) if orig_tokens is None else orig_tokens
+    src = torch.empty(total_tokens, dtype=torch.int32, device=device)
+    copies = torch.empty((orig_tokens, 2), dtype=torch.int32, device=device)
+    status = dev_status if dev_status is not None else torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib.opr_duplication_index(_ptr(tl), _ptr(cp), cp.numel() - 1, tl.numel() // 3, total_tokens, orig_tokens,
+                                     _ptr(src), _ptr(copies), _ptr(status), _stream(device)),
+           "opr_duplication_index")
+    src._inputs = (tl, cp, status)  # keep the device copies alive until the stream has used them
+    return src, copies
+
+
+def opr_gather_rows(x: torch.Tensor, src_index: torch.Tensor, out: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """out[i] = x[src_index[i]] along the first dimension (any dtype, rows contiguous)."""
+    _need_cuda(x, src_index)
+    rows = src_index.numel()
+    if out is None:
+        out = torch.empty((rows,) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
+    _need_cuda(out)
+    if out.shape[0] != rows or out.shape[1:] != x.shape[1:] or out.dtype != x.dtype:
+        raise OprError("opr_gather_rows: out must be [len(src_index)] rows of x's row shape and dtype")
+    row_bytes = x[0].numel() * x.element_size() if x.shape[0] > 0 else out[0].numel() * out.element_size()
+    _check(lib_call("opr_gather_rows", _ptr(x), x.shape[0], row_bytes, _ptr(src_index), rows, _ptr(out),
+                    _ptr(dev_status) if dev_status is not None else None, _stream(x.device)), "opr_gather_rows")
+    return out
+
+
+def opr_fold_rows(dy: torch.Tensor, copy_index: torch.Tensor, out: torch.Tensor | None = None,
+                  dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """Gradient of opr_gather_rows: out[o] = dy[copy_index[o, 0]] + dy[copy_index[o, 1]] (fp32)."""
+    _need_cuda(dy, copy_index)
+    if dy.dtype != torch.float32:
+        raise OprError("opr_fold_rows: dy must be fp32")
+    rows = copy_index.shape[0]
+    if out is None:
+        out = torch.empty((rows,) + tuple(dy.shape[1:]), dtype=torch.float32, device=dy.device)
+    _need_cuda(out)
+    width = int(np.prod(dy.shape[1:])) if dy.dim() > 1 else 1
+    _check(lib_call("opr_fold_rows", _ptr(dy), dy.shape[0], width, _ptr(copy_index), rows, _ptr(out),
+                    _ptr(dev_status) if dev_status is not None else None, _stream(dy.device)), "opr_fold_rows")
+    return out
+
+
+def lib_call(name: str, *args) -> int:
+    return int(getattr(load_library(), name)(*args))

@@ -14,6 +14,13 @@ cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, const CUtensorMap& tq, co
                             const CUtensorMap& tv, const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const BwdMaps& m, const BwdBuffers& b, const AttnParams& pq,
                             const AttnParams& pkv, int stages, cudaStream_t stream);
+cudaError_t launch_dup_index(const int32_t* turn_lens, const int32_t* conv_turn_ptr, int32_t n_convs, int32_t n_turns,
+                             int64_t total, int64_t orig_total, int32_t* src_index, int32_t* copy_index,
+                             int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_gather_rows(const void* x, int64_t orig_total, int64_t row_bytes, const int32_t* src_index,
+                               int64_t total, void* y, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_fold_rows(const float* dy, int64_t total, int64_t width, const int32_t* copy_index,
+                             int64_t orig_total, float* dx, int32_t* dev_status, cudaStream_t stream);
 
 namespace {
 
@@ -125,6 +132,42 @@ bool attn_args_ok(const void* q, const void* k, const void* v, int32_t hq, int32
 using namespace opr;
 
 extern "C" {
+
+opr_status opr_duplication_index(const int32_t* turn_lens, const int32_t* conv_turn_ptr, int32_t n_convs,
+                                 int32_t n_turns, int64_t total_tokens, int64_t orig_tokens, int32_t* src_index,
+                                 int32_t* copy_index, int32_t* dev_status, void* stream) {
+  if (n_convs < 0 || n_turns < 0 || total_tokens < 0 || orig_tokens < 0) return OPR_INVALID_ARG;
+  if (total_tokens >= (int64_t{1} << 31) || orig_tokens > total_tokens) return OPR_INVALID_ARG;
+  if (!conv_turn_ptr || !dev_status || (n_turns > 0 && !turn_lens) || (total_tokens > 0 && !src_index) ||
+      (orig_tokens > 0 && !copy_index))
+    return OPR_INVALID_ARG;
+  const opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  return status_of(launch_dup_index(turn_lens, conv_turn_ptr, n_convs, n_turns, total_tokens, orig_tokens, src_index,
+                                    copy_index, dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+opr_status opr_gather_rows(const void* x, int64_t orig_tokens, int64_t row_bytes, const int32_t* src_index,
+                           int64_t total_tokens, void* y, int32_t* dev_status, void* stream) {
+  if (orig_tokens < 0 || total_tokens < 0 || row_bytes <= 0) return OPR_INVALID_ARG;
+  if (total_tokens == 0) return OPR_OK;
+  if (!x || !src_index || !y) return OPR_INVALID_ARG;
+  const opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  return status_of(launch_gather_rows(x, orig_tokens, row_bytes, src_index, total_tokens, y, dev_status,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+opr_status opr_fold_rows(const float* dy, int64_t total_tokens, int64_t width, const int32_t* copy_index,
+                         int64_t orig_tokens, float* dx, int32_t* dev_status, void* stream) {
+  if (orig_tokens < 0 || total_tokens < 0 || width <= 0) return OPR_INVALID_ARG;
+  if (orig_tokens == 0) return OPR_OK;
+  if (!dy || !copy_index || !dx) return OPR_INVALID_ARG;
+  const opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  return status_of(launch_fold_rows(dy, total_tokens, width, copy_index, orig_tokens, dx, dev_status,
+                                    static_cast<cudaStream_t>(stream)));
+}
 
 const char* opr_version(void) { return "opr 0.1.0 sm_100a"; }
 

@@ -1,0 +1,250 @@
+// duplicate.cu - the step before the attention layer: token duplication.
+//
+// One-Pass to Reason wiki note, "Token 复制": each response r_i is stored
+// twice, as r_i^in (the context copy) and r_i^out (the copy that is trained
+// on), so the one-pass stream of a turn is h_i t_i r_i^in r_i^out while the
+// original stream holds h_i t_i r_i once.  Conversations follow each other in
+// index order in both streams.
+//
+//   dup_index_kernel   the map between the streams: src_index[i] = original
+//                      token of one-pass token i; copy_index[o] = the one-pass
+//                      positions of original token o (second = -1 for h, t);
+//   gather_rows_kernel one-pass rows as copies of original rows (token ids,
+//                      embeddings or any fixed-width row);
+//   fold_rows_kernel   the gradient of that copy: each original row sums its
+//                      copies' rows, first + second, in fp32.  A gather over
+//                      copy_index, so no atomics and the sum order is fixed.
+#include <cuda_runtime.h>
+
+#include "opr_internal.cuh"
+
+namespace opr {
+namespace {
+
+constexpr int kDupThreads = 1024;
+
+// Single block.  Turns are taken kDupThreads at a time: one thread per turn
+// loads (h, t, r), a block scan turns them into the turns' offsets in both
+// streams, then the whole block writes the indices of those turns' tokens.
+// Every write is bounds-checked against the sizes the caller gave; a total
+// that disagrees with the lengths sets OPR_DEV_TOTAL_MISMATCH.
+__global__ void __launch_bounds__(kDupThreads) dup_index_kernel(const int32_t* __restrict__ turn_lens,
+                                                                 const int32_t* __restrict__ conv_turn_ptr,
+                                                                 int32_t n_convs, int32_t n_turns, int64_t total,
+                                                                 int64_t orig_total, int32_t* __restrict__ src_index,
+                                                                 int32_t* __restrict__ copy_index,
+                                                                 int32_t* __restrict__ dev_status) {
+  __shared__ int64_t one_off[kDupThreads], orig_off[kDupThreads];
+  __shared__ int32_t lens[kDupThreads][3];
+  __shared__ int64_t warp_one[32], warp_orig[32];
+  __shared__ int64_t carry_one, carry_orig;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    carry_one = 0;
+    carry_orig = 0;
+    if (conv_turn_ptr[0] != 0 || conv_turn_ptr[n_convs] != n_turns) atomicOr(dev_status, OPR_DEV_BAD_INPUT);
+  }
+  __syncthreads();
+  bool bad = false;
+  for (int base = 0; base < n_turns; base += kDupThreads) {
+    const int t = base + tid;
+    int h = 0, tt = 0, r = 0;
+    if (t < n_turns) {
+      h = turn_lens[3 * t];
+      tt = turn_lens[3 * t + 1];
+      r = turn_lens[3 * t + 2];
+      if (h < 0 || tt < 0 || r < 0) bad = true;
+      h = max(h, 0);
+      tt = max(tt, 0);
+      r = max(r, 0);
+    }
+    lens[tid][0] = h;
+    lens[tid][1] = tt;
+    lens[tid][2] = r;
+    // inclusive warp scans of both streams' token counts, then across warps
+    int64_t a = static_cast<int64_t>(h) + tt + 2 * static_cast<int64_t>(r);
+    int64_t b = static_cast<int64_t>(h) + tt + r;
+    int64_t ia = a, ib = b;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int64_t ya = __shfl_up_sync(0xffffffffu, ia, d), yb = __shfl_up_sync(0xffffffffu, ib, d);
+      if (lane >= d) {
+        ia += ya;
+        ib += yb;
+      }
+    }
+    if (lane == 31) {
+      warp_one[warp] = ia;
+      warp_orig[warp] = ib;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int64_t wa = warp_one[lane], wb = warp_orig[lane];
+      int64_t xa = wa, xb = wb;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int64_t ya = __shfl_up_sync(0xffffffffu, xa, d), yb = __shfl_up_sync(0xffffffffu, xb, d);
+        if (lane >= d) {
+          xa += ya;
+          xb += yb;
+        }
+      }
+      warp_one[lane] = xa - wa;  // exclusive warp offsets
+      warp_orig[lane] = xb - wb;
+    }
+    __syncthreads();
+    const int64_t c1 = carry_one, c2 = carry_orig;
+    one_off[tid] = c1 + warp_one[warp] + ia - a;
+    orig_off[tid] = c2 + warp_orig[warp] + ib - b;
+    __syncthreads();
+    if (tid == kDupThreads - 1) {
+      carry_one = c1 + warp_one[warp] + ia;
+      carry_orig = c2 + warp_orig[warp] + ib;
+    }
+    // the tokens of this chunk's turns, one turn after another, the block across each turn
+    const int nt = min(kDupThreads, n_turns - base);
+    for (int u = 0; u < nt; ++u) {
+      const int hu = lens[u][0], tu = lens[u][1], ru = lens[u][2];
+      const int64_t o1 = one_off[u], o2 = orig_off[u];
+      const int n = hu + tu + 2 * ru;
+      for (int x = tid; x < n; x += kDupThreads) {
+        const int64_t i = o1 + x;
+        const int xo = x < hu + tu + ru ? x : x - ru;  // r^out copies r^in's originals
+        const int64_t o = o2 + xo;
+        if (i < total && o < orig_total) src_index[i] = static_cast<int32_t>(o);
+        if (x < hu + tu + ru && o < orig_total) {
+          const bool is_r = x >= hu + tu;
+          const int64_t second = is_r ? i + ru : -1;
+          copy_index[2 * o] = i < total ? static_cast<int32_t>(i) : -1;
+          copy_index[2 * o + 1] = (is_r && second < total) ? static_cast<int32_t>(second) : -1;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (bad) atomicOr(dev_status, OPR_DEV_BAD_INPUT);
+  if (tid == 0 && (carry_one != total || carry_orig != orig_total)) atomicOr(dev_status, OPR_DEV_TOTAL_MISMATCH);
+}
+
+// y[i] = x[src_index[i]], rows of row_units units of type U (16, 4 or 1 bytes).
+// Wide rows: one warp per row, lanes across the row (coalesced); narrow rows
+// (fewer than 32 units): one thread per row.
+template <typename U>
+__global__ void __launch_bounds__(256) gather_rows_kernel(const U* __restrict__ x, int64_t orig_total,
+                                                          int64_t row_units, const int32_t* __restrict__ src_index,
+                                                          int64_t total, U* __restrict__ y,
+                                                          int32_t* __restrict__ dev_status) {
+  const bool wide = row_units >= 32;
+  const int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t first = wide ? gid / 32 : gid, step = wide ? stride / 32 : stride;
+  const int64_t c0 = wide ? (threadIdx.x & 31) : 0, cs = wide ? 32 : 1;
+  bool bad = false;
+  for (int64_t i = first; i < total; i += step) {
+    const int32_t o = src_index[i];
+    if (o < 0 || o >= orig_total) {
+      bad = true;
+      continue;
+    }
+    const U* src = x + static_cast<int64_t>(o) * row_units;
+    U* dst = y + i * row_units;
+    for (int64_t c = c0; c < row_units; c += cs) dst[c] = src[c];
+  }
+  if (bad && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_BAD_INPUT);
+}
+
+// dx[o] = dy[first] + dy[second] (or dy[first] alone), V = float4 or float;
+// rows spread over warps or threads as in gather_rows_kernel.
+template <typename V>
+__device__ __forceinline__ V add_v(V a, V b);
+template <>
+__device__ __forceinline__ float add_v<float>(float a, float b) {
+  return a + b;
+}
+template <>
+__device__ __forceinline__ float4 add_v<float4>(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+template <typename V>
+__global__ void __launch_bounds__(256) fold_rows_kernel(const V* __restrict__ dy, int64_t total, int64_t row_units,
+                                                        const int32_t* __restrict__ copy_index, int64_t orig_total,
+                                                        V* __restrict__ dx, int32_t* __restrict__ dev_status) {
+  const bool wide = row_units >= 32;
+  const int64_t gid = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t first = wide ? gid / 32 : gid, step = wide ? stride / 32 : stride;
+  const int64_t c0 = wide ? (threadIdx.x & 31) : 0, cs = wide ? 32 : 1;
+  bool bad = false;
+  for (int64_t o = first; o < orig_total; o += step) {
+    const int32_t a = copy_index[2 * o], b = copy_index[2 * o + 1];
+    if (a < 0 || a >= total || b >= total) {
+      bad = true;
+      continue;
+    }
+    const V* ra = dy + static_cast<int64_t>(a) * row_units;
+    V* dst = dx + o * row_units;
+    if (b < 0) {
+      for (int64_t c = c0; c < row_units; c += cs) dst[c] = ra[c];
+    } else {
+      const V* rb = dy + static_cast<int64_t>(b) * row_units;
+      for (int64_t c = c0; c < row_units; c += cs) dst[c] = add_v(ra[c], rb[c]);
+    }
+  }
+  if (bad && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_BAD_INPUT);
+}
+
+// Blocks for `rows` rows of `units` units: a warp per wide row, a thread per narrow one;
+// at most 148 SMs x 16 blocks (grid-stride beyond).
+int64_t grid_for(int64_t rows, int64_t units) {
+  const int64_t threads = units >= 32 ? rows * 32 : rows;
+  const int64_t blocks = (threads + 255) / 256;
+  return blocks < 148 * 16 ? (blocks > 0 ? blocks : 1) : 148 * 16;
+}
+
+}  // namespace
+
+cudaError_t launch_dup_index(const int32_t* turn_lens, const int32_t* conv_turn_ptr, int32_t n_convs, int32_t n_turns,
+                             int64_t total, int64_t orig_total, int32_t* src_index, int32_t* copy_index,
+                             int32_t* dev_status, cudaStream_t stream) {
+  dup_index_kernel<<<1, kDupThreads, 0, stream>>>(turn_lens, conv_turn_ptr, n_convs, n_turns, total, orig_total,
+                                                  src_index, copy_index, dev_status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* x, int64_t orig_total, int64_t row_bytes, const int32_t* src_index,
+                               int64_t total, void* y, int32_t* dev_status, cudaStream_t stream) {
+  const bool a16 = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (reinterpret_cast<uintptr_t>(y) % 16 == 0);
+  const bool a4 = (reinterpret_cast<uintptr_t>(x) % 4 == 0) && (reinterpret_cast<uintptr_t>(y) % 4 == 0);
+  if (row_bytes % 16 == 0 && a16) {
+    const int64_t u = row_bytes / 16;
+    gather_rows_kernel<uint4><<<static_cast<unsigned>(grid_for(total, u)), 256, 0, stream>>>(
+        static_cast<const uint4*>(x), orig_total, u, src_index, total, static_cast<uint4*>(y), dev_status);
+  } else if (row_bytes % 4 == 0 && a4) {
+    const int64_t u = row_bytes / 4;
+    gather_rows_kernel<uint32_t><<<static_cast<unsigned>(grid_for(total, u)), 256, 0, stream>>>(
+        static_cast<const uint32_t*>(x), orig_total, u, src_index, total, static_cast<uint32_t*>(y), dev_status);
+  } else {
+    gather_rows_kernel<uint8_t><<<static_cast<unsigned>(grid_for(total, row_bytes)), 256, 0, stream>>>(
+        static_cast<const uint8_t*>(x), orig_total, row_bytes, src_index, total, static_cast<uint8_t*>(y),
+        dev_status);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fold_rows(const float* dy, int64_t total, int64_t width, const int32_t* copy_index,
+                             int64_t orig_total, float* dx, int32_t* dev_status, cudaStream_t stream) {
+  const bool a16 = (reinterpret_cast<uintptr_t>(dy) % 16 == 0) && (reinterpret_cast<uintptr_t>(dx) % 16 == 0);
+  if (width % 4 == 0 && a16) {
+    const int64_t u = width / 4;
+    fold_rows_kernel<float4><<<static_cast<unsigned>(grid_for(orig_total, u)), 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(dy), total, u, copy_index, orig_total, reinterpret_cast<float4*>(dx),
+        dev_status);
+  } else {
+    fold_rows_kernel<float><<<static_cast<unsigned>(grid_for(orig_total, width)), 256, 0, stream>>>(
+        dy, total, width, copy_index, orig_total, dx, dev_status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace opr

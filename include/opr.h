@@ -262,6 +262,55 @@ OPR_API opr_status opr_attn_bwd_noalloc(const void* q, const void* k, const void
                                         int32_t* dev_status, void* stream);
 
 /* Library version string, e.g. "opr 0.1.0 sm_100a". */
+/*
+ * Token duplication, the step before the attention layer (One-Pass to Reason
+ * wiki note, "Token 复制"): the one-pass stream of a turn is h, t, r^in,
+ * r^out, the original stream h, t, r, and conversations follow each other in
+ * index order in both.  The map is what a fine-tuning pipeline needs to build
+ * the one-pass input (token ids, or embeddings) from the original one and to
+ * take the gradient back.
+ *
+ * opr_duplication_index - the map between the two streams.
+ *   turn_lens       int32 [n_turns][3] (h, t, r), device, as for opr_build_layout
+ *   conv_turn_ptr   int32 [n_convs + 1], device
+ *   total_tokens    one-pass tokens, sum of h + t + 2r
+ *   orig_tokens     original tokens, sum of h + t + r
+ *   src_index       int32 [total_tokens] out: the original token each one-pass token copies
+ *   copy_index      int32 [orig_tokens][2] out: the one-pass positions of each original
+ *                   token; [o][1] = -1 for h and t tokens, the r^out copy for r tokens
+ *   dev_status      required; OPR_DEV_BAD_INPUT for a negative length or a conversation
+ *                   pointer that does not span the turns, OPR_DEV_TOTAL_MISMATCH when a
+ *                   total disagrees with the lengths (then only in-range entries are written)
+ * One thread block on `stream`.  OPR_INVALID_ARG for negative sizes or null pointers.
+ */
+OPR_API opr_status opr_duplication_index(const int32_t* turn_lens, const int32_t* conv_turn_ptr,
+                                         int32_t n_convs, int32_t n_turns, int64_t total_tokens,
+                                         int64_t orig_tokens, int32_t* src_index, int32_t* copy_index,
+                                         int32_t* dev_status, void* stream);
+
+/*
+ * opr_gather_rows - y[i] = x[src_index[i]] for i < total_tokens, rows of row_bytes bytes
+ * (token ids, embeddings, hidden states: any fixed-width row; 16-byte aligned
+ * tensors with row_bytes % 16 == 0 take 16-byte accesses).
+ *   x  [orig_tokens] rows, device;  y  [total_tokens] rows, device, caller-owned
+ *   dev_status  may be NULL; otherwise OPR_DEV_BAD_INPUT when an index is out of range
+ *               (that row is left unwritten)
+ */
+OPR_API opr_status opr_gather_rows(const void* x, int64_t orig_tokens, int64_t row_bytes,
+                                   const int32_t* src_index, int64_t total_tokens, void* y,
+                                   int32_t* dev_status, void* stream);
+
+/*
+ * opr_fold_rows - the gradient of opr_gather_rows w.r.t. x, fp32 rows of `width` values:
+ * dx[o] = dy[copy_index[o][0]] + dy[copy_index[o][1]], the first copy plus the second in that
+ * order (dy[copy_index[o][0]] alone when the second is -1).  No atomics; deterministic.
+ *   dy  fp32 [total_tokens][width];  dx  fp32 [orig_tokens][width], caller-owned
+ *   dev_status  may be NULL; otherwise OPR_DEV_BAD_INPUT for an out-of-range index
+ */
+OPR_API opr_status opr_fold_rows(const float* dy, int64_t total_tokens, int64_t width,
+                                 const int32_t* copy_index, int64_t orig_tokens, float* dx,
+                                 int32_t* dev_status, void* stream);
+
 OPR_API const char* opr_version(void);
 
 /*

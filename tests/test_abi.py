@@ -94,3 +94,18 @@ def test_npass_workload_is_causal_sequences():
     assert nw.n_seqs == 4 and [i for _, i in origin] == [0, 1, 2, 3]
     # N-pass sequence of turn i: sum_{j<i}(h+r) + h + t + r = 384 i + 896
     np.testing.assert_array_equal(nw.seq_lengths(), [896, 1280, 1664, 2048])
+
+
+def test_duplication_entry_points_check_arguments_on_the_host():
+    """Host-side checks return before any device work (fake pointers are never touched)."""
+    lib = opr.load_library()
+    fake = ctypes.c_void_p(1 << 20)
+    # negative sizes, a null status word, more original tokens than one-pass tokens
+    assert lib.opr_duplication_index(fake, fake, 1, -1, 10, 5, fake, fake, fake, None) == 1
+    assert lib.opr_duplication_index(fake, fake, 1, 2, 10, 5, fake, fake, None, None) == 1
+    assert lib.opr_duplication_index(fake, fake, 1, 2, 10, 11, fake, fake, fake, None) == 1
+    assert lib.opr_gather_rows(fake, 5, 0, fake, 10, fake, None, None) == 1
+    assert lib.opr_gather_rows(None, 5, 16, fake, 10, fake, None, None) == 1
+    assert lib.opr_gather_rows(fake, 5, 16, fake, 0, fake, None, None) == 0  # nothing to copy
+    assert lib.opr_fold_rows(fake, 10, 0, fake, 5, fake, None, None) == 1
+    assert lib.opr_fold_rows(fake, 10, 4, fake, 0, fake, None, None) == 0
