@@ -26,6 +26,9 @@ evaluated densely and slowly in float64 with numpy:
                      stream as copies of the original (h, t, r per turn) stream,
                      and the gradient of that copy, which sums the gradients of
                      r^in and r^out into their original token ("Token 复制").
+* ``kpass_plan`` / ``kpass_index``
+                     the K-pass arrangement ("K-Pass 中间方案"): each pass is a
+                     group of turns behind the history of the earlier turns.
 
 Pins (checked by the tests that do not need a GPU): a hand-derived worked
 example of positions, visibility and the duplication map, closed-form visible-pair counts per turn,
@@ -464,9 +467,98 @@ def gather_rows(x: np.ndarray, src: np.ndarray) -> np.ndarray:
 
 def fold_rows(dy: np.ndarray, copies: np.ndarray) -> np.ndarray:
     """Gradient of gather_rows w.r.t. x, in float32: each original row sums the
-    rows of its copies, first copy plus second copy (r tokens), in that order."""
+    rows of its copies (the non-negative entries of its row of `copies`), in
+    slot order, one float32 addition after another."""
     dy = np.asarray(dy, dtype=np.float32)
     out = np.zeros((len(copies),) + dy.shape[1:], dtype=np.float32)
-    for o, (a, b) in enumerate(copies):
-        out[o] = dy[a] if b < 0 else dy[a] + dy[b]
+    for o, row in enumerate(copies):
+        acc = None
+        for a in row:
+            if a < 0:
+                continue
+            acc = dy[a].copy() if acc is None else (acc + dy[a]).astype(np.float32)
+        out[o] = acc
     return out
+
+
+# --------------------------------------------------------------------------
+# K-pass ("K-Pass 中间方案"): between N-pass (K = N) and one-pass (K = 1).
+#
+# Reading (the pages give only the trade-off): a conversation's N turns are
+# split into K' = min(K, N) contiguous groups, group g holding turns
+# [floor(g N / K'), floor((g + 1) N / K')).  Pass g is one sequence-packed
+# conversation: first the history of the turns before the group, each turn j
+# as h_j followed by r_j in one causal context segment (the turn (h_j + r_j, 0, 0):
+# positions run on from h_j into r_j, exactly as h_j and r_j^in do in one pass),
+# then the group's turns (h, t, r) laid out one-pass.  Every loss row (t and
+# r^out) appears in exactly one pass; K = 1 is the one-pass layout.
+
+def kpass_groups(n: int, K: int):
+    """Turn boundaries b_0 = 0 < ... < b_K' = n of the K' = min(K, n) groups."""
+    k = min(K, n)
+    return [(g * n) // k for g in range(k + 1)] if k > 0 else [0]
+
+
+def kpass_plan(turn_lens, conv_turn_ptr, seq_conv_ptr, K: int):
+    """(turn_lens', conv_turn_ptr', seq_conv_ptr', turn_src): the K-pass
+    arrangement as a workload for the one-pass layout, one conversation per
+    pass, passes of a conversation back to back in its sequence; turn_src[u] =
+    (original turn, pass offset) with pass offset -1 for a turn of the pass's
+    own group and, for a history turn, (pass - group of the turn) >= 1."""
+    turn_lens = np.asarray(turn_lens, dtype=np.int64).reshape(-1, 3)
+    conv_turn_ptr = np.asarray(conv_turn_ptr, dtype=np.int64)
+    seq_conv_ptr = np.asarray(seq_conv_ptr, dtype=np.int64)
+    out_lens, out_conv, out_seq, src = [], [0], [0], []
+    conv_pass0 = []
+    n_out_convs = 0
+    for c in range(len(conv_turn_ptr) - 1):
+        t0, t1 = int(conv_turn_ptr[c]), int(conv_turn_ptr[c + 1])
+        b = kpass_groups(t1 - t0, K)
+        conv_pass0.append(n_out_convs)
+        for g in range(len(b) - 1):
+            for j in range(t0, t0 + b[g]):  # history: h_j then r_j as one context segment
+                h, _, r = (int(x) for x in turn_lens[j])
+                out_lens.append([h + r, 0, 0])
+                gj = next(q for q in range(len(b) - 1) if b[q] <= j - t0 < b[q + 1])
+                src.append([j, g - gj])
+            for j in range(t0 + b[g], t0 + b[g + 1]):
+                out_lens.append([int(x) for x in turn_lens[j]])
+                src.append([j, -1])
+            out_conv.append(len(out_lens))
+            n_out_convs += 1
+    conv_pass0.append(n_out_convs)
+    for s in range(len(seq_conv_ptr) - 1):
+        out_seq.append(conv_pass0[int(seq_conv_ptr[s + 1])])
+    return (np.asarray(out_lens, dtype=np.int32).reshape(-1, 3), np.asarray(out_conv, dtype=np.int32),
+            np.asarray(out_seq, dtype=np.int32), np.asarray(src, dtype=np.int32).reshape(-1, 2))
+
+
+def kpass_index(turn_lens, conv_turn_ptr, seq_conv_ptr, K: int):
+    """(src, copies): src[i] = original token of K-pass token i; copies[o] has K + 1
+    slots: 0 = the copy in the token's own pass (h, t or r^in), 1 = the r^out copy
+    (r tokens), 1 + d = the history copy in the pass d groups later (h and r tokens);
+    -1 where there is none.  The original stream is the one of duplication_index."""
+    turn_lens = np.asarray(turn_lens, dtype=np.int64).reshape(-1, 3)
+    orig_off = np.concatenate([[0], np.cumsum(turn_lens.sum(axis=1))])
+    lens2, _, _, tsrc = kpass_plan(turn_lens, conv_turn_ptr, seq_conv_ptr, K)
+    copies = -np.ones((int(orig_off[-1]), K + 1), dtype=np.int32)
+    src = []
+    pos = 0
+    for (n_h, _, _), (j, d) in zip(lens2, tsrc):
+        h, t, r = (int(x) for x in turn_lens[j])
+        o = int(orig_off[j])
+        if d >= 1:  # history turn: originals of h_j, then of r_j
+            ids = list(range(o, o + h)) + list(range(o + h + t, o + h + t + r))
+            for x, oi in enumerate(ids):
+                src.append(oi)
+                copies[oi, 1 + d] = pos + x
+            pos += len(ids)
+        else:
+            for x in range(h + t + r):
+                src.append(o + x)
+                copies[o + x, 0] = pos + x
+            for x in range(r):
+                src.append(o + h + t + x)
+                copies[o + h + t + x, 1] = pos + h + t + r + x
+            pos += h + t + 2 * r
+    return np.asarray(src, dtype=np.int32), copies
