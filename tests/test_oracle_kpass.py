@@ -95,10 +95,10 @@ def test_planted_history_order_is_caught():
     k_src, k_copies = orc.kpass_index(lens, ptr, seqs, 2)
     bad_src = k_src.copy()
     pos = 0
-    for (n, t, r), (j, dd) in zip(l2, tsrc):
+    for (n, t, r), (j, dd) in zip(l2, tsrc):  # noqa: B007
         n_tok = int(n) + int(t) + 2 * int(r)
         if dd >= 1:
-            h_j = int(lens[3 * j])
+            h_j = int(lens[j][0])
             seg = bad_src[pos:pos + n_tok].copy()
             bad_src[pos:pos + n_tok] = np.concatenate([seg[h_j:], seg[:h_j]])  # r_j first
         pos += n_tok
