@@ -407,6 +407,22 @@ def time_duplication(w: synth.Workload, device, hbm_gbs: float, hidden: int = 40
     }
 
 
+def kpass_workload(w: synth.Workload, K: int, device) -> synth.Workload:
+    """The K-pass arrangement of w, built on the GPU by opr_kpass (plan and token map)."""
+    import torch
+
+    import block_sparse_masked_segment_b200 as opr
+
+    kp = opr.opr_kpass(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, K, device=device)
+    torch.cuda.synchronize()
+    status = opr.read_status(kp.dev_status)
+    if status:
+        raise RuntimeError(f"device status after opr_kpass: {status}")
+    return synth.Workload(turn_lens=kp.turn_lens.cpu().numpy(), conv_turn_ptr=kp.conv_turn_ptr.cpu().numpy(),
+                          seq_conv_ptr=kp.seq_conv_ptr.cpu().numpy(), hq=w.hq, hkv=w.hkv, d=w.d, base=w.base,
+                          name=f"{w.name} [K={K}]")
+
+
 # ------------------------------------------------------------------ oracle timing
 def oracle_sample(w: synth.Workload, target_tokens: int):
     """The first conversation of the workload, cut after the turn that reaches
@@ -555,6 +571,18 @@ def main():
     _, _, hbm, _ = peaks()
     duplication = time_duplication(w, device, hbm)
 
+    # K-pass (K = 2) on the same conversations and kernels: speed and tokens against one-pass
+    kw = kpass_workload(w, 2, device)
+    rk = Runner(kw, seed=11 + rank, device=device)
+    k_ms, _ = time_runner(rk, args.steps, args.warmup, flush, barrier)
+    k_ms = max_over_ranks(k_ms)
+    k_conv_tps = sum_over_ranks(w.conversation_tokens() * args.steps) / (k_ms * 1e-3)
+    kpass = {"K": 2, "tokens_per_step": kw.total_tokens, "tokens_vs_one_pass": kw.total_tokens / w.total_tokens,
+             "ms_per_step": k_ms / args.steps, "conv_tokens_per_s": k_conv_tps,
+             "one_pass_vs_kpass": conv_tps / k_conv_tps}
+    del rk
+    torch.cuda.empty_cache()
+
     npass = None
     if not args.no_npass:
         nw, _ = synth.npass_workload(w)
@@ -568,6 +596,7 @@ def main():
                  "tokens_per_step": nw.total_tokens, "pairs_per_head": rn.pairs,
                  "kernel_ms": {k: statistics.mean(v) for k, v in n_per.items()},
                  "one_pass_speedup": conv_tps / n_conv_tps}
+        kpass["kpass_vs_npass"] = k_conv_tps / n_conv_tps
 
     # roofline of the dominant tensor-core kernel, timed live with CUDA events
     bf16_peak, bf16_sust, hbm, peak_src = peaks()
@@ -605,7 +634,7 @@ def main():
         "roofline": roofline,
         "e2e": e2e,
         "npass": npass,
-        "next_rows": {"token_duplication": duplication},
+        "next_rows": {"token_duplication": duplication, "kpass": kpass},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": dict(clocks.summary(), remeasured=remeasured),
         "cpu_baseline": cpu,

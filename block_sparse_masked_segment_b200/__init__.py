@@ -21,6 +21,8 @@ from ._abi import (  # noqa: F401
     opr_duplication_index,
     opr_gather_rows,
     opr_fold_rows,
+    opr_kpass,
+    KPass,
     BWD_ROW_TERMS,
     BWD_DQ,
     BWD_DKDV,

@@ -38,6 +38,10 @@ EXPORTED_SYMBOLS = (
     "opr_duplication_index",
     "opr_gather_rows",
     "opr_fold_rows",
+    "opr_kpass_sizes",
+    "opr_kpass_plan",
+    "opr_kpass_index_workspace_bytes",
+    "opr_kpass_index",
 )
 
 BWD_ROW_TERMS, BWD_DQ, BWD_DKDV = 1, 2, 4
@@ -78,7 +82,15 @@ def load_library() -> ctypes.CDLL:
     lib.opr_gather_rows.restype = ctypes.c_int
     lib.opr_gather_rows.argtypes = [P, I64, I64, P, I64, P, P, P]
     lib.opr_fold_rows.restype = ctypes.c_int
-    lib.opr_fold_rows.argtypes = [P, I64, I64, P, I64, P, P, P]
+    lib.opr_fold_rows.argtypes = [P, I64, I64, P, I32, I64, P, P, P]
+    lib.opr_kpass_sizes.restype = ctypes.c_int
+    lib.opr_kpass_sizes.argtypes = [P, I32, I32, P, P]
+    lib.opr_kpass_plan.restype = ctypes.c_int
+    lib.opr_kpass_plan.argtypes = [P, P, P, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P]
+    lib.opr_kpass_index_workspace_bytes.restype = ctypes.c_size_t
+    lib.opr_kpass_index_workspace_bytes.argtypes = [I32, I32]
+    lib.opr_kpass_index.restype = ctypes.c_int
+    lib.opr_kpass_index.argtypes = [P, I32, P, P, I32, I64, I64, I32, P, P, P, SZ, P, P]
     lib.opr_layout_workspace_bytes.restype = SZ
     lib.opr_layout_workspace_bytes.argtypes = [I32, I32, I32, I64, I32]
     lib.opr_build_layout.restype = I32
@@ -382,7 +394,8 @@ def opr_gather_rows(x: torch.Tensor, src_index: torch.Tensor, out: torch.Tensor 
 
 def opr_fold_rows(dy: torch.Tensor, copy_index: torch.Tensor, out: torch.Tensor | None = None,
                   dev_status: torch.Tensor | None = None) -> torch.Tensor:
-    """Gradient of opr_gather_rows: out[o] = dy[copy_index[o, 0]] + dy[copy_index[o, 1]] (fp32)."""
+    """Gradient of opr_gather_rows: out[o] = sum over the slots of copy_index[o] that are >= 0 of
+    dy[copy_index[o, k]], in slot order (fp32); copy_index [orig, slots]."""
     _need_cuda(dy, copy_index)
     if dy.dtype != torch.float32:
         raise OprError("opr_fold_rows: dy must be fp32")
@@ -391,10 +404,77 @@ def opr_fold_rows(dy: torch.Tensor, copy_index: torch.Tensor, out: torch.Tensor 
         out = torch.empty((rows,) + tuple(dy.shape[1:]), dtype=torch.float32, device=dy.device)
     _need_cuda(out)
     width = int(np.prod(dy.shape[1:])) if dy.dim() > 1 else 1
-    _check(lib_call("opr_fold_rows", _ptr(dy), dy.shape[0], width, _ptr(copy_index), rows, _ptr(out),
+    _check(lib_call("opr_fold_rows", _ptr(dy), dy.shape[0], width, _ptr(copy_index), copy_index.shape[1], rows, _ptr(out),
                     _ptr(dev_status) if dev_status is not None else None, _stream(dy.device)), "opr_fold_rows")
     return out
 
 
 def lib_call(name: str, *args) -> int:
     return int(getattr(load_library(), name)(*args))
+
+
+# ------------------------------------------------------------------ K-pass
+@dataclass
+class KPass:
+    """The K-pass arrangement of a batch as layout inputs, plus its token map."""
+
+    K: int
+    turn_lens: torch.Tensor        # int32 [n_out_turns, 3]
+    conv_turn_ptr: torch.Tensor    # int32 [n_out_convs + 1]
+    seq_conv_ptr: torch.Tensor     # int32 [n_seqs + 1]
+    turn_src: torch.Tensor         # int32 [n_out_turns, 2]
+    src_index: torch.Tensor        # int32 [total_tokens]
+    copy_index: torch.Tensor       # int32 [orig_tokens, K + 1]
+    total_tokens: int
+    max_seqlen: int
+    dev_status: torch.Tensor
+
+
+def opr_kpass(turn_lens, conv_turn_ptr, seq_conv_ptr, K: int, device="cuda") -> KPass:
+    """opr_kpass_sizes, opr_kpass_plan and opr_kpass_index in one call.  Length arrays are host
+    arrays (sizes are taken from them before the device work)."""
+    lib = load_library()
+    device = torch.device(device)
+    lens = np.asarray(turn_lens, dtype=np.int32).reshape(-1, 3)
+    cp = np.ascontiguousarray(np.asarray(conv_turn_ptr, dtype=np.int32))
+    sp = np.ascontiguousarray(np.asarray(seq_conv_ptr, dtype=np.int32))
+    n_turns, n_convs, n_seqs = lens.shape[0], cp.size - 1, sp.size - 1
+    nt, nc = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(lib.opr_kpass_sizes(cp.ctypes.data, n_convs, K, ctypes.byref(nt), ctypes.byref(nc)), "opr_kpass_sizes")
+    n_out_turns, n_out_convs = nt.value, nc.value
+    dev = lambda a: torch.as_tensor(a).to(device=device, dtype=torch.int32).contiguous()  # noqa: E731
+    tl, cpd, spd = dev(lens.reshape(-1)), dev(cp), dev(sp)
+    out_lens = torch.empty((n_out_turns, 3), dtype=torch.int32, device=device)
+    out_cp = torch.empty(n_out_convs + 1, dtype=torch.int32, device=device)
+    out_sp = torch.empty(n_seqs + 1, dtype=torch.int32, device=device)
+    out_src = torch.empty((n_out_turns, 2), dtype=torch.int32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib.opr_kpass_plan(_ptr(tl), _ptr(cpd), _ptr(spd), n_seqs, n_convs, n_turns, K, n_out_turns, n_out_convs,
+                              _ptr(out_lens), _ptr(out_cp), _ptr(out_sp), _ptr(out_src), _ptr(status),
+                              _stream(device)), "opr_kpass_plan")
+    # sizes of the arrangement, counted on the host from the same lengths (allocation only)
+    h, t, r = (np.maximum(lens[:, i].astype(np.int64), 0) for i in range(3))
+    total, seq_len, turn_hist = 0, [], []
+    for s in range(n_seqs):
+        L = 0
+        for c in range(int(sp[s]), int(sp[s + 1])):
+            t0, t1 = int(cp[c]), int(cp[c + 1])
+            n = t1 - t0
+            k = min(K, n)
+            for g in range(k):
+                b0, b1 = (g * n) // k, ((g + 1) * n) // k
+                L += int((h[t0:t0 + b0] + r[t0:t0 + b0]).sum() + (h + t + 2 * r)[t0 + b0:t0 + b1].sum())
+        seq_len.append(L)
+        total += L
+    orig = int((h + t + r).sum())
+    slots = K + 1
+    src = torch.empty(total, dtype=torch.int32, device=device)
+    copies = torch.empty((orig, slots), dtype=torch.int32, device=device)
+    ws = torch.empty(max(int(lib.opr_kpass_index_workspace_bytes(n_turns, n_out_turns)), 256), dtype=torch.uint8,
+                     device=device)
+    _check(lib.opr_kpass_index(_ptr(tl), n_turns, _ptr(out_lens), _ptr(out_src), n_out_turns, total, orig, slots,
+                               _ptr(src), _ptr(copies), _ptr(ws), ws.numel(), _ptr(status), _stream(device)),
+           "opr_kpass_index")
+    kp = KPass(K, out_lens, out_cp, out_sp, out_src, src, copies, total, max(seq_len) if seq_len else 0, status)
+    kp._keep = (tl, cpd, spd, ws)  # alive until the stream has used them
+    return kp

@@ -19,8 +19,17 @@ cudaError_t launch_dup_index(const int32_t* turn_lens, const int32_t* conv_turn_
                              int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_gather_rows(const void* x, int64_t orig_total, int64_t row_bytes, const int32_t* src_index,
                                int64_t total, void* y, int32_t* dev_status, cudaStream_t stream);
-cudaError_t launch_fold_rows(const float* dy, int64_t total, int64_t width, const int32_t* copy_index,
+cudaError_t launch_fold_rows(const float* dy, int64_t total, int64_t width, const int32_t* copy_index, int32_t slots,
                              int64_t orig_total, float* dx, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_kpass_plan(const int32_t* turn_lens, const int32_t* conv_turn_ptr, const int32_t* seq_conv_ptr,
+                              int32_t n_seqs, int32_t n_convs, int32_t n_turns, int32_t K, int32_t n_out_turns,
+                              int32_t n_out_convs, int32_t* out_turn_lens, int32_t* out_conv_turn_ptr,
+                              int32_t* out_seq_conv_ptr, int32_t* out_turn_src, int32_t* dev_status,
+                              cudaStream_t stream);
+cudaError_t launch_kpass_index(const int32_t* turn_lens, int32_t n_turns, const int32_t* out_turn_lens,
+                               const int32_t* out_turn_src, int32_t n_out_turns, int64_t total, int64_t orig_total,
+                               int32_t slots, int32_t* src_index, int32_t* copy_index, int64_t* ws,
+                               int32_t* dev_status, cudaStream_t stream);
 
 namespace {
 
@@ -159,14 +168,70 @@ opr_status opr_gather_rows(const void* x, int64_t orig_tokens, int64_t row_bytes
 }
 
 opr_status opr_fold_rows(const float* dy, int64_t total_tokens, int64_t width, const int32_t* copy_index,
-                         int64_t orig_tokens, float* dx, int32_t* dev_status, void* stream) {
-  if (orig_tokens < 0 || total_tokens < 0 || width <= 0) return OPR_INVALID_ARG;
+                         int32_t slots, int64_t orig_tokens, float* dx, int32_t* dev_status, void* stream) {
+  if (orig_tokens < 0 || total_tokens < 0 || width <= 0 || slots < 1 || slots > 64) return OPR_INVALID_ARG;
   if (orig_tokens == 0) return OPR_OK;
   if (!dy || !copy_index || !dx) return OPR_INVALID_ARG;
   const opr_status st = device_check();
   if (st != OPR_OK) return st;
-  return status_of(launch_fold_rows(dy, total_tokens, width, copy_index, orig_tokens, dx, dev_status,
+  return status_of(launch_fold_rows(dy, total_tokens, width, copy_index, slots, orig_tokens, dx, dev_status,
                                     static_cast<cudaStream_t>(stream)));
+}
+
+opr_status opr_kpass_sizes(const int32_t* conv_turn_ptr, int32_t n_convs, int32_t K, int64_t* n_out_turns,
+                           int64_t* n_out_convs) {
+  if (!conv_turn_ptr || !n_out_turns || !n_out_convs || n_convs < 0 || K < 1) return OPR_INVALID_ARG;
+  int64_t turns = 0, convs = 0;
+  for (int c = 0; c < n_convs; ++c) {
+    const int64_t n = conv_turn_ptr[c + 1] - conv_turn_ptr[c];
+    if (n < 0) return OPR_INVALID_ARG;
+    const int64_t k = n < K ? n : K;
+    for (int64_t g = 0; g < k; ++g) turns += ((g + 1) * n) / k;
+    convs += k;
+  }
+  if (turns >= (int64_t{1} << 31) || convs >= (int64_t{1} << 31)) return OPR_INVALID_ARG;
+  *n_out_turns = turns;
+  *n_out_convs = convs;
+  return OPR_OK;
+}
+
+opr_status opr_kpass_plan(const int32_t* turn_lens, const int32_t* conv_turn_ptr, const int32_t* seq_conv_ptr,
+                          int32_t n_seqs, int32_t n_convs, int32_t n_turns, int32_t K, int32_t n_out_turns,
+                          int32_t n_out_convs, int32_t* out_turn_lens, int32_t* out_conv_turn_ptr,
+                          int32_t* out_seq_conv_ptr, int32_t* out_turn_src, int32_t* dev_status, void* stream) {
+  if (n_seqs < 0 || n_convs < 0 || n_turns < 0 || K < 1 || n_out_turns < 0 || n_out_convs < 0) return OPR_INVALID_ARG;
+  if (!conv_turn_ptr || !seq_conv_ptr || !out_conv_turn_ptr || !out_seq_conv_ptr || !dev_status ||
+      (n_turns > 0 && !turn_lens) || (n_out_turns > 0 && (!out_turn_lens || !out_turn_src)))
+    return OPR_INVALID_ARG;
+  const opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  return status_of(launch_kpass_plan(turn_lens, conv_turn_ptr, seq_conv_ptr, n_seqs, n_convs, n_turns, K, n_out_turns,
+                                     n_out_convs, out_turn_lens, out_conv_turn_ptr, out_seq_conv_ptr, out_turn_src,
+                                     dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+size_t opr_kpass_index_workspace_bytes(int32_t n_turns, int32_t n_out_turns) {
+  if (n_turns < 0 || n_out_turns < 0) return 0;
+  return align_up(sizeof(int64_t) * (static_cast<size_t>(n_turns) + 1 + static_cast<size_t>(n_out_turns) + 1), 256);
+}
+
+opr_status opr_kpass_index(const int32_t* turn_lens, int32_t n_turns, const int32_t* out_turn_lens,
+                           const int32_t* out_turn_src, int32_t n_out_turns, int64_t total_tokens, int64_t orig_tokens,
+                           int32_t slots, int32_t* src_index, int32_t* copy_index, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (n_turns < 0 || n_out_turns < 0 || total_tokens < 0 || orig_tokens < 0 || slots < 2 || slots > 64)
+    return OPR_INVALID_ARG;
+  if (total_tokens >= (int64_t{1} << 31)) return OPR_INVALID_ARG;
+  if (!workspace || !dev_status || (n_turns > 0 && !turn_lens) || (n_out_turns > 0 && (!out_turn_lens || !out_turn_src)) ||
+      (total_tokens > 0 && !src_index) || (orig_tokens > 0 && !copy_index))
+    return OPR_INVALID_ARG;
+  if (workspace_bytes < opr_kpass_index_workspace_bytes(n_turns, n_out_turns)) return OPR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 8 != 0) return OPR_INVALID_ARG;
+  const opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  return status_of(launch_kpass_index(turn_lens, n_turns, out_turn_lens, out_turn_src, n_out_turns, total_tokens,
+                                      orig_tokens, slots, src_index, copy_index, static_cast<int64_t*>(workspace),
+                                      dev_status, static_cast<cudaStream_t>(stream)));
 }
 
 const char* opr_version(void) { return "opr 0.1.0 sm_100a"; }

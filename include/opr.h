@@ -302,14 +302,71 @@ OPR_API opr_status opr_gather_rows(const void* x, int64_t orig_tokens, int64_t r
 
 /*
  * opr_fold_rows - the gradient of opr_gather_rows w.r.t. x, fp32 rows of `width` values:
- * dx[o] = dy[copy_index[o][0]] + dy[copy_index[o][1]], the first copy plus the second in that
- * order (dy[copy_index[o][0]] alone when the second is -1).  No atomics; deterministic.
+ * dx[o] = sum of dy[copy_index[o][k]] over the slots k < slots with copy_index[o][k] >= 0, added
+ * in slot order (copy_index from opr_duplication_index has 2 slots, from opr_kpass_index K + 1).
+ * No atomics; deterministic.
  *   dy  fp32 [total_tokens][width];  dx  fp32 [orig_tokens][width], caller-owned
- *   dev_status  may be NULL; otherwise OPR_DEV_BAD_INPUT for an out-of-range index
+ *   dev_status  may be NULL; otherwise OPR_DEV_BAD_INPUT for an out-of-range index or a row
+ *               without any copy (left unwritten)
  */
 OPR_API opr_status opr_fold_rows(const float* dy, int64_t total_tokens, int64_t width,
-                                 const int32_t* copy_index, int64_t orig_tokens, float* dx,
-                                 int32_t* dev_status, void* stream);
+                                 const int32_t* copy_index, int32_t slots, int64_t orig_tokens,
+                                 float* dx, int32_t* dev_status, void* stream);
+
+/*
+ * K-pass, between N-pass (K = N) and one-pass (K = 1) (wiki note, "K-Pass 中间方案": a
+ * speed / memory trade-off).  The pages give only the trade-off; the reading built here:
+ * a conversation's N turns fall into K' = min(K, N) contiguous groups with bounds
+ * b_g = floor(g N / K'); pass g is one conversation holding the history of the turns
+ * before the group, each turn j as the single context segment (h_j + r_j, 0, 0) (h_j
+ * then r_j, positions running on, as h_j and r_j^in in one pass), then the group's own
+ * turns (h, t, r).  Every t and r^out row lies in exactly one pass, and the output is an
+ * ordinary input of opr_build_layout, so the attention calls serve every K unchanged.
+ *
+ * opr_kpass_sizes - output turn and conversation (pass) counts, from a HOST conv_turn_ptr.
+ */
+OPR_API opr_status opr_kpass_sizes(const int32_t* conv_turn_ptr, int32_t n_convs, int32_t K,
+                                   int64_t* n_out_turns, int64_t* n_out_convs);
+
+/*
+ * opr_kpass_plan - the K-pass arrangement as layout inputs (device arrays).
+ *   turn_lens, conv_turn_ptr, seq_conv_ptr  the one-pass inputs, as for opr_build_layout
+ *   n_out_turns, n_out_convs               from opr_kpass_sizes
+ *   out_turn_lens      int32 [n_out_turns][3]; out_conv_turn_ptr int32 [n_out_convs + 1];
+ *   out_seq_conv_ptr   int32 [n_seqs + 1] (the passes of a conversation stay in its sequence)
+ *   out_turn_src       int32 [n_out_turns][2]: (original turn, d) with d = -1 for a turn of
+ *                      the pass's own group and d >= 1 for a history turn d groups before
+ *   dev_status         required; OPR_DEV_BAD_INPUT, OPR_DEV_TOTAL_MISMATCH (sizes disagree)
+ * One thread block on `stream`.
+ */
+OPR_API opr_status opr_kpass_plan(const int32_t* turn_lens, const int32_t* conv_turn_ptr,
+                                  const int32_t* seq_conv_ptr, int32_t n_seqs, int32_t n_convs,
+                                  int32_t n_turns, int32_t K, int32_t n_out_turns, int32_t n_out_convs,
+                                  int32_t* out_turn_lens, int32_t* out_conv_turn_ptr,
+                                  int32_t* out_seq_conv_ptr, int32_t* out_turn_src, int32_t* dev_status,
+                                  void* stream);
+
+/* Bytes of device scratch (8-byte aligned) that opr_kpass_index needs: two turn-offset arrays. */
+OPR_API size_t opr_kpass_index_workspace_bytes(int32_t n_turns, int32_t n_out_turns);
+
+/*
+ * opr_kpass_index - the token map between the original stream (h, t, r per turn) and the
+ * K-pass stream of opr_kpass_plan's arrangement.
+ *   total_tokens   K-pass tokens (sum of h + t + 2r over the output turns)
+ *   orig_tokens    original tokens (sum of h + t + r over the input turns)
+ *   slots          K + 1 (or more)
+ *   src_index      int32 [total_tokens] out: the original token each K-pass token copies
+ *   copy_index     int32 [orig_tokens][slots] out: slot 0 the copy in the token's own pass
+ *                  (h, t or r^in), 1 the r^out copy, 1 + d the history copy d groups later;
+ *                  -1 where there is none (the call clears it first)
+ *   workspace      opr_kpass_index_workspace_bytes(n_turns, n_out_turns) bytes, caller-owned
+ * Fold gradients with opr_fold_rows(..., copy_index, slots, ...).
+ */
+OPR_API opr_status opr_kpass_index(const int32_t* turn_lens, int32_t n_turns, const int32_t* out_turn_lens,
+                                   const int32_t* out_turn_src, int32_t n_out_turns, int64_t total_tokens,
+                                   int64_t orig_tokens, int32_t slots, int32_t* src_index,
+                                   int32_t* copy_index, void* workspace, size_t workspace_bytes,
+                                   int32_t* dev_status, void* stream);
 
 OPR_API const char* opr_version(void);
 

@@ -107,5 +107,25 @@ def test_duplication_entry_points_check_arguments_on_the_host():
     assert lib.opr_gather_rows(fake, 5, 0, fake, 10, fake, None, None) == 1
     assert lib.opr_gather_rows(None, 5, 16, fake, 10, fake, None, None) == 1
     assert lib.opr_gather_rows(fake, 5, 16, fake, 0, fake, None, None) == 0  # nothing to copy
-    assert lib.opr_fold_rows(fake, 10, 0, fake, 5, fake, None, None) == 1
-    assert lib.opr_fold_rows(fake, 10, 4, fake, 0, fake, None, None) == 0
+    assert lib.opr_fold_rows(fake, 10, 0, fake, 2, 5, fake, None, None) == 1
+    assert lib.opr_fold_rows(fake, 10, 4, fake, 0, 5, fake, None, None) == 1  # no slots
+    assert lib.opr_fold_rows(fake, 10, 4, fake, 2, 0, fake, None, None) == 0
+    ws = lib.opr_kpass_index_workspace_bytes(10, 20)
+    assert ws >= 8 * (11 + 21)
+    assert lib.opr_kpass_index(fake, 10, fake, fake, 20, 100, 50, 3, fake, fake, fake, ws - 256, fake, None) == 4
+    assert lib.opr_kpass_plan(fake, fake, fake, 1, 1, 2, 0, 2, 1, fake, fake, fake, fake, fake, None) == 1  # K = 0
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 5])
+def test_kpass_sizes_match_the_oracle(K):
+    """opr_kpass_sizes is host code: checked against the oracle's arrangement without a GPU."""
+    import synth
+    from oracle import opr_oracle as orc
+
+    lib = opr.load_library()
+    w = synth.random_small_workload(21, max_convs=4, max_turns=6)
+    cp = np.ascontiguousarray(np.asarray(w.conv_turn_ptr, dtype=np.int32))
+    nt, nc = ctypes.c_int64(0), ctypes.c_int64(0)
+    assert lib.opr_kpass_sizes(cp.ctypes.data, cp.size - 1, K, ctypes.byref(nt), ctypes.byref(nc)) == 0
+    l2, c2, _, _ = orc.kpass_plan(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, K)
+    assert (nt.value, nc.value) == (len(l2), len(c2) - 1)
