@@ -29,6 +29,10 @@ evaluated densely and slowly in float64 with numpy:
 * ``kpass_plan`` / ``kpass_index``
                      the K-pass arrangement ("K-Pass 中间方案"): each pass is a
                      group of turns behind the history of the earlier turns.
+* ``loss_rows`` / ``cross_entropy``
+                     the step after the attention layer: the one-pass rows that
+                     carry the N-pass next-token losses (t and r^out, "Token 复制"),
+                     their targets, and softmax cross-entropy with its gradient.
 
 Pins (checked by the tests that do not need a GPU): a hand-derived worked
 example of positions, visibility and the duplication map, closed-form visible-pair counts per turn,
@@ -562,3 +566,56 @@ def kpass_index(turn_lens, conv_turn_ptr, seq_conv_ptr, K: int):
                 copies[o + h + t + x, 1] = pos + h + t + r + x
             pos += h + t + 2 * r
     return np.asarray(src, dtype=np.int32), copies
+
+
+# --------------------------------------------------------------------------
+# Loss side: which one-pass rows carry the N-pass next-token losses.
+#
+# Reading (the pages say the loss is that of the N-pass runs, "理论保证", and
+# that r^out is the copy trained on, "Token 复制"): in N-pass run i the
+# sequence is [H<i, h_i, t_i, r_i] and the losses are the next-token
+# predictions of t_i and r_i: from the last h_i row (target: the first t_i
+# token, or the first r_i token when t_i is empty), from each t_i row (target:
+# the next t_i token, or the first r_i token after the last), and from each
+# r_i row but the last (target: the next r_i token).  In one pass those rows
+# are the last h_i row, the t_i rows and the r_i^out rows (Theorem 2.1).
+
+def loss_rows(turn_lens, conv_turn_ptr):
+    """(rows, targets): one-pass row indices carrying a loss, in stream order, and the
+    original-stream index of each row's target token."""
+    turn_lens = np.asarray(turn_lens, dtype=np.int64).reshape(-1, 3)
+    conv_turn_ptr = np.asarray(conv_turn_ptr, dtype=np.int64)
+    rows, targets = [], []
+    one_pass = orig = 0
+    for c in range(len(conv_turn_ptr) - 1):
+        for t in range(conv_turn_ptr[c], conv_turn_ptr[c + 1]):
+            h, tt, r = (int(x) for x in turn_lens[t])
+            assistant = list(range(orig + h, orig + h + tt + r))  # original t then r tokens
+            if h > 0 and assistant:
+                rows.append(one_pass + h - 1)
+                targets.append(assistant[0])
+            for x in range(tt):  # t rows: the next assistant token
+                if x + 1 < len(assistant):
+                    rows.append(one_pass + h + x)
+                    targets.append(assistant[x + 1])
+            for x in range(r - 1):  # r^out rows but the last
+                rows.append(one_pass + h + tt + r + x)
+                targets.append(orig + h + tt + x + 1)
+            one_pass += h + tt + 2 * r
+            orig += h + tt + r
+    return np.asarray(rows, dtype=np.int32), np.asarray(targets, dtype=np.int32)
+
+
+def cross_entropy(logits: np.ndarray, target_ids: np.ndarray):
+    """Per-row softmax cross-entropy in float64 and its gradient w.r.t. the logits:
+    loss = logsumexp(z) - z[target], dz = softmax(z) - onehot(target)."""
+    z = np.asarray(logits, dtype=np.float64)
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    s = e.sum(axis=1, keepdims=True)
+    lse = (np.log(s) + m)[:, 0]
+    idx = np.asarray(target_ids, dtype=np.int64)
+    loss = lse - z[np.arange(len(idx)), idx]
+    dz = e / s
+    dz[np.arange(len(idx)), idx] -= 1.0
+    return loss, dz
