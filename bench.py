@@ -407,6 +407,43 @@ def time_duplication(w: synth.Workload, device, hbm_gbs: float, hidden: int = 40
     }
 
 
+def time_loss_side(w: synth.Workload, device, hbm_gbs: float, vocab: int = 151936, max_rows: int = 4096, reps: int = 5):
+    """The step after the attention layer: the loss-row map of this workload and the fused
+    cross-entropy (loss and gradient) over up to max_rows of its loss rows with bf16 logits of
+    the Qwen-3 vocabulary.  HBM-bound: two reads and one write of the logits."""
+    import torch
+
+    import block_sparse_masked_segment_b200 as opr
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    rows, targets = opr.opr_loss_rows(w.turn_lens, device=device)
+    t_rows = timed(lambda: opr.opr_loss_rows(w.turn_lens, device=device))
+    n = min(rows.numel(), max_rows)
+    logits = (torch.randn(n, vocab, device=device) * 3).to(torch.bfloat16)
+    tid = torch.randint(0, vocab, (n,), device=device, dtype=torch.int32)
+    t_ce = timed(lambda: opr.opr_cross_entropy(logits, tid, grad_scale=1.0 / n))
+    loss, _ = opr.opr_cross_entropy(logits, tid)
+    torch.cuda.synchronize()
+    status = opr.read_status(rows._inputs[1]) + opr.read_status(loss._status)
+    if status:
+        raise RuntimeError(f"device status after loss-side timing: {status}")
+    bytes_ = 3 * n * vocab * 2
+    return {"loss_rows": int(rows.numel()), "loss_rows_ms": t_rows, "ce_rows": n, "vocab": vocab,
+            "ce_ms": t_ce, "ce_gbs": bytes_ / (t_ce * 1e-3) / 1e9, "ce_frac_hbm": bytes_ / (t_ce * 1e-3) / 1e9 / hbm_gbs}
+
+
 def kpass_workload(w: synth.Workload, K: int, device) -> synth.Workload:
     """The K-pass arrangement of w, built on the GPU by opr_kpass (plan and token map)."""
     import torch
@@ -570,6 +607,7 @@ def main():
 
     _, _, hbm, _ = peaks()
     duplication = time_duplication(w, device, hbm)
+    loss_side = time_loss_side(w, device, hbm)
 
     # K-pass (K = 2) on the same conversations and kernels: speed and tokens against one-pass
     kw = kpass_workload(w, 2, device)
@@ -634,7 +672,7 @@ def main():
         "roofline": roofline,
         "e2e": e2e,
         "npass": npass,
-        "next_rows": {"token_duplication": duplication, "kpass": kpass},
+        "next_rows": {"token_duplication": duplication, "kpass": kpass, "loss_side": loss_side},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": dict(clocks.summary(), remeasured=remeasured),
         "cpu_baseline": cpu,

@@ -22,6 +22,8 @@ from ._abi import (  # noqa: F401
     opr_gather_rows,
     opr_fold_rows,
     opr_kpass,
+    opr_loss_rows,
+    opr_cross_entropy,
     KPass,
     BWD_ROW_TERMS,
     BWD_DQ,

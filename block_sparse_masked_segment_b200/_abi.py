@@ -42,6 +42,9 @@ EXPORTED_SYMBOLS = (
     "opr_kpass_plan",
     "opr_kpass_index_workspace_bytes",
     "opr_kpass_index",
+    "opr_loss_row_count",
+    "opr_loss_rows",
+    "opr_cross_entropy",
 )
 
 BWD_ROW_TERMS, BWD_DQ, BWD_DKDV = 1, 2, 4
@@ -89,6 +92,12 @@ def load_library() -> ctypes.CDLL:
     lib.opr_kpass_plan.argtypes = [P, P, P, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P]
     lib.opr_kpass_index_workspace_bytes.restype = ctypes.c_size_t
     lib.opr_kpass_index_workspace_bytes.argtypes = [I32, I32]
+    lib.opr_loss_row_count.restype = ctypes.c_int64
+    lib.opr_loss_row_count.argtypes = [P, I32]
+    lib.opr_loss_rows.restype = ctypes.c_int
+    lib.opr_loss_rows.argtypes = [P, I32, I64, I64, I64, P, P, P, P]
+    lib.opr_cross_entropy.restype = ctypes.c_int
+    lib.opr_cross_entropy.argtypes = [P, I32, I64, I32, P, P, P, F, P, P]
     lib.opr_kpass_index.restype = ctypes.c_int
     lib.opr_kpass_index.argtypes = [P, I32, P, P, I32, I64, I64, I32, P, P, P, SZ, P, P]
     lib.opr_layout_workspace_bytes.restype = SZ
@@ -478,3 +487,44 @@ def opr_kpass(turn_lens, conv_turn_ptr, seq_conv_ptr, K: int, device="cuda") -> 
     kp = KPass(K, out_lens, out_cp, out_sp, out_src, src, copies, total, max(seq_len) if seq_len else 0, status)
     kp._keep = (tl, cpd, spd, ws)  # alive until the stream has used them
     return kp
+
+
+# ------------------------------------------------------------------ loss side
+def opr_loss_rows(turn_lens, device="cuda", dev_status: torch.Tensor | None = None):
+    """(rows, targets) int32 device tensors: the one-pass rows carrying the N-pass next-token
+    losses and the original-stream index of each row's target token."""
+    lib = load_library()
+    device = torch.device(device)
+    lens = np.ascontiguousarray(np.asarray(turn_lens, dtype=np.int32).reshape(-1, 3))
+    n_turns = lens.shape[0]
+    n_rows = int(lib.opr_loss_row_count(lens.ctypes.data, n_turns))
+    if n_rows < 0:
+        raise OprError("opr_loss_row_count: negative lengths")
+    l64 = np.maximum(lens.astype(np.int64), 0)
+    total = int(l64[:, 0].sum() + l64[:, 1].sum() + 2 * l64[:, 2].sum())
+    orig = int(l64.sum())
+    tl = torch.as_tensor(lens.reshape(-1)).to(device)
+    rows = torch.empty(n_rows, dtype=torch.int32, device=device)
+    targets = torch.empty(n_rows, dtype=torch.int32, device=device)
+    status = dev_status if dev_status is not None else torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib.opr_loss_rows(_ptr(tl), n_turns, total, orig, n_rows, _ptr(rows), _ptr(targets), _ptr(status),
+                             _stream(device)), "opr_loss_rows")
+    rows._inputs = (tl, status)
+    return rows, targets
+
+
+def opr_cross_entropy(logits: torch.Tensor, target_ids: torch.Tensor, grad_scale: float = 1.0,
+                      with_grad: bool = True, dev_status: torch.Tensor | None = None):
+    """(loss fp32 [n], dlogits [n, V] in the logits' dtype or None): fused softmax cross-entropy."""
+    _need_cuda(logits, target_ids)
+    if logits.dtype not in (torch.bfloat16, torch.float32) or logits.dim() != 2:
+        raise OprError("opr_cross_entropy: logits must be [n, V] bf16 or fp32")
+    n, V = logits.shape
+    loss = torch.empty(n, dtype=torch.float32, device=logits.device)
+    dl = torch.empty_like(logits) if with_grad else None
+    status = dev_status if dev_status is not None else torch.zeros(1, dtype=torch.int32, device=logits.device)
+    _check(load_library().opr_cross_entropy(_ptr(logits), _DT[logits.dtype], n, V, _ptr(target_ids), _ptr(loss),
+                                            _ptr(dl), grad_scale, _ptr(status), _stream(logits.device)),
+           "opr_cross_entropy")
+    loss._status = status
+    return loss, dl

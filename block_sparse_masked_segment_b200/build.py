@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libopr.so")
-SOURCES = ["api.cu", "layout.cu", "rope.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu", "duplicate.cu"]
+SOURCES = ["api.cu", "layout.cu", "rope.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu", "duplicate.cu", "loss.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 

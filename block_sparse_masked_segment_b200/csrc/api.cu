@@ -26,6 +26,11 @@ cudaError_t launch_kpass_plan(const int32_t* turn_lens, const int32_t* conv_turn
                               int32_t n_out_convs, int32_t* out_turn_lens, int32_t* out_conv_turn_ptr,
                               int32_t* out_seq_conv_ptr, int32_t* out_turn_src, int32_t* dev_status,
                               cudaStream_t stream);
+cudaError_t launch_loss_rows(const int32_t* turn_lens, int32_t n_turns, int64_t total, int64_t orig_total,
+                             int64_t n_rows, int32_t* rows, int32_t* targets, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_cross_entropy(const void* logits, bool bf16, int64_t n_rows, int32_t V, const int32_t* target_ids,
+                                 float* loss, void* dlogits, float grad_scale, int32_t* dev_status,
+                                 cudaStream_t stream);
 cudaError_t launch_kpass_index(const int32_t* turn_lens, int32_t n_turns, const int32_t* out_turn_lens,
                                const int32_t* out_turn_src, int32_t n_out_turns, int64_t total, int64_t orig_total,
                                int32_t slots, int32_t* src_index, int32_t* copy_index, int64_t* ws,
@@ -232,6 +237,41 @@ opr_status opr_kpass_index(const int32_t* turn_lens, int32_t n_turns, const int3
   return status_of(launch_kpass_index(turn_lens, n_turns, out_turn_lens, out_turn_src, n_out_turns, total_tokens,
                                       orig_tokens, slots, src_index, copy_index, static_cast<int64_t*>(workspace),
                                       dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+int64_t opr_loss_row_count(const int32_t* turn_lens, int32_t n_turns) {
+  if (n_turns < 0 || (n_turns > 0 && !turn_lens)) return -1;
+  int64_t n = 0;
+  for (int i = 0; i < n_turns; ++i) {
+    const int64_t h = turn_lens[3 * i], t = turn_lens[3 * i + 1], r = turn_lens[3 * i + 2];
+    if (h < 0 || t < 0 || r < 0) return -1;
+    n += ((h > 0 && t + r > 0) ? 1 : 0) + (r > 0 ? t : (t > 0 ? t - 1 : 0)) + (r > 1 ? r - 1 : 0);
+  }
+  return n;
+}
+
+opr_status opr_loss_rows(const int32_t* turn_lens, int32_t n_turns, int64_t total_tokens, int64_t orig_tokens,
+                         int64_t n_rows, int32_t* rows, int32_t* targets, int32_t* dev_status, void* stream) {
+  if (n_turns < 0 || total_tokens < 0 || orig_tokens < 0 || n_rows < 0) return OPR_INVALID_ARG;
+  if (total_tokens >= (int64_t{1} << 31)) return OPR_INVALID_ARG;
+  if (!dev_status || (n_turns > 0 && !turn_lens) || (n_rows > 0 && (!rows || !targets))) return OPR_INVALID_ARG;
+  const opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  return status_of(launch_loss_rows(turn_lens, n_turns, total_tokens, orig_tokens, n_rows, rows, targets, dev_status,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+opr_status opr_cross_entropy(const void* logits, int32_t dtype, int64_t n_rows, int32_t vocab,
+                             const int32_t* target_ids, float* loss, void* dlogits, float grad_scale,
+                             int32_t* dev_status, void* stream) {
+  if (n_rows < 0 || vocab <= 0 || n_rows >= (int64_t{1} << 31)) return OPR_INVALID_ARG;
+  if (dtype != OPR_DTYPE_BF16 && dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
+  if (n_rows == 0) return OPR_OK;
+  if (!logits || !target_ids || !loss || !dev_status) return OPR_INVALID_ARG;
+  const opr_status st = device_check();
+  if (st != OPR_OK) return st;
+  return status_of(launch_cross_entropy(logits, dtype == OPR_DTYPE_BF16, n_rows, vocab, target_ids, loss, dlogits,
+                                        grad_scale, dev_status, static_cast<cudaStream_t>(stream)));
 }
 
 const char* opr_version(void) { return "opr 0.1.0 sm_100a"; }

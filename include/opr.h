@@ -368,6 +368,47 @@ OPR_API opr_status opr_kpass_index(const int32_t* turn_lens, int32_t n_turns, co
                                    int32_t* copy_index, void* workspace, size_t workspace_bytes,
                                    int32_t* dev_status, void* stream);
 
+/*
+ * The loss side, the step after the attention layer.  The pages prove that the one-pass
+ * loss equals the N-pass loss ("理论保证") and train on the r^out copies ("Token 复制").
+ * In N-pass run i the losses are the next-token predictions of t_i and r_i: from the last
+ * h_i row (target: the first t_i token, or r_i[0] when t_i is empty), from each t_i row
+ * (target: the next t_i token, or r_i[0] after the last) and from each r_i row but the last
+ * (target: the next r_i token).  In one pass those rows are the last h_i row, the t_i rows
+ * and the r_i^out rows.  (When h_i is empty the first assistant token has no loss row.)
+ *
+ * opr_loss_row_count - number of such rows, from HOST turn lengths; -1 for bad input.
+ */
+OPR_API int64_t opr_loss_row_count(const int32_t* turn_lens, int32_t n_turns);
+
+/*
+ * opr_loss_rows - the loss rows, in one-pass stream order, and the original-stream index of
+ * each row's target token (the original stream holds h, t, r once per turn, conversations in
+ * index order; a token id array of that stream gives the target ids).
+ *   turn_lens     int32 [n_turns][3], device
+ *   total_tokens  one-pass tokens; orig_tokens original tokens; n_rows from opr_loss_row_count
+ *   rows, targets int32 [n_rows] out
+ *   dev_status    required; OPR_DEV_BAD_INPUT, OPR_DEV_TOTAL_MISMATCH (sizes disagree)
+ * One thread block on `stream`.
+ */
+OPR_API opr_status opr_loss_rows(const int32_t* turn_lens, int32_t n_turns, int64_t total_tokens,
+                                 int64_t orig_tokens, int64_t n_rows, int32_t* rows, int32_t* targets,
+                                 int32_t* dev_status, void* stream);
+
+/*
+ * opr_cross_entropy - softmax cross-entropy of n_rows rows of logits, fused with its gradient:
+ * loss[i] = logsumexp(z_i) - z_i[target_ids[i]], and when dlogits is not NULL
+ * dlogits[i] = grad_scale * (softmax(z_i) - onehot(target_ids[i])).  fp32 arithmetic.
+ *   logits    [n_rows][vocab], dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32, device
+ *   target_ids int32 [n_rows]; a negative id marks a row to ignore (loss 0, gradient 0);
+ *             an id >= vocab sets OPR_DEV_BAD_INPUT and is ignored the same way
+ *   loss      fp32 [n_rows] out;  dlogits  [n_rows][vocab] in the logits' dtype, or NULL
+ * One CTA per row.
+ */
+OPR_API opr_status opr_cross_entropy(const void* logits, int32_t dtype, int64_t n_rows, int32_t vocab,
+                                     const int32_t* target_ids, float* loss, void* dlogits,
+                                     float grad_scale, int32_t* dev_status, void* stream);
+
 OPR_API const char* opr_version(void);
 
 /*

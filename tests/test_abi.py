@@ -129,3 +129,18 @@ def test_kpass_sizes_match_the_oracle(K):
     assert lib.opr_kpass_sizes(cp.ctypes.data, cp.size - 1, K, ctypes.byref(nt), ctypes.byref(nc)) == 0
     l2, c2, _, _ = orc.kpass_plan(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, K)
     assert (nt.value, nc.value) == (len(l2), len(c2) - 1)
+
+
+def test_loss_row_count_matches_the_oracle():
+    """opr_loss_row_count is host code: checked against the oracle's loss rows without a GPU."""
+    import synth
+    from oracle import opr_oracle as orc
+
+    lib = opr.load_library()
+    for seed in range(4):
+        w = synth.random_small_workload(seed, max_turns=6)
+        lens = np.ascontiguousarray(np.asarray(w.turn_lens, dtype=np.int32).reshape(-1, 3))
+        rows, _ = orc.loss_rows(w.turn_lens, w.conv_turn_ptr)
+        assert lib.opr_loss_row_count(lens.ctypes.data, lens.shape[0]) == len(rows)
+    bad = np.asarray([[1, -2, 3]], dtype=np.int32)
+    assert lib.opr_loss_row_count(bad.ctypes.data, 1) == -1
