@@ -16,6 +16,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cstdint>
 #include <type_traits>
 
 #include "opr_internal.cuh"
@@ -24,6 +25,12 @@ namespace opr {
 namespace {
 
 constexpr int kLossThreads = 1024;
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ int turn_loss_rows(int h, int t, int r) {
   return ((h > 0 && t + r > 0) ? 1 : 0) + (r > 0 ? t : (t > 0 ? t - 1 : 0)) + (r > 1 ? r - 1 : 0);
@@ -135,6 +142,56 @@ __global__ void __launch_bounds__(kLossThreads) loss_rows_kernel(const int32_t* 
     atomicOr(dev_status, OPR_DEV_TOTAL_MISMATCH);
 }
 
+// Online (max, sum 2^(x - max)) of a thread's values in base 2: a new maximum
+// rescales the running sum once, every other value adds one 2^(x - max).
+__device__ __forceinline__ void online_add(float& m, float& s, float x2) {
+  if (x2 == -INFINITY) return;  // a masked logit adds nothing
+  if (x2 > m) {
+    s = s * ex2f(m - x2) + 1.f;
+    m = x2;
+  } else {
+    s += ex2f(x2 - m);
+  }
+}
+
+__device__ __forceinline__ void merge_ms(float& m, float& s, float m2, float s2) {
+  const float mm = fmaxf(m, m2);
+  if (mm == -INFINITY) return;
+  s = s * ex2f(m - mm) + s2 * ex2f(m2 - mm);
+  m = mm;
+}
+
+// Eight consecutive logits of a row as floats (bf16: one 16-byte load; fp32: two).
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]) {
+  if constexpr (std::is_same_v<T, float>) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = __low2float(b2[k]);
+      v[2 * k + 1] = __high2float(b2[k]);
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store8(T* p, const float (&v)[8]) {
+  if constexpr (std::is_same_v<T, float>) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+    uint4 u;
+    __nv_bfloat162* b2 = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) b2[k] = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ float to_float(T v) {
   if constexpr (std::is_same_v<T, float>)
@@ -151,22 +208,18 @@ __device__ __forceinline__ T from_float(float v) {
     return __float2bfloat16_rn(v);
 }
 
-// Block-wide reduction of (max, sum of exp(z - max)) pairs.
-__device__ __forceinline__ void merge_ms(float& m, float& s, float m2, float s2) {
-  const float mm = fmaxf(m, m2);
-  if (mm == -INFINITY) return;
-  s = s * expf(m - mm) + s2 * expf(m2 - mm);
-  m = mm;
-}
-
-// One block of 256 threads per row.
-template <typename T>
+// One block of 256 threads per row; the arithmetic runs in base 2 on the SFU's
+// ex2 (scores pre-multiplied by log2 e).  Two reads of the row (statistics,
+// then the gradient) and one write.  VEC: the row is 16-byte aligned with
+// vocab % 8 == 0, read eight values at a time.
+template <typename T, bool VEC>
 __global__ void __launch_bounds__(256) cross_entropy_kernel(const T* __restrict__ logits, int64_t n_rows, int32_t V,
                                                             const int32_t* __restrict__ target_ids,
                                                             float* __restrict__ loss, T* __restrict__ dlogits,
                                                             float grad_scale, int32_t* __restrict__ dev_status) {
+  constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.69314718055994531f;
   __shared__ float red_m[8], red_s[8];
-  __shared__ float row_lse;
+  __shared__ float row_lse2;
   const int64_t row = blockIdx.x;
   if (row >= n_rows) return;
   const T* z = logits + row * V;
@@ -180,14 +233,15 @@ __global__ void __launch_bounds__(256) cross_entropy_kernel(const T* __restrict_
     return;
   }
   float m = -INFINITY, s = 0.f;
-  for (int j = tid; j < V; j += blockDim.x) {
-    const float x = to_float(z[j]);
-    if (x > m) {
-      s = s * expf(m - x) + 1.f;
-      m = x;
-    } else {
-      s += expf(x - m);
+  if constexpr (VEC) {
+    for (int j = tid * 8; j < V; j += blockDim.x * 8) {
+      float v[8];
+      load8(z + j, v);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) online_add(m, s, v[k] * kLog2e);
     }
+  } else {
+    for (int j = tid; j < V; j += blockDim.x) online_add(m, s, to_float(z[j]) * kLog2e);
   }
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) {
@@ -202,16 +256,25 @@ __global__ void __launch_bounds__(256) cross_entropy_kernel(const T* __restrict_
   if (tid == 0) {
     float mm = red_m[0], ss = red_s[0];
     for (int w = 1; w < 8; ++w) merge_ms(mm, ss, red_m[w], red_s[w]);
-    row_lse = mm + logf(ss);
-    loss[row] = row_lse - to_float(z[tgt]);
+    row_lse2 = mm + log2f(ss);
+    loss[row] = row_lse2 * kLn2 - to_float(z[tgt]);
   }
   __syncthreads();
-  if (dlogits != nullptr) {
-    const float lse = row_lse;
-    for (int j = tid; j < V; j += blockDim.x) {
-      const float p = expf(to_float(z[j]) - lse);
-      dlogits[row * V + j] = from_float<T>(grad_scale * (p - (j == tgt ? 1.f : 0.f)));
+  if (dlogits == nullptr) return;
+  const float lse2 = row_lse2;
+  T* dz = dlogits + row * V;
+  if constexpr (VEC) {
+    for (int j = tid * 8; j < V; j += blockDim.x * 8) {
+      float v[8];
+      load8(z + j, v);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        v[k] = grad_scale * (ex2f(fmaf(v[k], kLog2e, -lse2)) - (j + k == tgt ? 1.f : 0.f));
+      store8(dz + j, v);
     }
+  } else {
+    for (int j = tid; j < V; j += blockDim.x)
+      dz[j] = from_float<T>(grad_scale * (ex2f(fmaf(to_float(z[j]), kLog2e, -lse2)) - (j == tgt ? 1.f : 0.f)));
   }
 }
 
@@ -229,14 +292,28 @@ cudaError_t launch_cross_entropy(const void* logits, bool bf16, int64_t n_rows, 
                                  float* loss, void* dlogits, float grad_scale, int32_t* dev_status,
                                  cudaStream_t stream) {
   if (n_rows == 0) return cudaSuccess;
-  if (bf16)
-    cross_entropy_kernel<__nv_bfloat16><<<static_cast<unsigned>(n_rows), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(logits), n_rows, V, target_ids, loss,
-        static_cast<__nv_bfloat16*>(dlogits), grad_scale, dev_status);
-  else
-    cross_entropy_kernel<float><<<static_cast<unsigned>(n_rows), 256, 0, stream>>>(
-        static_cast<const float*>(logits), n_rows, V, target_ids, loss, static_cast<float*>(dlogits), grad_scale,
-        dev_status);
+  const unsigned grid = static_cast<unsigned>(n_rows);
+  const bool vec = V % 8 == 0 && reinterpret_cast<uintptr_t>(logits) % 16 == 0 &&
+                   (dlogits == nullptr || reinterpret_cast<uintptr_t>(dlogits) % 16 == 0);
+  if (bf16) {
+    const auto* z = static_cast<const __nv_bfloat16*>(logits);
+    auto* dz = static_cast<__nv_bfloat16*>(dlogits);
+    if (vec)
+      cross_entropy_kernel<__nv_bfloat16, true><<<grid, 256, 0, stream>>>(z, n_rows, V, target_ids, loss, dz,
+                                                                          grad_scale, dev_status);
+    else
+      cross_entropy_kernel<__nv_bfloat16, false><<<grid, 256, 0, stream>>>(z, n_rows, V, target_ids, loss, dz,
+                                                                           grad_scale, dev_status);
+  } else {
+    const auto* z = static_cast<const float*>(logits);
+    auto* dz = static_cast<float*>(dlogits);
+    if (vec)
+      cross_entropy_kernel<float, true><<<grid, 256, 0, stream>>>(z, n_rows, V, target_ids, loss, dz, grad_scale,
+                                                                  dev_status);
+    else
+      cross_entropy_kernel<float, false><<<grid, 256, 0, stream>>>(z, n_rows, V, target_ids, loss, dz, grad_scale,
+                                                                   dev_status);
+  }
   return cudaGetLastError();
 }
 

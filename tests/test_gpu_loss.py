@@ -39,10 +39,11 @@ def test_rows_many_turns_and_full_size():
     _check_rows(synth.make_workload(2))
 
 
+@pytest.mark.parametrize("V", [5003, 5008])  # scalar path, 16-byte path
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_cross_entropy_matches_oracle(dtype):
+def test_cross_entropy_matches_oracle(dtype, V):
     rng = np.random.default_rng(0)
-    n, V = 37, 5003
+    n = 37
     z = (rng.standard_normal((n, V)) * 4).astype(np.float32)
     tgt = rng.integers(0, V, size=n).astype(np.int32)
     tgt[3] = -1  # ignored row
@@ -60,6 +61,19 @@ def test_cross_entropy_matches_oracle(dtype):
     assert not g[3].any()
     tol = 1e-6 if dtype == torch.float32 else 0.5 * 2.0 ** -8  # bf16 output: one rounding
     np.testing.assert_allclose(g[keep], 0.5 * r_dz, atol=tol, rtol=tol)
+
+
+def test_cross_entropy_with_masked_logits():
+    """-inf logits (a masked vocabulary entry) contribute nothing and get a zero gradient."""
+    z = torch.randn(4, 64, device="cuda")
+    z[:, 5] = float("-inf")
+    tgt = torch.tensor([0, 1, 2, 3], dtype=torch.int32, device="cuda")
+    loss, dl = opr.opr_cross_entropy(z, tgt)
+    zz = z.clone()
+    zz[:, 5] = -1e30
+    ref = torch.nn.functional.cross_entropy(zz.double(), tgt.long(), reduction="none")
+    torch.testing.assert_close(loss.double(), ref, rtol=1e-5, atol=1e-5)
+    assert bool((dl[:, 5] == 0).all())
 
 
 def test_cross_entropy_flags_target_beyond_vocab():
