@@ -307,9 +307,11 @@ class Ranks:
         return self._reduce(x, self._dist.ReduceOp.SUM)
 
 
-def rank_workload(config: int, rank: int, turns: int | None = None) -> synth.Workload:
-    """This rank's batch: the configuration's shape and length mix, drawn from a rank-specific seed."""
-    return synth.make_workload(config, seed=1000 + config + 7919 * rank, n_turns=turns)
+def rank_workload(config: int, rank: int, turns: int | None = None, seed: int | None = None) -> synth.Workload:
+    """This rank's batch: the configuration's shape and length mix, drawn from a rank-specific seed
+    (base seed 1000 + config unless given)."""
+    base = 1000 + config if seed is None else seed
+    return synth.make_workload(config, seed=base + 7919 * rank, n_turns=turns)
 
 
 def time_runner(r: Runner, steps: int, warmup: int, flush, barrier):
@@ -533,7 +535,16 @@ def run_reference(args, cfg_index):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "conv_tokens_per_s": tok / total,
     }
-    print(json.dumps(line), flush=True)
+    emit(line, args.jsonl)
+
+
+def emit(line: dict, jsonl: str | None) -> None:
+    """Print the benchmark's one JSON line; with --jsonl, also append it to that file."""
+    text = json.dumps(line)
+    print(text, flush=True)
+    if jsonl:
+        with open(jsonl, "a") as fh:
+            fh.write(text + "\n")
 
 
 # ------------------------------------------------------------------ main
@@ -548,6 +559,8 @@ def main():
     ap.add_argument("--no-npass", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seed", type=int, default=None, help="base seed of the synthetic batch (default 1000 + config)")
+    ap.add_argument("--jsonl", default=None, help="also append the JSON line to this file")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -575,7 +588,7 @@ def main():
     flush = lambda: flush_buf.zero_()  # noqa: E731
 
     # every rank runs its own batch of the same shape (weak scaling, no data-path collective)
-    w = rank_workload(args.config, rank, args.turns)
+    w = rank_workload(args.config, rank, args.turns, args.seed)
     r = Runner(w, seed=11 + rank, device=device)
     pairs = r.pairs
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
@@ -677,7 +690,7 @@ def main():
         "clocks": dict(clocks.summary(), remeasured=remeasured),
         "cpu_baseline": cpu,
     }
-    print(json.dumps(line), flush=True)
+    emit(line, args.jsonl)
     if world > 1:
         dist.destroy_process_group()
 

@@ -3,6 +3,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <cstdint>
 #include <cstring>
 
@@ -53,6 +55,16 @@ EncodeTiledFn encode_fn() {
   }
   return fn;
 }
+
+// One NVTX range per entry-point call (named after the call), so that a
+// profiler timeline shows where each library call's launches begin and end.
+// Without an attached tool the push and pop cost a branch each.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // Text of the last OPR_CUDA_ERROR returned on this host thread (opr_last_error).
 thread_local const char* g_last_error = "no error";
@@ -150,6 +162,7 @@ extern "C" {
 opr_status opr_duplication_index(const int32_t* turn_lens, const int32_t* conv_turn_ptr, int32_t n_convs,
                                  int32_t n_turns, int64_t total_tokens, int64_t orig_tokens, int32_t* src_index,
                                  int32_t* copy_index, int32_t* dev_status, void* stream) {
+  CallRange range("opr_duplication_index");
   if (n_convs < 0 || n_turns < 0 || total_tokens < 0 || orig_tokens < 0) return OPR_INVALID_ARG;
   if (total_tokens >= (int64_t{1} << 31) || orig_tokens > total_tokens) return OPR_INVALID_ARG;
   if (!conv_turn_ptr || !dev_status || (n_turns > 0 && !turn_lens) || (total_tokens > 0 && !src_index) ||
@@ -163,6 +176,7 @@ opr_status opr_duplication_index(const int32_t* turn_lens, const int32_t* conv_t
 
 opr_status opr_gather_rows(const void* x, int64_t orig_tokens, int64_t row_bytes, const int32_t* src_index,
                            int64_t total_tokens, void* y, int32_t* dev_status, void* stream) {
+  CallRange range("opr_gather_rows");
   if (orig_tokens < 0 || total_tokens < 0 || row_bytes <= 0) return OPR_INVALID_ARG;
   if (total_tokens == 0) return OPR_OK;
   if (!x || !src_index || !y) return OPR_INVALID_ARG;
@@ -174,6 +188,7 @@ opr_status opr_gather_rows(const void* x, int64_t orig_tokens, int64_t row_bytes
 
 opr_status opr_fold_rows(const float* dy, int64_t total_tokens, int64_t width, const int32_t* copy_index,
                          int32_t slots, int64_t orig_tokens, float* dx, int32_t* dev_status, void* stream) {
+  CallRange range("opr_fold_rows");
   if (orig_tokens < 0 || total_tokens < 0 || width <= 0 || slots < 1 || slots > 64) return OPR_INVALID_ARG;
   if (orig_tokens == 0) return OPR_OK;
   if (!dy || !copy_index || !dx) return OPR_INVALID_ARG;
@@ -204,6 +219,7 @@ opr_status opr_kpass_plan(const int32_t* turn_lens, const int32_t* conv_turn_ptr
                           int32_t n_seqs, int32_t n_convs, int32_t n_turns, int32_t K, int32_t n_out_turns,
                           int32_t n_out_convs, int32_t* out_turn_lens, int32_t* out_conv_turn_ptr,
                           int32_t* out_seq_conv_ptr, int32_t* out_turn_src, int32_t* dev_status, void* stream) {
+  CallRange range("opr_kpass_plan");
   if (n_seqs < 0 || n_convs < 0 || n_turns < 0 || K < 1 || n_out_turns < 0 || n_out_convs < 0) return OPR_INVALID_ARG;
   if (!conv_turn_ptr || !seq_conv_ptr || !out_conv_turn_ptr || !out_seq_conv_ptr || !dev_status ||
       (n_turns > 0 && !turn_lens) || (n_out_turns > 0 && (!out_turn_lens || !out_turn_src)))
@@ -224,6 +240,7 @@ opr_status opr_kpass_index(const int32_t* turn_lens, int32_t n_turns, const int3
                            const int32_t* out_turn_src, int32_t n_out_turns, int64_t total_tokens, int64_t orig_tokens,
                            int32_t slots, int32_t* src_index, int32_t* copy_index, void* workspace,
                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  CallRange range("opr_kpass_index");
   if (n_turns < 0 || n_out_turns < 0 || total_tokens < 0 || orig_tokens < 0 || slots < 2 || slots > 64)
     return OPR_INVALID_ARG;
   if (total_tokens >= (int64_t{1} << 31)) return OPR_INVALID_ARG;
@@ -252,6 +269,7 @@ int64_t opr_loss_row_count(const int32_t* turn_lens, int32_t n_turns) {
 
 opr_status opr_loss_rows(const int32_t* turn_lens, int32_t n_turns, int64_t total_tokens, int64_t orig_tokens,
                          int64_t n_rows, int32_t* rows, int32_t* targets, int32_t* dev_status, void* stream) {
+  CallRange range("opr_loss_rows");
   if (n_turns < 0 || total_tokens < 0 || orig_tokens < 0 || n_rows < 0) return OPR_INVALID_ARG;
   if (total_tokens >= (int64_t{1} << 31)) return OPR_INVALID_ARG;
   if (!dev_status || (n_turns > 0 && !turn_lens) || (n_rows > 0 && (!rows || !targets))) return OPR_INVALID_ARG;
@@ -264,6 +282,7 @@ opr_status opr_loss_rows(const int32_t* turn_lens, int32_t n_turns, int64_t tota
 opr_status opr_cross_entropy(const void* logits, int32_t dtype, int64_t n_rows, int32_t vocab,
                              const int32_t* target_ids, float* loss, void* dlogits, float grad_scale,
                              int32_t* dev_status, void* stream) {
+  CallRange range("opr_cross_entropy");
   if (n_rows < 0 || vocab <= 0 || n_rows >= (int64_t{1} << 31)) return OPR_INVALID_ARG;
   if (dtype != OPR_DTYPE_BF16 && dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
   if (n_rows == 0) return OPR_OK;
@@ -289,6 +308,7 @@ opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* conv_turn_p
                             int32_t max_seqlen, int32_t* cu_seqlens, int8_t* token_type, int32_t* turn_idx,
                             int32_t* conv_idx, int32_t* pos_id, uint8_t* block_map, void* workspace,
                             size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  CallRange range("opr_build_layout");
   if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return OPR_INVALID_ARG;
   if (!conv_turn_ptr || !seq_conv_ptr || !cu_seqlens || !workspace || !dev_status) return OPR_INVALID_ARG;
   if (n_turns > 0 && !turn_lens) return OPR_INVALID_ARG;
@@ -305,6 +325,7 @@ opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* conv_turn_p
 opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, const int32_t* pos_id,
                     int64_t total_tokens, int32_t n_heads, int32_t head_dim, double base, int32_t inverse,
                     int32_t* dev_status, void* stream) {
+  CallRange range("opr_rope");
   if (total_tokens < 0 || n_heads < 0 || head_dim <= 0 || head_dim % 2 != 0 || head_dim > 256) return OPR_INVALID_ARG;
   auto known = [](int32_t t) { return t == OPR_DTYPE_BF16 || t == OPR_DTYPE_FP16 || t == OPR_DTYPE_FP32; };
   if (!known(x_dtype) || !known(y_dtype)) return OPR_UNSUPPORTED;
@@ -321,6 +342,7 @@ opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_
                         int32_t n_turns, int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv,
                         int32_t head_dim, float scale, void* o, int32_t o_dtype, float* lse, int32_t* dev_status,
                         void* stream) {
+  CallRange range("opr_attn_fwd");
   if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return OPR_INVALID_ARG;
   if (total_tokens == 0) return OPR_OK;
   if (!attn_args_ok(q, k, v, hq, hkv, head_dim, scale)) return OPR_INVALID_ARG;
@@ -375,6 +397,7 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
                                int32_t n_turns, int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv,
                                int32_t head_dim, float scale, float* dq, float* dk, float* dv, void* workspace,
                                size_t workspace_bytes, int32_t* dev_status, int32_t stages, void* stream) {
+  CallRange range("opr_attn_bwd_stages");
   if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return OPR_INVALID_ARG;
   if (stages & ~(OPR_BWD_ROW_TERMS | OPR_BWD_DQ | OPR_BWD_DKDV)) return OPR_INVALID_ARG;
   if (total_tokens == 0 || stages == 0) return OPR_OK;
