@@ -39,6 +39,15 @@ cudaError_t launch_kpass_index(const int32_t* turn_lens, int32_t n_turns, const 
                                int32_t* dev_status, cudaStream_t stream);
 
 namespace {
+thread_local const char* g_cuda_error_text = "no error";
+}  // namespace
+
+opr_status record_cuda_error(cudaError_t e) {
+  g_cuda_error_text = cudaGetErrorString(e);
+  return OPR_CUDA_ERROR;
+}
+
+namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -66,18 +75,12 @@ struct CallRange {
   CallRange& operator=(const CallRange&) = delete;
 };
 
-// Text of the last OPR_CUDA_ERROR returned on this host thread (opr_last_error).
-thread_local const char* g_last_error = "no error";
-
-opr_status cuda_fail(cudaError_t e) {
-  g_last_error = cudaGetErrorString(e);
-  return OPR_CUDA_ERROR;
-}
+opr_status cuda_fail(cudaError_t e) { return record_cuda_error(e); }
 
 opr_status status_of(cudaError_t e) { return e == cudaSuccess ? OPR_OK : cuda_fail(e); }
 
 opr_status map_fail() {
-  g_last_error = "TMA tensor map encoding failed (cuTensorMapEncodeTiled)";
+  g_cuda_error_text = "TMA tensor map encoding failed (cuTensorMapEncodeTiled)";
   return OPR_CUDA_ERROR;
 }
 
@@ -295,7 +298,7 @@ opr_status opr_cross_entropy(const void* logits, int32_t dtype, int64_t n_rows, 
 
 const char* opr_version(void) { return "opr 0.1.0 sm_100a"; }
 
-const char* opr_last_error(void) { return g_last_error; }
+const char* opr_last_error(void) { return g_cuda_error_text; }
 
 size_t opr_layout_workspace_bytes(int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
                                   int32_t max_seqlen) {

@@ -30,12 +30,15 @@ void* g_scratch_ptr[kMaxDevices] = {nullptr};
 // Device address of the array on the current device, looked up once per device.
 opr_status scratch_on_current_device(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return OPR_CUDA_ERROR;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_error(e);
   if (dev < 0 || dev >= kMaxDevices) return OPR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mutex);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return OPR_CUDA_ERROR;
+    const cudaError_t ea = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (ea != cudaSuccess) return record_cuda_error(ea);
+    if (p == nullptr) return record_cuda_error(cudaErrorInvalidSymbol);
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
