@@ -57,12 +57,13 @@ MEASURED_TRAFFIC = {
 }
 
 
-def measured_traffic(kernel: str, config_index: int, turns):
-    """Bytes per launch recorded for this kernel and workload, or None when absent or stale."""
+def measured_traffic(kernel: str, config_index: int, turns, seed=None):
+    """Bytes per launch recorded for this kernel and workload (the default seeded batch), or None
+    when absent, stale or measured on another batch."""
     import hashlib
 
     rec = MEASURED_TRAFFIC.get(kernel)
-    if rec is None or rec["config_index"] != config_index or turns is not None:
+    if rec is None or rec["config_index"] != config_index or turns is not None or seed is not None:
         return None
     h = hashlib.sha256()
     for f in rec["sources"]:
@@ -654,7 +655,7 @@ def main():
     dom = max(("attn_fwd", "bwd_dq", "bwd_dkdv"), key=lambda k: mean[k])
     achieved = fl[dom] / (mean[dom] * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
-                "frac": achieved / bf16_peak, "traffic": measured_traffic(dom, args.config, args.turns),
+                "frac": achieved / bf16_peak, "traffic": measured_traffic(dom, args.config, args.turns, args.seed),
                 "traffic_unit": "bytes per launch (ncu dram read + write)",
                 "peak_source": f"{peak_src} bf16_tflops (burst); sustained {bf16_sust}",
                 "frac_of_sustained": achieved / bf16_sust if bf16_sust else None,
