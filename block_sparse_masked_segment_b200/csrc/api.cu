@@ -9,6 +9,7 @@
 #include <cstring>
 
 #include "attn_common.cuh"
+#include "host_status.h"
 #include "opr_internal.cuh"
 
 namespace opr {

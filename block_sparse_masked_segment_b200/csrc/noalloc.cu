@@ -12,6 +12,7 @@
 
 #include <mutex>
 
+#include "host_status.h"
 #include "opr_internal.cuh"
 
 namespace opr {

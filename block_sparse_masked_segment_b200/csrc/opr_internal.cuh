@@ -116,10 +116,6 @@ cudaError_t launch_layout(const int32_t* turn_lens, const int32_t* conv_turn_ptr
                           int32_t* pos_id, uint8_t* block_map, void* ws, int32_t* dev_status,
                           cudaStream_t stream);
 
-// Records the text of a CUDA error for opr_last_error() on this host thread and
-// returns OPR_CUDA_ERROR (defined in api.cu).
-opr_status record_cuda_error(cudaError_t e);
-
 cudaError_t launch_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, const int32_t* pos_id,
                         int64_t total, int32_t n_heads, int32_t head_dim, double base, int32_t inverse,
                         int32_t* dev_status, cudaStream_t stream);
