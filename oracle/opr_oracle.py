@@ -13,7 +13,8 @@ evaluated densely and slowly in float64 with numpy:
   ``dense_mask``     the visibility rules of the four token types
   (same note, section "分块稀疏注意力掩码"; English note, "Method").
 * ``block_map``      classification of 128 x 128 tiles as empty / full / partial,
-  counted from the dense mask.
+  counted from the dense mask; ``key_half_map`` marks which 64-key halves of a
+  tile some query of the tile sees.
 * ``rope``           rotate-half rotary embedding by position id (the pages'
   "位置编码等价" argument in "理论保证" relies on it; Qwen-3 uses it).
 * ``attention_fwd`` / ``attention_bwd``
@@ -166,6 +167,27 @@ def block_map(lay: Layout, tile: int = TILE, max_seqlen: int | None = None) -> n
             counts[ql // tile, :len(edges)] += np.add.reduceat(row.astype(np.int64), edges)
         cls = np.where(counts == 0, EMPTY, np.where(counts == tile * tile, FULL, PARTIAL))
         out[s] = cls.astype(np.uint8)
+    return out
+
+
+def key_half_map(lay: Layout, tile: int = TILE, max_seqlen: int | None = None) -> np.ndarray:
+    """uint8 [n_seqs, T, T]: for each tile, bit h (h = 0, 1) set when some query of the
+    tile sees some key of its key half h (keys [h tile/2, (h + 1) tile/2) of the tile).
+    A non-empty tile with one bit clear has a key half that no query sees: the part of
+    the tile's products that sub-tile skipping leaves out."""
+    ms = lay.max_seqlen if max_seqlen is None else max_seqlen
+    nt = (ms + tile - 1) // tile
+    half = tile // 2
+    out = np.zeros((lay.n_seqs, nt, nt), dtype=np.uint8)
+    for s in range(lay.n_seqs):
+        a, b = int(lay.cu_seqlens[s]), int(lay.cu_seqlens[s + 1])
+        L = b - a
+        seen = np.zeros((nt, 2 * nt), dtype=bool)
+        edges = np.arange(0, L, half)
+        for ql in range(L):
+            row = mask_row(lay, a + ql, a, b)
+            seen[ql // tile, :len(edges)] |= np.logical_or.reduceat(row, edges)
+        out[s] = (seen[:, 0::2].astype(np.uint8) | (seen[:, 1::2].astype(np.uint8) << 1))
     return out
 
 

@@ -175,3 +175,36 @@ def test_visible_pairs_matches_closed_form():
     # by hand: turn 0 gives 8256 + 196864 + 65664 + 196736, turn 1 (A = 384)
     # gives 57408 + 393472 + 163968 + 295040
     assert orc.visible_pairs(lay) == expect == 1377408
+
+
+def test_key_half_map_by_brute_force():
+    """key_half_map against the dense mask, and consistent with the block map (a tile is empty
+    exactly when neither half is seen; a full tile has both halves seen)."""
+    w = synth.random_small_workload(8, n_seqs=2, max_convs=3, max_turns=4)
+    lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    km = orc.key_half_map(lay)
+    bm = orc.block_map(lay)
+    T = km.shape[1]
+    for s in range(lay.n_seqs):
+        m = orc.dense_mask(lay, s)
+        L = m.shape[0]
+        for I in range(T):
+            for J in range(T):
+                q = m[I * 128:min((I + 1) * 128, L)]
+                bits = 0
+                for h in range(2):
+                    ks = slice(J * 128 + 64 * h, min(J * 128 + 64 * (h + 1), L))
+                    if q.size and q[:, ks].size and q[:, ks].any():
+                        bits |= 1 << h
+                assert km[s, I, J] == bits
+                assert (bits == 0) == (bm[s, I, J] == orc.EMPTY)
+                if bm[s, I, J] == orc.FULL:
+                    assert bits == 3
+
+
+def test_key_half_map_of_a_causal_segment():
+    """One causal segment of 256 tokens: the diagonal tiles see both key halves, the tile above
+    the diagonal neither (closed form of the causal mask)."""
+    lay = orc.build_layout([[256, 0, 0]], [0, 1], [0, 1])
+    km = orc.key_half_map(lay)
+    assert km[0].tolist() == [[3, 0], [3, 3]]
