@@ -45,6 +45,7 @@ EXPORTED_SYMBOLS = (
     "opr_loss_row_count",
     "opr_loss_rows",
     "opr_cross_entropy",
+    "opr_testing_set_wait_limit_ns",
 )
 
 BWD_ROW_TERMS, BWD_DQ, BWD_DKDV = 1, 2, 4
@@ -87,7 +88,7 @@ def load_library() -> ctypes.CDLL:
     lib.opr_fold_rows.restype = ctypes.c_int
     lib.opr_fold_rows.argtypes = [P, I64, I64, P, I32, I64, P, P, P]
     lib.opr_kpass_sizes.restype = ctypes.c_int
-    lib.opr_kpass_sizes.argtypes = [P, I32, I32, P, P]
+    lib.opr_kpass_sizes.argtypes = [P, P, P, I32, I32, I32, I32, P, P, P, P, P]
     lib.opr_kpass_plan.restype = ctypes.c_int
     lib.opr_kpass_plan.argtypes = [P, P, P, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P]
     lib.opr_kpass_index_workspace_bytes.restype = ctypes.c_size_t
@@ -112,13 +113,15 @@ def load_library() -> ctypes.CDLL:
     lib.opr_attn_bwd_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.opr_attn_bwd.restype = I32
     lib.opr_attn_bwd.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F,
-                                 P, P, P, P, SZ, P, P]
+                                 P, P, P, P, D, P, SZ, P, P]
     lib.opr_attn_bwd_stages.restype = I32
     lib.opr_attn_bwd_stages.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32,
-                                        F, P, P, P, P, SZ, P, I32, P]
+                                        F, P, P, P, P, D, P, SZ, P, I32, P]
+    lib.opr_testing_set_wait_limit_ns.restype = ctypes.c_uint64
+    lib.opr_testing_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.opr_attn_bwd_noalloc.restype = I32
     lib.opr_attn_bwd_noalloc.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32,
-                                         F, P, P, P, P, P]
+                                         F, P, P, P, P, D, P, P]
     _lib = lib
     return lib
 
@@ -266,14 +269,29 @@ def opr_rope(x: torch.Tensor, pos_id: torch.Tensor, base: float, inverse: bool =
 
 def _attn_shapes(q, k, v, lay: Layout):
     _need_cuda(q, k, v)
-    if q.dtype not in (torch.float16, torch.bfloat16) or k.dtype != q.dtype:
-        raise OprError("q and k must both be fp16 or both bf16")
+    if q.dtype != torch.float16 or k.dtype != torch.float16:
+        raise OprError("q and k must be fp16 (rotated by opr_rope with an fp16 output)")
     if v.dtype != torch.bfloat16:
         raise OprError("v must be bf16")
     total, hq, d = q.shape
     if k.shape != v.shape or k.shape[0] != total or k.shape[2] != d or total != lay.total:
         raise OprError("shape mismatch between q, k, v and the layout")
     return total, hq, k.shape[1], d
+
+
+def _grad_buffers(out, q, total, hq, hkv, d):
+    """(dq, dk, dv): the caller's buffers after checking them, or new fp32 tensors."""
+    shapes = ((total, hq, d), (total, hkv, d), (total, hkv, d))
+    if out is None:
+        return tuple(torch.empty(sh, dtype=torch.float32, device=q.device) for sh in shapes)
+    if len(out) != 3:
+        raise OprError("out must be (dq, dk, dv)")
+    for name, t, sh in zip(("dq", "dk", "dv"), out, shapes):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or tuple(t.shape) != sh:
+            raise OprError(f"out {name} must be an fp32 tensor of shape {sh}")
+        if t.device != q.device or not t.is_contiguous():
+            raise OprError(f"out {name} must be contiguous on {q.device}")
+    return tuple(out)
 
 
 def opr_attn_fwd(q, k, v, lay: Layout, scale: float | None = None, out_dtype=torch.float32):
@@ -291,9 +309,18 @@ def opr_attn_fwd(q, k, v, lay: Layout, scale: float | None = None, out_dtype=tor
     return o, lse
 
 
+def _rope_args(rope_base, lay: Layout):
+    """(pos_id pointer, base) of the rotation the backward undoes in its epilogues, or (None, 0)."""
+    if rope_base is None:
+        return None, 0.0
+    return _ptr(lay.pos_id), float(rope_base)
+
+
 def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, workspace=None, out=None,
-                 stages: int | None = None):
-    """dQ [total, hq, d], dK and dV [total, hkv, d] (fp32), w.r.t. the rotated q, k and v.
+                 stages: int | None = None, rope_base: float | None = None):
+    """dQ [total, hq, d], dK and dV [total, hkv, d] (fp32), w.r.t. the rotated q, k and v; with
+    ``rope_base``, dQ and dK are rotated back by the layout's position ids in the kernels'
+    epilogues (the gradients w.r.t. the unrotated q and k).
 
     ``out`` = (dq, dk, dv) reuses buffers; ``stages`` (OR of BWD_ROW_TERMS,
     BWD_DQ, BWD_DKDV) runs only those kernels through opr_attn_bwd_stages, with
@@ -304,18 +331,14 @@ def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, w
     if do.dtype != torch.bfloat16 or lse.dtype != torch.float32:
         raise OprError("dout must be bf16 and lse fp32")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    if out is None:
-        out = (torch.empty((total, hq, d), dtype=torch.float32, device=q.device),
-               torch.empty((total, hkv, d), dtype=torch.float32, device=q.device),
-               torch.empty((total, hkv, d), dtype=torch.float32, device=q.device))
-    dq, dk, dv = out
+    dq, dk, dv = _grad_buffers(out, q, total, hq, hkv, d)
     wb = opr_attn_bwd_workspace_bytes(lay.n_seqs, lay.max_seqlen, hq, d)
     if workspace is None or workspace.numel() < wb:
         workspace = torch.empty(max(wb, 256), dtype=torch.uint8, device=q.device)
     args = (_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16, _ptr(do),
             _ptr(lse), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace), lay.n_seqs, lay.n_convs,
             lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
-            _ptr(workspace), workspace.numel(), _ptr(lay.dev_status))
+            *_rope_args(rope_base, lay), _ptr(workspace), workspace.numel(), _ptr(lay.dev_status))
     lib = load_library()
     if stages is None:
         _check(lib.opr_attn_bwd(*args, _stream(q.device)), "opr_attn_bwd")
@@ -324,12 +347,14 @@ def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, w
     return dq, dk, dv
 
 
-def opr_attn_bwd_stages(q, k, v, o, do, lse, lay: Layout, stages: int, workspace, out, scale=None):
+def opr_attn_bwd_stages(q, k, v, o, do, lse, lay: Layout, stages: int, workspace, out, scale=None, rope_base=None):
     """Run only the backward kernels selected by ``stages`` (see opr_attn_bwd)."""
-    return opr_attn_bwd(q, k, v, o, do, lse, lay, scale, workspace=workspace, out=out, stages=stages)
+    return opr_attn_bwd(q, k, v, o, do, lse, lay, scale, workspace=workspace, out=out, stages=stages,
+                        rope_base=rope_base)
 
 
-def opr_attn_bwd_noalloc(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, out=None):
+def opr_attn_bwd_noalloc(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, out=None,
+                         rope_base: float | None = None):
     """opr_attn_bwd with the scratch in the library's fixed device array (no workspace argument).
 
     For callers that cannot allocate device memory at the call; see the C
@@ -341,16 +366,13 @@ def opr_attn_bwd_noalloc(q, k, v, o, do, lse, lay: Layout, scale: float | None =
     if do.dtype != torch.bfloat16 or lse.dtype != torch.float32:
         raise OprError("dout must be bf16 and lse fp32")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    if out is None:
-        out = (torch.empty((total, hq, d), dtype=torch.float32, device=q.device),
-               torch.empty((total, hkv, d), dtype=torch.float32, device=q.device),
-               torch.empty((total, hkv, d), dtype=torch.float32, device=q.device))
-    dq, dk, dv = out
-    st = load_library().opr_attn_bwd_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16,
-        _ptr(do), _ptr(lse), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace), lay.n_seqs, lay.n_convs,
-        lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
-        _ptr(lay.dev_status), _stream(q.device))
+    dq, dk, dv = _grad_buffers(out, q, total, hq, hkv, d)
+    with torch.cuda.device(q.device):  # the library uses the current device's array
+        st = load_library().opr_attn_bwd_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16,
+            _ptr(do), _ptr(lse), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace), lay.n_seqs,
+            lay.n_convs, lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+            *_rope_args(rope_base, lay), _ptr(lay.dev_status), _stream(q.device))
     _check(st, "opr_attn_bwd_noalloc")
     return dq, dk, dv
 
@@ -448,9 +470,11 @@ def opr_kpass(turn_lens, conv_turn_ptr, seq_conv_ptr, K: int, device="cuda") -> 
     cp = np.ascontiguousarray(np.asarray(conv_turn_ptr, dtype=np.int32))
     sp = np.ascontiguousarray(np.asarray(seq_conv_ptr, dtype=np.int32))
     n_turns, n_convs, n_seqs = lens.shape[0], cp.size - 1, sp.size - 1
-    nt, nc = ctypes.c_int64(0), ctypes.c_int64(0)
-    _check(lib.opr_kpass_sizes(cp.ctypes.data, n_convs, K, ctypes.byref(nt), ctypes.byref(nc)), "opr_kpass_sizes")
-    n_out_turns, n_out_convs = nt.value, nc.value
+    sizes = [ctypes.c_int64(0) for _ in range(5)]
+    lens_flat = np.ascontiguousarray(lens.reshape(-1))
+    _check(lib.opr_kpass_sizes(lens_flat.ctypes.data, cp.ctypes.data, sp.ctypes.data, n_seqs, n_convs, n_turns, K,
+                               *(ctypes.byref(x) for x in sizes)), "opr_kpass_sizes")
+    n_out_turns, n_out_convs, total, max_seqlen, orig = (x.value for x in sizes)
     dev = lambda a: torch.as_tensor(a).to(device=device, dtype=torch.int32).contiguous()  # noqa: E731
     tl, cpd, spd = dev(lens.reshape(-1)), dev(cp), dev(sp)
     out_lens = torch.empty((n_out_turns, 3), dtype=torch.int32, device=device)
@@ -461,21 +485,6 @@ def opr_kpass(turn_lens, conv_turn_ptr, seq_conv_ptr, K: int, device="cuda") -> 
     _check(lib.opr_kpass_plan(_ptr(tl), _ptr(cpd), _ptr(spd), n_seqs, n_convs, n_turns, K, n_out_turns, n_out_convs,
                               _ptr(out_lens), _ptr(out_cp), _ptr(out_sp), _ptr(out_src), _ptr(status),
                               _stream(device)), "opr_kpass_plan")
-    # sizes of the arrangement, counted on the host from the same lengths (allocation only)
-    h, t, r = (np.maximum(lens[:, i].astype(np.int64), 0) for i in range(3))
-    total, seq_len, turn_hist = 0, [], []
-    for s in range(n_seqs):
-        L = 0
-        for c in range(int(sp[s]), int(sp[s + 1])):
-            t0, t1 = int(cp[c]), int(cp[c + 1])
-            n = t1 - t0
-            k = min(K, n)
-            for g in range(k):
-                b0, b1 = (g * n) // k, ((g + 1) * n) // k
-                L += int((h[t0:t0 + b0] + r[t0:t0 + b0]).sum() + (h + t + 2 * r)[t0 + b0:t0 + b1].sum())
-        seq_len.append(L)
-        total += L
-    orig = int((h + t + r).sum())
     slots = K + 1
     src = torch.empty(total, dtype=torch.int32, device=device)
     copies = torch.empty((orig, slots), dtype=torch.int32, device=device)
@@ -484,7 +493,7 @@ def opr_kpass(turn_lens, conv_turn_ptr, seq_conv_ptr, K: int, device="cuda") -> 
     _check(lib.opr_kpass_index(_ptr(tl), n_turns, _ptr(out_lens), _ptr(out_src), n_out_turns, total, orig, slots,
                                _ptr(src), _ptr(copies), _ptr(ws), ws.numel(), _ptr(status), _stream(device)),
            "opr_kpass_index")
-    kp = KPass(K, out_lens, out_cp, out_sp, out_src, src, copies, total, max(seq_len) if seq_len else 0, status)
+    kp = KPass(K, out_lens, out_cp, out_sp, out_src, src, copies, total, max_seqlen, status)
     kp._keep = (tl, cpd, spd, ws)  # alive until the stream has used them
     return kp
 

@@ -5,9 +5,13 @@
 
 #include <nvtx3/nvToolsExt.h>
 
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 
+#include <atomic>
+
+#include "../../include/opr_testing.h"
 #include "attn_common.cuh"
 #include "host_status.h"
 #include "opr_internal.cuh"
@@ -39,8 +43,23 @@ cudaError_t launch_kpass_index(const int32_t* turn_lens, int32_t n_turns, const 
                                int32_t slots, int32_t* src_index, int32_t* copy_index, int64_t* ws,
                                int32_t* dev_status, cudaStream_t stream);
 
+// Sizes every attention entry point accepts (declared in host_status.h).
+bool sizes_ok(int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total, int32_t max_seqlen) {
+  if (n_seqs < 0 || n_convs < 0 || n_turns < 0 || total < 0 || max_seqlen < 0) return false;
+  if (total >= (int64_t{1} << 31)) return false;  // token offsets are int32
+  if (n_seqs > 65535) return false;
+  const int64_t T = (max_seqlen + kTile - 1) / kTile;
+  if (T > 65535) return false;
+  if (static_cast<int64_t>(n_seqs) * T >= (int64_t{1} << 31)) return false;
+  // every sequence is at most max_seqlen long, so the tokens fit n_seqs * T tiles; the
+  // workspaces sized from (n_seqs, max_seqlen) rely on it
+  if (total > static_cast<int64_t>(n_seqs) * T * kTile) return false;
+  return true;
+}
+
 namespace {
 thread_local const char* g_cuda_error_text = "no error";
+std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};  // pipeline-wait limit of the attention kernels
 }  // namespace
 
 opr_status record_cuda_error(cudaError_t e) {
@@ -112,16 +131,6 @@ opr_status device_check() {
   return major == 10 ? OPR_OK : OPR_UNSUPPORTED;
 }
 
-bool sizes_ok(int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total, int32_t max_seqlen) {
-  if (n_seqs < 0 || n_convs < 0 || n_turns < 0 || total < 0 || max_seqlen < 0) return false;
-  if (total >= (int64_t{1} << 31)) return false;  // token offsets are int32
-  if (n_seqs > 65535) return false;
-  const int64_t T = (max_seqlen + kTile - 1) / kTile;
-  if (T > 65535) return false;
-  if (static_cast<int64_t>(n_seqs) * T >= (int64_t{1} << 31)) return false;
-  return true;
-}
-
 AttnParams base_params(const int32_t* cu_seqlens, const int32_t* conv_idx, const void* ws, int32_t n_seqs,
                        int32_t n_convs, int32_t n_turns, int64_t total, int32_t max_seqlen, int32_t hq, int32_t hkv,
                        float scale, int32_t* dev_status) {
@@ -144,6 +153,7 @@ AttnParams base_params(const int32_t* cu_seqlens, const int32_t* conv_idx, const
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.dev_status = dev_status;
+  p.wait_ns = g_wait_limit_ns.load();
   return p;
 }
 
@@ -202,20 +212,47 @@ opr_status opr_fold_rows(const float* dy, int64_t total_tokens, int64_t width, c
                                     static_cast<cudaStream_t>(stream)));
 }
 
-opr_status opr_kpass_sizes(const int32_t* conv_turn_ptr, int32_t n_convs, int32_t K, int64_t* n_out_turns,
-                           int64_t* n_out_convs) {
-  if (!conv_turn_ptr || !n_out_turns || !n_out_convs || n_convs < 0 || K < 1) return OPR_INVALID_ARG;
-  int64_t turns = 0, convs = 0;
-  for (int c = 0; c < n_convs; ++c) {
-    const int64_t n = conv_turn_ptr[c + 1] - conv_turn_ptr[c];
-    if (n < 0) return OPR_INVALID_ARG;
-    const int64_t k = n < K ? n : K;
-    for (int64_t g = 0; g < k; ++g) turns += ((g + 1) * n) / k;
-    convs += k;
+opr_status opr_kpass_sizes(const int32_t* turn_lens, const int32_t* conv_turn_ptr, const int32_t* seq_conv_ptr,
+                           int32_t n_seqs, int32_t n_convs, int32_t n_turns, int32_t K, int64_t* n_out_turns,
+                           int64_t* n_out_convs, int64_t* total_tokens, int64_t* max_seqlen, int64_t* orig_tokens) {
+  if (!conv_turn_ptr || !seq_conv_ptr || (n_turns > 0 && !turn_lens) || !n_out_turns || !n_out_convs ||
+      !total_tokens || !max_seqlen || !orig_tokens)
+    return OPR_INVALID_ARG;
+  if (n_seqs < 0 || n_convs < 0 || n_turns < 0 || K < 1) return OPR_INVALID_ARG;
+  if (conv_turn_ptr[0] != 0 || conv_turn_ptr[n_convs] != n_turns || seq_conv_ptr[0] != 0 ||
+      seq_conv_ptr[n_seqs] != n_convs)
+    return OPR_INVALID_ARG;
+  for (int i = 0; i < 3 * n_turns; ++i)
+    if (turn_lens[i] < 0) return OPR_INVALID_ARG;
+  int64_t turns = 0, convs = 0, total = 0, longest = 0, orig = 0;
+  for (int i = 0; i < n_turns; ++i) orig += int64_t{turn_lens[3 * i]} + turn_lens[3 * i + 1] + turn_lens[3 * i + 2];
+  for (int s = 0; s < n_seqs; ++s) {
+    if (seq_conv_ptr[s + 1] < seq_conv_ptr[s]) return OPR_INVALID_ARG;
+    int64_t seq_len = 0;
+    for (int c = seq_conv_ptr[s]; c < seq_conv_ptr[s + 1]; ++c) {
+      const int64_t t0 = conv_turn_ptr[c], n = conv_turn_ptr[c + 1] - t0;
+      if (n < 0) return OPR_INVALID_ARG;
+      const int64_t k = n < K ? n : K;  // K' = min(K, N) groups, bounds floor(g N / K')
+      for (int64_t g = 0; g < k; ++g) {
+        const int64_t b0 = (g * n) / k, b1 = ((g + 1) * n) / k;
+        for (int64_t j = t0; j < t0 + b0; ++j)  // history: h_j + r_j as one context segment
+          seq_len += int64_t{turn_lens[3 * j]} + turn_lens[3 * j + 2];
+        for (int64_t j = t0 + b0; j < t0 + b1; ++j)  // the group's own turns, laid out one-pass
+          seq_len += int64_t{turn_lens[3 * j]} + turn_lens[3 * j + 1] + 2 * int64_t{turn_lens[3 * j + 2]};
+        turns += b1;
+      }
+      convs += k;
+    }
+    total += seq_len;
+    longest = seq_len > longest ? seq_len : longest;
   }
-  if (turns >= (int64_t{1} << 31) || convs >= (int64_t{1} << 31)) return OPR_INVALID_ARG;
+  if (turns >= (int64_t{1} << 31) || convs >= (int64_t{1} << 31) || total >= (int64_t{1} << 31))
+    return OPR_INVALID_ARG;
   *n_out_turns = turns;
   *n_out_convs = convs;
+  *total_tokens = total;
+  *max_seqlen = longest;
+  *orig_tokens = orig;
   return OPR_OK;
 }
 
@@ -297,7 +334,9 @@ opr_status opr_cross_entropy(const void* logits, int32_t dtype, int64_t n_rows, 
                                         grad_scale, dev_status, static_cast<cudaStream_t>(stream)));
 }
 
-const char* opr_version(void) { return "opr 0.1.0 sm_100a"; }
+const char* opr_version(void) { return "opr 0.2.0 sm_100a"; }
+
+uint64_t opr_testing_set_wait_limit_ns(uint64_t limit_ns) { return g_wait_limit_ns.exchange(limit_ns); }
 
 const char* opr_last_error(void) { return g_cuda_error_text; }
 
@@ -352,7 +391,7 @@ opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_
   if (!attn_args_ok(q, k, v, hq, hkv, head_dim, scale)) return OPR_INVALID_ARG;
   if (!cu_seqlens || !conv_idx || !layout_ws || !o || !lse || !dev_status || !aligned16(o)) return OPR_INVALID_ARG;
   if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
-  if (qk_dtype != OPR_DTYPE_BF16 && qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
+  if (qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
   const bool f16 = qk_dtype == OPR_DTYPE_FP16;
   opr_status st = device_check();
   if (st != OPR_OK) return st;
@@ -373,18 +412,20 @@ namespace {
 // Backward scratch: the row terms, then fp16 copies of dO and V.  Token counts
 // are bounded by n_seqs * ceil(max_seqlen / 128) * 128 and the kv heads by hq.
 struct BwdWs {
-  size_t row_terms, dout16, v16, bytes;
+  size_t absmax, row_terms, dout16, v16, rope, bytes;
 };
 
 BwdWs bwd_ws_map(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
   const size_t T = (static_cast<size_t>(max_seqlen) + kTile - 1) / kTile;
   const size_t tokens = static_cast<size_t>(n_seqs) * T * kTile;
   BwdWs w;
-  w.row_terms = 0;
-  w.dout16 = align_up(2 * sizeof(float) * static_cast<size_t>(hq) * tokens, 256);
+  w.absmax = 0;
+  w.row_terms = 256;
+  w.dout16 = w.row_terms + align_up(2 * sizeof(float) * static_cast<size_t>(hq) * tokens, 256);
   const size_t copy = align_up(sizeof(uint16_t) * tokens * static_cast<size_t>(hq) * static_cast<size_t>(head_dim), 256);
   w.v16 = w.dout16 + copy;
-  w.bytes = w.v16 + copy;
+  w.rope = w.v16 + copy;  // (cos, sin) per position < max_seqlen and rotary pair
+  w.bytes = w.rope + align_up(sizeof(float) * 2 * static_cast<size_t>(max_seqlen) * (head_dim / 2), 256);
   return w;
 }
 }  // namespace
@@ -399,7 +440,8 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
                                const void* dout, const float* lse, const int32_t* cu_seqlens,
                                const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs, int32_t n_convs,
                                int32_t n_turns, int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv,
-                               int32_t head_dim, float scale, float* dq, float* dk, float* dv, void* workspace,
+                               int32_t head_dim, float scale, float* dq, float* dk, float* dv,
+                               const int32_t* rope_pos_id, double rope_base, void* workspace,
                                size_t workspace_bytes, int32_t* dev_status, int32_t stages, void* stream) {
   CallRange range("opr_attn_bwd_stages");
   if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return OPR_INVALID_ARG;
@@ -412,7 +454,8 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
     return OPR_INVALID_ARG;
   if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
-  if (qk_dtype != OPR_DTYPE_BF16 && qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
+  if (qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
+  if (rope_pos_id != nullptr && !(rope_base > 1.0)) return OPR_INVALID_ARG;
   const bool f16 = qk_dtype == OPR_DTYPE_FP16;
   if (workspace_bytes < opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim))
     return OPR_WORKSPACE_TOO_SMALL;
@@ -420,6 +463,7 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   if (st != OPR_OK) return st;
   const BwdWs bw = bwd_ws_map(n_seqs, max_seqlen, hq, head_dim);
   BwdBuffers buf;
+  buf.dout_absmax = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + bw.absmax);
   buf.o = o;
   buf.o_fp32 = o_dtype == OPR_DTYPE_FP32;
   buf.dout = static_cast<const __nv_bfloat16*>(dout);
@@ -427,6 +471,7 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   buf.row_terms = reinterpret_cast<float*>(static_cast<char*>(workspace) + bw.row_terms);
   buf.dout16 = reinterpret_cast<__half*>(static_cast<char*>(workspace) + bw.dout16);
   buf.v16 = reinterpret_cast<__half*>(static_cast<char*>(workspace) + bw.v16);
+  buf.rope_neg_log_base_over_half = rope_pos_id != nullptr ? -log(rope_base) / (head_dim / 2) : 0.0;
   BwdMaps maps;
   if (!make_map(&maps.q, q, total_tokens, hq, head_dim, f16) || !make_map(&maps.k, k, total_tokens, hkv, head_dim, f16) ||
       !make_map(&maps.v, v, total_tokens, hkv, head_dim) || !make_map(&maps.dout, dout, total_tokens, hq, head_dim) ||
@@ -437,11 +482,17 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   AttnParams pq = base_params(cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs, n_turns, total_tokens, max_seqlen,
                               hq, hkv, scale, dev_status);
   pq.lse_in = lse;
+  pq.dout_absmax = buf.dout_absmax;
   pq.d_tiles = buf.row_terms;
   pq.lse2_tiles = pq.d_tiles + static_cast<size_t>(hq) * pq.n_items * kTile;
   pq.dq = dq;
   pq.dk = dk;
   pq.dv = dv;
+  if (rope_pos_id != nullptr) {  // dq and dk w.r.t. the unrotated q and k
+    pq.pos_id = rope_pos_id;
+    pq.rope_cs = reinterpret_cast<const float2*>(static_cast<char*>(workspace) + bw.rope);
+    pq.rope_rows = max_seqlen;
+  }
   AttnParams pkv = pq;
   pkv.sched = ws_ptr<int32_t>(layout_ws, w.k_sched);
   cudaError_t e = launch_attn_bwd(head_dim, f16, maps, buf, pq, pkv, stages, static_cast<cudaStream_t>(stream));
@@ -453,11 +504,12 @@ opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int32_t qk_
                         const void* dout, const float* lse, const int32_t* cu_seqlens, const int32_t* conv_idx,
                         const void* layout_ws, int32_t n_seqs, int32_t n_convs, int32_t n_turns,
                         int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
-                        float scale, float* dq, float* dk, float* dv, void* workspace, size_t workspace_bytes,
-                        int32_t* dev_status, void* stream) {
+                        float scale, float* dq, float* dk, float* dv, const int32_t* rope_pos_id, double rope_base,
+                        void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
   return opr_attn_bwd_stages(q, k, v, qk_dtype, o, o_dtype, dout, lse, cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs,
-                             n_turns, total_tokens, max_seqlen, hq, hkv, head_dim, scale, dq, dk, dv, workspace,
-                             workspace_bytes, dev_status, OPR_BWD_ROW_TERMS | OPR_BWD_DQ | OPR_BWD_DKDV, stream);
+                             n_turns, total_tokens, max_seqlen, hq, hkv, head_dim, scale, dq, dk, dv, rope_pos_id,
+                             rope_base, workspace, workspace_bytes, dev_status,
+                             OPR_BWD_ROW_TERMS | OPR_BWD_DQ | OPR_BWD_DKDV, stream);
 }
 
 }  // extern "C"

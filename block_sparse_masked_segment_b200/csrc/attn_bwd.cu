@@ -34,13 +34,40 @@ constexpr int kListSmem = 1024;  // entries of a tile list kept in shared memory
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ----------------------------------------------------------------------------
+// max |dO| over the whole tensor, as float bits (non-negative floats order
+// like their bits), into *absmax (zeroed before the launch).  It fixes the
+// gradient scale 2^k of the call (grad_scale_exp).
+__global__ void __launch_bounds__(256) dout_absmax_kernel(const __nv_bfloat16* __restrict__ x, int64_t n8,
+                                                          uint32_t* __restrict__ absmax) {
+  float m = 0.f;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      // |bf16| of both halves: clear the sign bits, widen to fp32 by a shift
+      m = fmax3(m, __uint_as_float((w[k] & 0x7FFFu) << 16), __uint_as_float(w[k] & 0x7FFF0000u));
+    }
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+  __shared__ float wm[8];
+  if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wm[w]);
+    atomicMax(absmax, __float_as_uint(m));
+  }
+}
+
 // Row terms, stored negated and per 128-token tile so the kernels can
 // bulk-copy them and fold each into one fused multiply-add:
-// d_tiles[h][tile][c] = -sum_d dO * O and lse2_tiles[h][tile][c] = -LSE * log2(e)
+// d_tiles[h][tile][c] = -2^k sum_d dO * O and lse2_tiles[h][tile][c] = -LSE * log2(e)
 // of token c of tile (s, J); 0 and -inf past the end of the sequence.  The
-// kernel also writes dout16, the fp16 copy of dO that the dkdv kernel reads
-// (bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]; a larger one sets
-// OPR_DEV_FP16_RANGE).
+// kernel also writes dout16, the fp16 copy of 2^k dO that the dkdv kernel
+// reads (exact: 2^k dO lies in fp16's normal range except for entries below
+// 2^-10 of max |dO|; an inf or NaN sets OPR_DEV_FP16_RANGE).
 __device__ __forceinline__ bool fp16_range_ok(float x) { return fabsf(x) <= 65504.f; }
 
 // One block of 256 threads per (tile, head); each warp walks 16 of the tile's
@@ -51,9 +78,11 @@ __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o
                                                         const float* __restrict__ lse, const int32_t* __restrict__ cu_seqlens,
                                                         int64_t total, int32_t hq, int32_t T, float* __restrict__ d_tiles,
                                                         float* __restrict__ lse2_tiles, __half* __restrict__ dout16,
+                                                        const uint32_t* __restrict__ absmax,
                                                         int32_t* __restrict__ dev_status) {
   constexpr int kE = D / 32;  // elements per lane: 4 (D = 128) or 2 (D = 64)
   const int tile = blockIdx.x, h = blockIdx.y;
+  const float gs = pow2f(grad_scale_exp(*absmax));  // 2^k
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = tile / T, J = tile % T;
   const int seq0 = cu_seqlens[s];
@@ -75,12 +104,13 @@ __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o
     if constexpr (kE == 4) {
       const uint2 u = *reinterpret_cast<const uint2*>(dout + base);
       const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-      df[0] = __low2float(d2[0]); df[1] = __high2float(d2[0]); df[2] = __low2float(d2[1]); df[3] = __high2float(d2[1]);
+      df[0] = __low2float(d2[0]) * gs; df[1] = __high2float(d2[0]) * gs;
+      df[2] = __low2float(d2[1]) * gs; df[3] = __high2float(d2[1]) * gs;
       *reinterpret_cast<uint2*>(dout16 + base) = make_uint2(pack_f16x2(df[0], df[1]), pack_f16x2(df[2], df[3]));
     } else {
       const uint32_t u = *reinterpret_cast<const uint32_t*>(dout + base);
       const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(&u);
-      df[0] = __low2float(d2); df[1] = __high2float(d2);
+      df[0] = __low2float(d2) * gs; df[1] = __high2float(d2) * gs;
       *reinterpret_cast<uint32_t*>(dout16 + base) = pack_f16x2(df[0], df[1]);
     }
     if constexpr (sizeof(OT) == 4) {
@@ -104,6 +134,20 @@ __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o
     }
   }
   if (!in_range) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
+}
+
+// (cos, sin) of the rotary angle p base^(-2j/D) for positions p < rows and pairs
+// j < half, angle formed in fp64 as opr_rope forms it; read by the dQ and dK
+// epilogues that rotate the gradients back.
+__global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ cs, int32_t rows, int32_t half,
+                                                         double neg_log_base_over_half) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (i >= static_cast<int64_t>(rows) * half) return;
+  const int pos = static_cast<int>(i / half), j = static_cast<int>(i % half);
+  const double theta = exp(static_cast<double>(j) * neg_log_base_over_half);
+  double sd, cd;
+  sincos(static_cast<double>(pos) * theta, &sd, &cd);
+  cs[i] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
 }
 
 // fp16 copy of V for the dkdv kernel, eight values per thread (same range rule).
@@ -210,61 +254,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
         const int e = entry(j);
-        const int J = e >> 2;
-        if (j >= kStages && !mbar_wait(&sm.bar_kempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
+        const int J = entry_index(e);
+        if (j >= kStages && !mbar_wait(&sm.bar_kempty[st], ((j / kStages) + 1) & 1, abort_flag, p.wait_ns))
           break;
-        const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+        const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
         mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes + (partial ? sizeof(TileMeta) : 0));
         tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, seq0 + J * kTile);
         if (partial) bulk_load(&sm.kmeta[st], tmeta + J, sizeof(TileMeta), &sm.bar_kfull[st]);
         issued = j + 1;
       }
-      if (*abort_flag) {
-        mbar_wait(&sm.bar_qdo, 0, nullptr, kWaitLimitNs);
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-          mbar_wait(&sm.bar_kfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
-      }
+      // every copy issued has landed before the CTA exits (also after an abort, when
+      // no consumer waited for the last ones)
+      mbar_wait(&sm.bar_qdo, 0, nullptr, kWaitLimitNs);
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        mbar_wait(&sm.bar_kfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     } else if (lane == 1) {
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
-        if (j >= kStages && !mbar_wait(&sm.bar_vempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
+        if (j >= kStages && !mbar_wait(&sm.bar_vempty[st], ((j / kStages) + 1) & 1, abort_flag, p.wait_ns))
           break;
         mbar_arrive_expect_tx(&sm.bar_vfull[st], kTileBytes);
-        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + (entry(j) >> 2) * kTile);
+        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + entry_index(entry(j)) * kTile);
         issued = j + 1;
       }
-      if (*abort_flag)
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-          mbar_wait(&sm.bar_vfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        mbar_wait(&sm.bar_vfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // the whole warp runs this loop; elect.sync picks the issuing lane
-    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T (q/k type)
-    constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);      // dP = dO V^T (bf16)
-    constexpr uint32_t idesc_q = idesc_f32acc(128, D, QK16, 0, 1);    // dQ += dS K (K tile MN-major)
+    // On a partial tile of which no query sees one 64-key half, S and dP are the
+    // N = 64 products over the other half (in that half's columns) and dQ takes
+    // its 64 keys only.
+    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);   // S = Q K^T (q/k type)
+    constexpr uint32_t idesc_s64 = idesc_f32acc(128, 64, QK16, 0, 0);  // S over one key half
+    constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);       // dP = dO V^T (bf16)
+    constexpr uint32_t idesc_p64 = idesc_bf16_f32(128, 64, 0, 0);      // dP over one key half
+    constexpr uint32_t idesc_q = idesc_f32acc(128, D, QK16, 0, 1);     // dQ += dS K (K tile MN-major)
     const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
     // S(j) = Q K(j)^T
     auto issue_s = [&](int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
-      const uint32_t sk = smem_u32(sm.k[st]);
+      const int hv = entry_halves(entry(j));
+      const uint32_t k0 = hv == 2 ? kKeyHalf : 0;  // first key of the product
+      const uint64_t kb = desc_kmajor(smem_u32(sm.k[st]) + k0 * 128, 0);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + kDqColS, (desc_kmajor(sq, 0) + kmajor_step(kk)), (desc_kmajor(sk, 0) + kmajor_step(kk)), idesc_s, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kDqColS + k0, (desc_kmajor(sq, 0) + kmajor_step(kk)), kb + kmajor_step(kk),
+               hv == 3 ? idesc_s : idesc_s64, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_sfull);
       return true;
     };
     // dP(j) = dO V(j)^T; releases V(j)
     auto issue_dp = [&](int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_vfull[st], (j / kStages) & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_vfull[st], (j / kStages) & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
-      const uint32_t sv = smem_u32(sm.v[st]);
+      const int hv = entry_halves(entry(j));
+      const uint32_t k0 = hv == 2 ? kKeyHalf : 0;
+      const uint64_t vb = desc_kmajor(smem_u32(sm.v[st]) + k0 * 128, 0);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + kDqColDP, (desc_kmajor(sdo, 0) + kmajor_step(kk)), (desc_kmajor(sv, 0) + kmajor_step(kk)), idesc_p, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kDqColDP + k0, (desc_kmajor(sdo, 0) + kmajor_step(kk)), vb + kmajor_step(kk),
+               hv == 3 ? idesc_p : idesc_p64, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_dpfull);
       mma_commit(&sm.bar_vempty[st]);
       return true;
@@ -272,22 +326,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dQ += dS(j) K(j); releases K(j) and its metadata
     auto issue_dq = [&](int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_dsfull, j & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_dsfull, j & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
-      const uint32_t sk = smem_u32(sm.k[st]);
+      const int hv = entry_halves(entry(j));
+      const uint64_t kb = desc_mnmajor(smem_u32(sm.k[st]), 0);
+      uint32_t acc = j > 0 ? 1u : 0u;
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + kDqColAcc, tmem + kDqColDS + kk * 8, (desc_mnmajor(sk, 0) + mnmajor_step(kk)), idesc_q,
-               (j > 0 || kk > 0) ? 1u : 0u);
+      for (int half = 0; half < 2; ++half) {
+        if (!((hv >> half) & 1)) continue;  // no query of the tile sees these 64 keys
+#pragma unroll
+        for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
+          mma_ts(tmem + kDqColAcc, tmem + kDqColDS + kk * 8, kb + mnmajor_step(kk), idesc_q, acc);
+          acc = 1u;
+        }
+      }
       mma_commit(&sm.bar_kempty[st]);
       return true;
     };
     // Issue order S(0) dP(0) | S(1) dQ(0) dP(1) | S(2) dQ(1) dP(2) | ...: S(j+1) starts as
     // soon as the compute warps have read S(j), while they still form P(j) and dS(j).
-    bool ok = warp_wait(&sm.bar_qdo, 0, abort_flag) && issue_s(0) && issue_dp(0);
+    bool ok = warp_wait(&sm.bar_qdo, 0, abort_flag, p.wait_ns) && issue_s(0) && issue_dp(0);
     for (int j = 0; ok && j < n; ++j) {
       if (j + 1 < n) {
-        ok = warp_wait(&sm.bar_sfree, j & 1, abort_flag) && issue_s(j + 1);
+        ok = warp_wait(&sm.bar_sfree, j & 1, abort_flag, p.wait_ns) && issue_s(j + 1);
         if (!ok) break;
       }
       ok = issue_dq(j);
@@ -308,16 +369,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qmeta = qv ? p.tok_meta[qg] : 0;
     const size_t rt = (static_cast<size_t>(head) * p.n_items + tile_id) * kTile + row;
     const float nlse2 = qv ? p.lse2_tiles[rt] : 0.f;  // -LSE * log2(e)
-    const float nd = qv ? p.d_tiles[rt] : 0.f;        // -D
+    const float nd = qv ? p.d_tiles[rt] : 0.f;        // -2^k D
+    const int gk = grad_scale_exp(*p.dout_absmax);
+    const float gs = pow2f(gk);                       // dS is formed as 2^k P (dP - D)
     const uint64_t sl2x2 = f2(p.scale_log2, p.scale_log2), nlse2x2 = f2(nlse2, nlse2), ndx2 = f2(nd, nd);
+    const uint64_t gsx2 = f2(gs, gs);
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j % kStages;
       const int e = entry(j);
-      const bool partial = (e & 3) == OPR_TILE_PARTIAL;
-      const int kbase = seq0 + (e >> 2) * kTile;
+      const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
+      const int kbase = seq0 + entry_index(e) * kTile;
+      if (!((entry_halves(e) >> half) & 1)) {
+        // no query of the tile sees this thread's 64 keys: nothing to form, only the
+        // hand-offs (each wait orders this thread's arrival after the phase before)
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, p.wait_ns))) {
+          ok = false;
+          break;
+        }
+        mbar_arrive(&sm.bar_sfree);
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, p.wait_ns))) {
+          ok = false;
+          break;
+        }
+        mbar_arrive(&sm.bar_dsfull);
+        continue;
+      }
       if (partial &&
-          !__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs))) {
+          !__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / kStages) & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -329,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mm[0] = half ? m[2] : m[0];
         mm[1] = half ? m[3] : m[1];
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -351,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 64; ++c)
         if (!((mm[c >> 5] >> (c & 31)) & 1u)) pv[c] = 0.f;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -364,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            const uint64_t t = fadd2(f2(__uint_as_float(r[c * 32 + 2 * x]), __uint_as_float(r[c * 32 + 2 * x + 1])), ndx2);
+            const uint64_t t = ffma2(f2(__uint_as_float(r[c * 32 + 2 * x]), __uint_as_float(r[c * 32 + 2 * x + 1])), gsx2, ndx2);
             float d0, d1;
             f2_split(fmul2(f2(pv[c * 32 + 2 * x], pv[c * 32 + 2 * x + 1]), t), d0, d1);
             pk[x] = pack_x2<QK16>(d0, d1);
@@ -376,20 +455,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&sm.bar_dsfull);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_dqdone, 0, abort_flag, kWaitLimitNs))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_dqdone, 0, abort_flag, p.wait_ns))) {
       tc_fence_after();
       float* dst = p.dq + (static_cast<size_t>(qg) * p.hq + head) * D;
+      const float osc = p.scale * pow2f(-gk);  // undoes the gradient scale 2^k
+      if (p.rope_cs != nullptr) {
+        // the gradient w.r.t. the unrotated q: rotated back by the row's position
+        store_unrotated_row<D>(tl + kDqColAcc, half, osc, qv ? rope_row<D>(p, qg) : p.rope_cs, dst, qv);
+      } else {
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t r[32];
-        const int oc = half * (D / 2) + c * 32;
-        tmem_ld32(tl + kDqColAcc + oc, r);
-        if (qv) {
-          float4* d4 = reinterpret_cast<float4*>(dst + oc);
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t r[32];
+          const int oc = half * (D / 2) + c * 32;
+          tmem_ld32(tl + kDqColAcc + oc, r);
+          if (qv) {
+            float4* d4 = reinterpret_cast<float4*>(dst + oc);
 #pragma unroll
-          for (int x = 0; x < 8; ++x)
-            d4[x] = make_float4(__uint_as_float(r[4 * x]) * p.scale, __uint_as_float(r[4 * x + 1]) * p.scale,
-                                __uint_as_float(r[4 * x + 2]) * p.scale, __uint_as_float(r[4 * x + 3]) * p.scale);
+            for (int x = 0; x < 8; ++x)
+              d4[x] = make_float4(__uint_as_float(r[4 * x]) * osc, __uint_as_float(r[4 * x + 1]) * osc,
+                                  __uint_as_float(r[4 * x + 2]) * osc, __uint_as_float(r[4 * x + 3]) * osc);
+          }
         }
       }
     }
@@ -504,11 +589,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
         const int e = entry(j % cnt);
-        const int Iq = e >> 2;
+        const int Iq = entry_index(e);
         const int h = kvh * group + j / cnt;
-        if (j >= kStages && !mbar_wait(&sm.bar_qempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
+        if (j >= kStages && !mbar_wait(&sm.bar_qempty[st], ((j / kStages) + 1) & 1, abort_flag, p.wait_ns))
           break;
-        const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+        const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
         mbar_arrive_expect_tx(&sm.bar_qfull[st],
                               kTileBytes + 2 * kTile * sizeof(float) + (partial ? sizeof(TileMeta) : 0));
         tma_tile<D>(&tm_q, &sm.bar_qfull[st], sm.q[st], h, seq0 + Iq * kTile);
@@ -518,25 +603,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (partial) bulk_load(&sm.qmeta[st], tmeta + Iq, sizeof(TileMeta), &sm.bar_qfull[st]);
         issued = j + 1;
       }
-      if (*abort_flag) {
-        mbar_wait(&sm.bar_kv, 0, nullptr, kWaitLimitNs);
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-          mbar_wait(&sm.bar_qfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
-      }
+      // every copy issued has landed before the CTA exits (also after an abort, when
+      // no consumer waited for the last ones)
+      mbar_wait(&sm.bar_kv, 0, nullptr, kWaitLimitNs);
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        mbar_wait(&sm.bar_qfull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     } else if (lane == 1) {
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
         const int h = kvh * group + j / cnt;
-        if (j >= kStages && !mbar_wait(&sm.bar_doempty[st], ((j / kStages) + 1) & 1, abort_flag, kWaitLimitNs))
+        if (j >= kStages && !mbar_wait(&sm.bar_doempty[st], ((j / kStages) + 1) & 1, abort_flag, p.wait_ns))
           break;
         mbar_arrive_expect_tx(&sm.bar_dofull[st], kTileBytes);
-        tma_tile<D>(&tm_do16, &sm.bar_dofull[st], sm.dout[st], h, seq0 + (entry(j % cnt) >> 2) * kTile);
+        tma_tile<D>(&tm_do16, &sm.bar_dofull[st], sm.dout[st], h, seq0 + entry_index(entry(j % cnt)) * kTile);
         issued = j + 1;
       }
-      if (*abort_flag)
-        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-          mbar_wait(&sm.bar_dofull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
+      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+        mbar_wait(&sm.bar_dofull[j % kStages], (j / kStages) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // the whole warp runs this loop; elect.sync picks the issuing lane
@@ -549,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // memory, whose bandwidth a narrower N would spend faster than the tensor core.
     auto issue_s = [&](int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
       const uint64_t qb = desc_kmajor(smem_u32(sm.q[st]), 0);
 #pragma unroll
@@ -561,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dP^T(j) = V dO(j)^T
     auto issue_dp = [&](int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_dofull[st], (j / kStages) & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_dofull[st], (j / kStages) & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
       const uint64_t ob = desc_kmajor(smem_u32(sm.dout[st]), 0);
 #pragma unroll
@@ -573,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dV += P^T(j)[:, half h] dO(j)[half h]; the second half releases dO(j)
     auto issue_dv = [&](int h, int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_pfull[h], j & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_pfull[h], j & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
       const uint64_t ob = desc_mnmajor(smem_u32(sm.dout[st]), 4 * h);
 #pragma unroll
@@ -586,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dK += dS^T(j)[:, half h] Q(j)[half h]; the second half releases Q(j) and its column data
     auto issue_dk = [&](int h, int j) -> bool {
       const int st = j % kStages;
-      if (!warp_wait(&sm.bar_dsfull[h], j & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_dsfull[h], j & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
       const uint64_t qb = desc_mnmajor(smem_u32(sm.q[st]), 4 * h);
 #pragma unroll
@@ -600,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the next S^T is formed while the compute warps turn dP^T into dS^T, and
     // the next dP^T while they turn S^T into P^T; each half's dV (dK) product
     // starts as soon as that half's P^T (dS^T) is in place.
-    bool ok = warp_wait(&sm.bar_kv, 0, abort_flag) && issue_s(0) && issue_dp(0);
+    bool ok = warp_wait(&sm.bar_kv, 0, abort_flag, p.wait_ns) && issue_s(0) && issue_dp(0);
     for (int j = 0; ok && j < n; ++j) {
       const bool more = j + 1 < n;
       ok = issue_dv(0, j) && issue_dv(1, j);
@@ -629,9 +713,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n; ++j) {
       const int st = j % kStages;
       const int e = entry(j % cnt);
-      const bool partial = (e & 3) == OPR_TILE_PARTIAL;
-      const int qt0 = seq0 + (e >> 2) * kTile;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag, kWaitLimitNs))) {
+      const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
+      const int qt0 = seq0 + entry_index(e) * kTile;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -643,7 +727,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mm[0] = half ? m[2] : m[0];
         mm[1] = half ? m[3] : m[1];
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull, j & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -684,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.bar_pfull[half]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_dpfull, j & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -719,10 +803,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&sm.bar_dsfull[half]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_accdone, 0, abort_flag, kWaitLimitNs))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_accdone, 0, abort_flag, p.wait_ns))) {
       tc_fence_after();
       float* dvp = p.dv + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
       float* dkp = p.dk + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
+      const float vsc = pow2f(-grad_scale_exp(*p.dout_absmax));  // undoes the gradient scale 2^k
+      const float ksc = p.scale * vsc;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
@@ -732,21 +818,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           float4* d4 = reinterpret_cast<float4*>(dvp + oc);
 #pragma unroll
           for (int x = 0; x < 8; ++x)
-            d4[x] = make_float4(__uint_as_float(r[4 * x]), __uint_as_float(r[4 * x + 1]),
-                                __uint_as_float(r[4 * x + 2]), __uint_as_float(r[4 * x + 3]));
+            d4[x] = make_float4(__uint_as_float(r[4 * x]) * vsc, __uint_as_float(r[4 * x + 1]) * vsc,
+                                __uint_as_float(r[4 * x + 2]) * vsc, __uint_as_float(r[4 * x + 3]) * vsc);
         }
       }
+      if (p.rope_cs != nullptr) {
+        // the gradient w.r.t. the unrotated k: rotated back by the key's position
+        store_unrotated_row<D>(tl + kColDK, half, ksc, kvld ? rope_row<D>(p, kg) : p.rope_cs, dkp, kvld);
+      } else {
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t r[32];
-        const int oc = half * (D / 2) + c * 32;
-        tmem_ld32(tl + kColDK + oc, r);
-        if (kvld) {
-          float4* d4 = reinterpret_cast<float4*>(dkp + oc);
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t r[32];
+          const int oc = half * (D / 2) + c * 32;
+          tmem_ld32(tl + kColDK + oc, r);
+          if (kvld) {
+            float4* d4 = reinterpret_cast<float4*>(dkp + oc);
 #pragma unroll
-          for (int x = 0; x < 8; ++x)
-            d4[x] = make_float4(__uint_as_float(r[4 * x]) * p.scale, __uint_as_float(r[4 * x + 1]) * p.scale,
-                                __uint_as_float(r[4 * x + 2]) * p.scale, __uint_as_float(r[4 * x + 3]) * p.scale);
+            for (int x = 0; x < 8; ++x)
+              d4[x] = make_float4(__uint_as_float(r[4 * x]) * ksc, __uint_as_float(r[4 * x + 1]) * ksc,
+                                  __uint_as_float(r[4 * x + 2]) * ksc, __uint_as_float(r[4 * x + 3]) * ksc);
+          }
         }
       }
     }
@@ -779,18 +870,31 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
   cudaError_t e = cudaSuccess;
   // 1) row terms D and LSE * log2(e) per 128-token tile, and the fp16 copies of dO and V
   if ((stages & OPR_BWD_ROW_TERMS) && pq.n_items > 0) {
+    if ((e = cudaMemsetAsync(b.dout_absmax, 0, sizeof(uint32_t), stream)) != cudaSuccess) return e;
+    const int64_t n8_do = pq.total * pq.hq * D / 8;
+    if (n8_do > 0) {
+      const int64_t blocks = std::min<int64_t>((n8_do + 255) / 256, 148 * 8);
+      dout_absmax_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(b.dout, n8_do, b.dout_absmax);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     const dim3 grid(pq.n_items, pq.hq);
     float* row_d = b.row_terms;
     float* row_l = b.row_terms + static_cast<size_t>(pq.hq) * pq.n_items * kTile;
     if (b.o_fp32)
       row_terms_kernel<D, float><<<grid, 256, 0, stream>>>(static_cast<const float*>(b.o), b.dout, pq.lse_in,
                                                                pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d, row_l,
-                                                               b.dout16, pq.dev_status);
+                                                               b.dout16, b.dout_absmax, pq.dev_status);
     else
       row_terms_kernel<D, __nv_bfloat16><<<grid, 256, 0, stream>>>(
           static_cast<const __nv_bfloat16*>(b.o), b.dout, pq.lse_in, pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d,
-          row_l, b.dout16, pq.dev_status);
+          row_l, b.dout16, b.dout_absmax, pq.dev_status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (pq.rope_cs != nullptr) {
+      const int64_t n = static_cast<int64_t>(pq.rope_rows) * (D / 2);
+      rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+          const_cast<float2*>(pq.rope_cs), pq.rope_rows, D / 2, b.rope_neg_log_base_over_half);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     const int64_t n8 = pq.total * pq.hkv * D / 8;
     if (n8 > 0) {
       const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, 148 * 16);
@@ -824,11 +928,9 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
 
 cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const BwdMaps& m, const BwdBuffers& b, const AttnParams& pq,
                             const AttnParams& pkv, int stages, cudaStream_t stream) {
-  if (head_dim == 128)
-    return qk_f16 ? launch_bwd_t<128, true>(m, b, pq, pkv, stages, stream)
-                  : launch_bwd_t<128, false>(m, b, pq, pkv, stages, stream);
-  return qk_f16 ? launch_bwd_t<64, true>(m, b, pq, pkv, stages, stream)
-                : launch_bwd_t<64, false>(m, b, pq, pkv, stages, stream);
+  if (!qk_f16) return cudaErrorNotSupported;  // the entry points accept fp16 q and k only
+  if (head_dim == 128) return launch_bwd_t<128, true>(m, b, pq, pkv, stages, stream);
+  return launch_bwd_t<64, true>(m, b, pq, pkv, stages, stream);
 }
 
 }  // namespace opr

@@ -7,12 +7,17 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
+
 #include "opr_internal.cuh"
 #include "sm100.cuh"
 
 namespace opr {
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: any pipeline wait longer than this is a hang
+// 2 s: any pipeline wait longer than this is a hang.  The pipeline waits take their
+// limit from AttnParams::wait_ns (this value unless a test lowers it); the drains
+// before a CTA exits always use this one.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // CTA shape shared by the attention kernels: warp 0 TMA producer, warp 1 TMEM
 // owner / MMA issuer, warps 2..9 compute.  Two compute warps share each TMEM
@@ -22,8 +27,9 @@ constexpr int kThreads = 320;
 constexpr int kComputeThreads = 256;
 
 // Bounded mbarrier wait taken by a whole warp; the result is warp-uniform.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, kWaitLimitNs));
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, limit_ns));
 }
 
 // A 128-row tile of head_dim D bf16 values is stored as D/64 "chunks", each
@@ -143,6 +149,7 @@ struct BwdMaps {
 };
 
 struct BwdBuffers {
+  uint32_t* dout_absmax;  // one word: bits of max |dO|
   const void* o;
   int o_fp32;
   const __nv_bfloat16* dout;
@@ -150,6 +157,7 @@ struct BwdBuffers {
   float* row_terms;  // D tiles, then LSE * log2(e) tiles
   __half* dout16;
   __half* v16;
+  double rope_neg_log_base_over_half;  // -ln(base) / (D / 2) of the rotary table
 };
 
 struct AttnParams {
@@ -174,12 +182,94 @@ struct AttnParams {
   float* lse;
   // backward
   const float* lse_in;      // [hq, total]
-  const float* d_tiles;     // -D = -rowsum(dO * O), [hq][n_items][128]
+  const float* d_tiles;     // -2^k D = -2^k rowsum(dO * O), [hq][n_items][128]
   const float* lse2_tiles;  // -LSE * log2(e), [hq][n_items][128]
+  const uint32_t* dout_absmax;  // bits of max |dO| (a non-negative float), sets the scale 2^k
   float* dq;
   float* dk;
   float* dv;
+  // inverse rotary embedding of dq and dk in the epilogues (rope_cs null: none):
+  // (cos, sin) of position p and pair j at rope_cs[p * (D / 2) + j], p < rope_rows
+  const int32_t* pos_id;
+  const float2* rope_cs;
+  int32_t rope_rows;
   int32_t* dev_status;
+  uint64_t wait_ns;  // limit of the pipeline waits (kWaitLimitNs; 0: a wait not already done times out)
 };
+
+// ---------------------------------------------------------------- gradient scale
+// The backward is linear in dO, so it runs on 2^k dO and divides the results
+// by 2^k (exact: a power of two).  k puts max |2^k dO| in [8, 16): the fp16
+// copies of dO and the fp16 dS keep their 11-bit significands for small
+// upstream gradients (loss / token count, 1e-5 .. 1e-8), which fp16 would
+// otherwise hold as subnormals or zero, and large ones stay inside the fp16
+// range.  `bits` is max |dO| as float bits; zero, inf and NaN give k = 0.
+__host__ __device__ __forceinline__ int grad_scale_exp(uint32_t bits) {
+  const int e = static_cast<int>((bits >> 23) & 0xFFu);  // biased exponent
+  if (bits == 0u || e == 0xFF) return 0;
+  const int k = e == 0 ? 100 : 130 - e;  // max = 1.f * 2^(e - 127) -> 1.f * 2^(e - 127 + k) in [8, 16)
+  return k < -100 ? -100 : (k > 100 ? 100 : k);
+}
+
+// One thread's share of a gradient row held in TMEM (D fp32 columns from taddr in
+// this thread's lane), scaled by sc and rotated back by the row's rotary angles:
+// the gradient w.r.t. the unrotated q or k, x_j = y_j cos + y_{j+D/2} sin and
+// x_{j+D/2} = y_{j+D/2} cos - y_j sin.  Of the row's two threads, `part` takes
+// the pairs j = part D/4 .. part D/4 + D/4 - 1 (columns j and j + D/2).  cs is the
+// row's (cos, sin) table row; dst the row in global memory (written when valid).
+template <int D>
+__device__ __forceinline__ void store_unrotated_row(uint32_t taddr, int part, float sc, const float2* cs, float* dst,
+                                                    bool valid) {
+  constexpr int NP = D / 4;  // pairs per thread: 32 (D = 128) or 16 (D = 64)
+  const int j0 = part * NP;
+  uint32_t lo[NP], hi[NP];
+  if constexpr (NP == 32) {
+    tmem_ld32(taddr + j0, lo);
+    tmem_ld32(taddr + D / 2 + j0, hi);
+  } else {
+    tmem_ld16(taddr + j0, lo);
+    tmem_ld16(taddr + D / 2 + j0, hi);
+  }
+  if (!valid) return;
+  const float4* c4 = reinterpret_cast<const float4*>(cs + j0);  // two (cos, sin) pairs per float4
+  float xl[NP], xh[NP];
+#pragma unroll
+  for (int i = 0; i < NP; i += 2) {
+    const float4 w = c4[i / 2];
+    const float a0 = __uint_as_float(lo[i]) * sc, b0 = __uint_as_float(hi[i]) * sc;
+    const float a1 = __uint_as_float(lo[i + 1]) * sc, b1 = __uint_as_float(hi[i + 1]) * sc;
+    xl[i] = a0 * w.x + b0 * w.y;
+    xh[i] = b0 * w.x - a0 * w.y;
+    xl[i + 1] = a1 * w.z + b1 * w.w;
+    xh[i + 1] = b1 * w.z - a1 * w.w;
+  }
+  float4* dl = reinterpret_cast<float4*>(dst + j0);
+  float4* dh = reinterpret_cast<float4*>(dst + D / 2 + j0);
+#pragma unroll
+  for (int i = 0; i < NP / 4; ++i) {
+    dl[i] = make_float4(xl[4 * i], xl[4 * i + 1], xl[4 * i + 2], xl[4 * i + 3]);
+    dh[i] = make_float4(xh[4 * i], xh[4 * i + 1], xh[4 * i + 2], xh[4 * i + 3]);
+  }
+}
+
+// The (cos, sin) table row of a token's position; a position outside the table
+// (only with inconsistent inputs) sets OPR_DEV_BAD_INPUT and reads row 0 (no rotation).
+template <int D>
+__device__ __forceinline__ const float2* rope_row(const AttnParams& p, int64_t tok) {
+  int pos = p.pos_id[tok];
+  if (pos < 0 || pos >= p.rope_rows) {
+    atomicOr(p.dev_status, OPR_DEV_BAD_INPUT);
+    pos = 0;
+  }
+  return p.rope_cs + static_cast<size_t>(pos) * (D / 2);
+}
+
+// 2^k as a float, built from its bits (|k| <= 126).
+__host__ __device__ __forceinline__ float pow2f(int k) {
+  const uint32_t b = static_cast<uint32_t>(127 + k) << 23;
+  float f;
+  memcpy(&f, &b, sizeof f);
+  return f;
+}
 
 }  // namespace opr

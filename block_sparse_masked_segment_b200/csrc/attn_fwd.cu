@@ -4,7 +4,7 @@
 // visibility rules, evaluated block-sparsely (the pages use a FlexAttention
 // block mask on H100, "实现细节"; this is a hand-written Blackwell kernel).
 //
-// One CTA per (query tile of 128 rows, q head), 6 warps:
+// One CTA per (query tile of 128 rows, q head), 10 warps:
 //   warp 0      lane 0 loads Q once, then the K tiles of the row's non-empty
 //               tiles (3-stage ring) with TMA, plus, for partial tiles, the
 //               tile's precomputed key metadata (one bulk copy); lane 1
@@ -114,32 +114,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int st = j % kStagesK;
         const int e = entry(j);
-        const int J = e >> 2;
-        if (j >= kStagesK && !mbar_wait(&sm.bar_kempty[st], ((j / kStagesK) + 1) & 1, abort_flag, kWaitLimitNs))
+        const int J = entry_index(e);
+        if (j >= kStagesK && !mbar_wait(&sm.bar_kempty[st], ((j / kStagesK) + 1) & 1, abort_flag, p.wait_ns))
           break;
-        const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+        const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
         mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes + (partial ? sizeof(TileMeta) : 0));
         tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, seq0 + J * kTile);
         if (partial) bulk_load(&sm.kmeta[st], tmeta + J, sizeof(TileMeta), &sm.bar_kfull[st]);
         issued = j + 1;
       }
-      if (*abort_flag)  // let the copies already in flight land before the CTA exits
-        for (int j = (issued > kStagesK ? issued - kStagesK : 0); j < issued; ++j)
-          mbar_wait(&sm.bar_kfull[j % kStagesK], (j / kStagesK) & 1, nullptr, kWaitLimitNs);
+      // every copy issued has landed before the CTA exits (also after an abort, when
+      // no consumer waited for the last ones)
+      mbar_wait(&sm.bar_q, 0, nullptr, kWaitLimitNs);
+      for (int j = (issued > kStagesK ? issued - kStagesK : 0); j < issued; ++j)
+        mbar_wait(&sm.bar_kfull[j % kStagesK], (j / kStagesK) & 1, nullptr, kWaitLimitNs);
     } else if (lane == 1) {
       tma_prefetch_desc(&tm_v);
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStagesV;
-        if (j >= kStagesV && !mbar_wait(&sm.bar_vempty[st], ((j / kStagesV) + 1) & 1, abort_flag, kWaitLimitNs))
+        if (j >= kStagesV && !mbar_wait(&sm.bar_vempty[st], ((j / kStagesV) + 1) & 1, abort_flag, p.wait_ns))
           break;
         mbar_arrive_expect_tx(&sm.bar_vfull[st], kTileBytes);
-        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + (entry(j) >> 2) * kTile);
+        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + entry_index(entry(j)) * kTile);
         issued = j + 1;
       }
-      if (*abort_flag)
-        for (int j = (issued > kStagesV ? issued - kStagesV : 0); j < issued; ++j)
-          mbar_wait(&sm.bar_vfull[j % kStagesV], (j / kStagesV) & 1, nullptr, kWaitLimitNs);
+      for (int j = (issued > kStagesV ? issued - kStagesV : 0); j < issued; ++j)
+        mbar_wait(&sm.bar_vfull[j % kStagesV], (j / kStagesV) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // the whole warp runs this loop; elect.sync picks the issuing lane
@@ -147,11 +148,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
     constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);      // O += P V, P and V bf16
     const uint32_t sq = smem_u32(sm.q);
-    bool ok = warp_wait(&sm.bar_q, 0, abort_flag);
+    bool ok = warp_wait(&sm.bar_q, 0, abort_flag, p.wait_ns);
     auto issue_pv = [&](int jp) -> bool {
       const int bp = jp & 1, stp = jp % kStagesV;
-      if (!warp_wait(&sm.bar_pfull[bp], (jp >> 1) & 1, abort_flag)) return false;
-      if (!warp_wait(&sm.bar_vfull[stp], (jp / kStagesV) & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_pfull[bp], (jp >> 1) & 1, abort_flag, p.wait_ns)) return false;
+      if (!warp_wait(&sm.bar_vfull[stp], (jp / kStagesV) & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
       const uint32_t sv = smem_u32(sm.v[stp]);
 #pragma unroll
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     for (int j = 0; ok && j < n; ++j) {
       const int st = j % kStagesK, b = j & 1;
-      if (!warp_wait(&sm.bar_kfull[st], (j / kStagesK) & 1, abort_flag)) {
+      if (!warp_wait(&sm.bar_kfull[st], (j / kStagesK) & 1, abort_flag, p.wait_ns)) {
         ok = false;
         break;
       }
@@ -197,10 +198,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n; ++j) {
       const int b = j & 1, st = j % kStagesK;
       const int e = entry(j);
-      const bool partial = (e & 3) == OPR_TILE_PARTIAL;
-      const int kbase = seq0 + (e >> 2) * kTile;
+      const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
+      const int kbase = seq0 + entry_index(e) * kTile;
       // the K stage carries the tile's key metadata; it is released after this read
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / kStagesK) & 1, abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / kStagesK) & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mm[3] = half ? m[1] : m[3];
       }
       mbar_arrive(&sm.bar_kempty[st]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[b], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[b], (j >> 1) & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       // O may be rescaled only once the previous P V product has landed.
       if (j >= 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_odone, (j - 1) & 1, abort_flag, kWaitLimitNs))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_odone, (j - 1) & 1, abort_flag, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Every compute thread reaches this barrier exactly once (also after an abort).
     sm.lsum[half][row] = l_run;
     named_bar_sync(1, kComputeThreads);
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_odone, (n - 1) & 1, abort_flag, kWaitLimitNs))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_odone, (n - 1) & 1, abort_flag, p.wait_ns))) {
       tc_fence_after();
       const float l_tot = sm.lsum[0][row] + sm.lsum[1][row];
       const float inv = 1.f / l_tot;
@@ -337,6 +338,70 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
 // ----------------------------------------------------------------------------
+// Pieces of one thread's row of a tile in the head-pair kernel, for the NC keys
+// (128, or the 64 of the one key half that some query of the tile sees) that it
+// processes.
+
+// Row max of NC scores (NC a multiple of 16, at least 32): eight chains, each
+// over columns x, x + 8, x + 16, ..., mostly with the three-input max.
+template <int NC>
+__device__ __forceinline__ float row_max(const float (&sv)[NC]) {
+  constexpr int W = 8;
+  static_assert(NC % (2 * W) == 0 && NC >= 4 * W, "whole blocks of 16 columns");
+  constexpr int kPairs = (NC - 3 * W) / (2 * W);  // blocks of 8 taken two at a time
+  float mx[W];
+#pragma unroll
+  for (int x = 0; x < W; ++x) mx[x] = fmax3(sv[x], sv[W + x], sv[2 * W + x]);
+#pragma unroll
+  for (int b = 0; b < kPairs; ++b)
+#pragma unroll
+    for (int x = 0; x < W; ++x) mx[x] = fmax3(mx[x], sv[3 * W + 2 * W * b + x], sv[4 * W + 2 * W * b + x]);
+#pragma unroll
+  for (int x = 0; x < W; ++x) mx[x] = fmaxf(mx[x], sv[NC - W + x]);  // the last block of 8
+  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
+// P = 2^(S scale log2(e) - mb) of NC scores (the scale-and-shift on fp32 pairs),
+// stored as bf16 two per TMEM column from p_addr; returns the sum of P.
+template <int NC>
+__device__ __forceinline__ float exp_pack_row(const float (&sv)[NC], float sl2, float mb, uint32_t p_addr) {
+  const uint64_t sl2x2 = f2(sl2, sl2), nmb2 = f2(-mb, -mb);
+  float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < NC / 32; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      float a0, a1;
+      f2_split(ffma2(f2(sv[c * 32 + 2 * x], sv[c * 32 + 2 * x + 1]), sl2x2, nmb2), a0, a1);
+      const float p0 = fast_exp2(a0);
+      const float p1 = fast_exp2(a1);
+      rs8[x & 7] += p0 + p1;
+      pk[x] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(p_addr + c * 16, pk);
+  }
+  return ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+}
+
+// Running-max decision of a row after a tile whose masked row max is mx (scaled
+// to base 2 by sl2): P is taken against the old max unless the max grew by more
+// than 8 (a factor of 256), in which case O is rescaled to the new one.
+struct MaxStep {
+  float m_new;  // running max after the tile
+  bool need;    // rescale O and the row sum to m_new
+  float mb;     // the max P is taken against (0 while the row has seen nothing)
+};
+__device__ __forceinline__ MaxStep max_step(float m_run, float mx, float sl2) {
+  MaxStep r;
+  r.m_new = fmaxf(m_run, mx * sl2);
+  r.need = r.m_new > m_run + 8.f;  // also true on the first finite max
+  const float m_use = r.need ? r.m_new : m_run;
+  r.mb = (m_use == -INFINITY) ? 0.f : m_use;
+  return r;
+}
+
+// ----------------------------------------------------------------------------
 // Head-pair forward: one CTA per (query tile, two q heads of one GQA group).
 // Both heads read the same K/V tiles and the same mask, so the two heads are
 // two independent softmax streams on one K/V pipeline: while the tensor core
@@ -348,6 +413,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   warps 2..5  head A, warps 6..9 head B: one query row per thread, P (bf16)
 //               written over the first 64 columns of the thread's own row of S
 // TMEM columns: S_A 0, S_B 128, O_A 256, O_B 384.
+// Sub-tile skipping: on a partial tile of which no query sees one 64-key half,
+// S is the N = 64 product over the other half (written to that half's
+// columns), the softmax takes its 64 columns, and P V runs over its 64 keys.
 template <int D>
 struct FwdPairSmem {
   alignas(1024) uint8_t q[2][TileGeom<D>::kBytes];
@@ -426,58 +494,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int st = j % NS;
         const int e = entry(j);
-        const int J = e >> 2;
-        if (j >= NS && !mbar_wait(&sm.bar_kempty[st], ((j / NS) + 1) & 1, abort_flag, kWaitLimitNs)) break;
-        const bool partial = (e & 3) == OPR_TILE_PARTIAL;
+        const int J = entry_index(e);
+        if (j >= NS && !mbar_wait(&sm.bar_kempty[st], ((j / NS) + 1) & 1, abort_flag, p.wait_ns)) break;
+        const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
         mbar_arrive_expect_tx(&sm.bar_kfull[st], kTileBytes + (partial ? sizeof(TileMeta) : 0));
         tma_tile<D>(&tm_k, &sm.bar_kfull[st], sm.k[st], kvh, seq0 + J * kTile);
         if (partial) bulk_load(&sm.kmeta[st], tmeta + J, sizeof(TileMeta), &sm.bar_kfull[st]);
         issued = j + 1;
       }
-      if (*abort_flag) {
-        mbar_wait(&sm.bar_q, 0, nullptr, kWaitLimitNs);
-        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-          mbar_wait(&sm.bar_kfull[j % NS], (j / NS) & 1, nullptr, kWaitLimitNs);
-      }
+      // every copy issued has landed before the CTA exits (also after an abort, when
+      // no consumer waited for the last ones)
+      mbar_wait(&sm.bar_q, 0, nullptr, kWaitLimitNs);
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+        mbar_wait(&sm.bar_kfull[j % NS], (j / NS) & 1, nullptr, kWaitLimitNs);
     } else if (lane == 1) {
       tma_prefetch_desc(&tm_v);
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % NS;
-        if (j >= NS && !mbar_wait(&sm.bar_vempty[st], ((j / NS) + 1) & 1, abort_flag, kWaitLimitNs)) break;
+        if (j >= NS && !mbar_wait(&sm.bar_vempty[st], ((j / NS) + 1) & 1, abort_flag, p.wait_ns)) break;
         mbar_arrive_expect_tx(&sm.bar_vfull[st], kTileBytes);
-        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + (entry(j) >> 2) * kTile);
+        tma_tile<D>(&tm_v, &sm.bar_vfull[st], sm.v[st], kvh, seq0 + entry_index(entry(j)) * kTile);
         issued = j + 1;
       }
-      if (*abort_flag)
-        for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-          mbar_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, nullptr, kWaitLimitNs);
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+        mbar_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, nullptr, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // the whole warp runs this loop; elect.sync picks the issuing lane
-    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);        // O += P V, P and V bf16
+    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);   // S = Q K^T in the q/k type
+    constexpr uint32_t idesc_s64 = idesc_f32acc(128, 64, QK16, 0, 0);  // S over one 64-key half
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);         // O += P V, P and V bf16
     const uint32_t sq[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
     auto issue_s = [&](int h, int j) {
-      const uint32_t sk = smem_u32(sm.k[j % NS]);
+      const int hv = entry_halves(entry(j));
+      const uint32_t k0 = hv == 2 ? kKeyHalf : 0;  // first key of the product
+      const uint32_t idesc = hv == 3 ? idesc_s : idesc_s64;
+      // key row k0 of each 128-byte-row chunk (a multiple of the 8-row swizzle period)
+      const uint64_t kb = desc_kmajor(smem_u32(sm.k[j % NS]) + k0 * 128, 0);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + h * 128, (desc_kmajor(sq[h], 0) + kmajor_step(kk)), (desc_kmajor(sk, 0) + kmajor_step(kk)), idesc_s, kk > 0 ? 1u : 0u);
+        mma_ss(tmem + h * 128 + k0, (desc_kmajor(sq[h], 0) + kmajor_step(kk)), kb + kmajor_step(kk), idesc,
+               kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_sfull[h]);
     };
     auto issue_pv = [&](int h, int j) -> bool {
-      if (!warp_wait(&sm.bar_pfull[h], j & 1, abort_flag)) return false;
+      if (!warp_wait(&sm.bar_pfull[h], j & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
-      const uint32_t sv = smem_u32(sm.v[j % NS]);
+      const int hv = entry_halves(entry(j));
+      const uint64_t vb = desc_mnmajor(smem_u32(sm.v[j % NS]), 0);
+      uint32_t acc = j > 0 ? 1u : 0u;
 #pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, (desc_mnmajor(sv, 0) + mnmajor_step(kk)), idesc_o,
-               (j > 0 || kk > 0) ? 1u : 0u);
+      for (int half = 0; half < 2; ++half) {
+        if (!((hv >> half) & 1)) continue;  // no query of the tile sees these 64 keys
+#pragma unroll
+        for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
+          mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, vb + mnmajor_step(kk), idesc_o, acc);
+          acc = 1u;
+        }
+      }
       mma_commit(&sm.bar_odone[h]);
       return true;
     };
-    bool ok = warp_wait(&sm.bar_q, 0, abort_flag) &&
-              warp_wait(&sm.bar_kfull[0], 0, abort_flag);
+    bool ok = warp_wait(&sm.bar_q, 0, abort_flag, p.wait_ns) &&
+              warp_wait(&sm.bar_kfull[0], 0, abort_flag, p.wait_ns);
     if (ok) {
       tc_fence_after();
       issue_s(0, 0);
@@ -486,13 +566,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int j = 0; ok && j < n; ++j) {
       const bool more = j + 1 < n;
-      if (!warp_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, abort_flag)) {
+      if (!warp_wait(&sm.bar_vfull[j % NS], (j / NS) & 1, abort_flag, p.wait_ns)) {
         ok = false;
         break;
       }
       if (!(ok = issue_pv(0, j))) break;
       if (more) {
-        if (!warp_wait(&sm.bar_kfull[(j + 1) % NS], ((j + 1) / NS) & 1, abort_flag)) {
+        if (!warp_wait(&sm.bar_kfull[(j + 1) % NS], ((j + 1) / NS) & 1, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -525,9 +605,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < n; ++j) {
       const int st = j % NS;
       const int e = entry(j);
-      const bool partial = (e & 3) == OPR_TILE_PARTIAL;
-      const int kbase = seq0 + (e >> 2) * kTile;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / NS) & 1, abort_flag, kWaitLimitNs))) {
+      const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
+      const int kbase = seq0 + entry_index(e) * kTile;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_kfull[st], (j / NS) & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -535,65 +615,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (partial)
         query_row_mask(sm.kmeta[st], kbase, qg, qconv, qmeta, mm);
       mbar_arrive(&sm.bar_kempty[st]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[hx], j & 1, abort_flag, kWaitLimitNs))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_sfull[hx], j & 1, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sv[kTile];
-      {
-        uint32_t sr[kTile];
-        tmem_ld128(tl + scol, sr);
+      MaxStep ms;
+      float rs;
+      const int hv = entry_halves(e);
+      float sv[kTile];  // the row's scores; the first 64 hold the one seen key half of a half tile
+      if (hv == 3) {
+        {
+          uint32_t sr[kTile];
+          tmem_ld128(tl + scol, sr);
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) sv[c] = __uint_as_float(sr[c]);
-      }
-      if (partial) {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c)
-          if (!mask_bit(mm, c)) sv[c] = -INFINITY;
-      }
-      // row max: eight three-input chains
-      float mx8[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) mx8[x] = sv[x];
-#pragma unroll
-      for (int c = 8; c < kTile; c += 16)
-#pragma unroll
-        for (int x = 0; x < 8; ++x) mx8[x] = fmax3(mx8[x], sv[c + x], sv[c + 8 + x]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const bool need = m_new > m_run + 8.f;  // also true on the first finite max
-      const float m_use = need ? m_new : m_run;
-      const float mb = (m_use == -INFINITY) ? 0.f : m_use;
-      // P = 2^(S scale log2(e) - m), the scale-and-shift on fp32 pairs
-      const uint64_t sl2x2 = f2(sl2, sl2), nmb2 = f2(-mb, -mb);
-      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          float a0, a1;
-          f2_split(ffma2(f2(sv[c * 32 + 2 * x], sv[c * 32 + 2 * x + 1]), sl2x2, nmb2), a0, a1);
-          const float p0 = fast_exp2(a0);
-          const float p1 = fast_exp2(a1);
-          rs8[x & 7] += p0 + p1;
-          pk[x] = pack_bf16x2(p0, p1);
+          for (int c = 0; c < kTile; ++c) sv[c] = __uint_as_float(sr[c]);
         }
-        tmem_st16(tl + scol + c * 16, pk);  // own row, columns already read
+        if (partial) {
+#pragma unroll
+          for (int c = 0; c < kTile; ++c)
+            if (!mask_bit(mm, c)) sv[c] = -INFINITY;
+        }
+        ms = max_step(m_run, row_max<kTile>(sv), sl2);
+        rs = exp_pack_row<kTile>(sv, sl2, ms.mb, tl + scol);  // P over S's read columns
+      } else {
+        // the one key half that some query sees: its 64 S columns, its 32 P columns
+        const int k0 = hv == 2 ? kKeyHalf : 0;
+        float(&sh)[kKeyHalf] = *reinterpret_cast<float(*)[kKeyHalf]>(&sv[0]);
+        {
+          uint32_t sr[kKeyHalf];
+          tmem_ld64(tl + scol + k0, sr);
+#pragma unroll
+          for (int c = 0; c < kKeyHalf; ++c) sh[c] = __uint_as_float(sr[c]);
+        }
+        const uint32_t mh[2] = {hv == 2 ? mm[2] : mm[0], hv == 2 ? mm[3] : mm[1]};
+#pragma unroll
+        for (int c = 0; c < kKeyHalf; ++c)
+          if (!((mh[c >> 5] >> (c & 31)) & 1u)) sh[c] = -INFINITY;
+        ms = max_step(m_run, row_max<kKeyHalf>(sh), sl2);
+        rs = exp_pack_row<kKeyHalf>(sh, sl2, ms.mb, tl + scol + k0 / 2);
       }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       tmem_wait_st();
       if (j >= 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (j - 1) & 1, abort_flag, kWaitLimitNs))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (j - 1) & 1, abort_flag, p.wait_ns))) {
           ok = false;
           break;
         }
         tc_fence_after();
       }
-      const float factor = need ? fast_exp2(m_run - m_new) : 1.f;
-      if (__any_sync(0xffffffffu, need && j >= 1)) {
+      const float factor = ms.need ? fast_exp2(m_run - ms.m_new) : 1.f;
+      if (__any_sync(0xffffffffu, ms.need && j >= 1)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
@@ -605,11 +676,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       l_run = l_run * factor + rs;
-      if (need) m_run = m_new;
+      if (ms.need) m_run = ms.m_new;
       tc_fence_before();
       mbar_arrive(&sm.bar_pfull[hx]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (n - 1) & 1, abort_flag, kWaitLimitNs))) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (n - 1) & 1, abort_flag, p.wait_ns))) {
       tc_fence_after();
       const float inv = 1.f / l_run;
       const size_t orow = (static_cast<size_t>(qg) * p.hq + head) * D;
@@ -684,11 +755,9 @@ cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, cons
 
 cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const AttnParams& p, cudaStream_t stream) {
-  if (head_dim == 128)
-    return qk_f16 ? launch_attn_fwd_t<128, true>(tq, tk, tv, p, stream)
-                  : launch_attn_fwd_t<128, false>(tq, tk, tv, p, stream);
-  return qk_f16 ? launch_attn_fwd_t<64, true>(tq, tk, tv, p, stream)
-                : launch_attn_fwd_t<64, false>(tq, tk, tv, p, stream);
+  if (!qk_f16) return cudaErrorNotSupported;  // the entry points accept fp16 q and k only
+  if (head_dim == 128) return launch_attn_fwd_t<128, true>(tq, tk, tv, p, stream);
+  return launch_attn_fwd_t<64, true>(tq, tk, tv, p, stream);
 }
 
 }  // namespace opr

@@ -150,13 +150,15 @@ __global__ void fill_tokens_kernel(const int32_t* __restrict__ turn_lens, const 
 }
 
 // One block of 128 threads per tile (I, J) of sequence s; thread r owns query
-// row I*128 + r and counts its visible keys among the tile's 128 columns.
+// row I*128 + r and counts its visible keys among the tile's 128 columns, per
+// key half.  The tile's byte: class (empty / full / partial) | (key halves << 2),
+// bit h of the key halves set when some query sees a key of half h.
 __global__ void __launch_bounds__(128) block_map_kernel(const int32_t* __restrict__ cu_seqlens,
                                                         const int32_t* __restrict__ conv_idx,
                                                         const int32_t* __restrict__ tok_meta, int32_t T,
                                                         uint8_t* __restrict__ block_map) {
   __shared__ int32_t kconv[kTile], kmeta[kTile];
-  __shared__ int32_t warp_cnt[4];
+  __shared__ int32_t warp_cnt[4][2];
   const int J = blockIdx.x, I = blockIdx.y, s = blockIdx.z;
   const int r = threadIdx.x;
   const int seq0 = cu_seqlens[s];
@@ -182,22 +184,34 @@ __global__ void __launch_bounds__(128) block_map_kernel(const int32_t* __restric
     if (r == 0) *out = OPR_TILE_EMPTY;
     return;
   }
-  int cnt = 0;
+  int cnt[2] = {0, 0};
   const int qg = seq0 + qi;
-#pragma unroll 8
-  for (int c = 0; c < kTile; ++c) cnt += visible(qg, qconv, qmeta, seq0 + J * kTile + c, kconv[c], kmeta[c]) ? 1 : 0;
 #pragma unroll
-  for (int d = 16; d > 0; d >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, d);
-  if ((r & 31) == 0) warp_cnt[r >> 5] = cnt;
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll 8
+    for (int c = h * kKeyHalf; c < (h + 1) * kKeyHalf; ++c)
+      cnt[h] += visible(qg, qconv, qmeta, seq0 + J * kTile + c, kconv[c], kmeta[c]) ? 1 : 0;
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) cnt[h] += __shfl_xor_sync(0xffffffffu, cnt[h], d);
+    if ((r & 31) == 0) warp_cnt[r >> 5][h] = cnt[h];
+  }
   __syncthreads();
   if (r == 0) {
-    const int tot = warp_cnt[0] + warp_cnt[1] + warp_cnt[2] + warp_cnt[3];
-    *out = tot == 0 ? OPR_TILE_EMPTY : (tot == kTile * kTile ? OPR_TILE_FULL : OPR_TILE_PARTIAL);
+    int half_cnt[2];
+    for (int h = 0; h < 2; ++h) half_cnt[h] = warp_cnt[0][h] + warp_cnt[1][h] + warp_cnt[2][h] + warp_cnt[3][h];
+    const int tot = half_cnt[0] + half_cnt[1];
+    const int cls = tot == 0 ? OPR_TILE_EMPTY : (tot == kTile * kTile ? OPR_TILE_FULL : OPR_TILE_PARTIAL);
+    const int halves = (half_cnt[0] > 0 ? 1 : 0) | (half_cnt[1] > 0 ? 2 : 0);
+    *out = static_cast<uint8_t>(cls | (halves << 2));
   }
 }
 
 // One warp per row (blockIdx.y == 0) or column (== 1) of the tile grid of a
-// sequence: compact the non-empty tiles, in ascending order, into a list.
+// sequence: compact the non-empty tiles, in ascending order, into a list of
+// entries (index << 4) | block-map byte.
 __global__ void tile_lists_kernel(const uint8_t* __restrict__ block_map, int32_t T, int32_t* __restrict__ row_cnt,
                                   int32_t* __restrict__ row_list, int32_t* __restrict__ col_cnt,
                                   int32_t* __restrict__ col_list) {
@@ -210,10 +224,11 @@ __global__ void tile_lists_kernel(const uint8_t* __restrict__ block_map, int32_t
   int n = 0;
   for (int y0 = 0; y0 < T; y0 += 32) {
     const int y = y0 + lane;
-    int cls = 0;
-    if (y < T) cls = rows ? base[static_cast<size_t>(x) * T + y] : base[static_cast<size_t>(y) * T + x];
-    const unsigned m = __ballot_sync(0xffffffffu, cls != 0);
-    if (cls != 0) list[n + __popc(m & ((1u << lane) - 1u))] = (y << 2) | cls;
+    int byte = 0;  // class | (key halves << 2)
+    if (y < T) byte = rows ? base[static_cast<size_t>(x) * T + y] : base[static_cast<size_t>(y) * T + x];
+    const bool nonempty = (byte & 3) != OPR_TILE_EMPTY;
+    const unsigned m = __ballot_sync(0xffffffffu, nonempty);
+    if (nonempty) list[n + __popc(m & ((1u << lane) - 1u))] = (y << 4) | byte;
     n += __popc(m);
   }
   if (lane == 0) (rows ? row_cnt : col_cnt)[line] = n;

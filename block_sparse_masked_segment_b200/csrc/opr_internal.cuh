@@ -38,6 +38,14 @@ __host__ __device__ __forceinline__ bool visible(int32_t qg, int32_t qconv, int3
 
 __host__ __device__ __forceinline__ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// A block-map byte is class | (key halves << 2): class OPR_TILE_*, and bit h of the
+// key halves set when some query of the tile sees a key of half h (keys 64 h ..
+// 64 h + 63).  A tile-list entry is (tile index << 4) | block-map byte.
+__host__ __device__ __forceinline__ int entry_index(int e) { return e >> 4; }
+__host__ __device__ __forceinline__ int entry_class(int e) { return e & 3; }
+__host__ __device__ __forceinline__ int entry_halves(int e) { return (e >> 2) & 3; }
+constexpr int kKeyHalf = kTile / 2;
+
 // Key/query metadata of one 128-token tile of a sequence, precomputed by the
 // layout so that the attention kernels fetch it with one bulk copy: the tile's
 // tokens split into runs of equal (conversation, turn, type); run r covers
@@ -58,9 +66,9 @@ struct LayoutWs {
   int32_t n_tiles;    // n_seqs * T
   size_t tok_meta;    // int32 [total]          (turn << 2) | type
   size_t row_cnt;     // int32 [n_tiles]        non-empty tiles in row (s, I)
-  size_t row_list;    // int32 [n_tiles][T]     (J << 2) | class, ascending J
+  size_t row_list;    // int32 [n_tiles][T]     (J << 4) | block-map byte, ascending J
   size_t col_cnt;     // int32 [n_tiles]        non-empty tiles in column (s, J)
-  size_t col_list;    // int32 [n_tiles][T]     (I << 2) | class, ascending I
+  size_t col_list;    // int32 [n_tiles][T]     (I << 4) | block-map byte, ascending I
   size_t q_sched;     // int32 [n_tiles]        s * T + I, most tiles first
   size_t k_sched;     // int32 [n_tiles]        s * T + J, most tiles first
   size_t conv_off;    // int64 [n_convs + 1]    token offset of each conversation

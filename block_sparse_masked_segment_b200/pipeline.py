@@ -2,7 +2,8 @@
 
 forward:  opr_rope(q), opr_rope(k) by the layout's position ids (bf16 in,
           fp16 out) -> opr_attn_fwd
-backward: opr_attn_bwd -> opr_rope(inverse) on dq and dk
+backward: opr_attn_bwd with the position ids, whose epilogues rotate dq and dk
+          back (the gradients w.r.t. the unrotated q and k)
 (One-Pass to Reason: positions from "位置 ID 策略", mask from "分块稀疏注意力掩码").
 Every numerical step runs in libopr's CUDA kernels; this module only orders the
 calls and keeps buffers.
@@ -45,11 +46,10 @@ def useful_flops(pairs: int, hq: int, d: int, backward: bool) -> float:
     return f * 3.5 if backward else f
 
 
-def one_pass_forward(q_pre, k_pre, v, lay: Layout, base: float, scale=None, out_dtype=torch.float32,
-                     qk_dtype=torch.float16):
-    """RoPE (bf16 in, fp16 out by default) then masked attention.  Returns (o, lse, q_rot, k_rot)."""
-    q = torch.empty(q_pre.shape, dtype=qk_dtype, device=q_pre.device)
-    k = torch.empty(k_pre.shape, dtype=qk_dtype, device=k_pre.device)
+def one_pass_forward(q_pre, k_pre, v, lay: Layout, base: float, scale=None, out_dtype=torch.float32):
+    """RoPE (bf16 in, fp16 out) then masked attention.  Returns (o, lse, q_rot, k_rot)."""
+    q = torch.empty(q_pre.shape, dtype=torch.float16, device=q_pre.device)
+    k = torch.empty(k_pre.shape, dtype=torch.float16, device=k_pre.device)
     opr_rope(q_pre, lay.pos_id, base, out=q, dev_status=lay.dev_status)
     opr_rope(k_pre, lay.pos_id, base, out=k, dev_status=lay.dev_status)
     o, lse = opr_attn_fwd(q, k, v, lay, scale, out_dtype)
@@ -57,11 +57,8 @@ def one_pass_forward(q_pre, k_pre, v, lay: Layout, base: float, scale=None, out_
 
 
 def one_pass_backward(q_rot, k_rot, v, o, do, lse, lay: Layout, base: float, scale=None):
-    """Gradients w.r.t. the unrotated q, k and v."""
-    dq, dk, dv = opr_attn_bwd(q_rot, k_rot, v, o, do, lse, lay, scale)
-    opr_rope(dq, lay.pos_id, base, inverse=True)
-    opr_rope(dk, lay.pos_id, base, inverse=True)
-    return dq, dk, dv
+    """Gradients w.r.t. the unrotated q, k and v (the backward's epilogues rotate dq and dk back)."""
+    return opr_attn_bwd(q_rot, k_rot, v, o, do, lse, lay, scale, rope_base=base)
 
 
 class OnePassAttention:
@@ -76,8 +73,8 @@ class OnePassAttention:
         self.layout = opr_build_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, device=device)
         self.base = base
 
-    def forward(self, q_pre, k_pre, v, scale=None, out_dtype=torch.float32, qk_dtype=torch.float16):
-        return one_pass_forward(q_pre, k_pre, v, self.layout, self.base, scale, out_dtype, qk_dtype)
+    def forward(self, q_pre, k_pre, v, scale=None, out_dtype=torch.float32):
+        return one_pass_forward(q_pre, k_pre, v, self.layout, self.base, scale, out_dtype)
 
     def backward(self, q_rot, k_rot, v, o, do, lse, scale=None):
         return one_pass_backward(q_rot, k_rot, v, o, do, lse, self.layout, self.base, scale)

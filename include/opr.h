@@ -58,16 +58,18 @@ typedef int32_t opr_status;
 #define OPR_DEV_SEQ_TOO_LONG 4     /* a sequence is longer than max_seqlen */
 #define OPR_DEV_WAIT_TIMEOUT 8     /* a pipeline wait exceeded its time limit; outputs are invalid */
 #define OPR_DEV_FP16_RANGE 16      /* an fp16 value beyond +-65504 was written (opr_rope output, or the
-                                      backward's fp16 copies of dO and v) */
+                                      backward's fp16 copies of the scaled dO and of v) */
 
 #define OPR_DTYPE_BF16 0
 #define OPR_DTYPE_FP32 1
 #define OPR_DTYPE_FP16 2
 
 #define OPR_TILE 128               /* edge of a block-map tile, in tokens */
-#define OPR_TILE_EMPTY 0
+#define OPR_TILE_EMPTY 0           /* block-map classes (bits 0-1 of a block-map byte) */
 #define OPR_TILE_FULL 1
 #define OPR_TILE_PARTIAL 2
+#define OPR_TILE_KEY_HALF0 4       /* bits 2-3: a query of the tile sees a key of half 0 / half 1 */
+#define OPR_TILE_KEY_HALF1 8
 
 /*
  * Bytes of the layout workspace that opr_build_layout fills and the attention
@@ -100,10 +102,13 @@ OPR_API size_t opr_layout_workspace_bytes(int32_t n_seqs, int32_t n_convs, int32
  *   turn_idx       int32 [total]       turn index within the conversation (0-based)
  *   conv_idx       int32 [total]       global conversation index
  *   pos_id         int32 [total]       position id
- *   block_map      uint8 [n_seqs][T][T], T = ceil(max_seqlen / 128): tile (I, J)
- *                  of sequence s is 0 empty, 1 full (all 128 x 128 pairs
- *                  visible), 2 partial; indices past the sequence count as
- *                  not visible, so tail tiles are never full
+ *   block_map      uint8 [n_seqs][T][T], T = ceil(max_seqlen / 128).  Bits 0-1
+ *                  of the byte of tile (I, J) of sequence s: 0 empty, 1 full
+ *                  (all 128 x 128 pairs visible), 2 partial; indices past the
+ *                  sequence count as not visible, so tail tiles are never full.
+ *                  Bits 2-3: bit 2 + h set when some query of the tile sees a
+ *                  key of its half h (keys 64 h .. 64 h + 63); the attention
+ *                  calls skip the half that no query sees
  *   workspace      opr_layout_workspace_bytes(...) bytes, read by the attention calls
  *   dev_status     int32 word, OPR_DEV_* bits OR-ed in on inconsistent input
  * Returns OPR_INVALID_ARG for null pointers / negative sizes / n_seqs > n_convs
@@ -144,17 +149,28 @@ OPR_API opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_d
 /*
  * opr_attn_fwd - block-sparse masked attention forward (tcgen05 / TMEM / TMA).
  *
+ * Defined by the One-Pass to Reason wiki note, "分块稀疏注意力掩码" (one mask
+ * over the packed conversation: h_i sees H<i; t_i and r_i^in see H<i and h_i;
+ * r_i^out sees H<i, h_i and t_i; every segment causal within itself) and
+ * "实现细节" (the mask applied block-sparsely inside attention, with sequence
+ * packing); the English note's "Method" (items 1-2) states the same rules.
+ * The attention itself is softmax attention restricted to the visible keys:
  * O = softmax(scale * Q K^T restricted to visible keys) V for each q head;
  * q head h reads kv head h / (hq / hkv).  Tiles marked empty in the block map
  * are skipped, the visibility predicate is evaluated only on partial tiles.
- *   q            [total, hq, head_dim]   (already rotated), qk_dtype
- *   k            [total, hkv, head_dim]  (already rotated), qk_dtype
- *   qk_dtype     OPR_DTYPE_FP16 or OPR_DTYPE_BF16 (the type of the S = Q K^T MMA)
+ *   q            fp16 [total, hq, head_dim]   (already rotated, e.g. by opr_rope)
+ *   k            fp16 [total, hkv, head_dim]  (already rotated)
+ *   qk_dtype     OPR_DTYPE_FP16 (the type of the S = Q K^T MMA); any other
+ *                value returns OPR_UNSUPPORTED
  *   v            bf16 [total, hkv, head_dim]
  *   cu_seqlens, conv_idx, layout_ws: outputs of opr_build_layout for the same sizes
  *   o            [total, hq, head_dim], o_dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32
  *   lse          fp32 [hq, total]: natural-log sum of exp(scale * q.k) over visible keys
- * head_dim must be 64 or 128; all pointers 16-byte aligned.
+ * head_dim must be 64 or 128; all pointers 16-byte aligned; total_tokens at
+ * most n_seqs * ceil(max_seqlen / 128) * 128 (else OPR_INVALID_ARG).  All
+ * buffers are the caller's; the call reads q, k, v and the layout and writes
+ * o and lse only.  Errors: OPR_INVALID_ARG, OPR_UNSUPPORTED, OPR_CUDA_ERROR
+ * (text from opr_last_error); OPR_DEV_WAIT_TIMEOUT in *dev_status.
  */
 OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_dtype,
                         const int32_t* cu_seqlens,
@@ -167,48 +183,68 @@ OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int
 /*
  * Bytes of device scratch that opr_attn_bwd needs.  With
  * N = n_seqs * ceil(max_seqlen / 128) * 128 (a bound on the token count):
+ *   256 bytes for max |dO| (which sets the gradient scale below);
  *   the row terms D = rowsum(dO * O) and LSE * log2(e), stored per 128-token
  *   tile: 2 * 4 * hq * N bytes;
  *   an fp16 copy of dO: 2 * N * hq * head_dim bytes;
  *   an fp16 copy of v (kv heads bounded by hq): 2 * N * hq * head_dim bytes;
+ *   the rotary (cos, sin) table of the positions below max_seqlen:
+ *   8 * max_seqlen * (head_dim / 2) bytes (used when rope_pos_id is given);
  * each part rounded up to 256 bytes.  Returns 0 for negative arguments.
  */
 OPR_API size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq,
                                             int32_t head_dim);
 
 /*
- * opr_attn_bwd - gradients of opr_attn_fwd w.r.t. the rotated q, k and v.
+ * opr_attn_bwd - gradients of opr_attn_fwd w.r.t. q, k (rotated, or unrotated
+ * with rope_pos_id) and v.
  *
- * With P recomputed from LSE: D = rowsum(dO * O), dV = P^T dO,
- * dS = P * (dO V^T - D), dQ = scale dS K, dK = scale dS^T Q; dK and dV sum
- * over the q heads that share a kv head.  Deterministic (no atomics).
- *   q, k, v, o, dout  as in opr_attn_fwd (o in o_dtype, dout bf16); dS is formed
- *                     in qk_dtype for the dQ and dK products
+ * The pages fine-tune through this layer (wiki note, "理论保证": the one-pass
+ * loss equals the N-pass loss, so its gradients are the N-pass gradients;
+ * the mask is that of "分块稀疏注意力掩码").  These are the analytic gradients
+ * of softmax attention under that mask.  With P recomputed from LSE:
+ * D = rowsum(dO * O), dV = P^T dO, dS = P * (dO V^T - D), dQ = scale dS K,
+ * dK = scale dS^T Q; dK and dV sum over the q heads that share a kv head.
+ * Deterministic (no atomics).
+ *   q, k, v, o, dout  as in opr_attn_fwd (q, k fp16; o in o_dtype; dout bf16)
  *   lse               fp32 [hq, total] from opr_attn_fwd
  *   dq                fp32 [total, hq, head_dim]
  *   dk, dv            fp32 [total, hkv, head_dim]
+ *   rope_pos_id       NULL: dq and dk are the gradients w.r.t. the rotated q and k
+ *                     given.  Otherwise int32 [total] position ids (those q and k
+ *                     were rotated by, e.g. opr_build_layout's pos_id, each below
+ *                     max_seqlen) and rope_base > 1 their base: dq and dk are
+ *                     rotated back in the kernels' epilogues, giving the gradients
+ *                     w.r.t. the unrotated q and k, as opr_rope(inverse) on the
+ *                     first form would (a position outside [0, max_seqlen) sets
+ *                     OPR_DEV_BAD_INPUT and is left unrotated)
  *   workspace         opr_attn_bwd_workspace_bytes(...) bytes of device scratch,
  *                     16-byte aligned, owned by the caller; the call overwrites it
- * The dK/dV products use fp16 copies of dO and v (dV = P^T dO needs P^T with
- * more mantissa than bf16 has, and the two operands of one tensor-core product
- * share a type).  bf16 -> fp16 is exact for magnitudes in [2^-14, 65504];
- * smaller ones lose low bits and a larger one sets OPR_DEV_FP16_RANGE in
- * *dev_status (the results are then invalid).
+ * Precision: the tensor-core products take 16-bit operands.  The backward is
+ * linear in dO, so it runs on 2^k dO, with k chosen on the device from max |dO|
+ * so that max |2^k dO| lies in [8, 16), and divides dq, dk, dv by 2^k (exact).
+ * The fp16 copy of 2^k dO and the fp16 dS therefore keep 11 significant bits
+ * at any gradient magnitude (a loss divided by the token count, passed back
+ * through later layers, is often 1e-5 .. 1e-8).  v is copied to fp16 as it is:
+ * a |v| beyond 65504, or an inf or NaN in dO, sets OPR_DEV_FP16_RANGE in
+ * *dev_status (the results are then invalid).  Other errors as opr_attn_fwd.
  */
 OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int32_t qk_dtype,
                         const void* o, int32_t o_dtype, const void* dout, const float* lse,
                         const int32_t* cu_seqlens, const int32_t* conv_idx, const void* layout_ws,
                         int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
                         int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
-                        float scale, float* dq, float* dk, float* dv, void* workspace,
-                        size_t workspace_bytes, int32_t* dev_status, void* stream);
+                        float scale, float* dq, float* dk, float* dv, const int32_t* rope_pos_id,
+                        double rope_base, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, void* stream);
 
 /*
  * opr_attn_bwd_stages - the same computation as opr_attn_bwd, split into its
  * three kernels so that a caller can order, overlap or time them one by one.
  * `stages` is an OR of:
- *   OPR_BWD_ROW_TERMS  D = rowsum(dO * O) and the fp16 copies of dO and v into
- *                      `workspace` (needed by the other two)
+ *   OPR_BWD_ROW_TERMS  max |dO|, D = rowsum(dO * O), the fp16 copies of dO and v
+ *                      and (with rope_pos_id) the rotary table into `workspace`
+ *                      (needed by the other two)
  *   OPR_BWD_DQ         dq   (one CTA per query tile and q head)
  *   OPR_BWD_DKDV       dk, dv (one CTA per key tile and kv head; GQA group summed in the CTA)
  * Running all three, in this order on one stream, equals opr_attn_bwd.
@@ -224,8 +260,9 @@ OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void*
                                        const void* layout_ws, int32_t n_seqs, int32_t n_convs,
                                        int32_t n_turns, int64_t total_tokens, int32_t max_seqlen,
                                        int32_t hq, int32_t hkv, int32_t head_dim, float scale, float* dq,
-                                       float* dk, float* dv, void* workspace, size_t workspace_bytes,
-                                       int32_t* dev_status, int32_t stages, void* stream);
+                                       float* dk, float* dv, const int32_t* rope_pos_id, double rope_base,
+                                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                       int32_t stages, void* stream);
 
 /*
  * opr_attn_bwd_noalloc - opr_attn_bwd for callers that cannot allocate device
@@ -235,20 +272,21 @@ OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void*
  * not call cudaMalloc, which can block and synchronize the device.
  *
  * Same inputs, outputs and error behaviour as opr_attn_bwd, without the
- * workspace arguments: the scratch (the row terms and the fp16 copies of dO
- * and v) lives in one fixed
+ * workspace arguments: the scratch (max |dO|, the row terms, the fp16 copies
+ * of dO and v and the rotary table) lives in one fixed
  * library-owned device array of OPR_NOALLOC_SCRATCH_BYTES, allocated by the
  * CUDA loader on every GPU that loads the library and held until the process
  * exits.  The call allocates and frees nothing.
  *   - Returns OPR_SCRATCH_TOO_LARGE, before touching the device, when
  *     opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) exceeds
  *     OPR_NOALLOC_SCRATCH_BYTES.
+ *   - The array is the current device's: `stream` and every pointer must
+ *     belong to the device that is current on the calling thread.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
  *   - Every call on a device shares the one array and leaves its contents in
- *     it; nothing needs clearing because each call rewrites every entry it
- *     reads.  Calls whose work overlaps on the GPU (other streams, other host
+ *     it; each call clears (max |dO|) or rewrites every entry it reads.  Calls whose work overlaps on the GPU (other streams, other host
  *     threads) race on the array: order them on one stream.
  */
 #define OPR_NOALLOC_SCRATCH_BYTES (32u << 20)
@@ -259,6 +297,7 @@ OPR_API opr_status opr_attn_bwd_noalloc(const void* q, const void* k, const void
                                         int32_t n_convs, int32_t n_turns, int64_t total_tokens,
                                         int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
                                         float scale, float* dq, float* dk, float* dv,
+                                        const int32_t* rope_pos_id, double rope_base,
                                         int32_t* dev_status, void* stream);
 
 /* Library version string, e.g. "opr 0.1.0 sm_100a". */
@@ -323,10 +362,23 @@ OPR_API opr_status opr_fold_rows(const float* dy, int64_t total_tokens, int64_t 
  * turns (h, t, r).  Every t and r^out row lies in exactly one pass, and the output is an
  * ordinary input of opr_build_layout, so the attention calls serve every K unchanged.
  *
- * opr_kpass_sizes - output turn and conversation (pass) counts, from a HOST conv_turn_ptr.
+ * opr_kpass_sizes - the sizes of the K-pass arrangement, from HOST copies of the one-pass
+ * layout inputs (what a caller needs to allocate the outputs of opr_kpass_plan and
+ * opr_kpass_index and the buffers of the attention calls that follow):
+ *   turn_lens, conv_turn_ptr, seq_conv_ptr  host arrays, as for opr_build_layout
+ *   n_out_turns, n_out_convs   turns and conversations (passes) of the arrangement
+ *   total_tokens               its one-pass tokens, sum of h + t + 2r over the output turns
+ *   max_seqlen                 its longest sequence (the passes of a conversation stay in
+ *                              the conversation's sequence)
+ *   orig_tokens                tokens of the original stream, sum of h + t + r
+ * Returns OPR_INVALID_ARG for null pointers, K < 1, negative lengths, pointers that do not
+ * span the turns and conversations, or sizes beyond int32 token offsets.
  */
-OPR_API opr_status opr_kpass_sizes(const int32_t* conv_turn_ptr, int32_t n_convs, int32_t K,
-                                   int64_t* n_out_turns, int64_t* n_out_convs);
+OPR_API opr_status opr_kpass_sizes(const int32_t* turn_lens, const int32_t* conv_turn_ptr,
+                                   const int32_t* seq_conv_ptr, int32_t n_seqs, int32_t n_convs,
+                                   int32_t n_turns, int32_t K, int64_t* n_out_turns,
+                                   int64_t* n_out_convs, int64_t* total_tokens, int64_t* max_seqlen,
+                                   int64_t* orig_tokens);
 
 /*
  * opr_kpass_plan - the K-pass arrangement as layout inputs (device arrays).

@@ -1,6 +1,7 @@
 /* Plain C99 user of the C ABI: the host-only entry points, no GPU needed.
- * Prints the library version, the K-pass sizes and the loss-row count of a
- * two-conversation batch, one value per line. */
+ * Prints the library version, the K-pass sizes (turns, passes, tokens, longest
+ * sequence, original tokens) and the loss-row count of a two-conversation
+ * batch in one sequence, one value per line. */
 #include <stdint.h>
 #include <stdio.h>
 
@@ -10,11 +11,16 @@ int main(void) {
   /* two conversations: turns (2,3,2), (1,2,1) and (4,2,3) */
   const int32_t turn_lens[] = {2, 3, 2, 1, 2, 1, 4, 2, 3};
   const int32_t conv_turn_ptr[] = {0, 2, 3};
-  int64_t n_out_turns = -1, n_out_convs = -1;
+  const int32_t seq_conv_ptr[] = {0, 2};
+  int64_t n_out_turns = -1, n_out_convs = -1, total = -1, max_seqlen = -1, orig = -1;
   printf("%s\n", opr_version());
-  if (opr_kpass_sizes(conv_turn_ptr, 2, 2, &n_out_turns, &n_out_convs) != OPR_OK) return 1;
-  printf("%lld\n%lld\n", (long long)n_out_turns, (long long)n_out_convs);
+  if (opr_kpass_sizes(turn_lens, conv_turn_ptr, seq_conv_ptr, 1, 2, 3, 2, &n_out_turns, &n_out_convs, &total,
+                      &max_seqlen, &orig) != OPR_OK)
+    return 1;
+  printf("%lld\n%lld\n%lld\n%lld\n%lld\n", (long long)n_out_turns, (long long)n_out_convs, (long long)total,
+         (long long)max_seqlen, (long long)orig);
   printf("%lld\n", (long long)opr_loss_row_count(turn_lens, 3));
-  printf("%d\n", (int)(opr_kpass_sizes(conv_turn_ptr, 2, 0, &n_out_turns, &n_out_convs) == OPR_INVALID_ARG));
+  printf("%d\n", (int)(opr_kpass_sizes(turn_lens, conv_turn_ptr, seq_conv_ptr, 1, 2, 3, 0, &n_out_turns,
+                                        &n_out_convs, &total, &max_seqlen, &orig) == OPR_INVALID_ARG));
   return 0;
 }

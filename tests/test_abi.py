@@ -15,7 +15,7 @@ from block_sparse_masked_segment_b200.pipeline import visible_pairs_closed_form
 import synth
 from oracle import opr_oracle as orc
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "opr.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
 
 
 @pytest.fixture(scope="module")
@@ -25,7 +25,8 @@ def lib():
 
 
 def declared_symbols():
-    text = open(HEADER).read()
+    """Every entry point that a header under include/ declares."""
+    text = "".join(open(os.path.join(INCLUDE, f)).read() for f in sorted(os.listdir(INCLUDE)) if f.endswith(".h"))
     return sorted(set(re.findall(r"OPR_API\s+[\w\s\*]+?\b(opr_\w+)\s*\(", text)))
 
 
@@ -39,6 +40,14 @@ def test_exports_every_declared_symbol(lib):
 
 def test_version(lib):
     assert opr.opr_version().startswith("opr ")
+
+
+def test_wait_limit_hook_round_trips(lib):
+    """The test hook of include/opr_testing.h sets the pipeline-wait limit and returns the old one
+    (host code only: no kernel runs)."""
+    prev = lib.opr_testing_set_wait_limit_ns(12345)
+    assert prev == 2_000_000_000
+    assert lib.opr_testing_set_wait_limit_ns(prev) == 12345
 
 
 def test_workspace_queries(lib):
@@ -75,7 +84,26 @@ def test_host_argument_checks(lib):
                             fake, 0, fake, fake, N) == 2
     # opr_attn_bwd_stages: unknown stage bits
     assert lib.opr_attn_bwd_stages(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
-                                   4, 2, 128, 0.1, fake, fake, fake, fake, 1 << 20, fake, 8, N) == 1
+                                   4, 2, 128, 0.1, fake, fake, fake, N, 0.0, fake, 1 << 20, fake, 8, N) == 1
+    # a rotary position array without a valid base
+    assert lib.opr_attn_bwd(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
+                            4, 2, 128, 0.1, fake, fake, fake, fake, 0.5, fake, 1 << 30, fake, N) == 1
+    # q/k in bf16 are refused: the attention calls take the rotated q and k in fp16 only
+    assert lib.opr_attn_fwd(fake, fake, fake, 0, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
+                            fake, 0, fake, fake, N) == 2
+    assert lib.opr_attn_bwd(fake, fake, fake, 0, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
+                            4, 2, 128, 0.1, fake, fake, fake, N, 0.0, fake, 1 << 30, fake, N) == 2
+    # more tokens than n_seqs * ceil(max_seqlen / 128) * 128 (the bound every workspace is sized
+    # by): refused on the host, by every call that sizes buffers from (n_seqs, max_seqlen)
+    assert lib.opr_attn_fwd(fake, fake, fake, 2, fake, fake, fake, 1, 1, 1, 300, 100, 4, 2, 128, 0.1,
+                            fake, 0, fake, fake, N) == 1
+    assert lib.opr_attn_bwd(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 300, 100,
+                            4, 2, 128, 0.1, fake, fake, fake, N, 0.0, fake, 1 << 30, fake, N) == 1
+    assert lib.opr_attn_bwd_noalloc(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 300, 100,
+                                    4, 2, 128, 0.1, fake, fake, fake, N, 0.0, fake, N) == 1
+    assert lib.opr_build_layout(fake, fake, fake, 1, 1, 1, 300, 100, fake, fake, fake, fake, fake, fake, fake,
+                                1 << 30, fake, N) == 1
+    assert opr.opr_layout_workspace_bytes(1, 1, 1, 300, 100) == 0
     # empty problems are no-ops
     assert lib.opr_attn_fwd(N, N, N, 2, N, N, N, 0, 0, 0, 0, 0, 4, 2, 128, 0.1, N, 0, N, N, N) == 0
 
@@ -116,19 +144,35 @@ def test_duplication_entry_points_check_arguments_on_the_host():
     assert lib.opr_kpass_plan(fake, fake, fake, 1, 1, 2, 0, 2, 1, fake, fake, fake, fake, fake, None) == 1  # K = 0
 
 
+def _kpass_sizes(lib, w, K):
+    lens = np.ascontiguousarray(np.asarray(w.turn_lens, dtype=np.int32).reshape(-1))
+    cp = np.ascontiguousarray(np.asarray(w.conv_turn_ptr, dtype=np.int32))
+    sp = np.ascontiguousarray(np.asarray(w.seq_conv_ptr, dtype=np.int32))
+    out = [ctypes.c_int64(-1) for _ in range(5)]
+    st = lib.opr_kpass_sizes(lens.ctypes.data, cp.ctypes.data, sp.ctypes.data, sp.size - 1, cp.size - 1,
+                             lens.size // 3, K, *(ctypes.byref(x) for x in out))
+    return st, [x.value for x in out]
+
+
 @pytest.mark.parametrize("K", [1, 2, 3, 5])
 def test_kpass_sizes_match_the_oracle(K):
-    """opr_kpass_sizes is host code: checked against the oracle's arrangement without a GPU."""
-    import synth
-    from oracle import opr_oracle as orc
-
+    """opr_kpass_sizes is host code: every size it reports (turns, passes, tokens, longest
+    sequence, original tokens) is checked against the oracle's arrangement without a GPU."""
     lib = opr.load_library()
-    w = synth.random_small_workload(21, max_convs=4, max_turns=6)
-    cp = np.ascontiguousarray(np.asarray(w.conv_turn_ptr, dtype=np.int32))
-    nt, nc = ctypes.c_int64(0), ctypes.c_int64(0)
-    assert lib.opr_kpass_sizes(cp.ctypes.data, cp.size - 1, K, ctypes.byref(nt), ctypes.byref(nc)) == 0
-    l2, c2, _, _ = orc.kpass_plan(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, K)
-    assert (nt.value, nc.value) == (len(l2), len(c2) - 1)
+    for seed in (21, 22):
+        w = synth.random_small_workload(seed, n_seqs=3, max_convs=4, max_turns=6)
+        st, (nt, nc, total, max_seqlen, orig) = _kpass_sizes(lib, w, K)
+        assert st == 0
+        l2, c2, s2, _ = orc.kpass_plan(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, K)
+        lay = orc.build_layout(l2, c2, s2)
+        assert (nt, nc) == (len(l2), len(c2) - 1)
+        assert total == int(lay.cu_seqlens[-1])
+        assert max_seqlen == int(np.diff(lay.cu_seqlens).max())
+        assert orig == int(np.asarray(w.turn_lens, dtype=np.int64).sum())
+    # bad input: K = 0, a negative length, pointers that do not span the turns
+    assert _kpass_sizes(lib, w, 0)[0] == 1
+    bad = synth.make_custom_workload([[[(1, -2, 3)]]], hq=1, hkv=1, d=64, base=1e4)
+    assert _kpass_sizes(lib, bad, 2)[0] == 1
 
 
 def test_loss_row_count_matches_the_oracle():

@@ -1,7 +1,7 @@
 """GPU parity of opr_build_layout and opr_rope against the oracle.
 
-Layout, position ids and the block map must match bit for bit (One-Pass to
-Reason, "Token 复制", "位置 ID 策略", "分块稀疏注意力掩码").
+Layout, position ids, the block map and its key-half bits must match bit for
+bit (One-Pass to Reason, "Token 复制", "位置 ID 策略", "分块稀疏注意力掩码").
 """
 
 import numpy as np
@@ -26,8 +26,10 @@ def _compare_layout(w):
     np.testing.assert_array_equal(lay.turn_idx.cpu().numpy(), ref.turn_idx)
     np.testing.assert_array_equal(lay.conv_idx.cpu().numpy(), ref.conv_idx)
     np.testing.assert_array_equal(lay.pos_id.cpu().numpy(), ref.pos_id)
-    bm_ref = orc.block_map(ref, max_seqlen=lay.max_seqlen)
-    np.testing.assert_array_equal(lay.block_map.cpu().numpy(), bm_ref)
+    bm = lay.block_map.cpu().numpy()
+    # each byte: tile class in bits 0-1, key halves that some query sees in bits 2-3
+    np.testing.assert_array_equal(bm & 3, orc.block_map(ref, max_seqlen=lay.max_seqlen))
+    np.testing.assert_array_equal(bm >> 2, orc.key_half_map(ref, max_seqlen=lay.max_seqlen))
     return lay, ref
 
 
@@ -69,7 +71,7 @@ def test_layout_depth_sweep(n_turns):
 def test_layout_npass_is_causal():
     w, _ = synth.npass_workload(synth.make_workload(1))
     lay, ref = _compare_layout(w)
-    bm = lay.block_map.cpu().numpy()
+    bm = lay.block_map.cpu().numpy() & 3
     for s in range(lay.n_seqs):
         L = int(ref.cu_seqlens[s + 1] - ref.cu_seqlens[s])
         nt = (L + 127) // 128

@@ -16,7 +16,7 @@ import torch
 import block_sparse_masked_segment_b200 as opr
 from block_sparse_masked_segment_b200 import _abi
 import synth
-from parity_helpers import assert_close, inputs, to_dev
+from parity_helpers import inputs, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +34,8 @@ def test_noalloc_backward_matches_workspace_backward_twice():
         torch.cuda.synchronize()
         assert opr.read_status(lay.dev_status) == []
         for name, g, r in zip(("dQ", "dK", "dV"), got, ref):
-            assert_close(f"{name} (call {call})", g, r)
+            # the same deterministic kernels on the same inputs: identical bits
+            np.testing.assert_array_equal(g, r, err_msg=f"{name} (call {call})")
 
 
 def test_noalloc_rejects_scratch_beyond_the_limit():
@@ -44,5 +45,5 @@ def test_noalloc_rejects_scratch_beyond_the_limit():
     assert opr.opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, d) > _abi.NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check fails first
     st = lib.opr_attn_bwd_noalloc(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, n_seqs, 1, 1,
-                                  max_seqlen, max_seqlen, hq, 8, d, 0.1, fake, fake, fake, fake, None)
+                                  max_seqlen, max_seqlen, hq, 8, d, 0.1, fake, fake, fake, None, 0.0, fake, None)
     assert st == _abi.OPR_SCRATCH_TOO_LARGE
