@@ -310,7 +310,7 @@ def opr_attn_fwd(q, k, v, lay: Layout, scale: float | None = None, out_dtype=tor
 
 
 def _rope_args(rope_base, lay: Layout):
-    """(pos_id pointer, base) of the rotation the backward undoes in its epilogues, or (None, 0)."""
+    """(pos_id pointer, base) of the rotation the backward undoes, or (None, 0)."""
     if rope_base is None:
         return None, 0.0
     return _ptr(lay.pos_id), float(rope_base)
@@ -319,8 +319,8 @@ def _rope_args(rope_base, lay: Layout):
 def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, workspace=None, out=None,
                  stages: int | None = None, rope_base: float | None = None):
     """dQ [total, hq, d], dK and dV [total, hkv, d] (fp32), w.r.t. the rotated q, k and v; with
-    ``rope_base``, dQ and dK are rotated back by the layout's position ids in the kernels'
-    epilogues (the gradients w.r.t. the unrotated q and k).
+    ``rope_base``, dQ and dK are rotated back by the layout's position ids (the gradients
+    w.r.t. the unrotated q and k).
 
     ``out`` = (dq, dk, dv) reuses buffers; ``stages`` (OR of BWD_ROW_TERMS,
     BWD_DQ, BWD_DKDV) runs only those kernels through opr_attn_bwd_stages, with

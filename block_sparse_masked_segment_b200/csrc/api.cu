@@ -153,7 +153,8 @@ AttnParams base_params(const int32_t* cu_seqlens, const int32_t* conv_idx, const
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.dev_status = dev_status;
-  p.wait_ns = g_wait_limit_ns.load();
+  const uint64_t limit = g_wait_limit_ns.load();
+  p.wait_ns = limit > 0xFFFFFFFFull ? 0xFFFFFFFFu : static_cast<uint32_t>(limit);
   return p;
 }
 
@@ -412,7 +413,7 @@ namespace {
 // Backward scratch: the row terms, then fp16 copies of dO and V.  Token counts
 // are bounded by n_seqs * ceil(max_seqlen / 128) * 128 and the kv heads by hq.
 struct BwdWs {
-  size_t absmax, row_terms, dout16, v16, rope, bytes;
+  size_t absmax, row_terms, dout16, v16, bytes;
 };
 
 BwdWs bwd_ws_map(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
@@ -424,8 +425,7 @@ BwdWs bwd_ws_map(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_di
   w.dout16 = w.row_terms + align_up(2 * sizeof(float) * static_cast<size_t>(hq) * tokens, 256);
   const size_t copy = align_up(sizeof(uint16_t) * tokens * static_cast<size_t>(hq) * static_cast<size_t>(head_dim), 256);
   w.v16 = w.dout16 + copy;
-  w.rope = w.v16 + copy;  // (cos, sin) per position < max_seqlen and rotary pair
-  w.bytes = w.rope + align_up(sizeof(float) * 2 * static_cast<size_t>(max_seqlen) * (head_dim / 2), 256);
+  w.bytes = w.v16 + copy;
   return w;
 }
 }  // namespace
@@ -471,7 +471,8 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   buf.row_terms = reinterpret_cast<float*>(static_cast<char*>(workspace) + bw.row_terms);
   buf.dout16 = reinterpret_cast<__half*>(static_cast<char*>(workspace) + bw.dout16);
   buf.v16 = reinterpret_cast<__half*>(static_cast<char*>(workspace) + bw.v16);
-  buf.rope_neg_log_base_over_half = rope_pos_id != nullptr ? -log(rope_base) / (head_dim / 2) : 0.0;
+  buf.rope_pos = rope_pos_id;
+  buf.rope_base = rope_base;
   BwdMaps maps;
   if (!make_map(&maps.q, q, total_tokens, hq, head_dim, f16) || !make_map(&maps.k, k, total_tokens, hkv, head_dim, f16) ||
       !make_map(&maps.v, v, total_tokens, hkv, head_dim) || !make_map(&maps.dout, dout, total_tokens, hq, head_dim) ||
@@ -488,11 +489,6 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   pq.dq = dq;
   pq.dk = dk;
   pq.dv = dv;
-  if (rope_pos_id != nullptr) {  // dq and dk w.r.t. the unrotated q and k
-    pq.pos_id = rope_pos_id;
-    pq.rope_cs = reinterpret_cast<const float2*>(static_cast<char*>(workspace) + bw.rope);
-    pq.rope_rows = max_seqlen;
-  }
   AttnParams pkv = pq;
   pkv.sched = ws_ptr<int32_t>(layout_ws, w.k_sched);
   cudaError_t e = launch_attn_bwd(head_dim, f16, maps, buf, pq, pkv, stages, static_cast<cudaStream_t>(stream));

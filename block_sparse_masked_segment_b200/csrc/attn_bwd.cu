@@ -136,20 +136,6 @@ __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o
   if (!in_range) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
-// (cos, sin) of the rotary angle p base^(-2j/D) for positions p < rows and pairs
-// j < half, angle formed in fp64 as opr_rope forms it; read by the dQ and dK
-// epilogues that rotate the gradients back.
-__global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ cs, int32_t rows, int32_t half,
-                                                         double neg_log_base_over_half) {
-  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (i >= static_cast<int64_t>(rows) * half) return;
-  const int pos = static_cast<int>(i / half), j = static_cast<int>(i % half);
-  const double theta = exp(static_cast<double>(j) * neg_log_base_over_half);
-  double sd, cd;
-  sincos(static_cast<double>(pos) * theta, &sd, &cd);
-  cs[i] = make_float2(static_cast<float>(cd), static_cast<float>(sd));
-}
-
 // fp16 copy of V for the dkdv kernel, eight values per thread (same range rule).
 __global__ void __launch_bounds__(256) cast_f16_kernel(const __nv_bfloat16* __restrict__ x, __half* __restrict__ y,
                                                        int64_t n8, int32_t* __restrict__ dev_status) {
@@ -459,22 +445,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float* dst = p.dq + (static_cast<size_t>(qg) * p.hq + head) * D;
       const float osc = p.scale * pow2f(-gk);  // undoes the gradient scale 2^k
-      if (p.rope_cs != nullptr) {
-        // the gradient w.r.t. the unrotated q: rotated back by the row's position
-        store_unrotated_row<D>(tl + kDqColAcc, half, osc, qv ? rope_row<D>(p, qg) : p.rope_cs, dst, qv);
-      } else {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t r[32];
-          const int oc = half * (D / 2) + c * 32;
-          tmem_ld32(tl + kDqColAcc + oc, r);
-          if (qv) {
-            float4* d4 = reinterpret_cast<float4*>(dst + oc);
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+        const int oc = half * (D / 2) + c * 32;
+        tmem_ld32(tl + kDqColAcc + oc, r);
+        if (qv) {
+          float4* d4 = reinterpret_cast<float4*>(dst + oc);
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
-              d4[x] = make_float4(__uint_as_float(r[4 * x]) * osc, __uint_as_float(r[4 * x + 1]) * osc,
-                                  __uint_as_float(r[4 * x + 2]) * osc, __uint_as_float(r[4 * x + 3]) * osc);
-          }
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(r[4 * x]) * osc, __uint_as_float(r[4 * x + 1]) * osc,
+                                __uint_as_float(r[4 * x + 2]) * osc, __uint_as_float(r[4 * x + 3]) * osc);
         }
       }
     }
@@ -822,22 +803,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 __uint_as_float(r[4 * x + 2]) * vsc, __uint_as_float(r[4 * x + 3]) * vsc);
         }
       }
-      if (p.rope_cs != nullptr) {
-        // the gradient w.r.t. the unrotated k: rotated back by the key's position
-        store_unrotated_row<D>(tl + kColDK, half, ksc, kvld ? rope_row<D>(p, kg) : p.rope_cs, dkp, kvld);
-      } else {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t r[32];
-          const int oc = half * (D / 2) + c * 32;
-          tmem_ld32(tl + kColDK + oc, r);
-          if (kvld) {
-            float4* d4 = reinterpret_cast<float4*>(dkp + oc);
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t r[32];
+        const int oc = half * (D / 2) + c * 32;
+        tmem_ld32(tl + kColDK + oc, r);
+        if (kvld) {
+          float4* d4 = reinterpret_cast<float4*>(dkp + oc);
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
-              d4[x] = make_float4(__uint_as_float(r[4 * x]) * ksc, __uint_as_float(r[4 * x + 1]) * ksc,
-                                  __uint_as_float(r[4 * x + 2]) * ksc, __uint_as_float(r[4 * x + 3]) * ksc);
-          }
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(r[4 * x]) * ksc, __uint_as_float(r[4 * x + 1]) * ksc,
+                                __uint_as_float(r[4 * x + 2]) * ksc, __uint_as_float(r[4 * x + 3]) * ksc);
         }
       }
     }
@@ -889,12 +865,6 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
           static_cast<const __nv_bfloat16*>(b.o), b.dout, pq.lse_in, pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d,
           row_l, b.dout16, b.dout_absmax, pq.dev_status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (pq.rope_cs != nullptr) {
-      const int64_t n = static_cast<int64_t>(pq.rope_rows) * (D / 2);
-      rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
-          const_cast<float2*>(pq.rope_cs), pq.rope_rows, D / 2, b.rope_neg_log_base_over_half);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
     const int64_t n8 = pq.total * pq.hkv * D / 8;
     if (n8 > 0) {
       const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, 148 * 16);
@@ -910,6 +880,10 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
     if (bq > 0)
       attn_bwd_dq_kernel<D, QK16><<<static_cast<unsigned>(bq), kThreads, smem_q, stream>>>(m.q, m.k, m.v, m.dout, pq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (b.rope_pos != nullptr &&  // dq w.r.t. the unrotated q: one pass over the rows
+        (e = launch_rope(pq.dq, OPR_DTYPE_FP32, pq.dq, OPR_DTYPE_FP32, b.rope_pos, pq.total, pq.hq, D, b.rope_base, 1,
+                         pq.dev_status, stream)) != cudaSuccess)
+      return e;
   }
   // 3) dK, dV
   if (stages & OPR_BWD_DKDV) {
@@ -919,7 +893,10 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
     if (bkv > 0)
       attn_bwd_dkdv_kernel<D, QK16>
           <<<static_cast<unsigned>(bkv), kThreads, smem_kv, stream>>>(m.q, m.k, m.v16, m.dout16, pkv);
-    e = cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (b.rope_pos != nullptr)  // dk w.r.t. the unrotated k
+      e = launch_rope(pkv.dk, OPR_DTYPE_FP32, pkv.dk, OPR_DTYPE_FP32, b.rope_pos, pkv.total, pkv.hkv, D, b.rope_base, 1,
+                      pkv.dev_status, stream);
   }
   return e;
 }

@@ -157,7 +157,8 @@ struct BwdBuffers {
   float* row_terms;  // D tiles, then LSE * log2(e) tiles
   __half* dout16;
   __half* v16;
-  double rope_neg_log_base_over_half;  // -ln(base) / (D / 2) of the rotary table
+  const int32_t* rope_pos;  // not null: rotate dq and dk back by these positions (base rope_base)
+  double rope_base;
 };
 
 struct AttnParams {
@@ -188,13 +189,8 @@ struct AttnParams {
   float* dq;
   float* dk;
   float* dv;
-  // inverse rotary embedding of dq and dk in the epilogues (rope_cs null: none):
-  // (cos, sin) of position p and pair j at rope_cs[p * (D / 2) + j], p < rope_rows
-  const int32_t* pos_id;
-  const float2* rope_cs;
-  int32_t rope_rows;
   int32_t* dev_status;
-  uint64_t wait_ns;  // limit of the pipeline waits (kWaitLimitNs; 0: a wait not already done times out)
+  uint32_t wait_ns;  // limit of the pipeline waits (kWaitLimitNs; 0: a wait not already done times out)
 };
 
 // ---------------------------------------------------------------- gradient scale
@@ -211,57 +207,31 @@ __host__ __device__ __forceinline__ int grad_scale_exp(uint32_t bits) {
   return k < -100 ? -100 : (k > 100 ? 100 : k);
 }
 
-// One thread's share of a gradient row held in TMEM (D fp32 columns from taddr in
-// this thread's lane), scaled by sc and rotated back by the row's rotary angles:
-// the gradient w.r.t. the unrotated q or k, x_j = y_j cos + y_{j+D/2} sin and
-// x_{j+D/2} = y_{j+D/2} cos - y_j sin.  Of the row's two threads, `part` takes
-// the pairs j = part D/4 .. part D/4 + D/4 - 1 (columns j and j + D/2).  cs is the
-// row's (cos, sin) table row; dst the row in global memory (written when valid).
-template <int D>
-__device__ __forceinline__ void store_unrotated_row(uint32_t taddr, int part, float sc, const float2* cs, float* dst,
-                                                    bool valid) {
-  constexpr int NP = D / 4;  // pairs per thread: 32 (D = 128) or 16 (D = 64)
-  const int j0 = part * NP;
-  uint32_t lo[NP], hi[NP];
-  if constexpr (NP == 32) {
-    tmem_ld32(taddr + j0, lo);
-    tmem_ld32(taddr + D / 2 + j0, hi);
-  } else {
-    tmem_ld16(taddr + j0, lo);
-    tmem_ld16(taddr + D / 2 + j0, hi);
-  }
-  if (!valid) return;
-  const float4* c4 = reinterpret_cast<const float4*>(cs + j0);  // two (cos, sin) pairs per float4
-  float xl[NP], xh[NP];
-#pragma unroll
-  for (int i = 0; i < NP; i += 2) {
-    const float4 w = c4[i / 2];
-    const float a0 = __uint_as_float(lo[i]) * sc, b0 = __uint_as_float(hi[i]) * sc;
-    const float a1 = __uint_as_float(lo[i + 1]) * sc, b1 = __uint_as_float(hi[i + 1]) * sc;
-    xl[i] = a0 * w.x + b0 * w.y;
-    xh[i] = b0 * w.x - a0 * w.y;
-    xl[i + 1] = a1 * w.z + b1 * w.w;
-    xh[i + 1] = b1 * w.z - a1 * w.w;
-  }
-  float4* dl = reinterpret_cast<float4*>(dst + j0);
-  float4* dh = reinterpret_cast<float4*>(dst + D / 2 + j0);
-#pragma unroll
-  for (int i = 0; i < NP / 4; ++i) {
-    dl[i] = make_float4(xl[4 * i], xl[4 * i + 1], xl[4 * i + 2], xl[4 * i + 3]);
-    dh[i] = make_float4(xh[4 * i], xh[4 * i + 1], xh[4 * i + 2], xh[4 * i + 3]);
-  }
-}
-
-// The (cos, sin) table row of a token's position; a position outside the table
-// (only with inconsistent inputs) sets OPR_DEV_BAD_INPUT and reads row 0 (no rotation).
-template <int D>
-__device__ __forceinline__ const float2* rope_row(const AttnParams& p, int64_t tok) {
-  int pos = p.pos_id[tok];
-  if (pos < 0 || pos >= p.rope_rows) {
-    atomicOr(p.dev_status, OPR_DEV_BAD_INPUT);
-    pos = 0;
-  }
-  return p.rope_cs + static_cast<size_t>(pos) * (D / 2);
+// 2^x for a pair of fp32 values on the FMA and integer pipes instead of the
+// special-function unit (which the softmax otherwise saturates): x = n + f with
+// n = rint(x), taken by adding 1.5 * 2^23 (Cody and Waite's additive range
+// reduction); 2^f by the degree-3 Chebyshev interpolant of 2^f on [-1/2, 1/2]
+// (coefficients from csrc/exp2_poly.py, relative error below 1e-4); n added to
+// the exponent field.  Exact 0 for x below -125 (and for -inf), where the
+// exponent would leave the normal range (the special-function unit flushes
+// there too).
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23: its ulp is 1
+  constexpr float kC0 = 9.999245405e-01f, kC1 = 6.931367517e-01f, kC2 = 2.426394820e-01f, kC3 = 5.583828315e-02f;
+  const uint64_t t2 = fadd2(x2, f2(kShift, kShift));      // the low mantissa bits hold rint(x)
+  const uint64_t n2 = fadd2(t2, f2(-kShift, -kShift));    // rint(x)
+  const uint64_t fr = ffma2(n2, f2(-1.f, -1.f), x2);      // f = x - rint(x) in [-1/2, 1/2]
+  uint64_t p = ffma2(f2(kC3, kC3), fr, f2(kC2, kC2));
+  p = ffma2(p, fr, f2(kC1, kC1));
+  p = ffma2(p, fr, f2(kC0, kC0));
+  float xl, xh, pl, ph, tl, th;
+  f2_split(x2, xl, xh);
+  f2_split(p, pl, ph);
+  f2_split(t2, tl, th);
+  // bits(t) << 23 is rint(x) << 23 (the shifter's own bits vanish in the shift)
+  const float rl = __int_as_float(__float_as_int(pl) + (__float_as_int(tl) << 23));
+  const float rh = __int_as_float(__float_as_int(ph) + (__float_as_int(th) << 23));
+  return f2(xl >= -125.f ? rl : 0.f, xh >= -125.f ? rh : 0.f);
 }
 
 // 2^k as a float, built from its bits (|k| <= 126).

@@ -362,7 +362,11 @@ __device__ __forceinline__ float row_max(const float (&sv)[NC]) {
 }
 
 // P = 2^(S scale log2(e) - mb) of NC scores (the scale-and-shift on fp32 pairs),
-// stored as bf16 two per TMEM column from p_addr; returns the sum of P.
+// stored as bf16 two per TMEM column from p_addr; returns the sum of P.  One pair
+// in kFmaExpEvery takes the FMA-pipe exponential, the others the special-function
+// unit, so that the two pipes share the softmax's exponentials.
+constexpr int kFmaExpEvery = 3;
+
 template <int NC>
 __device__ __forceinline__ float exp_pack_row(const float (&sv)[NC], float sl2, float mb, uint32_t p_addr) {
   const uint64_t sl2x2 = f2(sl2, sl2), nmb2 = f2(-mb, -mb);
@@ -372,10 +376,16 @@ __device__ __forceinline__ float exp_pack_row(const float (&sv)[NC], float sl2, 
     uint32_t pk[16];
 #pragma unroll
     for (int x = 0; x < 16; ++x) {
-      float a0, a1;
-      f2_split(ffma2(f2(sv[c * 32 + 2 * x], sv[c * 32 + 2 * x + 1]), sl2x2, nmb2), a0, a1);
-      const float p0 = fast_exp2(a0);
-      const float p1 = fast_exp2(a1);
+      const uint64_t a2 = ffma2(f2(sv[c * 32 + 2 * x], sv[c * 32 + 2 * x + 1]), sl2x2, nmb2);
+      float p0, p1;
+      if (x % kFmaExpEvery == kFmaExpEvery - 1) {  // resolved at compile time (unrolled loop)
+        f2_split(exp2_fma2(a2), p0, p1);
+      } else {
+        float a0, a1;
+        f2_split(a2, a0, a1);
+        p0 = fast_exp2(a0);
+        p1 = fast_exp2(a1);
+      }
       rs8[x & 7] += p0 + p1;
       pk[x] = pack_bf16x2(p0, p1);
     }
@@ -413,9 +423,9 @@ __device__ __forceinline__ MaxStep max_step(float m_run, float mx, float sl2) {
 //   warps 2..5  head A, warps 6..9 head B: one query row per thread, P (bf16)
 //               written over the first 64 columns of the thread's own row of S
 // TMEM columns: S_A 0, S_B 128, O_A 256, O_B 384.
-// Sub-tile skipping: on a partial tile of which no query sees one 64-key half,
-// S is the N = 64 product over the other half (written to that half's
-// columns), the softmax takes its 64 columns, and P V runs over its 64 keys.
+// Full 128x128 products on every non-empty tile: the kernel is bound by its
+// softmax, not by the tensor core, and the 64-key half products measured slower
+// here (the dQ kernel uses them).
 template <int D>
 struct FwdPairSmem {
   alignas(1024) uint8_t q[2][TileGeom<D>::kBytes];
@@ -522,37 +532,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // the whole warp runs this loop; elect.sync picks the issuing lane
-    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);   // S = Q K^T in the q/k type
-    constexpr uint32_t idesc_s64 = idesc_f32acc(128, 64, QK16, 0, 0);  // S over one 64-key half
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);         // O += P V, P and V bf16
+    constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);        // O += P V, P and V bf16
     const uint32_t sq[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
     auto issue_s = [&](int h, int j) {
-      const int hv = entry_halves(entry(j));
-      const uint32_t k0 = hv == 2 ? kKeyHalf : 0;  // first key of the product
-      const uint32_t idesc = hv == 3 ? idesc_s : idesc_s64;
-      // key row k0 of each 128-byte-row chunk (a multiple of the 8-row swizzle period)
-      const uint64_t kb = desc_kmajor(smem_u32(sm.k[j % NS]) + k0 * 128, 0);
+      const uint32_t sk = smem_u32(sm.k[j % NS]);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        mma_ss(tmem + h * 128 + k0, (desc_kmajor(sq[h], 0) + kmajor_step(kk)), kb + kmajor_step(kk), idesc,
-               kk > 0 ? 1u : 0u);
+        mma_ss(tmem + h * 128, (desc_kmajor(sq[h], 0) + kmajor_step(kk)), (desc_kmajor(sk, 0) + kmajor_step(kk)), idesc_s, kk > 0 ? 1u : 0u);
       mma_commit(&sm.bar_sfull[h]);
     };
     auto issue_pv = [&](int h, int j) -> bool {
       if (!warp_wait(&sm.bar_pfull[h], j & 1, abort_flag, p.wait_ns)) return false;
       tc_fence_after();
-      const int hv = entry_halves(entry(j));
-      const uint64_t vb = desc_mnmajor(smem_u32(sm.v[j % NS]), 0);
-      uint32_t acc = j > 0 ? 1u : 0u;
+      const uint32_t sv = smem_u32(sm.v[j % NS]);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if (!((hv >> half) & 1)) continue;  // no query of the tile sees these 64 keys
-#pragma unroll
-        for (int kk = 4 * half; kk < 4 * half + 4; ++kk) {
-          mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, vb + mnmajor_step(kk), idesc_o, acc);
-          acc = 1u;
-        }
-      }
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        mma_ts(tmem + 256 + h * 128, tmem + h * 128 + kk * 8, (desc_mnmajor(sv, 0) + mnmajor_step(kk)), idesc_o,
+               (j > 0 || kk > 0) ? 1u : 0u);
       mma_commit(&sm.bar_odone[h]);
       return true;
     };
@@ -620,41 +617,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      MaxStep ms;
-      float rs;
-      const int hv = entry_halves(e);
-      float sv[kTile];  // the row's scores; the first 64 hold the one seen key half of a half tile
-      if (hv == 3) {
-        {
-          uint32_t sr[kTile];
-          tmem_ld128(tl + scol, sr);
+      float sv[kTile];
+      {
+        uint32_t sr[kTile];
+        tmem_ld128(tl + scol, sr);
 #pragma unroll
-          for (int c = 0; c < kTile; ++c) sv[c] = __uint_as_float(sr[c]);
-        }
-        if (partial) {
-#pragma unroll
-          for (int c = 0; c < kTile; ++c)
-            if (!mask_bit(mm, c)) sv[c] = -INFINITY;
-        }
-        ms = max_step(m_run, row_max<kTile>(sv), sl2);
-        rs = exp_pack_row<kTile>(sv, sl2, ms.mb, tl + scol);  // P over S's read columns
-      } else {
-        // the one key half that some query sees: its 64 S columns, its 32 P columns
-        const int k0 = hv == 2 ? kKeyHalf : 0;
-        float(&sh)[kKeyHalf] = *reinterpret_cast<float(*)[kKeyHalf]>(&sv[0]);
-        {
-          uint32_t sr[kKeyHalf];
-          tmem_ld64(tl + scol + k0, sr);
-#pragma unroll
-          for (int c = 0; c < kKeyHalf; ++c) sh[c] = __uint_as_float(sr[c]);
-        }
-        const uint32_t mh[2] = {hv == 2 ? mm[2] : mm[0], hv == 2 ? mm[3] : mm[1]};
-#pragma unroll
-        for (int c = 0; c < kKeyHalf; ++c)
-          if (!((mh[c >> 5] >> (c & 31)) & 1u)) sh[c] = -INFINITY;
-        ms = max_step(m_run, row_max<kKeyHalf>(sh), sl2);
-        rs = exp_pack_row<kKeyHalf>(sh, sl2, ms.mb, tl + scol + k0 / 2);
+        for (int c = 0; c < kTile; ++c) sv[c] = __uint_as_float(sr[c]);
       }
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (!mask_bit(mm, c)) sv[c] = -INFINITY;
+      }
+      const MaxStep ms = max_step(m_run, row_max<kTile>(sv), sl2);
+      const float rs = exp_pack_row<kTile>(sv, sl2, ms.mb, tl + scol);  // P over S's read columns
       tmem_wait_st();
       if (j >= 1) {
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (j - 1) & 1, abort_flag, p.wait_ns))) {

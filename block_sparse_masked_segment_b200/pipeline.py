@@ -2,8 +2,8 @@
 
 forward:  opr_rope(q), opr_rope(k) by the layout's position ids (bf16 in,
           fp16 out) -> opr_attn_fwd
-backward: opr_attn_bwd with the position ids, whose epilogues rotate dq and dk
-          back (the gradients w.r.t. the unrotated q and k)
+backward: opr_attn_bwd with the position ids, which rotates dq and dk back
+          (the gradients w.r.t. the unrotated q and k)
 (One-Pass to Reason: positions from "位置 ID 策略", mask from "分块稀疏注意力掩码").
 Every numerical step runs in libopr's CUDA kernels; this module only orders the
 calls and keeps buffers.
@@ -57,7 +57,7 @@ def one_pass_forward(q_pre, k_pre, v, lay: Layout, base: float, scale=None, out_
 
 
 def one_pass_backward(q_rot, k_rot, v, o, do, lse, lay: Layout, base: float, scale=None):
-    """Gradients w.r.t. the unrotated q, k and v (the backward's epilogues rotate dq and dk back)."""
+    """Gradients w.r.t. the unrotated q, k and v (the backward rotates dq and dk back)."""
     return opr_attn_bwd(q_rot, k_rot, v, o, do, lse, lay, scale, rope_base=base)
 
 

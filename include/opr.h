@@ -188,8 +188,6 @@ OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int
  *   tile: 2 * 4 * hq * N bytes;
  *   an fp16 copy of dO: 2 * N * hq * head_dim bytes;
  *   an fp16 copy of v (kv heads bounded by hq): 2 * N * hq * head_dim bytes;
- *   the rotary (cos, sin) table of the positions below max_seqlen:
- *   8 * max_seqlen * (head_dim / 2) bytes (used when rope_pos_id is given);
  * each part rounded up to 256 bytes.  Returns 0 for negative arguments.
  */
 OPR_API size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq,
@@ -212,12 +210,11 @@ OPR_API size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, 
  *   dk, dv            fp32 [total, hkv, head_dim]
  *   rope_pos_id       NULL: dq and dk are the gradients w.r.t. the rotated q and k
  *                     given.  Otherwise int32 [total] position ids (those q and k
- *                     were rotated by, e.g. opr_build_layout's pos_id, each below
- *                     max_seqlen) and rope_base > 1 their base: dq and dk are
- *                     rotated back in the kernels' epilogues, giving the gradients
- *                     w.r.t. the unrotated q and k, as opr_rope(inverse) on the
- *                     first form would (a position outside [0, max_seqlen) sets
- *                     OPR_DEV_BAD_INPUT and is left unrotated)
+ *                     were rotated by, e.g. opr_build_layout's pos_id) and
+ *                     rope_base > 1 their base: the call rotates dq and dk back
+ *                     (one pass over each, right after the kernel that writes it),
+ *                     giving the gradients w.r.t. the unrotated q and k, exactly
+ *                     as opr_rope(inverse) on the first form
  *   workspace         opr_attn_bwd_workspace_bytes(...) bytes of device scratch,
  *                     16-byte aligned, owned by the caller; the call overwrites it
  * Precision: the tensor-core products take 16-bit operands.  The backward is
@@ -242,11 +239,12 @@ OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int
  * opr_attn_bwd_stages - the same computation as opr_attn_bwd, split into its
  * three kernels so that a caller can order, overlap or time them one by one.
  * `stages` is an OR of:
- *   OPR_BWD_ROW_TERMS  max |dO|, D = rowsum(dO * O), the fp16 copies of dO and v
- *                      and (with rope_pos_id) the rotary table into `workspace`
- *                      (needed by the other two)
- *   OPR_BWD_DQ         dq   (one CTA per query tile and q head)
- *   OPR_BWD_DKDV       dk, dv (one CTA per key tile and kv head; GQA group summed in the CTA)
+ *   OPR_BWD_ROW_TERMS  max |dO|, D = rowsum(dO * O) and the fp16 copies of dO
+ *                      and v into `workspace` (needed by the other two)
+ *   OPR_BWD_DQ         dq   (one CTA per query tile and q head; then, with
+ *                      rope_pos_id, the rotation of dq back)
+ *   OPR_BWD_DKDV       dk, dv (one CTA per key tile and kv head; GQA group summed
+ *                      in the CTA; then, with rope_pos_id, the rotation of dk back)
  * Running all three, in this order on one stream, equals opr_attn_bwd.
  * Other arguments and error behaviour as for opr_attn_bwd; unknown bits give
  * OPR_INVALID_ARG.
@@ -272,8 +270,8 @@ OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void*
  * not call cudaMalloc, which can block and synchronize the device.
  *
  * Same inputs, outputs and error behaviour as opr_attn_bwd, without the
- * workspace arguments: the scratch (max |dO|, the row terms, the fp16 copies
- * of dO and v and the rotary table) lives in one fixed
+ * workspace arguments: the scratch (max |dO|, the row terms and the fp16
+ * copies of dO and v) lives in one fixed
  * library-owned device array of OPR_NOALLOC_SCRATCH_BYTES, allocated by the
  * CUDA loader on every GPU that loads the library and held until the process
  * exits.  The call allocates and frees nothing.
