@@ -3,12 +3,14 @@
 
 One step = the whole hot path over one batch of synthetic conversations:
 opr_build_layout -> opr_rope(q), opr_rope(k) -> opr_attn_fwd -> opr_attn_bwd
-(three kernels) -> opr_rope(inverse) on dq and dk.
+(row terms, dQ and dK/dV kernels) -> opr_rope(inverse) on dq and dk.
 
-Default workload: the Qwen-3-8B-like fwd+bwd configuration (32 q / 8 kv
-heads, head_dim 128, 8 turns per conversation, h~U[32,256], t~U[256,1024],
-r~U[64,512], two sequences packed to 32768 tokens), the first configuration
-on which the fwd+bwd metric is defined.
+Default workload: the Qwen-3-32B-like fwd+bwd configuration (64 q / 8 kv
+heads, head_dim 128, 16 turns per conversation, h~U[64,512], t~U[512,2048],
+r~U[128,1024], packed to 65536 tokens), the largest configuration that fits
+one GPU.  The line also carries the Qwen-3-8B-like fwd+bwd and Qwen-3-4B-like
+forward workloads and the depth sweep (one conversation of 2..16 turns) as
+extra keys, each against the same kernels run N-pass.
 
 Metric: useful TFLOP/s = 4 d P Hq (1 + 2.5) / step time, P the visible (q, k)
 pairs per head; plus conversation tokens/s (h + t + r per turn, no
@@ -38,9 +40,11 @@ import synth  # noqa: E402
 
 METRIC = "1-pass masked attn fwd+bwd useful TFLOP/s; conv tokens/s vs N-pass"
 UNIT = "TFLOP/s"
-DEFAULT_CONFIG = 2
+DEFAULT_CONFIG = 4
 L2_FLUSH_BYTES = 512 << 20
-KERNELS_PER_STEP = 8 + 2 + 1 + 4 + 2  # layout (8), rope x2, fwd, bwd (row terms, v cast, dq, dkdv), inverse rope x2
+# layout (8), rope x2, fwd, bwd (max |dO|, row terms, v cast, dq, dkdv), inverse rope x2
+KERNELS_PER_STEP = 8 + 2 + 1 + 5 + 2
+ORACLE_SAMPLE_TOKENS = 3000  # one-pass tokens of the oracle's sample (cpu_baseline and the reference arm)
 
 # DRAM bytes (read + write) per launch of a kernel, from one ncu capture of
 # dram__bytes_read.sum and dram__bytes_write.sum at full size (the capture is
@@ -48,11 +52,13 @@ KERNELS_PER_STEP = 8 + 2 + 1 + 4 + 2  # layout (8), rope x2, fwd, bwd (row terms
 # was taken on: the sources' hash is recorded with it and checked at run time.
 MEASURED_TRAFFIC = {
     "bwd_dkdv": {
-        "config_index": 2,
-        "bytes": 1891566336 + 499474176,
+        "config_index": 4,
+        "bytes": 30281906432 + 508292096,
         "sources": ["attn_bwd.cu", "attn_common.cuh", "sm100.cuh", "layout.cu", "opr_internal.cuh"],
-        "sha256": "6a3afaf9e69aa29f24263f1514d5061196df732f882aa2055b9d519402be02ae",
-        "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:attn_ -s 9 -c 3",
+        "sha256": "7a8f6b1733e471f94f781c3c1d0045bef454cf08cc8b2771afddc71c1f69577b",
+        "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
+                   "-k regex:attn_ -s 9 -c 3 --csv python bench.py --steps 1 --warmup 3 --no-extra --no-e2e "
+                   "--no-cpu-baseline --no-npass",
     },
 }
 
@@ -143,13 +149,14 @@ class Runner:
     timing uses set 0 with its inputs resident.
     """
 
-    def __init__(self, w: synth.Workload, seed: int, device):
+    def __init__(self, w: synth.Workload, seed: int, device, forward_only: bool = False):
         import torch
 
         import block_sparse_masked_segment_b200 as opr
         from block_sparse_masked_segment_b200.pipeline import visible_pairs_closed_form
 
         self.torch, self.opr, self.w, self.dev = torch, opr, w, device
+        self.forward_only = forward_only
         rng = np.random.default_rng(seed)
         n = w.total_tokens
         bf = torch.bfloat16
@@ -197,13 +204,20 @@ class Runner:
         rec(2)
         o, lse = opr.opr_attn_fwd(self.q_rot, self.k_rot, b["v"], lay, out_dtype=torch.bfloat16)
         rec(3)
+        if self.forward_only:
+            for i in (4, 5, 6, 7):
+                rec(i)
+            self.layout = lay
+            return lay
         args = (self.q_rot, self.k_rot, b["v"], o, b["do"], lse, lay)
-        opr.opr_attn_bwd(*args, workspace=self.bwd_ws, out=b["grads"], stages=opr.BWD_ROW_TERMS)
+        kw = dict(workspace=self.bwd_ws, out=b["grads"])
+        opr.opr_attn_bwd(*args, stages=opr.BWD_ROW_TERMS, **kw)
         rec(4)
-        opr.opr_attn_bwd(*args, workspace=self.bwd_ws, out=b["grads"], stages=opr.BWD_DQ)
+        opr.opr_attn_bwd(*args, stages=opr.BWD_DQ, **kw)
         rec(5)
-        opr.opr_attn_bwd(*args, workspace=self.bwd_ws, out=b["grads"], stages=opr.BWD_DKDV)
+        opr.opr_attn_bwd(*args, stages=opr.BWD_DKDV, **kw)
         rec(6)
+        # gradients w.r.t. the unrotated q and k
         opr.opr_rope(b["grads"][0], lay.pos_id, self.w.base, inverse=True)
         opr.opr_rope(b["grads"][1], lay.pos_id, self.w.base, inverse=True)
         rec(7)
@@ -496,7 +510,7 @@ def run_oracle_once(sub: synth.Workload, seed: int):
     return dt, 14.0 * sub.d * pairs * sub.hq, sub.conversation_tokens()
 
 
-def cpu_baseline(w: synth.Workload, seed: int, target_tokens=6000):
+def cpu_baseline(w: synth.Workload, seed: int, target_tokens=ORACLE_SAMPLE_TOKENS):
     sub = oracle_sample(w, target_tokens)
     dt, flops, conv_tok = run_oracle_once(sub, seed)
     cores = len(os.sched_getaffinity(0))
@@ -512,7 +526,7 @@ def run_reference(args, cfg_index):
     if rank != 0:
         return
     w = synth.make_workload(cfg_index)
-    sub = oracle_sample(w, 3000)
+    sub = oracle_sample(w, ORACLE_SAMPLE_TOKENS)
     for i in range(args.warmup):
         run_oracle_once(sub, 17 + i)
     t0 = time.perf_counter()
@@ -548,6 +562,57 @@ def emit(line: dict, jsonl: str | None) -> None:
             fh.write(text + "\n")
 
 
+# ------------------------------------------------------------------ other workloads
+def measure_workload(w: synth.Workload, device, steps: int, warmup: int, flush, forward_only: bool = False,
+                     compare: bool = True):
+    """One workload on this GPU: kernel times and useful TFLOP/s of one-pass steps, and (compare)
+    conversation tokens/s against the same kernels run N-pass and K-pass (K = 2)."""
+    import torch
+
+    nobar = lambda: None  # noqa: E731
+    r = Runner(w, seed=11, device=device, forward_only=forward_only)
+    ms, per = time_runner(r, steps, warmup, flush, nobar)
+    fl = r.flops()
+    useful = fl["useful_fwd"] + (0.0 if forward_only else fl["useful_bwd"])
+    out = {"workload": w.name, "tokens_per_step": w.total_tokens, "conv_tokens_per_step": w.conversation_tokens(),
+           "pairs_per_head": r.pairs, "ms_per_step": ms / steps,
+           "useful_tflops": useful * steps / (ms * 1e-3) / 1e12,
+           "kernel_ms": {k: statistics.mean(v) for k, v in per.items()},
+           "pass": "forward only" if forward_only else "forward + backward"}
+    bf16_peak = peaks()[0]
+    out["fraction_of_bf16_peak"] = out["useful_tflops"] / bf16_peak
+    k_fwd = statistics.mean(per["attn_fwd"])
+    out["attn_fwd_tflops"] = fl["attn_fwd"] / (k_fwd * 1e-3) / 1e12
+    conv_tps = w.conversation_tokens() * steps / (ms * 1e-3)
+    out["conv_tokens_per_s"] = conv_tps
+    del r
+    if compare:
+        for name, build in (("npass", lambda: synth.npass_workload(w)[0]), ("kpass2", lambda: kpass_workload(w, 2, device))):
+            torch.cuda.empty_cache()
+            ow = build()
+            ro = Runner(ow, seed=11, device=device, forward_only=forward_only)
+            o_ms, _ = time_runner(ro, steps, warmup, flush, nobar)
+            o_tps = w.conversation_tokens() * steps / (o_ms * 1e-3)
+            out[name] = {"tokens_per_step": ow.total_tokens, "ms_per_step": o_ms / steps, "conv_tokens_per_s": o_tps,
+                         "one_pass_vs": conv_tps / o_tps}
+            del ro
+    torch.cuda.empty_cache()
+    return out
+
+
+def other_workloads(device, steps: int, warmup: int, flush):
+    """The other workloads of the line: the Qwen-3-8B-like fwd+bwd batch, the Qwen-3-4B-like forward
+    batch, and the depth sweep (one conversation of N turns, fwd+bwd), each one-pass against N-pass."""
+    res = {"qwen3-8b-like fwd+bwd (2 x 32K)": measure_workload(synth.make_workload(2), device, steps, warmup, flush),
+           "qwen3-4b-like fwd (16K)": measure_workload(synth.make_workload(1), device, steps, warmup, flush,
+                                                      forward_only=True)}
+    sweep = {}
+    for n in synth.DEPTH_SWEEP_TURNS:
+        sweep[str(n)] = measure_workload(synth.make_workload(3, n_turns=n), device, steps, warmup, flush)
+    res["depth sweep (h128 t512 r256, fwd+bwd)"] = sweep
+    return res
+
+
 # ------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -560,6 +625,7 @@ def main():
     ap.add_argument("--no-npass", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads (8B-like, 4B-like, depth sweep)")
     ap.add_argument("--seed", type=int, default=None, help="base seed of the synthetic batch (default 1000 + config)")
     ap.add_argument("--jsonl", default=None, help="also append the JSON line to this file")
     args = ap.parse_args()
@@ -665,6 +731,11 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         return
+    extra = None
+    if world == 1 and not args.no_extra and args.turns is None:
+        r = None  # the main workload's buffers are no longer needed
+        torch.cuda.empty_cache()
+        extra = other_workloads(device, args.steps, args.warmup, flush)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, seed=5)
@@ -687,6 +758,7 @@ def main():
         "e2e": e2e,
         "npass": npass,
         "next_rows": {"token_duplication": duplication, "kpass": kpass, "loss_side": loss_side},
+        "other_workloads": extra,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": dict(clocks.summary(), remeasured=remeasured),
         "cpu_baseline": cpu,
