@@ -32,6 +32,7 @@ from ._abi import (  # noqa: F401
     opr_attn_bwd_workspace_bytes,
     opr_version,
     read_status,
+    layout_table_offsets,
     EXPORTED_SYMBOLS,
 )
 from .pipeline import OnePassAttention, one_pass_forward, one_pass_backward, useful_flops  # noqa: F401

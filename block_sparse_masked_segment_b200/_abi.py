@@ -16,11 +16,14 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "lib", "libopr.so")
+# OPR_DEBUG_CHECKS=1 selects the library built with device-side bounds checks
+# (same entry points; a failed check sets OPR_DEV_BOUNDS in the status word).
+_LIB_PATH = os.path.join(_HERE, "lib", "libopr_debug.so" if os.environ.get("OPR_DEBUG_CHECKS") == "1" else "libopr.so")
 
 OPR_OK, OPR_INVALID_ARG, OPR_UNSUPPORTED, OPR_CUDA_ERROR, OPR_WORKSPACE_TOO_SMALL = 0, 1, 2, 3, 4
 DEV_BITS = {1: "bad input", 2: "total mismatch", 4: "sequence longer than max_seqlen", 8: "pipeline wait timeout",
-            16: "fp16 range exceeded (rope output or backward fp16 copy)"}
+            16: "fp16 range exceeded (rope output or backward fp16 copy)",
+            32: "layout-table index out of range (debug checks)"}
 DTYPE_BF16, DTYPE_FP32, DTYPE_FP16 = 0, 1, 2
 TILE = 128
 
@@ -46,6 +49,7 @@ EXPORTED_SYMBOLS = (
     "opr_loss_rows",
     "opr_cross_entropy",
     "opr_testing_set_wait_limit_ns",
+    "opr_testing_layout_tables",
 )
 
 BWD_ROW_TERMS, BWD_DQ, BWD_DKDV = 1, 2, 4
@@ -119,6 +123,8 @@ def load_library() -> ctypes.CDLL:
                                         F, P, P, P, P, D, P, SZ, P, I32, P]
     lib.opr_testing_set_wait_limit_ns.restype = ctypes.c_uint64
     lib.opr_testing_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.opr_testing_layout_tables.restype = I32
+    lib.opr_testing_layout_tables.argtypes = [I32, I32, I32, I64, I32, P]
     lib.opr_attn_bwd_noalloc.restype = I32
     lib.opr_attn_bwd_noalloc.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32,
                                          F, P, P, P, P, D, P, P]
@@ -181,6 +187,15 @@ class Layout:
     @property
     def T(self) -> int:
         return (self.max_seqlen + TILE - 1) // TILE
+
+
+def layout_table_offsets(lay: "Layout") -> dict[str, int]:
+    """Byte offsets of the tile tables inside lay.workspace (test hook of include/opr_testing.h)."""
+    out = (ctypes.c_uint64 * 4)()
+    st = load_library().opr_testing_layout_tables(lay.n_seqs, lay.n_convs, lay.n_turns, lay.total, lay.max_seqlen,
+                                                  ctypes.cast(out, ctypes.c_void_p))
+    _check(st, "opr_testing_layout_tables")
+    return dict(zip(("row_cnt", "row_list", "col_cnt", "col_list"), (int(x) for x in out)))
 
 
 def read_status(dev_status: torch.Tensor) -> list[str]:

@@ -1,9 +1,15 @@
 """Build libopr.so (the CUDA library behind include/opr.h) for sm_100a, in-tree.
 
-    python -m block_sparse_masked_segment_b200.build [--verbose]
+    python -m block_sparse_masked_segment_b200.build [--verbose] [--force]
 
-nvcc cross-compiles without a GPU.  The shared library lands next to this
-file (``lib/libopr.so``) so that it travels with the source tree.
+nvcc cross-compiles without a GPU.  The shared libraries land next to this
+file so that they travel with the source tree:
+
+- ``lib/libopr.so``        the release library;
+- ``lib/libopr_debug.so``  the same sources built with ``-DOPR_DEBUG_CHECKS``: the
+  attention kernels check the indices they take from the layout tables and set
+  OPR_DEV_BOUNDS instead of using a bad one.  The binding loads it when the
+  environment sets ``OPR_DEBUG_CHECKS=1``.
 """
 
 from __future__ import annotations
@@ -18,6 +24,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libopr.so")
+LIB_DEBUG = os.path.join(LIB_DIR, "libopr_debug.so")
 SOURCES = ["api.cu", "layout.cu", "rope.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu", "duplicate.cu", "loss.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
@@ -35,39 +42,47 @@ def nvcc_flags(verbose: bool = False) -> list[str]:
     return flags
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     inc = os.path.join(ROOT, "include")
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(inc, f) for f in os.listdir(inc)]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build the release library (or, with debug=True, the bounds-checking one); returns its path."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not _stale(lib):
+        return lib
     os.makedirs(LIB_DIR, exist_ok=True)
     objs = []
+    extra = ["-DOPR_DEBUG_CHECKS"] if debug else []
     for src in SOURCES:
-        obj = os.path.join(LIB_DIR, src.replace(".cu", ".o"))
-        cmd = [NVCC, *nvcc_flags(verbose), "-c", os.path.join(CSRC, src), "-o", obj]
+        obj = os.path.join(LIB_DIR, src.replace(".cu", "_debug.o" if debug else ".o"))
+        cmd = [NVCC, *nvcc_flags(verbose), *extra, "-c", os.path.join(CSRC, src), "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0 or verbose:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}")
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs, "-lcudart"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("link of libopr.so failed")
-    os.replace(tmp, LIB)
+        raise RuntimeError(f"link of {os.path.basename(lib)} failed")
+    os.replace(tmp, lib)
     for o in objs:
         os.remove(o)
-    return LIB
+    return lib
+
+
+def build_all(force: bool = False) -> list[str]:
+    """Both libraries: release and debug checks."""
+    return [build(force=force), build(force=force, debug=True)]
 
 
 if __name__ == "__main__":
@@ -76,3 +91,4 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     a = ap.parse_args()
     print(build(force=a.force or a.verbose, verbose=a.verbose))
+    print(build(force=a.force, debug=True))

@@ -335,9 +335,27 @@ opr_status opr_cross_entropy(const void* logits, int32_t dtype, int64_t n_rows, 
                                         grad_scale, dev_status, static_cast<cudaStream_t>(stream)));
 }
 
-const char* opr_version(void) { return "opr 0.2.0 sm_100a"; }
+const char* opr_version(void) {
+#ifdef OPR_DEBUG_CHECKS
+  return "opr 0.2.0 sm_100a debug-checks";
+#else
+  return "opr 0.2.0 sm_100a";
+#endif
+}
 
 uint64_t opr_testing_set_wait_limit_ns(uint64_t limit_ns) { return g_wait_limit_ns.exchange(limit_ns); }
+
+int opr_testing_layout_tables(int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
+                              int32_t max_seqlen, uint64_t offsets[4]) {
+  if (offsets == nullptr || n_seqs < 0 || n_convs < 0 || n_turns < 0 || total_tokens < 0 || max_seqlen < 0)
+    return OPR_INVALID_ARG;
+  const LayoutWs w = layout_ws_map(n_seqs, n_convs, n_turns, total_tokens, max_seqlen);
+  offsets[0] = w.row_cnt;
+  offsets[1] = w.row_list;
+  offsets[2] = w.col_cnt;
+  offsets[3] = w.col_list;
+  return OPR_OK;
+}
 
 const char* opr_last_error(void) { return g_cuda_error_text; }
 

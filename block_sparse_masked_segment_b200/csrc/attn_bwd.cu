@@ -87,6 +87,12 @@ __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o
   const int s = tile / T, J = tile % T;
   const int seq0 = cu_seqlens[s];
   const int L = cu_seqlens[s + 1] - seq0;
+  if constexpr (kDebugChecks) {  // the sequence must lie inside the token range
+    if (seq0 < 0 || L < 0 || seq0 + L > total) {
+      if (threadIdx.x == 0) atomicOr(dev_status, OPR_DEV_BOUNDS);
+      return;
+    }
+  }
   bool in_range = true;
   for (int i = 0; i < kTile / 8; ++i) {
     const int c = warp * (kTile / 8) + i;
@@ -192,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int head = blockIdx.x / p.n_items;
   const int tile_id = p.sched[blockIdx.x % p.n_items];
   if (head >= p.hq) return;
+  if (!debug_tile_ok(p, tile_id, p.row_cnt, p.row_list)) return;
   const int n = p.row_cnt[tile_id];
   if (n == 0) return;
   const int s = tile_id / p.T, I = tile_id % p.T;
@@ -517,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kvh = blockIdx.x / p.n_items;
   const int tile_id = p.sched[blockIdx.x % p.n_items];
   if (kvh >= p.hkv) return;
+  if (!debug_tile_ok(p, tile_id, p.col_cnt, p.col_list)) return;
   const int cnt = p.col_cnt[tile_id];
   if (cnt == 0) return;
   const int group = p.hq / p.hkv;

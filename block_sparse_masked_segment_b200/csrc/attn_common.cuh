@@ -19,6 +19,12 @@ namespace opr {
 // before a CTA exits always use this one.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+#ifdef OPR_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
 // CTA shape shared by the attention kernels: warp 0 TMA producer, warp 1 TMEM
 // owner / MMA issuer, warps 2..9 compute.  Two compute warps share each TMEM
 // lane quadrant (warp % 4): warps 2..5 own columns 0..63 of their rows, warps
@@ -141,6 +147,42 @@ __device__ __forceinline__ void key_row_mask(const TileMeta& t, int qbase, int k
 }
 
 __device__ __forceinline__ bool mask_bit(const uint32_t (&m)[4], int c) { return (m[c >> 5] >> (c & 31)) & 1u; }
+
+// Debug builds (OPR_DEBUG_CHECKS) check, before their first use, the indices an
+// attention CTA takes from the layout tables: its tile id, the sequence bounds of
+// the tile, the length of its tile list and each entry of the list (a tile inside
+// the sequence, class full or partial).  On a failure every thread of the CTA
+// returns false (one block-wide vote, taken before any barrier, TMEM allocation or
+// copy) and OPR_DEV_BOUNDS is set; the caller then returns without touching
+// memory through those indices.  Release builds compile it to `true`.
+template <typename Params>
+__device__ __forceinline__ bool debug_tile_ok(const Params& p, int tile_id, const int32_t* cnt_tab,
+                                              const int32_t* list_tab) {
+  if constexpr (!kDebugChecks) {
+    return true;
+  } else {
+    bool bad = p.T <= 0 || tile_id < 0 || tile_id >= p.n_items;
+    int n = 0, seq_len = 0;
+    if (!bad) {
+      const int s = tile_id / p.T, I = tile_id % p.T;
+      const int a = p.cu_seqlens[s], b = p.cu_seqlens[s + 1];
+      n = cnt_tab[tile_id];
+      seq_len = b - a;
+      bad = a < 0 || b < a || b > p.total || n < 0 || n > p.T || (n > 0 && I * kTile >= seq_len);
+    }
+    if (!bad) {
+      const int32_t* list = list_tab + static_cast<size_t>(tile_id) * p.T;
+      for (int x = threadIdx.x; x < n && !bad; x += blockDim.x) {
+        const int e = list[x];
+        const int idx = entry_index(e), cls = entry_class(e);
+        bad = idx < 0 || idx >= p.T || idx * kTile >= seq_len || (cls != OPR_TILE_FULL && cls != OPR_TILE_PARTIAL);
+      }
+    }
+    bad = __syncthreads_or(bad) != 0;
+    if (bad && threadIdx.x == 0) atomicOr(p.dev_status, OPR_DEV_BOUNDS);
+    return !bad;
+  }
+}
 
 // Tensor maps and buffers of one backward call (built by the entry point).
 struct BwdMaps {

@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int head = blockIdx.x / p.n_items;
   const int tile_id = p.sched[blockIdx.x % p.n_items];
   if (head >= p.hq) return;
+  if (!debug_tile_ok(p, tile_id, p.row_cnt, p.row_list)) return;
   const int n = p.row_cnt[tile_id];
   if (n == 0) return;  // tile past the end of its sequence
   const int s = tile_id / p.T, I = tile_id % p.T;
@@ -454,6 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pair = blockIdx.x / p.n_items;
   const int tile_id = p.sched[blockIdx.x % p.n_items];
   if (pair >= p.hq / 2) return;
+  if (!debug_tile_ok(p, tile_id, p.row_cnt, p.row_list)) return;
   const int n = p.row_cnt[tile_id];
   if (n == 0) return;
   const int s = tile_id / p.T, I = tile_id % p.T;

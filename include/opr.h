@@ -59,6 +59,11 @@ typedef int32_t opr_status;
 #define OPR_DEV_WAIT_TIMEOUT 8     /* a pipeline wait exceeded its time limit; outputs are invalid */
 #define OPR_DEV_FP16_RANGE 16      /* an fp16 value beyond +-65504 was written (opr_rope output, or the
                                       backward's fp16 copies of the scaled dO and of v) */
+#define OPR_DEV_BOUNDS 32          /* debug library (libopr_debug.so, built with OPR_DEBUG_CHECKS) only:
+                                      an index an attention kernel takes from the layout tables (tile id,
+                                      sequence bounds, tile-list length or entry) is out of range; the
+                                      kernel's CTA for that tile skipped all of its work, so the outputs
+                                      are invalid.  Release builds do not check and never set it. */
 
 #define OPR_DTYPE_BF16 0
 #define OPR_DTYPE_FP32 1

@@ -30,6 +30,20 @@ extern "C" {
  */
 OPR_API uint64_t opr_testing_set_wait_limit_ns(uint64_t limit_ns);
 
+/*
+ * Byte offsets, inside the layout workspace that opr_build_layout fills for
+ * these sizes, of the tile tables the attention kernels read:
+ *   offsets[0] row counts   int32 [n_seqs * T]       (T = ceil(max_seqlen / 128))
+ *   offsets[1] row lists    int32 [n_seqs * T][T]    entry (J << 4) | block-map byte
+ *   offsets[2] column counts int32 [n_seqs * T]
+ *   offsets[3] column lists int32 [n_seqs * T][T]    entry (I << 4) | block-map byte
+ * A test of the debug library (OPR_DEBUG_CHECKS) writes an out-of-range value
+ * there to see OPR_DEV_BOUNDS set.  Returns OPR_INVALID_ARG for a null pointer
+ * or negative sizes, else OPR_OK.
+ */
+OPR_API int opr_testing_layout_tables(int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
+                                      int32_t max_seqlen, uint64_t offsets[4]);
+
 #ifdef __cplusplus
 }
 #endif

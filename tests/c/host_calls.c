@@ -1,11 +1,14 @@
 /* Plain C99 user of the C ABI: the host-only entry points, no GPU needed.
  * Prints the library version, the K-pass sizes (turns, passes, tokens, longest
  * sequence, original tokens) and the loss-row count of a two-conversation
- * batch in one sequence, one value per line. */
+ * batch in one sequence, the refusal of a K of 0, and whether the test hook of
+ * opr_testing.h places the row counts first in the layout workspace, one
+ * value per line. */
 #include <stdint.h>
 #include <stdio.h>
 
 #include "opr.h"
+#include "opr_testing.h"
 
 int main(void) {
   /* two conversations: turns (2,3,2), (1,2,1) and (4,2,3) */
@@ -22,5 +25,10 @@ int main(void) {
   printf("%lld\n", (long long)opr_loss_row_count(turn_lens, 3));
   printf("%d\n", (int)(opr_kpass_sizes(turn_lens, conv_turn_ptr, seq_conv_ptr, 1, 2, 3, 0, &n_out_turns,
                                         &n_out_convs, &total, &max_seqlen, &orig) == OPR_INVALID_ARG));
+  {
+    uint64_t off[4] = {0, 0, 0, 0};
+    const int st = opr_testing_layout_tables(1, 2, 3, total, max_seqlen, off);
+    printf("%d\n", (int)(st == OPR_OK && off[0] < off[1] && off[1] < off[2] && off[2] < off[3]));
+  }
   return 0;
 }

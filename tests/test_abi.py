@@ -50,6 +50,48 @@ def test_wait_limit_hook_round_trips(lib):
     assert lib.opr_testing_set_wait_limit_ns(prev) == 12345
 
 
+def test_layout_tables_hook(lib):
+    """Offsets of the tile tables inside the layout workspace: in order, non-overlapping, inside it."""
+    n_seqs, n_convs, n_turns, total, max_seqlen = 2, 5, 20, 30000, 16384
+    out = (ctypes.c_uint64 * 4)()
+    assert lib.opr_testing_layout_tables(n_seqs, n_convs, n_turns, total, max_seqlen,
+                                         ctypes.cast(out, ctypes.c_void_p)) == 0
+    T = (max_seqlen + 127) // 128
+    n_tiles = n_seqs * T
+    row_cnt, row_list, col_cnt, col_list = (int(x) for x in out)
+    assert row_list - row_cnt >= 4 * n_tiles and col_cnt - row_list >= 4 * n_tiles * T
+    assert col_list - col_cnt >= 4 * n_tiles
+    assert col_list + 4 * n_tiles * T <= opr.opr_layout_workspace_bytes(n_seqs, n_convs, n_turns, total, max_seqlen)
+    assert lib.opr_testing_layout_tables(-1, n_convs, n_turns, total, max_seqlen, ctypes.cast(out, ctypes.c_void_p)) == 1
+    assert lib.opr_testing_layout_tables(n_seqs, n_convs, n_turns, total, max_seqlen, None) == 1
+
+
+def test_debug_library_builds_and_exports_the_same_symbols(lib):
+    """The bounds-checking build (OPR_DEBUG_CHECKS) has every entry point and says so in its version."""
+    path = opr_build.build(debug=True)
+    assert path.endswith("libopr_debug.so")
+    dbg = ctypes.CDLL(path)
+    for name in declared_symbols():
+        assert hasattr(dbg, name), name
+    dbg.opr_version.restype = ctypes.c_char_p
+    assert dbg.opr_version().decode().endswith("debug-checks")
+    assert not opr.opr_version().endswith("debug-checks")
+
+
+def test_binding_loads_the_debug_library_on_request(lib):
+    """OPR_DEBUG_CHECKS=1 in the environment points the binding at libopr_debug.so."""
+    import subprocess
+    import sys
+    opr_build.build(debug=True)
+    root = os.path.dirname(INCLUDE)
+    code = "import block_sparse_masked_segment_b200 as o; o.load_library(); print(o.library_path()); print(o.opr_version())"
+    env = dict(os.environ, OPR_DEBUG_CHECKS="1")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    path, version = r.stdout.split("\n")[:2]
+    assert path.endswith("libopr_debug.so") and version.endswith("debug-checks")
+
+
 def test_workspace_queries(lib):
     b = opr.opr_layout_workspace_bytes(2, 5, 20, 30000, 16384)
     assert b > 4 * 30000 and b % 256 == 0

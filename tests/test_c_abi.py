@@ -33,6 +33,6 @@ def test_header_is_c99_and_host_calls_work():
     l2, c2, s2, _ = orc.kpass_plan(turns, [0, 2, 3], [0, 2], 2)
     lay = orc.build_layout(l2, c2, s2)
     rows, _ = orc.loss_rows(turns, [0, 2, 3])
-    vals = [int(x) for x in lines[-7:]]
+    vals = [int(x) for x in lines[-8:]]
     total = int(lay.cu_seqlens[-1])
-    assert vals == [len(l2), len(c2) - 1, total, total, 20, len(rows), 1]
+    assert vals == [len(l2), len(c2) - 1, total, total, 20, len(rows), 1, 1]
