@@ -42,8 +42,18 @@ METRIC = "1-pass masked attn fwd+bwd useful TFLOP/s; conv tokens/s vs N-pass"
 UNIT = "TFLOP/s"
 DEFAULT_CONFIG = 4
 L2_FLUSH_BYTES = 512 << 20
-# layout (8), rope x2, fwd, bwd (max |dO|, row terms, v cast, dq, dkdv), inverse rope x2
-KERNELS_PER_STEP = 8 + 2 + 1 + 5 + 2
+# layout (8), rope of q and k and the fp16 copy of v (3), fwd, bwd (max |dO|, row terms,
+# v cast, dq, dkdv), inverse rope x2
+KERNELS_PER_STEP = 8 + 3 + 1 + 5 + 2
+
+
+def kernels_per_step(w) -> int:
+    """Library kernels one step launches: one more (the GQA partial sum) when the dK/dV stage
+    splits its long columns by q head, which include/opr.h states for a grid below 4 x 148 CTAs
+    with GQA and the recommended workspace (which reserves the partials while tiles x Hq <= 4736)."""
+    tiles = w.n_seqs * ((w.max_seqlen + 127) // 128)
+    split = w.hq > w.hkv and tiles * w.hkv < 4 * 148 and tiles * w.hq <= 4 * 148 * 8
+    return KERNELS_PER_STEP + (1 if split else 0)
 ORACLE_SAMPLE_TOKENS = 3000  # one-pass tokens of the oracle's sample (cpu_baseline and the reference arm)
 
 # DRAM bytes (read + write) per launch of a kernel, from one ncu capture of
@@ -177,6 +187,7 @@ class Runner:
                           torch.empty((n, w.hkv, w.d), dtype=torch.float32, device=device))})
         self.q_rot = torch.empty(self.h_q.shape, dtype=torch.float16, device=device)
         self.k_rot = torch.empty(self.h_k.shape, dtype=torch.float16, device=device)
+        self.v16 = torch.empty(self.h_v.shape, dtype=torch.float16, device=device)
         self.h_grads = tuple(torch.empty(g.shape, dtype=g.dtype).pin_memory() for g in self.sets[0]["grads"])
         self.bwd_ws = torch.empty(max(opr.opr_attn_bwd_workspace_bytes(w.n_seqs, w.max_seqlen, w.hq, w.d), 256),
                                   dtype=torch.uint8, device=device)
@@ -201,8 +212,9 @@ class Runner:
         rec(1)
         opr.opr_rope(b["q"], lay.pos_id, self.w.base, out=self.q_rot, dev_status=lay.dev_status)
         opr.opr_rope(b["k"], lay.pos_id, self.w.base, out=self.k_rot, dev_status=lay.dev_status)
+        opr.opr_rope(b["v"], None, self.w.base, out=self.v16, dev_status=lay.dev_status)  # fp16 v: P V in fp16
         rec(2)
-        o, lse = opr.opr_attn_fwd(self.q_rot, self.k_rot, b["v"], lay, out_dtype=torch.bfloat16)
+        o, lse = opr.opr_attn_fwd(self.q_rot, self.k_rot, self.v16, lay, out_dtype=torch.bfloat16)
         rec(3)
         if self.forward_only:
             for i in (4, 5, 6, 7):
@@ -759,7 +771,7 @@ def main():
         "npass": npass,
         "next_rows": {"token_duplication": duplication, "kpass": kpass, "loss_side": loss_side},
         "other_workloads": extra,
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": kernels_per_step(w) * args.steps,
         "clocks": dict(clocks.summary(), remeasured=remeasured),
         "cpu_baseline": cpu,
     }

@@ -30,6 +30,7 @@ from ._abi import (  # noqa: F401
     BWD_DKDV,
     opr_layout_workspace_bytes,
     opr_attn_bwd_workspace_bytes,
+    opr_attn_bwd_min_workspace_bytes,
     opr_version,
     read_status,
     layout_table_offsets,

@@ -35,6 +35,7 @@ EXPORTED_SYMBOLS = (
     "opr_rope",
     "opr_attn_fwd",
     "opr_attn_bwd_workspace_bytes",
+    "opr_attn_bwd_min_workspace_bytes",
     "opr_attn_bwd",
     "opr_attn_bwd_stages",
     "opr_attn_bwd_noalloc",
@@ -112,9 +113,11 @@ def load_library() -> ctypes.CDLL:
     lib.opr_rope.restype = I32
     lib.opr_rope.argtypes = [P, I32, P, I32, P, I64, I32, I32, D, I32, P, P]
     lib.opr_attn_fwd.restype = I32
-    lib.opr_attn_fwd.argtypes = [P, P, P, I32, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F, P, I32, P, P, P]
+    lib.opr_attn_fwd.argtypes = [P, P, P, I32, I32, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F, P, I32, P, P, P]
     lib.opr_attn_bwd_workspace_bytes.restype = SZ
     lib.opr_attn_bwd_workspace_bytes.argtypes = [I32, I32, I32, I32]
+    lib.opr_attn_bwd_min_workspace_bytes.restype = SZ
+    lib.opr_attn_bwd_min_workspace_bytes.argtypes = [I32, I32, I32, I32]
     lib.opr_attn_bwd.restype = I32
     lib.opr_attn_bwd.argtypes = [P, P, P, I32, P, I32, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F,
                                  P, P, P, P, D, P, SZ, P, P]
@@ -164,6 +167,10 @@ def opr_layout_workspace_bytes(n_seqs, n_convs, n_turns, total_tokens, max_seqle
 
 def opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) -> int:
     return int(load_library().opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim))
+
+
+def opr_attn_bwd_min_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) -> int:
+    return int(load_library().opr_attn_bwd_min_workspace_bytes(n_seqs, max_seqlen, hq, head_dim))
 
 
 @dataclass
@@ -263,14 +270,15 @@ def opr_build_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, total_tokens=None, 
 _DT = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16, torch.float32: DTYPE_FP32}
 
 
-def opr_rope(x: torch.Tensor, pos_id: torch.Tensor, base: float, inverse: bool = False,
+def opr_rope(x: torch.Tensor, pos_id: torch.Tensor | None, base: float, inverse: bool = False,
              out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None) -> torch.Tensor:
     """Rotate x [total, heads, head_dim] by position id, into ``out`` (default: in place).
 
-    x and out may be bf16, fp16 or fp32 (types may differ when out is not x).
+    x and out may be bf16, fp16 or fp32 (types may differ when out is not x).  With
+    ``pos_id`` None there is no rotation, only the type conversion.
     """
     out = x if out is None else out
-    _need_cuda(x, pos_id, out)
+    _need_cuda(x, out, *(() if pos_id is None else (pos_id,)))
     if x.dtype not in _DT or out.dtype not in _DT:
         raise OprError("opr_rope takes bf16, fp16 or fp32")
     if out.shape != x.shape:
@@ -282,12 +290,12 @@ def opr_rope(x: torch.Tensor, pos_id: torch.Tensor, base: float, inverse: bool =
     return out
 
 
-def _attn_shapes(q, k, v, lay: Layout):
+def _attn_shapes(q, k, v, lay: Layout, v_types=(torch.bfloat16,)):
     _need_cuda(q, k, v)
     if q.dtype != torch.float16 or k.dtype != torch.float16:
         raise OprError("q and k must be fp16 (rotated by opr_rope with an fp16 output)")
-    if v.dtype != torch.bfloat16:
-        raise OprError("v must be bf16")
+    if v.dtype not in v_types:
+        raise OprError("v must be " + " or ".join(str(t).replace("torch.", "") for t in v_types))
     total, hq, d = q.shape
     if k.shape != v.shape or k.shape[0] != total or k.shape[2] != d or total != lay.total:
         raise OprError("shape mismatch between q, k, v and the layout")
@@ -310,14 +318,15 @@ def _grad_buffers(out, q, total, hq, hkv, d):
 
 
 def opr_attn_fwd(q, k, v, lay: Layout, scale: float | None = None, out_dtype=torch.float32):
-    """O [total, hq, d] (out_dtype) and LSE [hq, total] fp32."""
-    total, hq, hkv, d = _attn_shapes(q, k, v, lay)
+    """O [total, hq, d] (out_dtype) and LSE [hq, total] fp32.  v is fp16 (P V in fp16, see
+    include/opr.h) or bf16."""
+    total, hq, hkv, d = _attn_shapes(q, k, v, lay, v_types=(torch.float16, torch.bfloat16))
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty((total, hq, d), dtype=out_dtype, device=q.device)
     lse = torch.empty((hq, total), dtype=torch.float32, device=q.device)
     st = load_library().opr_attn_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace),
-        lay.n_seqs, lay.n_convs, lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale),
+        _ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _DT[v.dtype], _ptr(lay.cu_seqlens), _ptr(lay.conv_idx),
+        _ptr(lay.workspace), lay.n_seqs, lay.n_convs, lay.n_turns, total, lay.max_seqlen, hq, hkv, d, float(scale),
         _ptr(o), DTYPE_FP32 if out_dtype == torch.float32 else DTYPE_BF16, _ptr(lse), _ptr(lay.dev_status),
         _stream(q.device))
     _check(st, "opr_attn_fwd")
@@ -339,7 +348,9 @@ def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, w
 
     ``out`` = (dq, dk, dv) reuses buffers; ``stages`` (OR of BWD_ROW_TERMS,
     BWD_DQ, BWD_DKDV) runs only those kernels through opr_attn_bwd_stages, with
-    the row terms kept in ``workspace`` between calls.
+    the row terms kept in ``workspace`` between calls.  A ``workspace`` below
+    opr_attn_bwd_min_workspace_bytes is replaced by one of the recommended size;
+    one between the two sizes is used as given (the dK/dV stage then runs unsplit).
     """
     total, hq, hkv, d = _attn_shapes(q, k, v, lay)
     _need_cuda(o, do, lse)
@@ -348,7 +359,7 @@ def opr_attn_bwd(q, k, v, o, do, lse, lay: Layout, scale: float | None = None, w
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dq, dk, dv = _grad_buffers(out, q, total, hq, hkv, d)
     wb = opr_attn_bwd_workspace_bytes(lay.n_seqs, lay.max_seqlen, hq, d)
-    if workspace is None or workspace.numel() < wb:
+    if workspace is None or workspace.numel() < opr_attn_bwd_min_workspace_bytes(lay.n_seqs, lay.max_seqlen, hq, d):
         workspace = torch.empty(max(wb, 256), dtype=torch.uint8, device=q.device)
     args = (_ptr(q), _ptr(k), _ptr(v), _DT[q.dtype], _ptr(o), DTYPE_FP32 if o.dtype == torch.float32 else DTYPE_BF16, _ptr(do),
             _ptr(lse), _ptr(lay.cu_seqlens), _ptr(lay.conv_idx), _ptr(lay.workspace), lay.n_seqs, lay.n_convs,

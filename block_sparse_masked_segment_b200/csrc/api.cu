@@ -17,7 +17,7 @@
 #include "opr_internal.cuh"
 
 namespace opr {
-cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, bool v_f16, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_attn_bwd(int head_dim, bool qk_f16, const BwdMaps& m, const BwdBuffers& b, const AttnParams& pq,
                             const AttnParams& pkv, int stages, cudaStream_t stream);
@@ -392,14 +392,15 @@ opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, co
   auto known = [](int32_t t) { return t == OPR_DTYPE_BF16 || t == OPR_DTYPE_FP16 || t == OPR_DTYPE_FP32; };
   if (!known(x_dtype) || !known(y_dtype)) return OPR_UNSUPPORTED;
   if (!(base > 1.0)) return OPR_INVALID_ARG;
-  if (total_tokens > 0 && n_heads > 0 && (!x || !y || !pos_id)) return OPR_INVALID_ARG;
+  if (total_tokens > 0 && n_heads > 0 && (!x || !y)) return OPR_INVALID_ARG;
   if (x == y && x_dtype != y_dtype) return OPR_INVALID_ARG;
   cudaError_t e = launch_rope(x, x_dtype, y, y_dtype, pos_id, total_tokens, n_heads, head_dim, base, inverse,
                               dev_status, static_cast<cudaStream_t>(stream));
   return status_of(e);
 }
 
-opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_dtype, const int32_t* cu_seqlens,
+opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_dtype, int32_t v_dtype,
+                        const int32_t* cu_seqlens,
                         const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs, int32_t n_convs,
                         int32_t n_turns, int64_t total_tokens, int32_t max_seqlen, int32_t hq, int32_t hkv,
                         int32_t head_dim, float scale, void* o, int32_t o_dtype, float* lse, int32_t* dev_status,
@@ -411,39 +412,60 @@ opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_
   if (!cu_seqlens || !conv_idx || !layout_ws || !o || !lse || !dev_status || !aligned16(o)) return OPR_INVALID_ARG;
   if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
   if (qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
+  if (v_dtype != OPR_DTYPE_FP16 && v_dtype != OPR_DTYPE_BF16) return OPR_UNSUPPORTED;
   const bool f16 = qk_dtype == OPR_DTYPE_FP16;
+  const bool v16 = v_dtype == OPR_DTYPE_FP16;
   opr_status st = device_check();
   if (st != OPR_OK) return st;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, total_tokens, hq, head_dim, f16) || !make_map(&tk, k, total_tokens, hkv, head_dim, f16) ||
-      !make_map(&tv, v, total_tokens, hkv, head_dim))
+      !make_map(&tv, v, total_tokens, hkv, head_dim, v16))
     return map_fail();
   AttnParams p = base_params(cu_seqlens, conv_idx, layout_ws, n_seqs, n_convs, n_turns, total_tokens, max_seqlen, hq,
                              hkv, scale, dev_status);
   p.o = o;
   p.o_fp32 = o_dtype == OPR_DTYPE_FP32;
   p.lse = lse;
-  cudaError_t e = launch_attn_fwd(head_dim, f16, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_attn_fwd(head_dim, f16, v16, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
   return status_of(e);
 }
 
 namespace {
-// Backward scratch: the row terms, then fp16 copies of dO and V.  Token counts
-// are bounded by n_seqs * ceil(max_seqlen / 128) * 128 and the kv heads by hq.
+// The dK/dV stage runs one CTA per (key tile, kv head), each walking the whole
+// column for every q head of its GQA group.  When that grid is short of a few
+// waves of the 148 SMs, the longest columns set the stage's time; the stage is
+// then split by q head (one CTA per key tile and q head, per-head partials summed
+// afterwards), which needs room for the partials in the workspace.
+constexpr int64_t kSplitGridCtas = 4 * 148;         // split below this many (key tile, kv head) CTAs
+constexpr int64_t kSplitMaxHeadTiles = 4 * 148 * 8;  // partials reserved while tiles * hq stays at or below
+// A key column is split when its whole-group walk (query tiles x group) reaches
+// kSplitColumnRatio x T iterations; shorter columns stay whole (one CTA, no partials).
+constexpr double kSplitColumnRatio = 2.0;
+
+// Backward scratch: the row terms, then fp16 copies of dO and V (the minimum),
+// then, for small problems, the per-q-head dK and dV partials of the split dK/dV
+// stage.  Token counts are bounded by n_seqs * ceil(max_seqlen / 128) * 128 and
+// the kv heads by hq.
 struct BwdWs {
-  size_t absmax, row_terms, dout16, v16, bytes;
+  size_t absmax, row_terms, dout16, v16, min_bytes, dk_part, dv_part, bytes;
 };
 
 BwdWs bwd_ws_map(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
   const size_t T = (static_cast<size_t>(max_seqlen) + kTile - 1) / kTile;
-  const size_t tokens = static_cast<size_t>(n_seqs) * T * kTile;
+  const size_t tiles = static_cast<size_t>(n_seqs) * T;
+  const size_t tokens = tiles * kTile;
   BwdWs w;
   w.absmax = 0;
   w.row_terms = 256;
   w.dout16 = w.row_terms + align_up(2 * sizeof(float) * static_cast<size_t>(hq) * tokens, 256);
   const size_t copy = align_up(sizeof(uint16_t) * tokens * static_cast<size_t>(hq) * static_cast<size_t>(head_dim), 256);
   w.v16 = w.dout16 + copy;
-  w.bytes = w.v16 + copy;
+  w.min_bytes = w.v16 + copy;
+  const bool reserve = tiles * static_cast<size_t>(hq) <= static_cast<size_t>(kSplitMaxHeadTiles);
+  const size_t part = reserve ? 2 * copy : 0;  // fp32 [hq][tokens][head_dim]
+  w.dk_part = w.min_bytes;
+  w.dv_part = w.dk_part + part;
+  w.bytes = w.dv_part + part;
   return w;
 }
 }  // namespace
@@ -451,6 +473,11 @@ BwdWs bwd_ws_map(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_di
 size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
   if (n_seqs < 0 || max_seqlen < 0 || hq < 0 || head_dim < 0) return 0;
   return bwd_ws_map(n_seqs, max_seqlen, hq, head_dim).bytes;
+}
+
+size_t opr_attn_bwd_min_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq, int32_t head_dim) {
+  if (n_seqs < 0 || max_seqlen < 0 || hq < 0 || head_dim < 0) return 0;
+  return bwd_ws_map(n_seqs, max_seqlen, hq, head_dim).min_bytes;
 }
 
 opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int32_t qk_dtype, const void* o,
@@ -475,7 +502,7 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   if (qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;
   if (rope_pos_id != nullptr && !(rope_base > 1.0)) return OPR_INVALID_ARG;
   const bool f16 = qk_dtype == OPR_DTYPE_FP16;
-  if (workspace_bytes < opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim))
+  if (workspace_bytes < opr_attn_bwd_min_workspace_bytes(n_seqs, max_seqlen, hq, head_dim))
     return OPR_WORKSPACE_TOO_SMALL;
   opr_status st = device_check();
   if (st != OPR_OK) return st;
@@ -509,6 +536,16 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   pq.dv = dv;
   AttnParams pkv = pq;
   pkv.sched = ws_ptr<int32_t>(layout_ws, w.k_sched);
+  // dK/dV split by q head: GQA, a grid short of kSplitGridCtas, and room for the partials
+  pkv.dkdv_split = hq > hkv && static_cast<int64_t>(w.n_tiles) * hkv < kSplitGridCtas && bw.bytes > bw.min_bytes &&
+                   workspace_bytes >= bw.bytes;
+  if (pkv.dkdv_split) {
+    const int group = hq / hkv;
+    const double c = std::ceil(kSplitColumnRatio * w.T / group);
+    pkv.split_min_cnt = c < 1.0 ? 1 : static_cast<int32_t>(c);
+  }
+  pkv.dk_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + bw.dk_part);
+  pkv.dv_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + bw.dv_part);
   cudaError_t e = launch_attn_bwd(head_dim, f16, maps, buf, pq, pkv, stages, static_cast<cudaStream_t>(stream));
   return status_of(e);
 }

@@ -520,15 +520,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // kv-head-major grid over a schedule grouped by sequence: the CTAs that run
   // together stream the Q and dO tiles of one kv head group and sequence,
-  // which stay in L2
-  const int kvh = blockIdx.x / p.n_items;
+  // which stay in L2.  In split mode (p.dkdv_split) the grid's major index is the
+  // q head: a long column (split_col) is walked for that head only, a short one by
+  // the group's first head for the whole group, as in the unsplit grid.
+  const int group = p.hq / p.hkv;
+  const int major = blockIdx.x / p.n_items;
   const int tile_id = p.sched[blockIdx.x % p.n_items];
-  if (kvh >= p.hkv) return;
+  if (major >= (p.dkdv_split ? p.hq : p.hkv)) return;
+  const int kvh = p.dkdv_split ? major / group : major;
   if (!debug_tile_ok(p, tile_id, p.col_cnt, p.col_list)) return;
   const int cnt = p.col_cnt[tile_id];
   if (cnt == 0) return;
-  const int group = p.hq / p.hkv;
-  const int n = cnt * group;
+  const bool split_col = p.dkdv_split && cnt >= p.split_min_cnt;
+  if (p.dkdv_split && !split_col && major % group != 0) return;
+  const int n = split_col ? cnt : cnt * group;
+  // q head of iteration j (query tile entry(j % cnt))
+  auto head_of = [&](int j) { return split_col ? major : kvh * group + j / cnt; };
   const int s = tile_id / p.T, J = tile_id % p.T;
   const int32_t* list = p.col_list + static_cast<size_t>(tile_id) * p.T;
   const int seq0 = p.cu_seqlens[s];
@@ -567,8 +574,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // lane 0: K and V once, then the Q ring with each query tile's column data;
-    // lane 1: the dO ring.  Iteration j covers q head kvh * group + j / cnt and
-    // query tile entry(j % cnt).
+    // lane 1: the dO ring.  Iteration j covers q head head_of(j) and query tile
+    // entry(j % cnt).
     if (lane == 0) {
       const TileMeta* tmeta = p.tile_meta + static_cast<size_t>(s) * p.T;
       mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
@@ -579,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = j % kStages;
         const int e = entry(j % cnt);
         const int Iq = entry_index(e);
-        const int h = kvh * group + j / cnt;
+        const int h = head_of(j);
         if (j >= kStages && !mbar_wait(&sm.bar_qempty[st], ((j / kStages) + 1) & 1, abort_flag, p.wait_ns))
           break;
         const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
@@ -601,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
-        const int h = kvh * group + j / cnt;
+        const int h = head_of(j);
         if (j >= kStages && !mbar_wait(&sm.bar_doempty[st], ((j / kStages) + 1) & 1, abort_flag, p.wait_ns))
           break;
         mbar_arrive_expect_tx(&sm.bar_dofull[st], kTileBytes);
@@ -794,8 +801,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_accdone, 0, abort_flag, p.wait_ns))) {
       tc_fence_after();
-      float* dvp = p.dv + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
-      float* dkp = p.dk + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
+      float* dvp = split_col ? p.dv_part + (static_cast<size_t>(major) * p.total + kg) * D
+                             : p.dv + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
+      float* dkp = split_col ? p.dk_part + (static_cast<size_t>(major) * p.total + kg) * D
+                             : p.dk + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
       const float vsc = pow2f(-grad_scale_exp(*p.dout_absmax));  // undoes the gradient scale 2^k
       const float ksc = p.scale * vsc;
 #pragma unroll
@@ -835,6 +844,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
   if (threadIdx.x == 0 && sm.abort_flag) atomicOr(p.dev_status, OPR_DEV_WAIT_TIMEOUT);
+}
+
+// dK, dV [total][hkv][D] of the tokens of split key columns (at least min_cnt
+// query tiles) = the sum over the q heads of each GQA group of the per-head
+// partials [hq][total][D] the split dK/dV kernel wrote (head order kvh * group +
+// 0, 1, ...; one float4 of dK and of dV per thread and step).  The tokens of
+// shorter columns were written whole by the dK/dV kernel and are left alone.
+template <int D>
+__global__ void __launch_bounds__(256) gqa_sum_kernel(const float* __restrict__ dk_part,
+                                                      const float* __restrict__ dv_part, int64_t total, int32_t hq,
+                                                      int32_t hkv, const int32_t* __restrict__ cu_seqlens,
+                                                      int32_t n_seqs, int32_t T, const int32_t* __restrict__ col_cnt,
+                                                      int32_t min_cnt, float* __restrict__ dk, float* __restrict__ dv) {
+  const int group = hq / hkv;
+  const int64_t n4 = total * hkv * (D / 4);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int c4 = static_cast<int>(i % (D / 4));
+    const int64_t tk = i / (D / 4);  // token * hkv + kv head
+    const int kvh = static_cast<int>(tk % hkv);
+    const int64_t tok = tk / hkv;
+    int lo = 0, hi = n_seqs - 1;  // sequence of tok: the last s with cu_seqlens[s] <= tok
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cu_seqlens[mid] <= tok) lo = mid; else hi = mid - 1;
+    }
+    const int J = static_cast<int>((tok - cu_seqlens[lo]) / kTile);
+    if (J >= T || col_cnt[lo * T + J] < min_cnt) continue;
+    float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
+    for (int g = 0; g < group; ++g) {
+      const size_t src = ((static_cast<size_t>(kvh) * group + g) * total + tok) * (D / 4) + c4;
+      const float4 a = reinterpret_cast<const float4*>(dk_part)[src];
+      const float4 b = reinterpret_cast<const float4*>(dv_part)[src];
+      sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
+      sv.x += b.x; sv.y += b.y; sv.z += b.z; sv.w += b.w;
+    }
+    reinterpret_cast<float4*>(dk)[i] = sk;
+    reinterpret_cast<float4*>(dv)[i] = sv;
+  }
 }
 
 template <typename K>
@@ -897,11 +945,21 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
   if (stages & OPR_BWD_DKDV) {
     const size_t smem_kv = smem_request(sizeof(DkdvSmem<D>) + 1024);
     if ((e = set_smem(attn_bwd_dkdv_kernel<D, QK16>, smem_kv, conf_kv)) != cudaSuccess) return e;
-    const int64_t bkv = static_cast<int64_t>(pkv.n_items) * pkv.hkv;
+    const int64_t bkv = static_cast<int64_t>(pkv.n_items) * (pkv.dkdv_split ? pkv.hq : pkv.hkv);
     if (bkv > 0)
       attn_bwd_dkdv_kernel<D, QK16>
           <<<static_cast<unsigned>(bkv), kThreads, smem_kv, stream>>>(m.q, m.k, m.v16, m.dout16, pkv);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (pkv.dkdv_split) {  // sum each GQA group's per-head partials, in head order
+      const int64_t n4 = pkv.total * pkv.hkv * (D / 4);
+      if (n4 > 0) {
+        const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 148 * 16);
+        gqa_sum_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+            pkv.dk_part, pkv.dv_part, pkv.total, pkv.hq, pkv.hkv, pkv.cu_seqlens, pkv.n_items / pkv.T, pkv.T,
+            pkv.col_cnt, pkv.split_min_cnt, pkv.dk, pkv.dv);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      }
+    }
     if (b.rope_pos != nullptr)  // dk w.r.t. the unrotated k
       e = launch_rope(pkv.dk, OPR_DTYPE_FP32, pkv.dk, OPR_DTYPE_FP32, b.rope_pos, pkv.total, pkv.hkv, D, b.rope_base, 1,
                       pkv.dev_status, stream);

@@ -231,6 +231,15 @@ struct AttnParams {
   float* dq;
   float* dk;
   float* dv;
+  // dK/dV split by q head (small grids): the dK/dV grid has one CTA per (key tile,
+  // q head).  A key column of at least split_min_cnt query tiles is split: each CTA
+  // writes its head's dK and dV to dk_part / dv_part [hq][total][D], which a second
+  // kernel sums per GQA group into dk / dv.  A shorter column is done whole by the
+  // CTA of the group's first head, which writes dk / dv itself.
+  int32_t dkdv_split;
+  int32_t split_min_cnt;
+  float* dk_part;
+  float* dv_part;
   int32_t* dev_status;
   uint32_t wait_ns;  // limit of the pipeline waits (kWaitLimitNs; 0: a wait not already done times out)
 };

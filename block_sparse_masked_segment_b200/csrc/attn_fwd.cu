@@ -15,14 +15,15 @@
 //               key columns: read S from TMEM, apply the visibility mask on
 //               partial tiles only, online softmax in base 2 (the row max is
 //               taken over all 128 columns by both threads, so no exchange is
-//               needed), write their half of P (bf16) to TMEM, rescale
+//               needed), write their half of P (V's type) to TMEM, rescale
 //               their half of O in TMEM only when the running max grows by
 //               more than 2^8; epilogue O / l and the log-sum-exp.
 // TMEM columns: S buffer 0 at 0, buffer 1 at 128, O at 256, P buffers at 384
 // and 448 (512 allocated).
 // Q and K may be bf16 or fp16 (QK16: the rotated q, k stored in fp16, whose
-// 11-bit significand keeps the rounding of the rotation 8x smaller); V and P
-// are bf16.
+// 11-bit significand keeps the rounding of the rotation 8x smaller).  V and P
+// share one 16-bit type: fp16 (V16; P keeps 11 bits, so O, and the backward's
+// D = rowsum(dO * O), are about 8x closer to exact) or bf16.
 #include "attn_common.cuh"
 
 namespace opr {
@@ -49,7 +50,7 @@ struct FwdSmem {
   int abort_flag;
 };
 
-template <int D, bool QK16>
+template <int D, bool QK16, bool V16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the whole warp runs this loop; elect.sync picks the issuing lane
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);      // O += P V, P and V bf16
+    constexpr uint32_t idesc_o = idesc_f32acc(128, D, V16, 0, 1);  // O += P V, P and V fp16 (V16) or bf16
     const uint32_t sq = smem_u32(sm.q);
     bool ok = warp_wait(&sm.bar_q, 0, abort_flag, p.wait_ns);
     auto issue_pv = [&](int jp) -> bool {
@@ -258,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float p0 = fast_exp2(fmaf(sv[c * 32 + 2 * x], sl2, -mb));
           const float p1 = fast_exp2(fmaf(sv[c * 32 + 2 * x + 1], sl2, -mb));
           rs8[x & 7] += p0 + p1;
-          pk[x] = pack_bf16x2(p0, p1);
+          pk[x] = pack_x2<V16>(p0, p1);
         }
         tmem_st16(tl + kPCol + b * 64 + half * 32 + c * 16, pk);
       }
@@ -363,12 +364,13 @@ __device__ __forceinline__ float row_max(const float (&sv)[NC]) {
 }
 
 // P = 2^(S scale log2(e) - mb) of NC scores (the scale-and-shift on fp32 pairs),
-// stored as bf16 two per TMEM column from p_addr; returns the sum of P.  One pair
+// stored two per TMEM column from p_addr, in the type of V (fp16 when V16, else
+// bf16); returns the sum of the unrounded P.  One pair
 // in kFmaExpEvery takes the FMA-pipe exponential, the others the special-function
 // unit, so that the two pipes share the softmax's exponentials.
 constexpr int kFmaExpEvery = 3;
 
-template <int NC>
+template <int NC, bool V16>
 __device__ __forceinline__ float exp_pack_row(const float (&sv)[NC], float sl2, float mb, uint32_t p_addr) {
   const uint64_t sl2x2 = f2(sl2, sl2), nmb2 = f2(-mb, -mb);
   float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -388,7 +390,7 @@ __device__ __forceinline__ float exp_pack_row(const float (&sv)[NC], float sl2, 
         p1 = fast_exp2(a1);
       }
       rs8[x & 7] += p0 + p1;
-      pk[x] = pack_bf16x2(p0, p1);
+      pk[x] = pack_x2<V16>(p0, p1);
     }
     tmem_st16(p_addr + c * 16, pk);
   }
@@ -421,7 +423,7 @@ __device__ __forceinline__ MaxStep max_step(float m_run, float mx, float sl2) {
 //               partial tiles); lane 1: the V ring
 //   warp 1      TMEM owner, MMA issuer: S_A(0) S_B(0) | P_A V, S_A(j+1),
 //               P_B V, S_B(j+1) | ...
-//   warps 2..5  head A, warps 6..9 head B: one query row per thread, P (bf16)
+//   warps 2..5  head A, warps 6..9 head B: one query row per thread, P (V's type)
 //               written over the first 64 columns of the thread's own row of S
 // TMEM columns: S_A 0, S_B 128, O_A 256, O_B 384.
 // Full 128x128 products on every non-empty tile: the kernel is bound by its
@@ -441,7 +443,7 @@ struct FwdPairSmem {
   int abort_flag;
 };
 
-template <int D, bool QK16>
+template <int D, bool QK16, bool V16>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -535,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // the whole warp runs this loop; elect.sync picks the issuing lane
     constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);  // S = Q K^T in the q/k type
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);        // O += P V, P and V bf16
+    constexpr uint32_t idesc_o = idesc_f32acc(128, D, V16, 0, 1);    // O += P V, P and V fp16 (V16) or bf16
     const uint32_t sq[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
     auto issue_s = [&](int h, int j) {
       const uint32_t sk = smem_u32(sm.k[j % NS]);
@@ -632,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mask_bit(mm, c)) sv[c] = -INFINITY;
       }
       const MaxStep ms = max_step(m_run, row_max<kTile>(sv), sl2);
-      const float rs = exp_pack_row<kTile>(sv, sl2, ms.mb, tl + scol);  // P over S's read columns
+      const float rs = exp_pack_row<kTile, V16>(sv, sl2, ms.mb, tl + scol);  // P over S's read columns
       tmem_wait_st();
       if (j >= 1) {
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (j - 1) & 1, abort_flag, p.wait_ns))) {
@@ -700,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int D, bool QK16>
+template <int D, bool QK16, bool V16>
 cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const AttnParams& p, cudaStream_t stream) {
   static int configured[64] = {0};
@@ -710,10 +712,10 @@ cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, cons
   const size_t smem_single = smem_request(sizeof(FwdSmem<D>) + 1024);
   const size_t smem_pair = smem_request(sizeof(FwdPairSmem<D>) + 1024);
   if (dev < 64 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, QK16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, QK16, V16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem_single));
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_fwd_pair_kernel<D, QK16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      e = cudaFuncSetAttribute(attn_fwd_pair_kernel<D, QK16, V16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_pair));
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
@@ -722,20 +724,23 @@ cudaError_t launch_attn_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, cons
     // two q heads of one GQA group per CTA
     const int64_t blocks = static_cast<int64_t>(p.n_items) * (p.hq / 2);
     if (blocks == 0) return cudaSuccess;
-    attn_fwd_pair_kernel<D, QK16><<<static_cast<unsigned>(blocks), kThreads, smem_pair, stream>>>(tq, tk, tv, p);
+    attn_fwd_pair_kernel<D, QK16, V16><<<static_cast<unsigned>(blocks), kThreads, smem_pair, stream>>>(tq, tk, tv, p);
   } else {
     const int64_t blocks = static_cast<int64_t>(p.n_items) * p.hq;
     if (blocks == 0) return cudaSuccess;
-    attn_fwd_kernel<D, QK16><<<static_cast<unsigned>(blocks), kThreads, smem_single, stream>>>(tq, tk, tv, p);
+    attn_fwd_kernel<D, QK16, V16><<<static_cast<unsigned>(blocks), kThreads, smem_single, stream>>>(tq, tk, tv, p);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, const CUtensorMap& tq, const CUtensorMap& tk,
+cudaError_t launch_attn_fwd(int head_dim, bool qk_f16, bool v_f16, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tv, const AttnParams& p, cudaStream_t stream) {
   if (!qk_f16) return cudaErrorNotSupported;  // the entry points accept fp16 q and k only
-  if (head_dim == 128) return launch_attn_fwd_t<128, true>(tq, tk, tv, p, stream);
-  return launch_attn_fwd_t<64, true>(tq, tk, tv, p, stream);
+  if (head_dim == 128)
+    return v_f16 ? launch_attn_fwd_t<128, true, true>(tq, tk, tv, p, stream)
+                 : launch_attn_fwd_t<128, true, false>(tq, tk, tv, p, stream);
+  return v_f16 ? launch_attn_fwd_t<64, true, true>(tq, tk, tv, p, stream)
+               : launch_attn_fwd_t<64, true, false>(tq, tk, tv, p, stream);
 }
 
 }  // namespace opr

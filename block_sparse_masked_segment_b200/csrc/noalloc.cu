@@ -20,8 +20,9 @@ namespace opr {
 namespace {
 
 // Largest backward scratch this entry point serves (OPR_NOALLOC_SCRATCH_BYTES):
-// a call is accepted when opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq,
-// head_dim) -- max |dO|, the row terms and both fp16 copies -- fits.
+// a call is accepted when opr_attn_bwd_min_workspace_bytes(n_seqs, max_seqlen,
+// hq, head_dim) -- max |dO|, the row terms and both fp16 copies -- fits.  The
+// dK/dV stage is split by q head only when its partials fit as well.
 constexpr size_t kNoAllocScratchBytes = OPR_NOALLOC_SCRATCH_BYTES;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -61,7 +62,7 @@ opr_status opr_attn_bwd_noalloc(const void* q, const void* k, const void* v, int
                                 int32_t head_dim, float scale, float* dq, float* dk, float* dv,
                                 const int32_t* rope_pos_id, double rope_base, int32_t* dev_status, void* stream) {
   if (!opr::sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen) || hq < 0) return OPR_INVALID_ARG;
-  if (opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) > opr::kNoAllocScratchBytes)
+  if (opr_attn_bwd_min_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) > opr::kNoAllocScratchBytes)
     return OPR_SCRATCH_TOO_LARGE;
   void* scratch = nullptr;
   const opr_status st = opr::scratch_on_current_device(&scratch);

@@ -16,6 +16,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <type_traits>
 
@@ -159,9 +160,31 @@ __global__ void __launch_bounds__(256) rope_vec_kernel(const TI* x, TO* y, const
   if (out_of_range && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
+// No position ids: the rotation by angle 0, i.e. a plain type conversion, one
+// element per thread and step (e.g. the fp16 copy of v that lets the forward's
+// P V product take P in fp16).
+template <typename TI, typename TO>
+__global__ void __launch_bounds__(256) convert_kernel(const TI* x, TO* y, int64_t n, int32_t* __restrict__ dev_status) {
+  bool out_of_range = false;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = to_f<TI>(x[i]);
+    if constexpr (std::is_same<TO, __half>::value) out_of_range |= !(fabsf(v) <= 65504.f);
+    y[i] = from_f<TO>(v);
+  }
+  if (out_of_range && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
+}
+
 template <typename TI, typename TO>
 cudaError_t launch_t(const void* x, void* y, const int32_t* pos_id, int64_t total, int32_t n_heads, int32_t half,
                      double nl, double sign, int32_t* dev_status, cudaStream_t stream) {
+  if (pos_id == nullptr) {
+    const int64_t n = total * n_heads * 2 * half;
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
+    convert_kernel<TI, TO><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const TI*>(x),
+                                                                              static_cast<TO*>(y), n, dev_status);
+    return cudaGetLastError();
+  }
   const bool vec = half % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0 &&
                    (reinterpret_cast<uintptr_t>(y) & 15u) == 0;
   if (vec) {

@@ -47,12 +47,15 @@ def useful_flops(pairs: int, hq: int, d: int, backward: bool) -> float:
 
 
 def one_pass_forward(q_pre, k_pre, v, lay: Layout, base: float, scale=None, out_dtype=torch.float32):
-    """RoPE (bf16 in, fp16 out) then masked attention.  Returns (o, lse, q_rot, k_rot)."""
+    """RoPE (bf16 in, fp16 out), an fp16 copy of v (so that P V runs with fp16 P), then
+    masked attention.  Returns (o, lse, q_rot, k_rot)."""
     q = torch.empty(q_pre.shape, dtype=torch.float16, device=q_pre.device)
     k = torch.empty(k_pre.shape, dtype=torch.float16, device=k_pre.device)
+    v16 = torch.empty(v.shape, dtype=torch.float16, device=v.device)
     opr_rope(q_pre, lay.pos_id, base, out=q, dev_status=lay.dev_status)
     opr_rope(k_pre, lay.pos_id, base, out=k, dev_status=lay.dev_status)
-    o, lse = opr_attn_fwd(q, k, v, lay, scale, out_dtype)
+    opr_rope(v, None, base, out=v16, dev_status=lay.dev_status)
+    o, lse = opr_attn_fwd(q, k, v16, lay, scale, out_dtype)
     return o, lse, q, k
 
 

@@ -139,9 +139,11 @@ OPR_API opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* con
  *   x, y     [total_tokens, n_heads, head_dim]; x_dtype, y_dtype each one of
  *            OPR_DTYPE_BF16 / OPR_DTYPE_FP16 / OPR_DTYPE_FP32.  y may equal x
  *            (in place) only when the two types are the same.
- *   pos_id   int32 [total_tokens]
+ *   pos_id   int32 [total_tokens]; NULL: no rotation, only the type conversion
+ *            (e.g. the fp16 copy of v that opr_attn_fwd takes for an fp16 P V
+ *            product)
  *   dev_status  may be NULL; otherwise OPR_DEV_FP16_RANGE is OR-ed in when an
- *            fp16 output overflows.
+ *            fp16 output overflows (an inf or NaN input included).
  * head_dim must be even and <= 256.  The attention calls take the rotated q
  * and k in fp16 (bf16 in, fp16 out here): same MMA rate as bf16, 8x smaller
  * rounding of the rotation.
@@ -167,7 +169,11 @@ OPR_API opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_d
  *   k            fp16 [total, hkv, head_dim]  (already rotated)
  *   qk_dtype     OPR_DTYPE_FP16 (the type of the S = Q K^T MMA); any other
  *                value returns OPR_UNSUPPORTED
- *   v            bf16 [total, hkv, head_dim]
+ *   v            [total, hkv, head_dim], v_dtype OPR_DTYPE_FP16 or OPR_DTYPE_BF16:
+ *                the type of the O += P V MMA, whose P is rounded to the same
+ *                type.  fp16 (v copied by opr_rope with no position ids) keeps
+ *                P to 11 bits: O, and D = rowsum(dO * O) in the backward, are
+ *                then about 8x closer to exact than with bf16 P.
  *   cu_seqlens, conv_idx, layout_ws: outputs of opr_build_layout for the same sizes
  *   o            [total, hq, head_dim], o_dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32
  *   lse          fp32 [hq, total]: natural-log sum of exp(scale * q.k) over visible keys
@@ -178,7 +184,7 @@ OPR_API opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_d
  * (text from opr_last_error); OPR_DEV_WAIT_TIMEOUT in *dev_status.
  */
 OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int32_t qk_dtype,
-                        const int32_t* cu_seqlens,
+                        int32_t v_dtype, const int32_t* cu_seqlens,
                         const int32_t* conv_idx, const void* layout_ws, int32_t n_seqs,
                         int32_t n_convs, int32_t n_turns, int64_t total_tokens,
                         int32_t max_seqlen, int32_t hq, int32_t hkv, int32_t head_dim,
@@ -186,17 +192,31 @@ OPR_API opr_status opr_attn_fwd(const void* q, const void* k, const void* v, int
                         void* stream);
 
 /*
- * Bytes of device scratch that opr_attn_bwd needs.  With
- * N = n_seqs * ceil(max_seqlen / 128) * 128 (a bound on the token count):
- *   256 bytes for max |dO| (which sets the gradient scale below);
- *   the row terms D = rowsum(dO * O) and LSE * log2(e), stored per 128-token
- *   tile: 2 * 4 * hq * N bytes;
- *   an fp16 copy of dO: 2 * N * hq * head_dim bytes;
- *   an fp16 copy of v (kv heads bounded by hq): 2 * N * hq * head_dim bytes;
- * each part rounded up to 256 bytes.  Returns 0 for negative arguments.
+ * Bytes of device scratch for opr_attn_bwd.  With N = n_seqs * ceil(max_seqlen
+ * / 128) * 128 (a bound on the token count) and n_tiles = N / 128:
+ *   opr_attn_bwd_min_workspace_bytes, the least a call accepts:
+ *     256 bytes for max |dO| (which sets the gradient scale below);
+ *     the row terms D = rowsum(dO * O) and LSE * log2(e), stored per 128-token
+ *     tile: 2 * 4 * hq * N bytes;
+ *     an fp16 copy of dO: 2 * N * hq * head_dim bytes;
+ *     an fp16 copy of v (kv heads bounded by hq): 2 * N * hq * head_dim bytes;
+ *   opr_attn_bwd_workspace_bytes, the recommended size: the minimum, plus, when
+ *     n_tiles * hq <= 4736, room for per-q-head fp32 dK and dV partials
+ *     (2 * 4 * N * hq * head_dim bytes).  With it, a call whose dK/dV grid
+ *     (n_tiles * hkv CTAs) is below 4 * 148 and that has more q heads than kv
+ *     heads splits the long key columns of the dK/dV stage by q head: a column
+ *     seen by at least 2 * T / (hq / hkv) query tiles (T = max_seqlen / 128,
+ *     rounded up) gets one CTA per q head, and a pass sums each group's partials
+ *     in head order; shorter columns keep one CTA for the group.  Short grids
+ *     (short or few sequences) are otherwise bound by their longest key column.
+ *     The two forms differ in the order of the group sum, within fp32 rounding;
+ *     each is deterministic.
+ * each part rounded up to 256 bytes.  Both return 0 for negative arguments.
  */
 OPR_API size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq,
                                             int32_t head_dim);
+OPR_API size_t opr_attn_bwd_min_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, int32_t hq,
+                                                int32_t head_dim);
 
 /*
  * opr_attn_bwd - gradients of opr_attn_fwd w.r.t. q, k (rotated, or unrotated
@@ -220,7 +240,8 @@ OPR_API size_t opr_attn_bwd_workspace_bytes(int32_t n_seqs, int32_t max_seqlen, 
  *                     (one pass over each, right after the kernel that writes it),
  *                     giving the gradients w.r.t. the unrotated q and k, exactly
  *                     as opr_rope(inverse) on the first form
- *   workspace         opr_attn_bwd_workspace_bytes(...) bytes of device scratch,
+ *   workspace         at least opr_attn_bwd_min_workspace_bytes(...) bytes of device
+ *                     scratch (opr_attn_bwd_workspace_bytes(...) recommended),
  *                     16-byte aligned, owned by the caller; the call overwrites it
  * Precision: the tensor-core products take 16-bit operands.  The backward is
  * linear in dO, so it runs on 2^k dO, with k chosen on the device from max |dO|
@@ -248,8 +269,10 @@ OPR_API opr_status opr_attn_bwd(const void* q, const void* k, const void* v, int
  *                      and v into `workspace` (needed by the other two)
  *   OPR_BWD_DQ         dq   (one CTA per query tile and q head; then, with
  *                      rope_pos_id, the rotation of dq back)
- *   OPR_BWD_DKDV       dk, dv (one CTA per key tile and kv head; GQA group summed
- *                      in the CTA; then, with rope_pos_id, the rotation of dk back)
+ *   OPR_BWD_DKDV       dk, dv (one CTA per key tile and kv head, GQA group summed
+ *                      in the CTA; or, split as opr_attn_bwd_workspace_bytes says,
+ *                      one CTA per key tile and q head and a group-sum pass; then,
+ *                      with rope_pos_id, the rotation of dk back)
  * Running all three, in this order on one stream, equals opr_attn_bwd.
  * Other arguments and error behaviour as for opr_attn_bwd; unknown bits give
  * OPR_INVALID_ARG.
@@ -281,8 +304,9 @@ OPR_API opr_status opr_attn_bwd_stages(const void* q, const void* k, const void*
  * CUDA loader on every GPU that loads the library and held until the process
  * exits.  The call allocates and frees nothing.
  *   - Returns OPR_SCRATCH_TOO_LARGE, before touching the device, when
- *     opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) exceeds
- *     OPR_NOALLOC_SCRATCH_BYTES.
+ *     opr_attn_bwd_min_workspace_bytes(n_seqs, max_seqlen, hq, head_dim) exceeds
+ *     OPR_NOALLOC_SCRATCH_BYTES.  The dK/dV stage is split by q head (as in
+ *     opr_attn_bwd) only when opr_attn_bwd_workspace_bytes(...) fits too.
  *   - The array is the current device's: `stream` and every pointer must
  *     belong to the device that is current on the calling thread.
  *   - The first call on each device looks up the array's device address

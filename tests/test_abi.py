@@ -115,14 +115,17 @@ def test_host_argument_checks(lib):
     assert lib.opr_rope(N, 0, N, 0, N, 10, 2, 64, 1e4, 0, N, N) == 1
     assert lib.opr_rope(fake, 0, fake, 2, fake, 10, 2, 64, 1e4, 0, N, N) == 1
     # opr_attn_fwd: null q; hq % hkv != 0; head_dim 96
-    assert lib.opr_attn_fwd(N, fake, fake, 2, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
+    assert lib.opr_attn_fwd(N, fake, fake, 2, 0, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
                             fake, 0, fake, fake, N) == 1
-    assert lib.opr_attn_fwd(fake, fake, fake, 2, fake, fake, fake, 1, 1, 1, 100, 100, 6, 4, 128, 0.1,
+    assert lib.opr_attn_fwd(fake, fake, fake, 2, 0, fake, fake, fake, 1, 1, 1, 100, 100, 6, 4, 128, 0.1,
                             fake, 0, fake, fake, N) == 1
-    assert lib.opr_attn_fwd(fake, fake, fake, 2, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 96, 0.1,
+    assert lib.opr_attn_fwd(fake, fake, fake, 2, 0, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 96, 0.1,
                             fake, 0, fake, fake, N) == 1
+    # v of fp32 is not an MMA type (fp16 or bf16 only)
+    assert lib.opr_attn_fwd(fake, fake, fake, 2, 1, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
+                            fake, 0, fake, fake, N) == 2
     # q/k of fp32 are not an MMA type
-    assert lib.opr_attn_fwd(fake, fake, fake, 1, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
+    assert lib.opr_attn_fwd(fake, fake, fake, 1, 0, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
                             fake, 0, fake, fake, N) == 2
     # opr_attn_bwd_stages: unknown stage bits
     assert lib.opr_attn_bwd_stages(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
@@ -131,13 +134,13 @@ def test_host_argument_checks(lib):
     assert lib.opr_attn_bwd(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
                             4, 2, 128, 0.1, fake, fake, fake, fake, 0.5, fake, 1 << 30, fake, N) == 1
     # q/k in bf16 are refused: the attention calls take the rotated q and k in fp16 only
-    assert lib.opr_attn_fwd(fake, fake, fake, 0, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
+    assert lib.opr_attn_fwd(fake, fake, fake, 0, 0, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
                             fake, 0, fake, fake, N) == 2
     assert lib.opr_attn_bwd(fake, fake, fake, 0, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 100, 100,
                             4, 2, 128, 0.1, fake, fake, fake, N, 0.0, fake, 1 << 30, fake, N) == 2
     # more tokens than n_seqs * ceil(max_seqlen / 128) * 128 (the bound every workspace is sized
     # by): refused on the host, by every call that sizes buffers from (n_seqs, max_seqlen)
-    assert lib.opr_attn_fwd(fake, fake, fake, 2, fake, fake, fake, 1, 1, 1, 300, 100, 4, 2, 128, 0.1,
+    assert lib.opr_attn_fwd(fake, fake, fake, 2, 0, fake, fake, fake, 1, 1, 1, 300, 100, 4, 2, 128, 0.1,
                             fake, 0, fake, fake, N) == 1
     assert lib.opr_attn_bwd(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 300, 100,
                             4, 2, 128, 0.1, fake, fake, fake, N, 0.0, fake, 1 << 30, fake, N) == 1
@@ -147,7 +150,7 @@ def test_host_argument_checks(lib):
                                 1 << 30, fake, N) == 1
     assert opr.opr_layout_workspace_bytes(1, 1, 1, 300, 100) == 0
     # empty problems are no-ops
-    assert lib.opr_attn_fwd(N, N, N, 2, N, N, N, 0, 0, 0, 0, 0, 4, 2, 128, 0.1, N, 0, N, N, N) == 0
+    assert lib.opr_attn_fwd(N, N, N, 2, 0, N, N, N, 0, 0, 0, 0, 0, 4, 2, 128, 0.1, N, 0, N, N, N) == 0
 
 
 def test_closed_form_pair_count_matches_oracle():

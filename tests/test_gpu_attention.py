@@ -110,6 +110,27 @@ def test_fwd_bwd_segment_edges():
     _dense_check(w, 3)
 
 
+def test_forward_p_v_in_fp16_and_bf16():
+    """The forward's O += P V takes P in v's type.  With v in fp16 (the pipeline's choice) P keeps
+    11 bits; with v in bf16, 8.  Both meet the standard on O and LSE; the fp16 form's O error is
+    several times smaller (the bf16 rounding of P dominates the bf16 form's)."""
+    w = synth.random_small_workload(8, n_seqs=2, max_convs=2, max_turns=4, hq=8, hkv=2, d=128, base=1e4)
+    q, k, v, _ = inputs(w, 4200, with_do=False)
+    lo = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    o_ref, lse_ref = orc.forward(q, k, v, lo, w.base)
+    att = opr.OnePassAttention(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, base=w.base)
+    o16, lse16, qr, kr = att.forward(to_dev(q), to_dev(k), to_dev(v))  # fp16 copy of v inside
+    o_bf, lse_bf = opr.opr_attn_fwd(qr, kr, to_dev(v), att.layout)     # bf16 v as given
+    torch.cuda.synchronize()
+    assert opr.read_status(att.layout.dev_status) == []
+    e16, _ = assert_close("O (fp16 P)", o16.cpu().numpy(), o_ref)
+    ebf, _ = assert_close("O (bf16 P)", o_bf.cpu().numpy(), o_ref)
+    assert_close("LSE (fp16 P)", lse16.cpu().numpy(), lse_ref)
+    assert_close("LSE (bf16 P)", lse_bf.cpu().numpy(), lse_ref)
+    np.testing.assert_array_equal(lse16.cpu().numpy(), lse_bf.cpu().numpy())  # P's type does not enter LSE
+    assert e16 < ebf / 3, (e16, ebf)
+
+
 def test_fwd_bf16_output_is_rounded_fp32():
     w = synth.random_small_workload(11, hq=2, hkv=1, d=128)
     q, k, v, _ = inputs(w, 11, with_do=False)
@@ -269,6 +290,63 @@ def test_backward_with_positions_equals_rotation_afterwards(d):
     assert opr.read_status(lay.dev_status) == []
     for name, a, b in (("dQ", dq0, dq1), ("dK", dk0, dk1), ("dV", dv0, dv1)):
         np.testing.assert_array_equal(b.cpu().numpy(), a.cpu().numpy(), err_msg=name)
+
+
+@pytest.mark.parametrize("case", ["ragged_8q2kv", "gqa_8q1kv", "depth4_32q8kv"])
+def test_dkdv_split_by_q_head_and_unsplit_agree(case):
+    """Short dK/dV grids (few key tiles x kv heads) split their long key columns by q head:
+    per-head partials in the workspace, then a group sum.  A workspace of the minimum size keeps
+    the stage unsplit.  Both
+    forms match the oracle; they differ from each other only by the order of the fp32 group sum
+    (a few 1e-6 of the largest gradient, far inside the oracle tolerance; dQ, which the split
+    does not touch, is bit-identical)."""
+    if case == "ragged_8q2kv":
+        w = synth.random_small_workload(5, n_seqs=2, max_convs=2, max_turns=4, hq=8, hkv=2, d=128, base=1e4)
+    elif case == "gqa_8q1kv":
+        w = synth.random_small_workload(6, n_seqs=1, max_convs=2, max_turns=3, hq=8, hkv=1, d=128, base=1e4)
+    else:
+        w = synth.make_workload(3, n_turns=4)
+    q, k, v, do = inputs(w, 4100)
+    att = opr.OnePassAttention(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, base=w.base)
+    qd, kd, vd, dod = to_dev(q), to_dev(k), to_dev(v), to_dev(do)
+    o, lse, qr, kr = att.forward(qd, kd, vd)
+    lay = att.layout
+    assert w.hq > w.hkv and lay.n_seqs * lay.T * w.hkv < 4 * 148  # a grid the split applies to
+    full = opr.opr_attn_bwd_workspace_bytes(lay.n_seqs, lay.max_seqlen, w.hq, w.d)
+    least = opr.opr_attn_bwd_min_workspace_bytes(lay.n_seqs, lay.max_seqlen, w.hq, w.d)
+    assert full > least
+    ws_full = torch.full((full,), 0xFF, dtype=torch.uint8, device="cuda")
+    split = opr.opr_attn_bwd(qr, kr, vd, o, dod, lse, lay, workspace=ws_full, rope_base=w.base)
+    unsplit = opr.opr_attn_bwd(qr, kr, vd, o, dod, lse, lay, rope_base=w.base,
+                               workspace=torch.empty(least, dtype=torch.uint8, device="cuda"))
+    torch.cuda.synchronize()
+    assert opr.read_status(lay.dev_status) == []
+    # the split form ran on the long columns (seen by >= 2T / group query tiles, include/opr.h):
+    # it wrote per-head partials past the minimum workspace
+    lo = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    col_cnt = (orc.block_map(lo) > 0).sum(axis=1)  # [n_seqs, key tile]
+    min_cnt = -(-2 * lay.T // (w.hq // w.hkv))
+    assert int(col_cnt.max()) >= min_cnt
+    assert bool((ws_full[least:] != 0xFF).any())
+    split = [t.cpu().numpy() for t in split]
+    unsplit = [t.cpu().numpy() for t in unsplit]
+    np.testing.assert_array_equal(split[0], unsplit[0], err_msg="dQ")
+    for name, a, b in zip(("dK", "dV"), split[1:], unsplit[1:]):
+        np.testing.assert_allclose(a, b, rtol=1e-4, atol=2e-5 * float(np.abs(b).max()), err_msg=name)
+    if case == "depth4_32q8kv":  # one GQA group densely (the whole problem is too large for the oracle)
+        grp = w.hq // w.hkv
+        g = 5
+        hs = slice(g * grp, (g + 1) * grp)
+        qg, kg, vg, dog = q[:, hs], k[:, g:g + 1], v[:, g:g + 1], do[:, hs]
+        oo, ll = orc.forward(qg, kg, vg, lo, w.base)
+        ref = orc.backward(qg, kg, vg, oo, dog, ll, lo, w.base)
+        got = [split[0][:, hs], split[1][:, g:g + 1], split[2][:, g:g + 1]]
+    else:
+        oo, ll = orc.forward(q, k, v, lo, w.base)
+        ref = orc.backward(q, k, v, oo, do, ll, lo, w.base)
+        got = split
+    for name, g_, r in zip(("dQ", "dK", "dV"), got, ref):
+        assert_close(name, g_, r)
 
 
 def test_deterministic_backward():

@@ -156,3 +156,22 @@ def test_rope_fp16_overflow_is_flagged():
     opr.opr_rope(x, lay.pos_id, 1e4, out=y, dev_status=lay.dev_status)
     torch.cuda.synchronize()
     assert _abi.DEV_BITS[16] in opr.read_status(lay.dev_status)
+
+
+@pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
+def test_rope_without_positions_is_a_type_conversion(in_dtype):
+    """pos_id NULL: no rotation, the value rounded once to the output type (the fp16 copy of v
+    that the forward's P V product takes): bit for bit torch's round-to-nearest conversion;
+    a value beyond the fp16 range is flagged."""
+    rng = np.random.default_rng(7)
+    x = torch.from_numpy(rng.standard_normal((1000, 3, 64)).astype(np.float32) * 100).to("cuda", in_dtype)
+    y = torch.empty(x.shape, dtype=torch.float16, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    opr.opr_rope(x, None, 1e4, out=y, dev_status=st)
+    torch.cuda.synchronize()
+    assert opr.read_status(st) == []
+    assert torch.equal(y.view(torch.int16), x.to(torch.float16).view(torch.int16))
+    x[17, 1, 5] = 1e5
+    opr.opr_rope(x, None, 1e4, out=y, dev_status=st)
+    torch.cuda.synchronize()
+    assert _abi.DEV_BITS[16] in opr.read_status(st)

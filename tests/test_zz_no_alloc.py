@@ -42,7 +42,7 @@ def test_noalloc_rejects_scratch_beyond_the_limit():
     """Sizes whose scratch exceeds the fixed array are refused before any device work."""
     lib = opr.load_library()
     n_seqs, max_seqlen, hq, d = 1, 100000, 64, 128
-    assert opr.opr_attn_bwd_workspace_bytes(n_seqs, max_seqlen, hq, d) > _abi.NOALLOC_SCRATCH_BYTES
+    assert opr.opr_attn_bwd_min_workspace_bytes(n_seqs, max_seqlen, hq, d) > _abi.NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check fails first
     st = lib.opr_attn_bwd_noalloc(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, n_seqs, 1, 1,
                                   max_seqlen, max_seqlen, hq, 8, d, 0.1, fake, fake, fake, None, 0.0, fake, None)
