@@ -63,9 +63,9 @@ ORACLE_SAMPLE_TOKENS = 3000  # one-pass tokens of the oracle's sample (cpu_basel
 MEASURED_TRAFFIC = {
     "bwd_dkdv": {
         "config_index": 4,
-        "bytes": 30281906432 + 508292096,
+        "bytes": 31602076928 + 509505536,
         "sources": ["attn_bwd.cu", "attn_common.cuh", "sm100.cuh", "layout.cu", "opr_internal.cuh"],
-        "sha256": "7a8f6b1733e471f94f781c3c1d0045bef454cf08cc8b2771afddc71c1f69577b",
+        "sha256": "7bb406e6c5decf1732f9fceb856ae021595865457315f240794a7958015e895a",
         "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                    "-k regex:attn_ -s 9 -c 3 --csv python bench.py --steps 1 --warmup 3 --no-extra --no-e2e "
                    "--no-cpu-baseline --no-npass",
@@ -208,11 +208,14 @@ class Runner:
         b = self.sets[s]
         rec = (lambda i: events[i].record()) if events is not None else (lambda i: None)
         rec(0)
-        lay = opr.opr_build_layout(*b["lens"], total_tokens=self.total, max_seqlen=self.max_seqlen, device=self.dev)
+        lay = opr.opr_build_layout(*b["lens"], total_tokens=self.total, max_seqlen=self.max_seqlen, device=self.dev,
+                                   block_map=False)  # the attention calls use the layout's internal block map
         rec(1)
-        opr.opr_rope(b["q"], lay.pos_id, self.w.base, out=self.q_rot, dev_status=lay.dev_status)
-        opr.opr_rope(b["k"], lay.pos_id, self.w.base, out=self.k_rot, dev_status=lay.dev_status)
-        opr.opr_rope(b["v"], None, self.w.base, out=self.v16, dev_status=lay.dev_status)  # fp16 v: P V in fp16
+        # rotated q, k and the fp16 copy of v (P V in fp16), in the attention order
+        am = lay.attn_pos
+        opr.opr_rope(b["q"], lay.pos_id, self.w.base, out=self.q_rot, dev_status=lay.dev_status, row_map=am)
+        opr.opr_rope(b["k"], lay.pos_id, self.w.base, out=self.k_rot, dev_status=lay.dev_status, row_map=am)
+        opr.opr_rope(b["v"], None, self.w.base, out=self.v16, dev_status=lay.dev_status, row_map=am)
         rec(2)
         o, lse = opr.opr_attn_fwd(self.q_rot, self.k_rot, self.v16, lay, out_dtype=torch.bfloat16)
         rec(3)

@@ -109,9 +109,9 @@ def load_library() -> ctypes.CDLL:
     lib.opr_layout_workspace_bytes.restype = SZ
     lib.opr_layout_workspace_bytes.argtypes = [I32, I32, I32, I64, I32]
     lib.opr_build_layout.restype = I32
-    lib.opr_build_layout.argtypes = [P, P, P, I32, I32, I32, I64, I32, P, P, P, P, P, P, P, SZ, P, P]
+    lib.opr_build_layout.argtypes = [P, P, P, I32, I32, I32, I64, I32, P, P, P, P, P, P, P, P, SZ, P, P]
     lib.opr_rope.restype = I32
-    lib.opr_rope.argtypes = [P, I32, P, I32, P, I64, I32, I32, D, I32, P, P]
+    lib.opr_rope.argtypes = [P, I32, P, I32, P, P, I64, I32, I32, D, I32, P, P]
     lib.opr_attn_fwd.restype = I32
     lib.opr_attn_fwd.argtypes = [P, P, P, I32, I32, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, F, P, I32, P, P, P]
     lib.opr_attn_bwd_workspace_bytes.restype = SZ
@@ -187,7 +187,8 @@ class Layout:
     turn_idx: torch.Tensor
     conv_idx: torch.Tensor
     pos_id: torch.Tensor
-    block_map: torch.Tensor
+    attn_pos: torch.Tensor  # row of each stream token in the attention order (q, k, v of the attention calls)
+    block_map: torch.Tensor | None
     workspace: torch.Tensor
     dev_status: torch.Tensor
 
@@ -228,8 +229,9 @@ def sizes_from_lengths(turn_lens, conv_turn_ptr, seq_conv_ptr) -> tuple[int, int
 
 
 def opr_build_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, total_tokens=None, max_seqlen=None,
-                     device="cuda") -> Layout:
-    """Run opr_build_layout.  Length arrays may be host (copied in) or device int32 tensors."""
+                     device="cuda", block_map: bool = True) -> Layout:
+    """Run opr_build_layout.  Length arrays may be host (copied in) or device int32 tensors.
+    ``block_map=False`` skips the stream-order block map (the attention calls do not read it)."""
     lib = load_library()
     device = torch.device(device)
     if total_tokens is None or max_seqlen is None:
@@ -254,14 +256,16 @@ def opr_build_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, total_tokens=None, 
         turn_idx=torch.empty(total_tokens, dtype=torch.int32, device=device),
         conv_idx=torch.empty(total_tokens, dtype=torch.int32, device=device),
         pos_id=torch.empty(total_tokens, dtype=torch.int32, device=device),
-        block_map=torch.empty((n_seqs, T, T), dtype=torch.uint8, device=device),
+        attn_pos=torch.empty(total_tokens, dtype=torch.int32, device=device),
+        block_map=torch.empty((n_seqs, T, T), dtype=torch.uint8, device=device) if block_map else None,
         workspace=torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device),
         dev_status=torch.zeros(1, dtype=torch.int32, device=device),
     )
     st = lib.opr_build_layout(
         _ptr(tl), _ptr(cp), _ptr(sp), n_seqs, n_convs, n_turns, total_tokens, max_seqlen,
         _ptr(lay.cu_seqlens), _ptr(lay.token_type), _ptr(lay.turn_idx), _ptr(lay.conv_idx), _ptr(lay.pos_id),
-        _ptr(lay.block_map), _ptr(lay.workspace), lay.workspace.numel(), _ptr(lay.dev_status), _stream(device))
+        _ptr(lay.attn_pos), _ptr(lay.block_map), _ptr(lay.workspace), lay.workspace.numel(), _ptr(lay.dev_status),
+        _stream(device))
     _check(st, "opr_build_layout")
     lay._inputs = (tl, cp, sp)  # keep the device copies alive until the stream has used them
     return lay
@@ -271,20 +275,25 @@ _DT = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16, torch.float32: DTY
 
 
 def opr_rope(x: torch.Tensor, pos_id: torch.Tensor | None, base: float, inverse: bool = False,
-             out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None) -> torch.Tensor:
+             out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
+             row_map: torch.Tensor | None = None) -> torch.Tensor:
     """Rotate x [total, heads, head_dim] by position id, into ``out`` (default: in place).
 
     x and out may be bf16, fp16 or fp32 (types may differ when out is not x).  With
-    ``pos_id`` None there is no rotation, only the type conversion.
+    ``pos_id`` None there is no rotation, only the type conversion.  With ``row_map``
+    (e.g. a layout's attn_pos) row t of x goes to row row_map[t] of out (out must not be x).
     """
     out = x if out is None else out
-    _need_cuda(x, out, *(() if pos_id is None else (pos_id,)))
+    _need_cuda(x, out, *(() if pos_id is None else (pos_id,)), *(() if row_map is None else (row_map,)))
+    if row_map is not None and (row_map.dtype != torch.int32 or row_map.numel() != x.shape[0]):
+        raise OprError("row_map must be int32 with one entry per row of x")
     if x.dtype not in _DT or out.dtype not in _DT:
         raise OprError("opr_rope takes bf16, fp16 or fp32")
     if out.shape != x.shape:
         raise OprError("opr_rope: out must have the shape of x")
     total, heads, d = x.shape
-    st = load_library().opr_rope(_ptr(x), _DT[x.dtype], _ptr(out), _DT[out.dtype], _ptr(pos_id), total, heads, d,
+    st = load_library().opr_rope(_ptr(x), _DT[x.dtype], _ptr(out), _DT[out.dtype], _ptr(pos_id), _ptr(row_map),
+                                 total, heads, d,
                                  float(base), int(bool(inverse)), _ptr(dev_status), _stream(x.device))
     _check(st, "opr_rope")
     return out

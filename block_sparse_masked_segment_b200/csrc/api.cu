@@ -135,10 +135,12 @@ AttnParams base_params(const int32_t* cu_seqlens, const int32_t* conv_idx, const
                        int32_t n_convs, int32_t n_turns, int64_t total, int32_t max_seqlen, int32_t hq, int32_t hkv,
                        float scale, int32_t* dev_status) {
   const LayoutWs w = layout_ws_map(n_seqs, n_convs, n_turns, total, max_seqlen);
+  (void)conv_idx;  // the kernels read the layout's attention-order copy
   AttnParams p{};
   p.cu_seqlens = cu_seqlens;
-  p.conv_idx = conv_idx;
-  p.tok_meta = ws_ptr<int32_t>(ws, w.tok_meta);
+  p.conv_idx = ws_ptr<int32_t>(ws, w.attn_conv);
+  p.tok_meta = ws_ptr<int32_t>(ws, w.attn_meta);
+  p.stream_of = ws_ptr<int32_t>(ws, w.stream_of);
   p.row_cnt = ws_ptr<int32_t>(ws, w.row_cnt);
   p.row_list = ws_ptr<int32_t>(ws, w.row_list);
   p.col_cnt = ws_ptr<int32_t>(ws, w.col_cnt);
@@ -368,34 +370,33 @@ size_t opr_layout_workspace_bytes(int32_t n_seqs, int32_t n_convs, int32_t n_tur
 opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* conv_turn_ptr, const int32_t* seq_conv_ptr,
                             int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total_tokens,
                             int32_t max_seqlen, int32_t* cu_seqlens, int8_t* token_type, int32_t* turn_idx,
-                            int32_t* conv_idx, int32_t* pos_id, uint8_t* block_map, void* workspace,
-                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
+                            int32_t* conv_idx, int32_t* pos_id, int32_t* attn_pos, uint8_t* block_map,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
   CallRange range("opr_build_layout");
   if (!sizes_ok(n_seqs, n_convs, n_turns, total_tokens, max_seqlen)) return OPR_INVALID_ARG;
   if (!conv_turn_ptr || !seq_conv_ptr || !cu_seqlens || !workspace || !dev_status) return OPR_INVALID_ARG;
   if (n_turns > 0 && !turn_lens) return OPR_INVALID_ARG;
-  if (total_tokens > 0 && (!token_type || !turn_idx || !conv_idx || !pos_id)) return OPR_INVALID_ARG;
-  if (max_seqlen > 0 && n_seqs > 0 && !block_map) return OPR_INVALID_ARG;
+  if (total_tokens > 0 && (!token_type || !turn_idx || !conv_idx || !pos_id || !attn_pos)) return OPR_INVALID_ARG;
   if (workspace_bytes < layout_ws_map(n_seqs, n_convs, n_turns, total_tokens, max_seqlen).bytes)
     return OPR_WORKSPACE_TOO_SMALL;
   cudaError_t e = launch_layout(turn_lens, conv_turn_ptr, seq_conv_ptr, n_seqs, n_convs, n_turns, total_tokens,
-                                max_seqlen, cu_seqlens, token_type, turn_idx, conv_idx, pos_id, block_map, workspace,
-                                dev_status, static_cast<cudaStream_t>(stream));
+                                max_seqlen, cu_seqlens, token_type, turn_idx, conv_idx, pos_id, attn_pos, block_map,
+                                workspace, dev_status, static_cast<cudaStream_t>(stream));
   return status_of(e);
 }
 
 opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, const int32_t* pos_id,
-                    int64_t total_tokens, int32_t n_heads, int32_t head_dim, double base, int32_t inverse,
-                    int32_t* dev_status, void* stream) {
+                    const int32_t* row_map, int64_t total_tokens, int32_t n_heads, int32_t head_dim, double base,
+                    int32_t inverse, int32_t* dev_status, void* stream) {
   CallRange range("opr_rope");
   if (total_tokens < 0 || n_heads < 0 || head_dim <= 0 || head_dim % 2 != 0 || head_dim > 256) return OPR_INVALID_ARG;
   auto known = [](int32_t t) { return t == OPR_DTYPE_BF16 || t == OPR_DTYPE_FP16 || t == OPR_DTYPE_FP32; };
   if (!known(x_dtype) || !known(y_dtype)) return OPR_UNSUPPORTED;
   if (!(base > 1.0)) return OPR_INVALID_ARG;
   if (total_tokens > 0 && n_heads > 0 && (!x || !y)) return OPR_INVALID_ARG;
-  if (x == y && x_dtype != y_dtype) return OPR_INVALID_ARG;
-  cudaError_t e = launch_rope(x, x_dtype, y, y_dtype, pos_id, total_tokens, n_heads, head_dim, base, inverse,
-                              dev_status, static_cast<cudaStream_t>(stream));
+  if (x == y && (x_dtype != y_dtype || row_map != nullptr)) return OPR_INVALID_ARG;
+  cudaError_t e = launch_rope(x, x_dtype, y, y_dtype, pos_id, row_map, total_tokens, n_heads, head_dim, base,
+                              inverse, dev_status, static_cast<cudaStream_t>(stream));
   return status_of(e);
 }
 

@@ -76,6 +76,7 @@ __device__ __forceinline__ bool fp16_range_ok(float x) { return fabsf(x) <= 6550
 template <int D, typename OT>
 __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                                                         const float* __restrict__ lse, const int32_t* __restrict__ cu_seqlens,
+                                                        const int32_t* __restrict__ stream_of,
                                                         int64_t total, int32_t hq, int32_t T, float* __restrict__ d_tiles,
                                                         float* __restrict__ lse2_tiles, __half* __restrict__ dout16,
                                                         const uint32_t* __restrict__ absmax,
@@ -104,27 +105,36 @@ __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o
       }
       continue;
     }
-    const int64_t tok = seq0 + J * kTile + c;
+    const int64_t tok = seq0 + J * kTile + c;  // attention position: tiles and the dO copy
+    const int64_t src = stream_of[tok];         // stream row: O, dO and LSE
+    if (src < 0 || src >= total) {
+      if (lane == 0) {
+        d_tiles[out] = 0.f;
+        lse2_tiles[out] = -INFINITY;
+      }
+      continue;
+    }
     const size_t base = (static_cast<size_t>(tok) * hq + h) * D + lane * kE;
+    const size_t sbase = (static_cast<size_t>(src) * hq + h) * D + lane * kE;
     float df[kE], ov[kE];
     if constexpr (kE == 4) {
-      const uint2 u = *reinterpret_cast<const uint2*>(dout + base);
+      const uint2 u = *reinterpret_cast<const uint2*>(dout + sbase);
       const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&u);
       df[0] = __low2float(d2[0]) * gs; df[1] = __high2float(d2[0]) * gs;
       df[2] = __low2float(d2[1]) * gs; df[3] = __high2float(d2[1]) * gs;
       *reinterpret_cast<uint2*>(dout16 + base) = make_uint2(pack_f16x2(df[0], df[1]), pack_f16x2(df[2], df[3]));
     } else {
-      const uint32_t u = *reinterpret_cast<const uint32_t*>(dout + base);
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(dout + sbase);
       const __nv_bfloat162 d2 = *reinterpret_cast<const __nv_bfloat162*>(&u);
       df[0] = __low2float(d2) * gs; df[1] = __high2float(d2) * gs;
       *reinterpret_cast<uint32_t*>(dout16 + base) = pack_f16x2(df[0], df[1]);
     }
     if constexpr (sizeof(OT) == 4) {
 #pragma unroll
-      for (int k = 0; k < kE; ++k) ov[k] = static_cast<const float*>(o)[base + k];
+      for (int k = 0; k < kE; ++k) ov[k] = static_cast<const float*>(o)[sbase + k];
     } else {
 #pragma unroll
-      for (int k = 0; k < kE; ++k) ov[k] = __bfloat162float(o[base + k]);
+      for (int k = 0; k < kE; ++k) ov[k] = __bfloat162float(o[sbase + k]);
     }
     float acc = 0.f;
 #pragma unroll
@@ -136,19 +146,28 @@ __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o
     for (int m = 16; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
     if (lane == 0) {
       d_tiles[out] = -acc;
-      lse2_tiles[out] = -lse[static_cast<size_t>(h) * total + tok] * kLog2e;
+      lse2_tiles[out] = -lse[static_cast<size_t>(h) * total + src] * kLog2e;
     }
   }
   if (!in_range) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
 // fp16 copy of V for the dkdv kernel, eight values per thread (same range rule).
+// Row t of y (attention order) is row stream_of[t] of x (stream order); a row
+// holds row8 groups of eight values.
 __global__ void __launch_bounds__(256) cast_f16_kernel(const __nv_bfloat16* __restrict__ x, __half* __restrict__ y,
-                                                       int64_t n8, int32_t* __restrict__ dev_status) {
+                                                       int64_t n8, int64_t row8, int64_t total,
+                                                       const int32_t* __restrict__ stream_of,
+                                                       int32_t* __restrict__ dev_status) {
   bool in_range = true;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+    const int64_t src_row = stream_of[i / row8];
+    if (src_row < 0 || src_row >= total) {
+      reinterpret_cast<uint4*>(y)[i] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint4 u = reinterpret_cast<const uint4*>(x)[src_row * row8 + i % row8];
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
     float f[8];
 #pragma unroll
@@ -281,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // its 64 keys only.
     constexpr uint32_t idesc_s = idesc_f32acc(128, 128, QK16, 0, 0);   // S = Q K^T (q/k type)
     constexpr uint32_t idesc_s64 = idesc_f32acc(128, 64, QK16, 0, 0);  // S over one key half
-    constexpr uint32_t idesc_p = idesc_bf16_f32(128, 128, 0, 0);       // dP = dO V^T (bf16)
-    constexpr uint32_t idesc_p64 = idesc_bf16_f32(128, 64, 0, 0);      // dP over one key half
+    constexpr uint32_t idesc_p = idesc_f32acc(128, 128, true, 0, 0);   // dP = 2^k dO V^T (fp16 copies)
+    constexpr uint32_t idesc_p64 = idesc_f32acc(128, 64, true, 0, 0);  // dP over one key half
     constexpr uint32_t idesc_q = idesc_f32acc(128, D, QK16, 0, 1);     // dQ += dS K (K tile MN-major)
     const uint32_t sq = smem_u32(sm.q), sdo = smem_u32(sm.dout);
     // S(j) = Q K(j)^T
@@ -364,9 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float nlse2 = qv ? p.lse2_tiles[rt] : 0.f;  // -LSE * log2(e)
     const float nd = qv ? p.d_tiles[rt] : 0.f;        // -2^k D
     const int gk = grad_scale_exp(*p.dout_absmax);
-    const float gs = pow2f(gk);                       // dS is formed as 2^k P (dP - D)
+    // dP comes from the fp16 copy of 2^k dO, so dS is formed as 2^k P (dP - D)
     const uint64_t sl2x2 = f2(p.scale_log2, p.scale_log2), nlse2x2 = f2(nlse2, nlse2), ndx2 = f2(nd, nd);
-    const uint64_t gsx2 = f2(gs, gs);
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j % kStages;
@@ -436,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int x = 0; x < 16; ++x) {
-            const uint64_t t = ffma2(f2(__uint_as_float(r[c * 32 + 2 * x]), __uint_as_float(r[c * 32 + 2 * x + 1])), gsx2, ndx2);
+            const uint64_t t = fadd2(f2(__uint_as_float(r[c * 32 + 2 * x]), __uint_as_float(r[c * 32 + 2 * x + 1])), ndx2);
             float d0, d1;
             f2_split(fmul2(f2(pv[c * 32 + 2 * x], pv[c * 32 + 2 * x + 1]), t), d0, d1);
             pk[x] = pack_x2<QK16>(d0, d1);
@@ -450,14 +468,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_dqdone, 0, abort_flag, p.wait_ns))) {
       tc_fence_after();
-      float* dst = p.dq + (static_cast<size_t>(qg) * p.hq + head) * D;
+      const int srow = qv ? p.stream_of[qg] : -1;  // stream row of this query's dQ
+      const bool qw = srow >= 0 && srow < p.total;
+      float* dst = p.dq + (static_cast<size_t>(qw ? srow : 0) * p.hq + head) * D;
       const float osc = p.scale * pow2f(-gk);  // undoes the gradient scale 2^k
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
         const int oc = half * (D / 2) + c * 32;
         tmem_ld32(tl + kDqColAcc + oc, r);
-        if (qv) {
+        if (qw) {
           float4* d4 = reinterpret_cast<float4*>(dst + oc);
 #pragma unroll
           for (int x = 0; x < 8; ++x)
@@ -801,10 +821,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_accdone, 0, abort_flag, p.wait_ns))) {
       tc_fence_after();
+      // partials at the attention position, final rows at the stream row
+      const int srow = kvld ? p.stream_of[kg] : -1;
+      const bool kw = kvld && (split_col || (srow >= 0 && srow < p.total));
+      const size_t fin = static_cast<size_t>(srow >= 0 && srow < p.total ? srow : 0);
       float* dvp = split_col ? p.dv_part + (static_cast<size_t>(major) * p.total + kg) * D
-                             : p.dv + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
+                             : p.dv + (fin * p.hkv + kvh) * D;
       float* dkp = split_col ? p.dk_part + (static_cast<size_t>(major) * p.total + kg) * D
-                             : p.dk + (static_cast<size_t>(kg) * p.hkv + kvh) * D;
+                             : p.dk + (fin * p.hkv + kvh) * D;
       const float vsc = pow2f(-grad_scale_exp(*p.dout_absmax));  // undoes the gradient scale 2^k
       const float ksc = p.scale * vsc;
 #pragma unroll
@@ -812,7 +836,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         const int oc = half * (D / 2) + c * 32;
         tmem_ld32(tl + kKvColDV + oc, r);
-        if (kvld) {
+        if (kw) {
           float4* d4 = reinterpret_cast<float4*>(dvp + oc);
 #pragma unroll
           for (int x = 0; x < 8; ++x)
@@ -825,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         const int oc = half * (D / 2) + c * 32;
         tmem_ld32(tl + kColDK + oc, r);
-        if (kvld) {
+        if (kw) {
           float4* d4 = reinterpret_cast<float4*>(dkp + oc);
 #pragma unroll
           for (int x = 0; x < 8; ++x)
@@ -846,15 +870,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && sm.abort_flag) atomicOr(p.dev_status, OPR_DEV_WAIT_TIMEOUT);
 }
 
-// dK, dV [total][hkv][D] of the tokens of split key columns (at least min_cnt
-// query tiles) = the sum over the q heads of each GQA group of the per-head
-// partials [hq][total][D] the split dK/dV kernel wrote (head order kvh * group +
-// 0, 1, ...; one float4 of dK and of dV per thread and step).  The tokens of
-// shorter columns were written whole by the dK/dV kernel and are left alone.
+// dK, dV [total][hkv][D] (stream rows) of the tokens of split key columns (at
+// least min_cnt query tiles) = the sum over the q heads of each GQA group of the
+// per-head partials [hq][total][D] (attention positions) the split dK/dV kernel
+// wrote (head order kvh * group + 0, 1, ...; one float4 of dK and of dV per
+// thread and step).  The tokens of shorter columns were written whole by the
+// dK/dV kernel and are left alone.
 template <int D>
 __global__ void __launch_bounds__(256) gqa_sum_kernel(const float* __restrict__ dk_part,
                                                       const float* __restrict__ dv_part, int64_t total, int32_t hq,
                                                       int32_t hkv, const int32_t* __restrict__ cu_seqlens,
+                                                      const int32_t* __restrict__ stream_of,
                                                       int32_t n_seqs, int32_t T, const int32_t* __restrict__ col_cnt,
                                                       int32_t min_cnt, float* __restrict__ dk, float* __restrict__ dv) {
   const int group = hq / hkv;
@@ -871,7 +897,7 @@ __global__ void __launch_bounds__(256) gqa_sum_kernel(const float* __restrict__ 
       if (cu_seqlens[mid] <= tok) lo = mid; else hi = mid - 1;
     }
     const int J = static_cast<int>((tok - cu_seqlens[lo]) / kTile);
-    if (J >= T || col_cnt[lo * T + J] < min_cnt) continue;
+    if (J < 0 || J >= T || col_cnt[lo * T + J] < min_cnt) continue;
     float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
     for (int g = 0; g < group; ++g) {
       const size_t src = ((static_cast<size_t>(kvh) * group + g) * total + tok) * (D / 4) + c4;
@@ -880,8 +906,11 @@ __global__ void __launch_bounds__(256) gqa_sum_kernel(const float* __restrict__ 
       sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
       sv.x += b.x; sv.y += b.y; sv.z += b.z; sv.w += b.w;
     }
-    reinterpret_cast<float4*>(dk)[i] = sk;
-    reinterpret_cast<float4*>(dv)[i] = sv;
+    const int64_t srow = stream_of[tok];
+    if (srow < 0 || srow >= total) continue;
+    const int64_t o = (srow * hkv + kvh) * (D / 4) + c4;  // stream row of the attention position tok
+    reinterpret_cast<float4*>(dk)[o] = sk;
+    reinterpret_cast<float4*>(dv)[o] = sv;
   }
 }
 
@@ -914,17 +943,18 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
     float* row_l = b.row_terms + static_cast<size_t>(pq.hq) * pq.n_items * kTile;
     if (b.o_fp32)
       row_terms_kernel<D, float><<<grid, 256, 0, stream>>>(static_cast<const float*>(b.o), b.dout, pq.lse_in,
-                                                               pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d, row_l,
-                                                               b.dout16, b.dout_absmax, pq.dev_status);
+                                                               pq.cu_seqlens, pq.stream_of, pq.total, pq.hq, pq.T,
+                                                               row_d, row_l, b.dout16, b.dout_absmax, pq.dev_status);
     else
       row_terms_kernel<D, __nv_bfloat16><<<grid, 256, 0, stream>>>(
-          static_cast<const __nv_bfloat16*>(b.o), b.dout, pq.lse_in, pq.cu_seqlens, pq.total, pq.hq, pq.T, row_d,
-          row_l, b.dout16, b.dout_absmax, pq.dev_status);
+          static_cast<const __nv_bfloat16*>(b.o), b.dout, pq.lse_in, pq.cu_seqlens, pq.stream_of, pq.total, pq.hq,
+          pq.T, row_d, row_l, b.dout16, b.dout_absmax, pq.dev_status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t n8 = pq.total * pq.hkv * D / 8;
     if (n8 > 0) {
       const int64_t blocks = std::min<int64_t>((n8 + 255) / 256, 148 * 16);
-      cast_f16_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(b.v, b.v16, n8, pq.dev_status);
+      cast_f16_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(b.v, b.v16, n8, pq.hkv * D / 8, pq.total,
+                                                                         pq.stream_of, pq.dev_status);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
@@ -934,10 +964,11 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
     if ((e = set_smem(attn_bwd_dq_kernel<D, QK16>, smem_q, conf_dq)) != cudaSuccess) return e;
     const int64_t bq = static_cast<int64_t>(pq.n_items) * pq.hq;
     if (bq > 0)
-      attn_bwd_dq_kernel<D, QK16><<<static_cast<unsigned>(bq), kThreads, smem_q, stream>>>(m.q, m.k, m.v, m.dout, pq);
+      attn_bwd_dq_kernel<D, QK16><<<static_cast<unsigned>(bq), kThreads, smem_q, stream>>>(m.q, m.k, m.v16, m.dout16,
+                                                                                          pq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (b.rope_pos != nullptr &&  // dq w.r.t. the unrotated q: one pass over the rows
-        (e = launch_rope(pq.dq, OPR_DTYPE_FP32, pq.dq, OPR_DTYPE_FP32, b.rope_pos, pq.total, pq.hq, D, b.rope_base, 1,
+        (e = launch_rope(pq.dq, OPR_DTYPE_FP32, pq.dq, OPR_DTYPE_FP32, b.rope_pos, nullptr, pq.total, pq.hq, D, b.rope_base, 1,
                          pq.dev_status, stream)) != cudaSuccess)
       return e;
   }
@@ -955,13 +986,14 @@ cudaError_t launch_bwd_t(const BwdMaps& m, const BwdBuffers& b, const AttnParams
       if (n4 > 0) {
         const int64_t blocks = std::min<int64_t>((n4 + 255) / 256, 148 * 16);
         gqa_sum_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-            pkv.dk_part, pkv.dv_part, pkv.total, pkv.hq, pkv.hkv, pkv.cu_seqlens, pkv.n_items / pkv.T, pkv.T,
+            pkv.dk_part, pkv.dv_part, pkv.total, pkv.hq, pkv.hkv, pkv.cu_seqlens, pkv.stream_of, pkv.n_items / pkv.T,
+            pkv.T,
             pkv.col_cnt, pkv.split_min_cnt, pkv.dk, pkv.dv);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
       }
     }
     if (b.rope_pos != nullptr)  // dk w.r.t. the unrotated k
-      e = launch_rope(pkv.dk, OPR_DTYPE_FP32, pkv.dk, OPR_DTYPE_FP32, b.rope_pos, pkv.total, pkv.hkv, D, b.rope_base, 1,
+      e = launch_rope(pkv.dk, OPR_DTYPE_FP32, pkv.dk, OPR_DTYPE_FP32, b.rope_pos, nullptr, pkv.total, pkv.hkv, D, b.rope_base, 1,
                       pkv.dev_status, stream);
   }
   return e;

@@ -106,10 +106,7 @@ __device__ __forceinline__ void set_range128(uint64_t& lo, uint64_t& hi, int a, 
 }
 
 // Does a query of meta qmeta see a key of meta kmeta (same conversation, key not after the query)?
-__device__ __forceinline__ bool type_rule(int32_t qmeta, int32_t kmeta) {
-  const uint32_t bits = (kmeta < (qmeta & ~3)) ? kPrevTurnBits : ((kSameTurnBits >> ((qmeta & 3) * 4)) & 0xFu);
-  return (bits >> (kmeta & 3)) & 1u;
-}
+__device__ __forceinline__ bool type_rule(int32_t qmeta, int32_t kmeta) { return turn_type_rule(qmeta, kmeta); }
 
 // Mask of the keys kbase + c (c < 128) visible from query qg: one rule test per
 // run of the key tile, with the causal limit k <= qg.  m[w] holds columns 32w..32w+31.
@@ -203,8 +200,13 @@ struct BwdBuffers {
   double rope_base;
 };
 
+// Token rows of the attention kernels are attention positions (the layout's
+// attention order): q, k and v tiles, conv_idx and tok_meta are in that order;
+// stream_of maps a position to the stream row that O, LSE, dO, dQ, dK and dV
+// (and v in the backward) use.
 struct AttnParams {
   const int32_t* cu_seqlens;
+  const int32_t* stream_of;
   const int32_t* conv_idx;
   const int32_t* tok_meta;
   const int32_t* row_cnt;

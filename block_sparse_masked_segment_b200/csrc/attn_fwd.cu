@@ -299,13 +299,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const float l_tot = sm.lsum[0][row] + sm.lsum[1][row];
       const float inv = 1.f / l_tot;
-      const size_t orow = (static_cast<size_t>(qg) * p.hq + head) * D;
+      const int srow = qv ? p.stream_of[qg] : -1;  // stream row of this query's O and LSE
+      const bool qw = srow >= 0 && srow < p.total;
+      const size_t orow = (static_cast<size_t>(qw ? srow : 0) * p.hq + head) * D;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t r[32];
         const int oc = half * (D / 2) + c * 32;
         tmem_ld32(tl + kOCol + oc, r);
-        if (qv) {
+        if (qw) {
           if (p.o_fp32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + oc);
 #pragma unroll
@@ -323,8 +325,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (qv && half == 0)
-        p.lse[static_cast<size_t>(head) * p.total + qg] = (m_run + __log2f(l_tot)) * 0.69314718055994531f;
+      if (qw && half == 0)
+        p.lse[static_cast<size_t>(head) * p.total + srow] = (m_run + __log2f(l_tot)) * 0.69314718055994531f;
     }
   }
 
@@ -663,12 +665,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && __all_sync(0xffffffffu, mbar_wait(&sm.bar_odone[hx], (n - 1) & 1, abort_flag, p.wait_ns))) {
       tc_fence_after();
       const float inv = 1.f / l_run;
-      const size_t orow = (static_cast<size_t>(qg) * p.hq + head) * D;
+      const int srow = qv ? p.stream_of[qg] : -1;  // stream row of this query's O and LSE
+      const bool qw = srow >= 0 && srow < p.total;
+      const size_t orow = (static_cast<size_t>(qw ? srow : 0) * p.hq + head) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tl + ocol + c * 32, r);
-        if (qv) {
+        if (qw) {
           if (p.o_fp32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + orow + c * 32);
 #pragma unroll
@@ -686,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (qv) p.lse[static_cast<size_t>(head) * p.total + qg] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (qw) p.lse[static_cast<size_t>(head) * p.total + srow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
   }
 

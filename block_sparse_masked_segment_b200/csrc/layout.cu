@@ -13,18 +13,21 @@ namespace opr {
 namespace {
 
 // One thread per conversation: walk its turns, record each turn's first
-// position id (cursor p), its token offset inside the conversation and the
-// conversation's token count (h + t + 2r per turn).
+// position id (cursor p), its token offset inside the conversation, the
+// conversation's token count (h + t + 2r per turn) and its count of context
+// tokens (h + r^in per turn, which is also the final cursor p).
 __global__ void conv_walk_kernel(const int32_t* __restrict__ turn_lens, const int32_t* __restrict__ conv_turn_ptr,
                                  int32_t n_convs, int32_t n_turns, int64_t* __restrict__ conv_tokens,
                                  int64_t* __restrict__ turn_off, int32_t* __restrict__ turn_pos0,
-                                 int32_t* __restrict__ turn_conv, int32_t* __restrict__ dev_status) {
+                                 int32_t* __restrict__ turn_conv, int32_t* __restrict__ conv_ctx,
+                                 int32_t* __restrict__ dev_status) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= n_convs) return;
   const int t0 = conv_turn_ptr[c], t1 = conv_turn_ptr[c + 1];
   if (t0 < 0 || t1 < t0 || t1 > n_turns) {
     atomicOr(dev_status, OPR_DEV_BAD_INPUT);
     conv_tokens[c] = 0;
+    conv_ctx[c] = 0;
     return;
   }
   int64_t off = 0;
@@ -44,6 +47,7 @@ __global__ void conv_walk_kernel(const int32_t* __restrict__ turn_lens, const in
     p += static_cast<int64_t>(h) + r;  // next h starts right after r^in ends
   }
   conv_tokens[c] = off;
+  conv_ctx[c] = static_cast<int32_t>(p);
 }
 
 // Single block: exclusive scan of conversation token counts (in place, with
@@ -109,13 +113,22 @@ __global__ void seq_scan_kernel(int64_t* __restrict__ conv_off, const int32_t* _
 }
 
 // One block per turn: write type, turn index, conversation and position of
-// each of its h + t + 2r tokens (segment order h, t, r^in, r^out).
+// each of its h + t + 2r tokens (segment order h, t, r^in, r^out), and the
+// token's attention position.  The attention order stores each conversation as
+// its context tokens h_1 r^in_1 ... h_N r^in_N, then its trained tokens t_1
+// r^out_1 ... t_N r^out_N (each segment in stream order): the mask is the same,
+// every visible key still comes before its query, and the context part is one
+// causal block and the trained part one staircase, which leaves far fewer
+// partially visible 128x128 tiles than the interleaved stream order.
 __global__ void fill_tokens_kernel(const int32_t* __restrict__ turn_lens, const int32_t* __restrict__ conv_turn_ptr,
                                    const int64_t* __restrict__ conv_off, const int64_t* __restrict__ turn_off,
                                    const int32_t* __restrict__ turn_pos0, const int32_t* __restrict__ turn_conv,
-                                   int32_t n_convs, int64_t total, int8_t* __restrict__ token_type,
-                                   int32_t* __restrict__ turn_idx, int32_t* __restrict__ conv_idx,
-                                   int32_t* __restrict__ pos_id, int32_t* __restrict__ tok_meta) {
+                                   const int32_t* __restrict__ conv_ctx, int32_t n_convs, int64_t total,
+                                   int8_t* __restrict__ token_type, int32_t* __restrict__ turn_idx,
+                                   int32_t* __restrict__ conv_idx, int32_t* __restrict__ pos_id,
+                                   int32_t* __restrict__ tok_meta, int32_t* __restrict__ attn_pos,
+                                   int32_t* __restrict__ attn_conv, int32_t* __restrict__ attn_meta,
+                                   int32_t* __restrict__ stream_of) {
   const int t = blockIdx.x;
   const int c = turn_conv[t];
   if (c < 0 || c >= n_convs) return;
@@ -123,29 +136,44 @@ __global__ void fill_tokens_kernel(const int32_t* __restrict__ turn_lens, const 
   const int i = t - conv_turn_ptr[c];
   const int p = turn_pos0[t];
   const int64_t base = conv_off[c] + turn_off[t];
+  // attention order: this turn's context tokens start at its cursor p (the
+  // context tokens of the earlier turns), its trained ones after the
+  // conversation's conv_ctx context tokens and the earlier turns' t + r^out
+  const int64_t ctx0 = conv_off[c] + p;
+  const int64_t trn0 = conv_off[c] + conv_ctx[c] + (turn_off[t] - p);
   const int n = h + tt + 2 * r;
   for (int x = threadIdx.x; x < n; x += blockDim.x) {
     int type, pos;
+    int64_t ap;
     if (x < h) {
       type = kTypeH;
       pos = p + x;
+      ap = ctx0 + x;
     } else if (x < h + tt) {
       type = kTypeT;
       pos = p + x;  // t starts at p + h
+      ap = trn0 + (x - h);
     } else if (x < h + tt + r) {
       type = kTypeRin;
       pos = p + h + (x - h - tt);
+      ap = ctx0 + h + (x - h - tt);
     } else {
       type = kTypeRout;
       pos = p + h + tt + (x - h - tt - r);
+      ap = trn0 + tt + (x - h - tt - r);
     }
     const int64_t g = base + x;
-    if (g < 0 || g >= total) continue;
+    if (g < 0 || g >= total || ap < 0 || ap >= total) continue;
+    const int meta = (i << 2) | type;
     token_type[g] = static_cast<int8_t>(type);
     turn_idx[g] = i;
     conv_idx[g] = c;
     pos_id[g] = pos;
-    tok_meta[g] = (i << 2) | type;
+    tok_meta[g] = meta;
+    attn_pos[g] = static_cast<int32_t>(ap);
+    attn_conv[ap] = c;
+    attn_meta[ap] = meta;
+    stream_of[ap] = static_cast<int32_t>(g);
   }
 }
 
@@ -317,36 +345,50 @@ __global__ void __launch_bounds__(1024) sched_kernel(const int32_t* __restrict__
 cudaError_t launch_layout(const int32_t* turn_lens, const int32_t* conv_turn_ptr, const int32_t* seq_conv_ptr,
                           int32_t n_seqs, int32_t n_convs, int32_t n_turns, int64_t total, int32_t max_seqlen,
                           int32_t* cu_seqlens, int8_t* token_type, int32_t* turn_idx, int32_t* conv_idx,
-                          int32_t* pos_id, uint8_t* block_map, void* ws, int32_t* dev_status,
+                          int32_t* pos_id, int32_t* attn_pos, uint8_t* block_map, void* ws, int32_t* dev_status,
                           cudaStream_t stream) {
   const LayoutWs w = layout_ws_map(n_seqs, n_convs, n_turns, total, max_seqlen);
   int64_t* conv_off = ws_ptr<int64_t>(ws, w.conv_off);
   int64_t* turn_off = ws_ptr<int64_t>(ws, w.turn_off);
   int32_t* turn_pos0 = ws_ptr<int32_t>(ws, w.turn_pos0);
   int32_t* turn_conv = ws_ptr<int32_t>(ws, w.turn_conv);
+  int32_t* conv_ctx = ws_ptr<int32_t>(ws, w.conv_ctx);
   int32_t* tok_meta = ws_ptr<int32_t>(ws, w.tok_meta);
+  int32_t* attn_conv = ws_ptr<int32_t>(ws, w.attn_conv);
+  int32_t* attn_meta = ws_ptr<int32_t>(ws, w.attn_meta);
+  int32_t* stream_of = ws_ptr<int32_t>(ws, w.stream_of);
+  uint8_t* attn_bmap = ws_ptr<uint8_t>(ws, w.attn_bmap);
 
-  if (n_turns > 0) {
-    cudaError_t e = cudaMemsetAsync(turn_conv, 0xFF, sizeof(int32_t) * n_turns, stream);  // -1: no conversation
-    if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (n_turns > 0 && (e = cudaMemsetAsync(turn_conv, 0xFF, sizeof(int32_t) * n_turns, stream)) != cudaSuccess)
+    return e;  // -1: no conversation
+  if (total > 0) {
+    // -1 where an inconsistent input leaves an attention position unwritten: no
+    // conversation (never visible), and no stream row (the kernels skip it)
+    if ((e = cudaMemsetAsync(attn_conv, 0xFF, sizeof(int32_t) * total, stream)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(stream_of, 0xFF, sizeof(int32_t) * total, stream)) != cudaSuccess) return e;
   }
   if (n_convs > 0)
     conv_walk_kernel<<<(n_convs + 127) / 128, 128, 0, stream>>>(turn_lens, conv_turn_ptr, n_convs, n_turns,
-                                                                conv_off, turn_off, turn_pos0, turn_conv,
+                                                                conv_off, turn_off, turn_pos0, turn_conv, conv_ctx,
                                                                 dev_status);
   seq_scan_kernel<<<1, 1024, 0, stream>>>(conv_off, conv_turn_ptr, seq_conv_ptr, n_seqs, n_convs, n_turns, total,
                                           max_seqlen, cu_seqlens, dev_status);
   if (n_turns > 0)
     fill_tokens_kernel<<<n_turns, 256, 0, stream>>>(turn_lens, conv_turn_ptr, conv_off, turn_off, turn_pos0,
-                                                    turn_conv, n_convs, total, token_type, turn_idx, conv_idx,
-                                                    pos_id, tok_meta);
+                                                    turn_conv, conv_ctx, n_convs, total, token_type, turn_idx,
+                                                    conv_idx, pos_id, tok_meta, attn_pos, attn_conv, attn_meta,
+                                                    stream_of);
   if (w.n_tiles > 0) {
     dim3 grid(w.T, w.T, n_seqs);
-    block_map_kernel<<<grid, 128, 0, stream>>>(cu_seqlens, conv_idx, tok_meta, w.T, block_map);
-    tile_meta_kernel<<<w.n_tiles, 128, 0, stream>>>(cu_seqlens, conv_idx, tok_meta, w.T,
+    if (block_map != nullptr)  // the stream-order block map (an output for the caller)
+      block_map_kernel<<<grid, 128, 0, stream>>>(cu_seqlens, conv_idx, tok_meta, w.T, block_map);
+    // the attention order's block map, run tables and tile lists (the kernels' view)
+    block_map_kernel<<<grid, 128, 0, stream>>>(cu_seqlens, attn_conv, attn_meta, w.T, attn_bmap);
+    tile_meta_kernel<<<w.n_tiles, 128, 0, stream>>>(cu_seqlens, attn_conv, attn_meta, w.T,
                                                     ws_ptr<TileMeta>(ws, w.tile_meta));
     tile_lists_kernel<<<dim3(w.n_tiles, 2), 32, 0, stream>>>(
-        block_map, w.T, ws_ptr<int32_t>(ws, w.row_cnt), ws_ptr<int32_t>(ws, w.row_list),
+        attn_bmap, w.T, ws_ptr<int32_t>(ws, w.row_cnt), ws_ptr<int32_t>(ws, w.row_list),
         ws_ptr<int32_t>(ws, w.col_cnt), ws_ptr<int32_t>(ws, w.col_list));
     int np = 1;
     while (np < w.n_tiles) np <<= 1;

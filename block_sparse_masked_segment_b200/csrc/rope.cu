@@ -56,9 +56,9 @@ __device__ __forceinline__ __half from_f<__half>(float v) {
 
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) rope_kernel(const TI* x, TO* y, const int32_t* __restrict__ pos_id,
-                                                   int64_t total, int32_t n_heads, int32_t half,
-                                                   double neg_log_base_over_half, double sign,
-                                                   int32_t* __restrict__ dev_status) {
+                                                   const int32_t* __restrict__ row_map, int64_t total,
+                                                   int32_t n_heads, int32_t half, double neg_log_base_over_half,
+                                                   double sign, int32_t* __restrict__ dev_status) {
   const int tokens_per_block = blockDim.x / half;
   const int64_t tok = static_cast<int64_t>(blockIdx.x) * tokens_per_block + threadIdx.x / half;
   const int j = threadIdx.x % half;
@@ -69,16 +69,18 @@ __global__ void __launch_bounds__(256) rope_kernel(const TI* x, TO* y, const int
   double sd, cd;
   sincos(ang, &sd, &cd);
   const float c = static_cast<float>(cd), s = static_cast<float>(sd);
-  const int64_t row = tok * n_heads * (2 * half);
+  const int64_t orow_tok = row_map != nullptr ? row_map[tok] : tok;
+  if (orow_tok < 0 || orow_tok >= total) return;
+  const int64_t row = tok * n_heads * (2 * half), orow = orow_tok * n_heads * (2 * half);
   bool out_of_range = false;
   for (int h = 0; h < n_heads; ++h) {
-    const int64_t o = row + static_cast<int64_t>(h) * 2 * half;
+    const int64_t o = row + static_cast<int64_t>(h) * 2 * half, oo = orow + static_cast<int64_t>(h) * 2 * half;
     const float a = to_f(x[o + j]), b = to_f(x[o + j + half]);
     const float ya = a * c - b * s, yb = b * c + a * s;
     if constexpr (sizeof(TO) == 2 && !std::is_same_v<TO, __nv_bfloat16>)
       out_of_range |= !(fabsf(ya) <= 65504.f) || !(fabsf(yb) <= 65504.f);
-    y[o + j] = from_f<TO>(ya);
-    y[o + j + half] = from_f<TO>(yb);
+    y[oo + j] = from_f<TO>(ya);
+    y[oo + j + half] = from_f<TO>(yb);
   }
   if (out_of_range && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
@@ -120,9 +122,9 @@ constexpr int kRopeTok = 8;
 
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) rope_vec_kernel(const TI* x, TO* y, const int32_t* __restrict__ pos_id,
-                                                       int64_t total, int32_t n_heads, int32_t half,
-                                                       double neg_log_base_over_half, double sign,
-                                                       int32_t* __restrict__ dev_status) {
+                                                       const int32_t* __restrict__ row_map, int64_t total,
+                                                       int32_t n_heads, int32_t half, double neg_log_base_over_half,
+                                                       double sign, int32_t* __restrict__ dev_status) {
   extern __shared__ float2 cs[];  // [kRopeTok][half]: (cos, sin)
   const int64_t tok0 = static_cast<int64_t>(blockIdx.x) * kRopeTok;
   const int ntok = static_cast<int>(total - tok0 < kRopeTok ? total - tok0 : kRopeTok);
@@ -141,7 +143,10 @@ __global__ void __launch_bounds__(256) rope_vec_kernel(const TI* x, TO* y, const
   for (int it = threadIdx.x; it < items; it += blockDim.x) {
     const int c = it % chunks, th = it / chunks;
     const int h = th % n_heads, t = th / n_heads;
+    const int64_t otok = row_map != nullptr ? row_map[tok0 + t] : tok0 + t;
+    if (otok < 0 || otok >= total) continue;
     const int64_t o = ((tok0 + t) * n_heads + h) * static_cast<int64_t>(2 * half) + 8 * c;
+    const int64_t oo = (otok * n_heads + h) * static_cast<int64_t>(2 * half) + 8 * c;
     float a[8], b[8], ya[8], yb[8];
     load8(x + o, a);
     load8(x + o + half, b);
@@ -154,35 +159,66 @@ __global__ void __launch_bounds__(256) rope_vec_kernel(const TI* x, TO* y, const
       if constexpr (sizeof(TO) == 2 && !std::is_same_v<TO, __nv_bfloat16>)
         out_of_range |= !(fabsf(ya[k]) <= 65504.f) || !(fabsf(yb[k]) <= 65504.f);
     }
-    store8(y + o, ya);
-    store8(y + o + half, yb);
+    store8(y + oo, ya);
+    store8(y + oo + half, yb);
   }
   if (out_of_range && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
-// No position ids: the rotation by angle 0, i.e. a plain type conversion, one
-// element per thread and step (e.g. the fp16 copy of v that lets the forward's
-// P V product take P in fp16).
+// No position ids: the rotation by angle 0, i.e. a plain type conversion (e.g.
+// the fp16 copy of v that lets the forward's P V product take P in fp16).  Eight
+// elements per thread and step when both tensors are 16-byte aligned and n is a
+// multiple of 8 (16-byte accesses), else one.
 template <typename TI, typename TO>
-__global__ void __launch_bounds__(256) convert_kernel(const TI* x, TO* y, int64_t n, int32_t* __restrict__ dev_status) {
+__global__ void __launch_bounds__(256) convert_kernel(const TI* x, TO* y, const int32_t* __restrict__ row_map,
+                                                      int64_t total, int64_t row_len, bool vec,
+                                                      int32_t* __restrict__ dev_status) {
+  constexpr bool kF16 = std::is_same<TO, __half>::value;
   bool out_of_range = false;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float v = to_f<TI>(x[i]);
-    if constexpr (std::is_same<TO, __half>::value) out_of_range |= !(fabsf(v) <= 65504.f);
-    y[i] = from_f<TO>(v);
+  const int64_t n = total * row_len;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  // output element of input element e (row e / row_len moved to row_map[row])
+  auto out_at = [&](int64_t e) -> int64_t {
+    if (row_map == nullptr) return e;
+    const int64_t r = row_map[e / row_len];
+    return (r < 0 || r >= total) ? -1 : r * row_len + e % row_len;
+  };
+  if (vec) {  // row_len is a multiple of 8: eight elements never straddle two rows
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n / 8; i += stride) {
+      const int64_t o = out_at(8 * i);
+      if (o < 0) continue;
+      float v[8];
+      load8(x + 8 * i, v);
+      if constexpr (kF16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) out_of_range |= !(fabsf(v[k]) <= 65504.f);
+      }
+      store8(y + o, v);
+    }
+  } else {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n; i += stride) {
+      const int64_t o = out_at(i);
+      if (o < 0) continue;
+      const float v = to_f<TI>(x[i]);
+      if constexpr (kF16) out_of_range |= !(fabsf(v) <= 65504.f);
+      y[o] = from_f<TO>(v);
+    }
   }
   if (out_of_range && dev_status != nullptr) atomicOr(dev_status, OPR_DEV_FP16_RANGE);
 }
 
 template <typename TI, typename TO>
-cudaError_t launch_t(const void* x, void* y, const int32_t* pos_id, int64_t total, int32_t n_heads, int32_t half,
-                     double nl, double sign, int32_t* dev_status, cudaStream_t stream) {
+cudaError_t launch_t(const void* x, void* y, const int32_t* pos_id, const int32_t* row_map, int64_t total,
+                     int32_t n_heads, int32_t half, double nl, double sign, int32_t* dev_status, cudaStream_t stream) {
   if (pos_id == nullptr) {
-    const int64_t n = total * n_heads * 2 * half;
-    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 16);
-    convert_kernel<TI, TO><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const TI*>(x),
-                                                                              static_cast<TO*>(y), n, dev_status);
+    const int64_t row_len = static_cast<int64_t>(n_heads) * 2 * half;
+    const int64_t n = total * row_len;
+    const bool vec = row_len % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(y) & 15u) == 0;
+    const int64_t items = vec ? n / 8 : n;
+    const int64_t blocks = std::min<int64_t>((items + 255) / 256, 148 * 16);
+    convert_kernel<TI, TO><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const TI*>(x), static_cast<TO*>(y), row_map, total, row_len, vec, dev_status);
     return cudaGetLastError();
   }
   const bool vec = half % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0 &&
@@ -191,42 +227,42 @@ cudaError_t launch_t(const void* x, void* y, const int32_t* pos_id, int64_t tota
     const int64_t blocks = (total + kRopeTok - 1) / kRopeTok;
     const size_t smem = sizeof(float2) * kRopeTok * half;
     rope_vec_kernel<TI, TO><<<static_cast<unsigned>(blocks), 256, smem, stream>>>(
-        static_cast<const TI*>(x), static_cast<TO*>(y), pos_id, total, n_heads, half, nl, sign, dev_status);
+        static_cast<const TI*>(x), static_cast<TO*>(y), pos_id, row_map, total, n_heads, half, nl, sign, dev_status);
     return cudaGetLastError();
   }
   const int threads = 256 / half * half;
   const int tpb = threads / half;
   const int64_t blocks = (total + tpb - 1) / tpb;
   rope_kernel<TI, TO><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-      static_cast<const TI*>(x), static_cast<TO*>(y), pos_id, total, n_heads, half, nl, sign, dev_status);
+      static_cast<const TI*>(x), static_cast<TO*>(y), pos_id, row_map, total, n_heads, half, nl, sign, dev_status);
   return cudaGetLastError();
 }
 
 template <typename TI>
-cudaError_t launch_in(const void* x, int32_t y_dtype, void* y, const int32_t* pos_id, int64_t total,
-                      int32_t n_heads, int32_t half, double nl, double sign, int32_t* dev_status,
+cudaError_t launch_in(const void* x, int32_t y_dtype, void* y, const int32_t* pos_id, const int32_t* row_map,
+                      int64_t total, int32_t n_heads, int32_t half, double nl, double sign, int32_t* dev_status,
                       cudaStream_t stream) {
   if (y_dtype == OPR_DTYPE_BF16)
-    return launch_t<TI, __nv_bfloat16>(x, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
+    return launch_t<TI, __nv_bfloat16>(x, y, pos_id, row_map, total, n_heads, half, nl, sign, dev_status, stream);
   if (y_dtype == OPR_DTYPE_FP16)
-    return launch_t<TI, __half>(x, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
-  return launch_t<TI, float>(x, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
+    return launch_t<TI, __half>(x, y, pos_id, row_map, total, n_heads, half, nl, sign, dev_status, stream);
+  return launch_t<TI, float>(x, y, pos_id, row_map, total, n_heads, half, nl, sign, dev_status, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype, const int32_t* pos_id,
-                        int64_t total, int32_t n_heads, int32_t head_dim, double base, int32_t inverse,
-                        int32_t* dev_status, cudaStream_t stream) {
+                        const int32_t* row_map, int64_t total, int32_t n_heads, int32_t head_dim, double base,
+                        int32_t inverse, int32_t* dev_status, cudaStream_t stream) {
   if (total == 0 || n_heads == 0) return cudaSuccess;
   const int half = head_dim / 2;
   const double nl = -log(base) / static_cast<double>(half);
   const double sign = inverse ? -1.0 : 1.0;
   if (x_dtype == OPR_DTYPE_BF16)
-    return launch_in<__nv_bfloat16>(x, y_dtype, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
+    return launch_in<__nv_bfloat16>(x, y_dtype, y, pos_id, row_map, total, n_heads, half, nl, sign, dev_status, stream);
   if (x_dtype == OPR_DTYPE_FP16)
-    return launch_in<__half>(x, y_dtype, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
-  return launch_in<float>(x, y_dtype, y, pos_id, total, n_heads, half, nl, sign, dev_status, stream);
+    return launch_in<__half>(x, y_dtype, y, pos_id, row_map, total, n_heads, half, nl, sign, dev_status, stream);
+  return launch_in<float>(x, y_dtype, y, pos_id, row_map, total, n_heads, half, nl, sign, dev_status, stream);
 }
 
 }  // namespace opr

@@ -47,14 +47,17 @@ def useful_flops(pairs: int, hq: int, d: int, backward: bool) -> float:
 
 
 def one_pass_forward(q_pre, k_pre, v, lay: Layout, base: float, scale=None, out_dtype=torch.float32):
-    """RoPE (bf16 in, fp16 out), an fp16 copy of v (so that P V runs with fp16 P), then
-    masked attention.  Returns (o, lse, q_rot, k_rot)."""
+    """RoPE (bf16 in, fp16 out), an fp16 copy of v (so that P V runs with fp16 P), all three
+    written in the layout's attention order, then masked attention.  Returns (o, lse, q_rot,
+    k_rot): o and lse in the stream order, q_rot and k_rot in the attention order (the form
+    one_pass_backward takes)."""
     q = torch.empty(q_pre.shape, dtype=torch.float16, device=q_pre.device)
     k = torch.empty(k_pre.shape, dtype=torch.float16, device=k_pre.device)
     v16 = torch.empty(v.shape, dtype=torch.float16, device=v.device)
-    opr_rope(q_pre, lay.pos_id, base, out=q, dev_status=lay.dev_status)
-    opr_rope(k_pre, lay.pos_id, base, out=k, dev_status=lay.dev_status)
-    opr_rope(v, None, base, out=v16, dev_status=lay.dev_status)
+    # rotated q, k and the fp16 v go to the attention order (rows lay.attn_pos)
+    opr_rope(q_pre, lay.pos_id, base, out=q, dev_status=lay.dev_status, row_map=lay.attn_pos)
+    opr_rope(k_pre, lay.pos_id, base, out=k, dev_status=lay.dev_status, row_map=lay.attn_pos)
+    opr_rope(v, None, base, out=v16, dev_status=lay.dev_status, row_map=lay.attn_pos)
     o, lse = opr_attn_fwd(q, k, v16, lay, scale, out_dtype)
     return o, lse, q, k
 

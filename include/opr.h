@@ -107,7 +107,20 @@ OPR_API size_t opr_layout_workspace_bytes(int32_t n_seqs, int32_t n_convs, int32
  *   turn_idx       int32 [total]       turn index within the conversation (0-based)
  *   conv_idx       int32 [total]       global conversation index
  *   pos_id         int32 [total]       position id
- *   block_map      uint8 [n_seqs][T][T], T = ceil(max_seqlen / 128).  Bits 0-1
+ *   attn_pos       int32 [total]       the token's row in the attention order, the
+ *                  order of the q, k and v rows that opr_attn_fwd and opr_attn_bwd
+ *                  take (opr_rope writes them there with row_map = attn_pos).  Per
+ *                  conversation: the context tokens h_1 r_1^in ... h_N r_N^in, then
+ *                  the trained tokens t_1 r_1^out ... t_N r_N^out, each segment in
+ *                  stream order, inside the conversation's own rows.  The mask is the
+ *                  same in both orders (every visible key comes before its query in
+ *                  both), but the context part is one causal block and the trained
+ *                  part a staircase, so far fewer 128 x 128 tiles are partly visible
+ *                  (a storage choice of this library; the pages state the segments,
+ *                  "Token 复制", and pack them, "实现细节")
+ *   block_map      NULL, or uint8 [n_seqs][T][T], T = ceil(max_seqlen / 128), in the
+ *                  stream order (the attention calls use their own, internal block
+ *                  map of the attention order).  Bits 0-1
  *                  of the byte of tile (I, J) of sequence s: 0 empty, 1 full
  *                  (all 128 x 128 pairs visible), 2 partial; indices past the
  *                  sequence count as not visible, so tail tiles are never full.
@@ -123,7 +136,7 @@ OPR_API opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* con
                             const int32_t* seq_conv_ptr, int32_t n_seqs, int32_t n_convs,
                             int32_t n_turns, int64_t total_tokens, int32_t max_seqlen,
                             int32_t* cu_seqlens, int8_t* token_type, int32_t* turn_idx,
-                            int32_t* conv_idx, int32_t* pos_id, uint8_t* block_map,
+                            int32_t* conv_idx, int32_t* pos_id, int32_t* attn_pos, uint8_t* block_map,
                             void* workspace, size_t workspace_bytes, int32_t* dev_status,
                             void* stream);
 
@@ -142,6 +155,9 @@ OPR_API opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* con
  *   pos_id   int32 [total_tokens]; NULL: no rotation, only the type conversion
  *            (e.g. the fp16 copy of v that opr_attn_fwd takes for an fp16 P V
  *            product)
+ *   row_map  NULL (row t of y is row t of x), or int32 [total_tokens]: row t of x
+ *            is written to row row_map[t] of y (opr_build_layout's attn_pos puts
+ *            q, k and v in the attention order); y must not be x
  *   dev_status  may be NULL; otherwise OPR_DEV_FP16_RANGE is OR-ed in when an
  *            fp16 output overflows (an inf or NaN input included).
  * head_dim must be even and <= 256.  The attention calls take the rotated q
@@ -149,7 +165,7 @@ OPR_API opr_status opr_build_layout(const int32_t* turn_lens, const int32_t* con
  * rounding of the rotation.
  */
 OPR_API opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_dtype,
-                            const int32_t* pos_id, int64_t total_tokens, int32_t n_heads,
+                            const int32_t* pos_id, const int32_t* row_map, int64_t total_tokens, int32_t n_heads,
                             int32_t head_dim, double base, int32_t inverse, int32_t* dev_status,
                             void* stream);
 
@@ -165,18 +181,22 @@ OPR_API opr_status opr_rope(const void* x, int32_t x_dtype, void* y, int32_t y_d
  * O = softmax(scale * Q K^T restricted to visible keys) V for each q head;
  * q head h reads kv head h / (hq / hkv).  Tiles marked empty in the block map
  * are skipped, the visibility predicate is evaluated only on partial tiles.
- *   q            fp16 [total, hq, head_dim]   (already rotated, e.g. by opr_rope)
- *   k            fp16 [total, hkv, head_dim]  (already rotated)
+ *   q            fp16 [total, hq, head_dim]   rotated, rows in the attention order
+ *                (opr_rope with row_map = opr_build_layout's attn_pos)
+ *   k            fp16 [total, hkv, head_dim]  rotated, attention order
  *   qk_dtype     OPR_DTYPE_FP16 (the type of the S = Q K^T MMA); any other
  *                value returns OPR_UNSUPPORTED
- *   v            [total, hkv, head_dim], v_dtype OPR_DTYPE_FP16 or OPR_DTYPE_BF16:
+ *   v            [total, hkv, head_dim] in the attention order, v_dtype
+ *                OPR_DTYPE_FP16 or OPR_DTYPE_BF16:
  *                the type of the O += P V MMA, whose P is rounded to the same
  *                type.  fp16 (v copied by opr_rope with no position ids) keeps
  *                P to 11 bits: O, and D = rowsum(dO * O) in the backward, are
  *                then about 8x closer to exact than with bf16 P.
  *   cu_seqlens, conv_idx, layout_ws: outputs of opr_build_layout for the same sizes
- *   o            [total, hq, head_dim], o_dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32
- *   lse          fp32 [hq, total]: natural-log sum of exp(scale * q.k) over visible keys
+ *   o            [total, hq, head_dim] in the stream order (row = stream token),
+ *                o_dtype OPR_DTYPE_BF16 or OPR_DTYPE_FP32
+ *   lse          fp32 [hq, total], stream order: natural-log sum of exp(scale * q.k)
+ *                over visible keys
  * head_dim must be 64 or 128; all pointers 16-byte aligned; total_tokens at
  * most n_seqs * ceil(max_seqlen / 128) * 128 (else OPR_INVALID_ARG).  All
  * buffers are the caller's; the call reads q, k, v and the layout and writes
@@ -229,10 +249,12 @@ OPR_API size_t opr_attn_bwd_min_workspace_bytes(int32_t n_seqs, int32_t max_seql
  * D = rowsum(dO * O), dV = P^T dO, dS = P * (dO V^T - D), dQ = scale dS K,
  * dK = scale dS^T Q; dK and dV sum over the q heads that share a kv head.
  * Deterministic (no atomics).
- *   q, k, v, o, dout  as in opr_attn_fwd (q, k fp16; o in o_dtype; dout bf16)
- *   lse               fp32 [hq, total] from opr_attn_fwd
- *   dq                fp32 [total, hq, head_dim]
- *   dk, dv            fp32 [total, hkv, head_dim]
+ *   q, k              as in opr_attn_fwd (fp16, rotated, attention order)
+ *   v                 bf16 [total, hkv, head_dim], stream order
+ *   o, dout           stream order, o in o_dtype, dout bf16 [total, hq, head_dim]
+ *   lse               fp32 [hq, total] from opr_attn_fwd (stream order)
+ *   dq                fp32 [total, hq, head_dim], stream order
+ *   dk, dv            fp32 [total, hkv, head_dim], stream order
  *   rope_pos_id       NULL: dq and dk are the gradients w.r.t. the rotated q and k
  *                     given.  Otherwise int32 [total] position ids (those q and k
  *                     were rotated by, e.g. opr_build_layout's pos_id) and

@@ -38,10 +38,13 @@ def run(lay, w, q, k, v, do):
     """Rope, forward, backward; returns (outputs, fwd status bits, bwd status bits)."""
     qr = torch.empty(q.shape, dtype=torch.float16, device=q.device)
     kr = torch.empty(k.shape, dtype=torch.float16, device=q.device)
-    opr.opr_rope(q, lay.pos_id, w.base, out=qr)
-    opr.opr_rope(k, lay.pos_id, w.base, out=kr)
+    va = torch.empty(v.shape, dtype=torch.bfloat16, device=q.device)
+    # the attention calls take q, k and v in the layout's attention order
+    opr.opr_rope(q, lay.pos_id, w.base, out=qr, row_map=lay.attn_pos)
+    opr.opr_rope(k, lay.pos_id, w.base, out=kr, row_map=lay.attn_pos)
+    opr.opr_rope(v, None, w.base, out=va, row_map=lay.attn_pos)
     lay.dev_status.zero_()
-    o, lse = opr.opr_attn_fwd(qr, kr, v, lay, out_dtype=torch.bfloat16)
+    o, lse = opr.opr_attn_fwd(qr, kr, va, lay, out_dtype=torch.bfloat16)
     fwd_bits = int(lay.dev_status.item())
     lay.dev_status.zero_()
     dq, dk, dv = opr.opr_attn_bwd(qr, kr, v, o, do, lse, lay)

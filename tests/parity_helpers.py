@@ -42,3 +42,41 @@ def inputs(w, seed, with_do=True):
 
 def to_dev(x):
     return torch.from_numpy(np.ascontiguousarray(x)).to(device="cuda", dtype=torch.bfloat16)
+
+
+def attention_order(lay) -> np.ndarray:
+    """Stream index of each attention position (the order the attention calls take q, k and v
+    in, include/opr.h attn_pos): per conversation its context tokens (h, r^in), then its trained
+    tokens (t, r^out), each group in stream order.  Conversation ids grow along the stream, so
+    one stable sort by (conversation, trained?) gives it; `lay` is an oracle layout."""
+    from oracle import opr_oracle as orc
+
+    idx = np.arange(len(lay.token_type))
+    trained = (lay.token_type == orc.T) | (lay.token_type == orc.ROUT)
+    return idx[np.lexsort((idx, trained.astype(np.int64), lay.conv_idx.astype(np.int64)))]
+
+
+def block_map_in_order(lay, order, tile: int = 128) -> np.ndarray:
+    """uint8 [n_seqs, T, T] block-map bytes (class | seen key halves << 2) of the oracle mask
+    with rows and columns taken in `order` (stream index of each position)."""
+    from oracle import opr_oracle as orc
+
+    nt = (lay.max_seqlen + tile - 1) // tile
+    out = np.zeros((lay.n_seqs, nt, nt), dtype=np.uint8)
+    for s in range(lay.n_seqs):
+        a, b = int(lay.cu_seqlens[s]), int(lay.cu_seqlens[s + 1])
+        L = b - a
+        perm = order[a:b]
+        cnt = np.zeros((nt, nt, 2), dtype=np.int64)
+        half_edges = np.arange(0, L, tile // 2)
+        for qpos in range(L):
+            row = orc.mask_row(lay, int(perm[qpos]), a, b)[perm - a].astype(np.int64)
+            hs = np.add.reduceat(row, half_edges) if L else np.zeros(0, dtype=np.int64)
+            hh = np.zeros(2 * nt, dtype=np.int64)
+            hh[:len(hs)] = hs
+            cnt[qpos // tile] += hh.reshape(nt, 2)
+        tot = cnt.sum(axis=2)
+        cls = np.where(tot == 0, orc.EMPTY, np.where(tot == tile * tile, orc.FULL, orc.PARTIAL))
+        halves = (cnt[:, :, 0] > 0).astype(np.int64) | ((cnt[:, :, 1] > 0).astype(np.int64) << 1)
+        out[s] = (cls | (halves << 2)).astype(np.uint8)
+    return out

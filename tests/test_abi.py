@@ -105,15 +105,17 @@ def test_host_argument_checks(lib):
     (1) before any CUDA call, so this runs without a GPU."""
     N = None
     # opr_build_layout with null outputs
-    assert lib.opr_build_layout(N, N, N, 1, 1, 1, 10, 10, N, N, N, N, N, N, N, 0, N, N) == 1
+    assert lib.opr_build_layout(N, N, N, 1, 1, 1, 10, 10, N, N, N, N, N, N, N, N, 0, N, N) == 1
     # negative sizes
-    assert lib.opr_build_layout(N, N, N, -1, 1, 1, 10, 10, N, N, N, N, N, N, N, 0, N, N) == 1
+    assert lib.opr_build_layout(N, N, N, -1, 1, 1, 10, 10, N, N, N, N, N, N, N, N, 0, N, N) == 1
     fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the checks fail first
     # opr_rope: odd head_dim, bad dtype, null pointer, in place with two types
-    assert lib.opr_rope(N, 0, N, 0, N, 10, 2, 63, 1e4, 0, N, N) == 1
-    assert lib.opr_rope(N, 7, N, 0, N, 10, 2, 64, 1e4, 0, N, N) == 2
-    assert lib.opr_rope(N, 0, N, 0, N, 10, 2, 64, 1e4, 0, N, N) == 1
-    assert lib.opr_rope(fake, 0, fake, 2, fake, 10, 2, 64, 1e4, 0, N, N) == 1
+    assert lib.opr_rope(N, 0, N, 0, N, N, 10, 2, 63, 1e4, 0, N, N) == 1
+    assert lib.opr_rope(N, 7, N, 0, N, N, 10, 2, 64, 1e4, 0, N, N) == 2
+    assert lib.opr_rope(N, 0, N, 0, N, N, 10, 2, 64, 1e4, 0, N, N) == 1
+    assert lib.opr_rope(fake, 0, fake, 2, fake, N, 10, 2, 64, 1e4, 0, N, N) == 1
+    # a row map writes rows elsewhere, so it cannot work in place
+    assert lib.opr_rope(fake, 0, fake, 0, fake, fake, 10, 2, 64, 1e4, 0, N, N) == 1
     # opr_attn_fwd: null q; hq % hkv != 0; head_dim 96
     assert lib.opr_attn_fwd(N, fake, fake, 2, 0, fake, fake, fake, 1, 1, 1, 100, 100, 4, 2, 128, 0.1,
                             fake, 0, fake, fake, N) == 1
@@ -146,7 +148,7 @@ def test_host_argument_checks(lib):
                             4, 2, 128, 0.1, fake, fake, fake, N, 0.0, fake, 1 << 30, fake, N) == 1
     assert lib.opr_attn_bwd_noalloc(fake, fake, fake, 2, fake, 0, fake, fake, fake, fake, fake, 1, 1, 1, 300, 100,
                                     4, 2, 128, 0.1, fake, fake, fake, N, 0.0, fake, N) == 1
-    assert lib.opr_build_layout(fake, fake, fake, 1, 1, 1, 300, 100, fake, fake, fake, fake, fake, fake, fake,
+    assert lib.opr_build_layout(fake, fake, fake, 1, 1, 1, 300, 100, fake, fake, fake, fake, fake, fake, fake, fake,
                                 1 << 30, fake, N) == 1
     assert opr.opr_layout_workspace_bytes(1, 1, 1, 300, 100) == 0
     # empty problems are no-ops

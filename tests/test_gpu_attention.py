@@ -13,7 +13,7 @@ import torch
 import block_sparse_masked_segment_b200 as opr
 import synth
 from oracle import opr_oracle as orc
-from parity_helpers import assert_close, inputs, to_dev
+from parity_helpers import assert_close, attention_order, block_map_in_order, inputs, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -120,7 +120,9 @@ def test_forward_p_v_in_fp16_and_bf16():
     o_ref, lse_ref = orc.forward(q, k, v, lo, w.base)
     att = opr.OnePassAttention(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr, base=w.base)
     o16, lse16, qr, kr = att.forward(to_dev(q), to_dev(k), to_dev(v))  # fp16 copy of v inside
-    o_bf, lse_bf = opr.opr_attn_fwd(qr, kr, to_dev(v), att.layout)     # bf16 v as given
+    v_bf = torch.empty((w.total_tokens, w.hkv, w.d), dtype=torch.bfloat16, device="cuda")
+    opr.opr_rope(to_dev(v), None, w.base, out=v_bf, row_map=att.layout.attn_pos)  # bf16 v, attention order
+    o_bf, lse_bf = opr.opr_attn_fwd(qr, kr, v_bf, att.layout)
     torch.cuda.synchronize()
     assert opr.read_status(att.layout.dev_status) == []
     e16, _ = assert_close("O (fp16 P)", o16.cpu().numpy(), o_ref)
@@ -324,7 +326,7 @@ def test_dkdv_split_by_q_head_and_unsplit_agree(case):
     # the split form ran on the long columns (seen by >= 2T / group query tiles, include/opr.h):
     # it wrote per-head partials past the minimum workspace
     lo = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
-    col_cnt = (orc.block_map(lo) > 0).sum(axis=1)  # [n_seqs, key tile]
+    col_cnt = ((block_map_in_order(lo, attention_order(lo)) & 3) > 0).sum(axis=1)  # [n_seqs, key tile]
     min_cnt = -(-2 * lay.T // (w.hq // w.hkv))
     assert int(col_cnt.max()) >= min_cnt
     assert bool((ws_full[least:] != 0xFF).any())

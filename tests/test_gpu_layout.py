@@ -2,6 +2,9 @@
 
 Layout, position ids, the block map and its key-half bits must match bit for
 bit (One-Pass to Reason, "Token 复制", "位置 ID 策略", "分块稀疏注意力掩码").
+So must the attention order (each token's row for the attention calls) and the
+internal tile lists the attention kernels walk, which describe the oracle's mask
+with rows and columns taken in that order.
 """
 
 import numpy as np
@@ -12,11 +15,28 @@ import block_sparse_masked_segment_b200 as opr
 from block_sparse_masked_segment_b200 import _abi
 import synth
 from oracle import opr_oracle as orc
+from parity_helpers import attention_order, block_map_in_order
 
 pytestmark = pytest.mark.gpu
 
 
-def _compare_layout(w):
+def _internal_block_map(lay):
+    """The attention kernels' block map, read back from the layout's row lists
+    (entries (J << 4) | block-map byte of the non-empty tiles of each tile row)."""
+    off = opr.layout_table_offsets(lay)
+    T, n_tiles = lay.T, lay.n_seqs * lay.T
+    ws = lay.workspace.cpu().numpy()
+    cnt = ws[off["row_cnt"]:off["row_cnt"] + 4 * n_tiles].view(np.int32)
+    lists = ws[off["row_list"]:off["row_list"] + 4 * n_tiles * T].view(np.int32).reshape(n_tiles, T)
+    bm = np.zeros((lay.n_seqs, T, T), dtype=np.uint8)
+    for row in range(n_tiles):
+        s, i = divmod(row, T)
+        for e in lists[row, :cnt[row]]:
+            bm[s, i, e >> 4] = e & 15
+    return bm
+
+
+def _compare_layout(w, internal=True):
     lay = opr.opr_build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
     ref = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
     torch.cuda.synchronize()
@@ -30,6 +50,13 @@ def _compare_layout(w):
     # each byte: tile class in bits 0-1, key halves that some query sees in bits 2-3
     np.testing.assert_array_equal(bm & 3, orc.block_map(ref, max_seqlen=lay.max_seqlen))
     np.testing.assert_array_equal(bm >> 2, orc.key_half_map(ref, max_seqlen=lay.max_seqlen))
+    # attention order: attn_pos is the inverse of the order (stream index of each position)
+    order = attention_order(ref)
+    expect_pos = np.empty_like(order)
+    expect_pos[order] = np.arange(len(order))
+    np.testing.assert_array_equal(lay.attn_pos.cpu().numpy(), expect_pos)
+    if internal:
+        np.testing.assert_array_equal(_internal_block_map(lay), block_map_in_order(ref, order))
     return lay, ref
 
 
@@ -158,20 +185,21 @@ def test_rope_fp16_overflow_is_flagged():
     assert _abi.DEV_BITS[16] in opr.read_status(lay.dev_status)
 
 
+@pytest.mark.parametrize("shape", [(1000, 3, 64), (1001, 3, 2)])  # 16-byte vector form; element form
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
-def test_rope_without_positions_is_a_type_conversion(in_dtype):
+def test_rope_without_positions_is_a_type_conversion(in_dtype, shape):
     """pos_id NULL: no rotation, the value rounded once to the output type (the fp16 copy of v
     that the forward's P V product takes): bit for bit torch's round-to-nearest conversion;
     a value beyond the fp16 range is flagged."""
     rng = np.random.default_rng(7)
-    x = torch.from_numpy(rng.standard_normal((1000, 3, 64)).astype(np.float32) * 100).to("cuda", in_dtype)
+    x = torch.from_numpy(rng.standard_normal(shape).astype(np.float32) * 100).to("cuda", in_dtype)
     y = torch.empty(x.shape, dtype=torch.float16, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     opr.opr_rope(x, None, 1e4, out=y, dev_status=st)
     torch.cuda.synchronize()
     assert opr.read_status(st) == []
     assert torch.equal(y.view(torch.int16), x.to(torch.float16).view(torch.int16))
-    x[17, 1, 5] = 1e5
+    x[17, 1, 1] = 1e5
     opr.opr_rope(x, None, 1e4, out=y, dev_status=st)
     torch.cuda.synchronize()
     assert _abi.DEV_BITS[16] in opr.read_status(st)

@@ -208,3 +208,41 @@ def test_key_half_map_of_a_causal_segment():
     lay = orc.build_layout([[256, 0, 0]], [0, 1], [0, 1])
     km = orc.key_half_map(lay)
     assert km[0].tolist() == [[3, 0], [3, 3]]
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_attention_order_keeps_every_visible_key_before_its_query(seed):
+    """The attention kernels take tokens in the attention order (per conversation: context h,
+    r^in, then trained t, r^out) and rely on "key not after query" there too: the mask with rows
+    and columns in that order must stay lower triangular, each segment in stream order."""
+    from parity_helpers import attention_order
+
+    w = synth.random_small_workload(100 + seed, n_seqs=2, max_convs=3, max_turns=5)
+    lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    order = attention_order(lay)
+    assert sorted(order.tolist()) == list(range(len(order)))
+    for s in range(lay.n_seqs):
+        a, b = int(lay.cu_seqlens[s]), int(lay.cu_seqlens[s + 1])
+        perm = order[a:b]
+        assert perm.min() >= a and perm.max() < b  # a permutation inside the sequence
+        m = orc.dense_mask(lay, s)[np.ix_(perm - a, perm - a)]
+        assert not np.triu(m, 1).any()
+        # inside a conversation: every context token before every trained token
+        ty = lay.token_type[perm]
+        cv = lay.conv_idx[perm]
+        for c in np.unique(cv):
+            t = ty[cv == c]
+            trained = (t == orc.T) | (t == orc.ROUT)
+            assert not (trained[:-1] & ~trained[1:]).any()
+
+
+def test_block_map_in_order_reduces_to_the_oracle_block_map():
+    """The test helper that builds the attention-order block map gives the oracle's block map
+    and key-half map for the identity order."""
+    from parity_helpers import block_map_in_order
+
+    w = synth.random_small_workload(7, n_seqs=2, max_convs=3, max_turns=4)
+    lay = orc.build_layout(w.turn_lens, w.conv_turn_ptr, w.seq_conv_ptr)
+    got = block_map_in_order(lay, np.arange(len(lay.token_type)))
+    np.testing.assert_array_equal(got & 3, orc.block_map(lay))
+    np.testing.assert_array_equal(got >> 2, orc.key_half_map(lay))
