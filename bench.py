@@ -63,9 +63,9 @@ ORACLE_SAMPLE_TOKENS = 3000  # one-pass tokens of the oracle's sample (cpu_basel
 MEASURED_TRAFFIC = {
     "bwd_dkdv": {
         "config_index": 4,
-        "bytes": 31602076928 + 509505536,
+        "bytes": 20950449664 + 511457536,
         "sources": ["attn_bwd.cu", "attn_common.cuh", "sm100.cuh", "layout.cu", "opr_internal.cuh"],
-        "sha256": "7bb406e6c5decf1732f9fceb856ae021595865457315f240794a7958015e895a",
+        "sha256": "f08c45677a724fa4187561153cb07c04e0206ee69d6b77e85388014d7c6f755c",
         "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                    "-k regex:attn_ -s 9 -c 3 --csv python bench.py --steps 1 --warmup 3 --no-extra --no-e2e "
                    "--no-cpu-baseline --no-npass",
