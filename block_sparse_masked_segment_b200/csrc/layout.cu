@@ -237,6 +237,71 @@ __global__ void __launch_bounds__(128) block_map_kernel(const int32_t* __restric
   }
 }
 
+// The block map again, from the key tile's run table (tile_meta_kernel): thread
+// r owns query row I*128 + r and counts, per key half, its visible keys run by
+// run (one rule test per run instead of per key).  Same bytes as
+// block_map_kernel; the attention order has few runs per tile.
+__global__ void __launch_bounds__(128) block_map_runs_kernel(const int32_t* __restrict__ cu_seqlens,
+                                                             const int32_t* __restrict__ conv_idx,
+                                                             const int32_t* __restrict__ tok_meta,
+                                                             const TileMeta* __restrict__ tmeta, int32_t T,
+                                                             uint8_t* __restrict__ block_map) {
+  __shared__ TileMeta km;
+  __shared__ int32_t warp_cnt[4][2];
+  const int J = blockIdx.x, I = blockIdx.y, s = blockIdx.z;
+  const int r = threadIdx.x;
+  const int seq0 = cu_seqlens[s];
+  const int L = cu_seqlens[s + 1] - seq0;
+  uint8_t* out = block_map + (static_cast<size_t>(s) * T + I) * T + J;
+  if (J > I || I * kTile >= L || J * kTile >= L) {  // above the diagonal or past the end: empty
+    if (r == 0) *out = OPR_TILE_EMPTY;
+    return;
+  }
+  // Quick exit: every key of the tile belongs to a conversation that ends
+  // before the tile's first query row (conversation ids grow along a sequence).
+  const int first_q_conv = conv_idx[seq0 + I * kTile];
+  const int last_k = min(L, (J + 1) * kTile) - 1;
+  if (conv_idx[seq0 + last_k] < first_q_conv) {
+    if (r == 0) *out = OPR_TILE_EMPTY;
+    return;
+  }
+  {
+    const int4* src = reinterpret_cast<const int4*>(tmeta + static_cast<size_t>(s) * T + J);
+    int4* dst = reinterpret_cast<int4*>(&km);
+    for (int x = r; x < static_cast<int>(sizeof(TileMeta) / sizeof(int4)); x += blockDim.x) dst[x] = src[x];
+  }
+  __syncthreads();
+  const int qi = I * kTile + r;
+  int cnt[2] = {0, 0};
+  if (qi < L) {
+    const int qconv = conv_idx[seq0 + qi];
+    const int qmeta = tok_meta[seq0 + qi];
+    const int lim = min(max(qi - J * kTile + 1, 0), kTile);  // keys not after the query
+    const int nr = min(km.nruns, kTile);
+    for (int x = 0; x < nr; ++x) {
+      const int a = km.bound[x], b = min(km.bound[x + 1], lim);
+      if (a >= b || km.conv[x] != qconv || !turn_type_rule(qmeta, km.meta[x])) continue;
+      cnt[0] += max(0, min(b, kKeyHalf) - a);
+      cnt[1] += max(0, b - max(a, kKeyHalf));
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) cnt[h] += __shfl_xor_sync(0xffffffffu, cnt[h], d);
+    if ((r & 31) == 0) warp_cnt[r >> 5][h] = cnt[h];
+  }
+  __syncthreads();
+  if (r == 0) {
+    int half_cnt[2];
+    for (int h = 0; h < 2; ++h) half_cnt[h] = warp_cnt[0][h] + warp_cnt[1][h] + warp_cnt[2][h] + warp_cnt[3][h];
+    const int tot = half_cnt[0] + half_cnt[1];
+    const int cls = tot == 0 ? OPR_TILE_EMPTY : (tot == kTile * kTile ? OPR_TILE_FULL : OPR_TILE_PARTIAL);
+    const int halves = (half_cnt[0] > 0 ? 1 : 0) | (half_cnt[1] > 0 ? 2 : 0);
+    *out = static_cast<uint8_t>(cls | (halves << 2));
+  }
+}
+
 // One warp per row (blockIdx.y == 0) or column (== 1) of the tile grid of a
 // sequence: compact the non-empty tiles, in ascending order, into a list of
 // entries (index << 4) | block-map byte.
@@ -383,10 +448,11 @@ cudaError_t launch_layout(const int32_t* turn_lens, const int32_t* conv_turn_ptr
     dim3 grid(w.T, w.T, n_seqs);
     if (block_map != nullptr)  // the stream-order block map (an output for the caller)
       block_map_kernel<<<grid, 128, 0, stream>>>(cu_seqlens, conv_idx, tok_meta, w.T, block_map);
-    // the attention order's block map, run tables and tile lists (the kernels' view)
-    block_map_kernel<<<grid, 128, 0, stream>>>(cu_seqlens, attn_conv, attn_meta, w.T, attn_bmap);
+    // the attention order's run tables, block map and tile lists (the kernels' view)
     tile_meta_kernel<<<w.n_tiles, 128, 0, stream>>>(cu_seqlens, attn_conv, attn_meta, w.T,
                                                     ws_ptr<TileMeta>(ws, w.tile_meta));
+    block_map_runs_kernel<<<grid, 128, 0, stream>>>(cu_seqlens, attn_conv, attn_meta,
+                                                    ws_ptr<TileMeta>(ws, w.tile_meta), w.T, attn_bmap);
     tile_lists_kernel<<<dim3(w.n_tiles, 2), 32, 0, stream>>>(
         attn_bmap, w.T, ws_ptr<int32_t>(ws, w.row_cnt), ws_ptr<int32_t>(ws, w.row_list),
         ws_ptr<int32_t>(ws, w.col_cnt), ws_ptr<int32_t>(ws, w.col_list));
