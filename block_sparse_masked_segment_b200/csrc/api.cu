@@ -497,7 +497,8 @@ opr_status opr_attn_bwd_stages(const void* q, const void* k, const void* v, int3
   if (!o || !dout || !lse || !cu_seqlens || !conv_idx || !layout_ws || !dq || !dk || !dv || !workspace ||
       !dev_status)
     return OPR_INVALID_ARG;
-  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+  if (!aligned16(o) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace))
     return OPR_INVALID_ARG;
   if (o_dtype != OPR_DTYPE_BF16 && o_dtype != OPR_DTYPE_FP32) return OPR_UNSUPPORTED;
   if (qk_dtype != OPR_DTYPE_FP16) return OPR_UNSUPPORTED;

@@ -130,11 +130,21 @@ __global__ void __launch_bounds__(256) row_terms_kernel(const OT* __restrict__ o
       *reinterpret_cast<uint32_t*>(dout16 + base) = pack_f16x2(df[0], df[1]);
     }
     if constexpr (sizeof(OT) == 4) {
-#pragma unroll
-      for (int k = 0; k < kE; ++k) ov[k] = static_cast<const float*>(o)[sbase + k];
+      if constexpr (kE == 4) {
+        const float4 f = *reinterpret_cast<const float4*>(static_cast<const float*>(o) + sbase);
+        ov[0] = f.x; ov[1] = f.y; ov[2] = f.z; ov[3] = f.w;
+      } else {
+        const float2 f = *reinterpret_cast<const float2*>(static_cast<const float*>(o) + sbase);
+        ov[0] = f.x; ov[1] = f.y;
+      }
+    } else if constexpr (kE == 4) {  // four bf16 values in one 8-byte load
+      const uint2 u = *reinterpret_cast<const uint2*>(o + sbase);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+      ov[0] = __low2float(o2[0]); ov[1] = __high2float(o2[0]); ov[2] = __low2float(o2[1]); ov[3] = __high2float(o2[1]);
     } else {
-#pragma unroll
-      for (int k = 0; k < kE; ++k) ov[k] = __bfloat162float(o[sbase + k]);
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(o + sbase);
+      const __nv_bfloat162 o2 = *reinterpret_cast<const __nv_bfloat162*>(&u);
+      ov[0] = __low2float(o2); ov[1] = __high2float(o2);
     }
     float acc = 0.f;
 #pragma unroll
