@@ -63,9 +63,9 @@ ORACLE_SAMPLE_TOKENS = 3000  # one-pass tokens of the oracle's sample (cpu_basel
 MEASURED_TRAFFIC = {
     "bwd_dkdv": {
         "config_index": 4,
-        "bytes": 20950449664 + 511457536,
+        "bytes": 21588765952 + 513224448,
         "sources": ["attn_bwd.cu", "attn_common.cuh", "sm100.cuh", "layout.cu", "opr_internal.cuh"],
-        "sha256": "f08c45677a724fa4187561153cb07c04e0206ee69d6b77e85388014d7c6f755c",
+        "sha256": "7e566c73dcad049578cb10f0c0f0ce6b1809dbe8fa08cb2e28d1755028e56cd0",
         "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                    "-k regex:attn_ -s 9 -c 3 --csv python bench.py --steps 1 --warmup 3 --no-extra --no-e2e "
                    "--no-cpu-baseline --no-npass",
