@@ -63,9 +63,9 @@ ORACLE_SAMPLE_TOKENS = 3000  # one-pass tokens of the oracle's sample (cpu_basel
 MEASURED_TRAFFIC = {
     "bwd_dkdv": {
         "config_index": 4,
-        "bytes": 21588765952 + 513224448,
+        "bytes": 23265346560 + 512066560,
         "sources": ["attn_bwd.cu", "attn_common.cuh", "sm100.cuh", "layout.cu", "opr_internal.cuh"],
-        "sha256": "7e566c73dcad049578cb10f0c0f0ce6b1809dbe8fa08cb2e28d1755028e56cd0",
+        "sha256": "2ea88915d3b3f98b75dd4dbb6158f29bf0a7f7211dfe4ba0572e705af9635d03",
         "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                    "-k regex:attn_ -s 9 -c 3 --csv python bench.py --steps 1 --warmup 3 --no-extra --no-e2e "
                    "--no-cpu-baseline --no-npass",

@@ -9,14 +9,15 @@
 // Deterministic split into two tcgen05 kernels (no atomics):
 //   dq kernel    one CTA per (query tile, q head), loops over the row's
 //                non-empty key tiles: S, dP -> dS (TMEM) -> dQ += dS K;
-//   dkdv kernel  one CTA per (key tile, kv head), loops over the q heads of
-//                the group and the column's non-empty query tiles:
+//   dkdv kernel  one CTA per (key tile, kv head), loops over the column's
+//                non-empty query tiles and, for each, the q heads of the group:
 //                S^T = K Q^T, dP^T = V dO^T -> P^T, dS^T (TMEM) ->
 //                dV += P^T dO, dK += dS^T Q.
 // Q/K and the dS operand share one 16-bit type (fp16 when QK16, else bf16).
-// The dq kernel forms dP from the bf16 dO and V; the dkdv kernel works on
-// fp16 copies of dO and V (written by the row-terms stage), so that P^T is
-// an fp16 operand of dV = P^T dO (bf16 P^T loses too much there).
+// Both kernels form dP from fp16 copies of 2^k dO and of V, which the row-terms
+// stage writes in the attention order; P^T is an fp16 operand of dV = P^T dO
+// (bf16 P^T loses too much there).  Q, K, the copies and the tile lists are in
+// the attention order; dQ, dK, dV rows go back to their stream rows.
 // Warp roles as in the forward: warp 0 TMA producer (+ metadata lanes),
 // warp 1 TMEM owner and MMA issuer, warps 2..9 two threads per TMEM lane
 // (row), each owning 64 of the tile's 128 columns.
@@ -564,8 +565,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool split_col = p.dkdv_split && cnt >= p.split_min_cnt;
   if (p.dkdv_split && !split_col && major % group != 0) return;
   const int n = split_col ? cnt : cnt * group;
-  // q head of iteration j (query tile entry(j % cnt))
-  auto head_of = [&](int j) { return split_col ? major : kvh * group + j / cnt; };
+  // Iteration j covers query tile entry(tile_of(j)) of q head head_of(j): a whole
+  // column walks its query tiles in order and, for each, the group's q heads in
+  // turn (tile-outer: the CTAs that run together touch fewer distinct Q and dO
+  // tiles at a time than with the heads outermost).
+  auto head_of = [&](int j) { return split_col ? major : kvh * group + j % group; };
+  auto tile_of = [&](int j) { return split_col ? j : j / group; };
   const int s = tile_id / p.T, J = tile_id % p.T;
   const int32_t* list = p.col_list + static_cast<size_t>(tile_id) * p.T;
   const int seq0 = p.cu_seqlens[s];
@@ -605,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // lane 0: K and V once, then the Q ring with each query tile's column data;
     // lane 1: the dO ring.  Iteration j covers q head head_of(j) and query tile
-    // entry(j % cnt).
+    // entry(tile_of(j)).
     if (lane == 0) {
       const TileMeta* tmeta = p.tile_meta + static_cast<size_t>(s) * p.T;
       mbar_arrive_expect_tx(&sm.bar_kv, 2 * kTileBytes);
@@ -614,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
-        const int e = entry(j % cnt);
+        const int e = entry(tile_of(j));
         const int Iq = entry_index(e);
         const int h = head_of(j);
         if (j >= kStages && !mbar_wait(&sm.bar_qempty[st], ((j / kStages) + 1) & 1, abort_flag, p.wait_ns))
@@ -642,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= kStages && !mbar_wait(&sm.bar_doempty[st], ((j / kStages) + 1) & 1, abort_flag, p.wait_ns))
           break;
         mbar_arrive_expect_tx(&sm.bar_dofull[st], kTileBytes);
-        tma_tile<D>(&tm_do16, &sm.bar_dofull[st], sm.dout[st], h, seq0 + entry_index(entry(j % cnt)) * kTile);
+        tma_tile<D>(&tm_do16, &sm.bar_dofull[st], sm.dout[st], h, seq0 + entry_index(entry(tile_of(j))) * kTile);
         issued = j + 1;
       }
       for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
@@ -738,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int st = j % kStages;
-      const int e = entry(j % cnt);
+      const int e = entry(tile_of(j));
       const bool partial = entry_class(e) == OPR_TILE_PARTIAL;
       const int qt0 = seq0 + entry_index(e) * kTile;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.bar_qfull[st], (j / kStages) & 1, abort_flag, p.wait_ns))) {
