@@ -287,6 +287,10 @@ def opr_rope(x: torch.Tensor, pos_id: torch.Tensor | None, base: float, inverse:
     _need_cuda(x, out, *(() if pos_id is None else (pos_id,)), *(() if row_map is None else (row_map,)))
     if row_map is not None and (row_map.dtype != torch.int32 or row_map.numel() != x.shape[0]):
         raise OprError("row_map must be int32 with one entry per row of x")
+    if pos_id is not None and (pos_id.dtype != torch.int32 or pos_id.numel() != x.shape[0]):
+        raise OprError("pos_id must be int32 with one entry per row of x")
+    if out.device != x.device or any(t is not None and t.device != x.device for t in (pos_id, row_map)):
+        raise OprError("opr_rope: every tensor must be on x's device")
     if x.dtype not in _DT or out.dtype not in _DT:
         raise OprError("opr_rope takes bf16, fp16 or fp32")
     if out.shape != x.shape:
@@ -446,12 +450,14 @@ def opr_gather_rows(x: torch.Tensor, src_index: torch.Tensor, out: torch.Tensor 
                     dev_status: torch.Tensor | None = None) -> torch.Tensor:
     """out[i] = x[src_index[i]] along the first dimension (any dtype, rows contiguous)."""
     _need_cuda(x, src_index)
+    if src_index.dtype != torch.int32 or src_index.device != x.device:
+        raise OprError("opr_gather_rows: src_index must be int32 on x's device")
     rows = src_index.numel()
     if out is None:
         out = torch.empty((rows,) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
     _need_cuda(out)
-    if out.shape[0] != rows or out.shape[1:] != x.shape[1:] or out.dtype != x.dtype:
-        raise OprError("opr_gather_rows: out must be [len(src_index)] rows of x's row shape and dtype")
+    if out.shape[0] != rows or out.shape[1:] != x.shape[1:] or out.dtype != x.dtype or out.device != x.device:
+        raise OprError("opr_gather_rows: out must be [len(src_index)] rows of x's row shape and dtype, on x's device")
     row_bytes = x[0].numel() * x.element_size() if x.shape[0] > 0 else out[0].numel() * out.element_size()
     _check(lib_call("opr_gather_rows", _ptr(x), x.shape[0], row_bytes, _ptr(src_index), rows, _ptr(out),
                     _ptr(dev_status) if dev_status is not None else None, _stream(x.device)), "opr_gather_rows")
@@ -465,10 +471,14 @@ def opr_fold_rows(dy: torch.Tensor, copy_index: torch.Tensor, out: torch.Tensor 
     _need_cuda(dy, copy_index)
     if dy.dtype != torch.float32:
         raise OprError("opr_fold_rows: dy must be fp32")
+    if copy_index.dtype != torch.int32 or copy_index.dim() != 2 or copy_index.device != dy.device:
+        raise OprError("opr_fold_rows: copy_index must be int32 [orig, slots] on dy's device")
     rows = copy_index.shape[0]
     if out is None:
         out = torch.empty((rows,) + tuple(dy.shape[1:]), dtype=torch.float32, device=dy.device)
     _need_cuda(out)
+    if out.dtype != torch.float32 or tuple(out.shape) != (rows,) + tuple(dy.shape[1:]) or out.device != dy.device:
+        raise OprError("opr_fold_rows: out must be fp32 [len(copy_index)] rows of dy's row shape, on dy's device")
     width = int(np.prod(dy.shape[1:])) if dy.dim() > 1 else 1
     _check(lib_call("opr_fold_rows", _ptr(dy), dy.shape[0], width, _ptr(copy_index), copy_index.shape[1], rows, _ptr(out),
                     _ptr(dev_status) if dev_status is not None else None, _stream(dy.device)), "opr_fold_rows")

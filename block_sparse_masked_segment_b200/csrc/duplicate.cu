@@ -181,15 +181,31 @@ __global__ void __launch_bounds__(256) fold_rows_kernel(const V* __restrict__ dy
   for (int64_t o = first; o < orig_total; o += step) {
     const int32_t* cp = copy_index + o * slots;
     int n = 0;
+    int32_t a0 = -1, a1 = -1;  // the first two valid copies, in slot order
     for (int k = 0; k < slots; ++k) {
-      if (cp[k] >= total) bad = true;
-      n += (cp[k] >= 0 && cp[k] < total) ? 1 : 0;
+      const int32_t a = cp[k];
+      if (a >= total) bad = true;
+      if (a < 0 || a >= total) continue;
+      if (n == 0) a0 = a;
+      else if (n == 1) a1 = a;
+      ++n;
     }
     if (n == 0) {  // every original token has at least its first copy
       bad = true;
       continue;
     }
     V* dst = dx + o * row_units;
+    if (n <= 2) {  // the common case (one response copy more): both source rows known up front
+      const V* s0 = dy + static_cast<int64_t>(a0) * row_units;
+      const V* s1 = dy + static_cast<int64_t>(n == 2 ? a1 : a0) * row_units;
+#pragma unroll 4
+      for (int64_t c = c0; c < row_units; c += cs) {
+        V v = s0[c];
+        if (n == 2) v = add_v(v, s1[c]);
+        dst[c] = v;
+      }
+      continue;
+    }
     for (int64_t c = c0; c < row_units; c += cs) {
       bool have = false;
       V acc;
@@ -446,12 +462,16 @@ __global__ void __launch_bounds__(256) kpass_index_kernel(
 }
 
 // Blocks for `rows` rows of `units` units: a warp per wide row, a thread per narrow one;
-// at most 148 SMs x 16 blocks (grid-stride beyond).
-int64_t grid_for(int64_t rows, int64_t units) {
+// at most 148 SMs x max_per_sm blocks (grid-stride beyond).
+int64_t grid_for(int64_t rows, int64_t units, int64_t max_per_sm = 16) {
   const int64_t threads = units >= 32 ? rows * 32 : rows;
   const int64_t blocks = (threads + 255) / 256;
-  return blocks < 148 * 16 ? (blocks > 0 ? blocks : 1) : 148 * 16;
+  return blocks < 148 * max_per_sm ? (blocks > 0 ? blocks : 1) : 148 * max_per_sm;
 }
+
+// The fold's rows differ in cost (one or two source rows), so its grid covers
+// more rows at once and the block scheduler evens the load out.
+constexpr int64_t kFoldBlocksPerSm = 64;
 
 }  // namespace
 
@@ -488,11 +508,11 @@ cudaError_t launch_fold_rows(const float* dy, int64_t total, int64_t width, cons
   const bool a16 = (reinterpret_cast<uintptr_t>(dy) % 16 == 0) && (reinterpret_cast<uintptr_t>(dx) % 16 == 0);
   if (width % 4 == 0 && a16) {
     const int64_t u = width / 4;
-    fold_rows_kernel<float4><<<static_cast<unsigned>(grid_for(orig_total, u)), 256, 0, stream>>>(
+    fold_rows_kernel<float4><<<static_cast<unsigned>(grid_for(orig_total, u, kFoldBlocksPerSm)), 256, 0, stream>>>(
         reinterpret_cast<const float4*>(dy), total, u, copy_index, slots, orig_total, reinterpret_cast<float4*>(dx),
         dev_status);
   } else {
-    fold_rows_kernel<float><<<static_cast<unsigned>(grid_for(orig_total, width)), 256, 0, stream>>>(
+    fold_rows_kernel<float><<<static_cast<unsigned>(grid_for(orig_total, width, kFoldBlocksPerSm)), 256, 0, stream>>>(
         dy, total, width, copy_index, slots, orig_total, dx, dev_status);
   }
   return cudaGetLastError();

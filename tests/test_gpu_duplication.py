@@ -103,3 +103,25 @@ def test_total_mismatch_is_flagged_without_overrun():
     torch.cuda.synchronize()
     assert _abi.DEV_BITS[2] in opr.read_status(status)
     assert bool((buf_src[total - 5:] == -7).all()) and bool((buf_cp[(orig - 5) * 2:] == -7).all())
+
+
+def test_binding_rejects_bad_index_and_out_tensors():
+    """The binding refuses, before any launch, index tensors of the wrong type or rank and
+    output buffers of the wrong type or shape (the library would read or write past them)."""
+    w = synth.random_small_workload(14)
+    src, copies, _, r_copies = _check_maps(w)
+    n_orig = r_copies.shape[0]
+    x = torch.randn(n_orig, 8, device="cuda")
+    dy = torch.randn(src.numel(), 8, device="cuda")
+    with pytest.raises(opr.OprError):
+        opr.opr_gather_rows(x, src.long())
+    with pytest.raises(opr.OprError):
+        opr.opr_fold_rows(dy, copies.long())
+    with pytest.raises(opr.OprError):
+        opr.opr_fold_rows(dy, copies.reshape(-1))
+    with pytest.raises(opr.OprError):
+        opr.opr_fold_rows(dy, copies, out=torch.empty(n_orig - 1, 8, device="cuda"))
+    with pytest.raises(opr.OprError):
+        opr.opr_fold_rows(dy, copies, out=torch.empty(n_orig, 8, device="cuda", dtype=torch.float16))
+    torch.testing.assert_close(opr.opr_fold_rows(dy, copies, out=torch.empty(n_orig, 8, device="cuda")),
+                               opr.opr_fold_rows(dy, copies), rtol=0, atol=0)

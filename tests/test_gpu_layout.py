@@ -185,6 +185,16 @@ def test_rope_fp16_overflow_is_flagged():
     assert _abi.DEV_BITS[16] in opr.read_status(lay.dev_status)
 
 
+def test_rope_binding_rejects_bad_positions():
+    """pos_id must be int32 with one entry per row: the kernel reads pos_id[t] for every row t."""
+    lay = opr.opr_build_layout([[4, 0, 0]], [0, 1], [0, 1])
+    x = torch.zeros((4, 1, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(opr.OprError):
+        opr.opr_rope(x, lay.pos_id.long(), 1e4)
+    with pytest.raises(opr.OprError):
+        opr.opr_rope(x, lay.pos_id[:3], 1e4)
+
+
 @pytest.mark.parametrize("shape", [(1000, 3, 64), (1001, 3, 2)])  # 16-byte vector form; element form
 @pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
 def test_rope_without_positions_is_a_type_conversion(in_dtype, shape):
