@@ -65,7 +65,7 @@ MEASURED_TRAFFIC = {
         "config_index": 4,
         "bytes": 23265346560 + 512066560,
         "sources": ["attn_bwd.cu", "attn_common.cuh", "sm100.cuh", "layout.cu", "opr_internal.cuh"],
-        "sha256": "2ea88915d3b3f98b75dd4dbb6158f29bf0a7f7211dfe4ba0572e705af9635d03",
+        "sha256": "2d56eddae8ae839a614b7c25bf15a93698298f9d3b609a247da58566ccbfb24a",
         "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                    "-k regex:attn_ -s 9 -c 3 --csv python bench.py --steps 1 --warmup 3 --no-extra --no-e2e "
                    "--no-cpu-baseline --no-npass",

@@ -567,8 +567,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n = split_col ? cnt : cnt * group;
   // Iteration j covers query tile entry(tile_of(j)) of q head head_of(j): a whole
   // column walks its query tiles in order and, for each, the group's q heads in
-  // turn (tile-outer: the CTAs that run together touch fewer distinct Q and dO
-  // tiles at a time than with the heads outermost).
+  // turn.  Against the heads-outermost walk this takes fewer SM cycles (fewer
+  // long-scoreboard stalls) at the cost of more L2 misses on Q and dO, which at
+  // this kernel's DRAM rate cost no bandwidth.
   auto head_of = [&](int j) { return split_col ? major : kvh * group + j % group; };
   auto tile_of = [&](int j) { return split_col ? j : j / group; };
   const int s = tile_id / p.T, J = tile_id % p.T;
