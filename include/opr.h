@@ -125,8 +125,9 @@ OPR_API size_t opr_layout_workspace_bytes(int32_t n_seqs, int32_t n_convs, int32
  *                  (all 128 x 128 pairs visible), 2 partial; indices past the
  *                  sequence count as not visible, so tail tiles are never full.
  *                  Bits 2-3: bit 2 + h set when some query of the tile sees a
- *                  key of its half h (keys 64 h .. 64 h + 63); the attention
- *                  calls skip the half that no query sees
+ *                  key of its half h (keys 64 h .. 64 h + 63); the dQ kernel,
+ *                  from the same bits of its internal map, skips the half that
+ *                  no query of a tile sees
  *   workspace      opr_layout_workspace_bytes(...) bytes, read by the attention calls
  *   dev_status     int32 word, OPR_DEV_* bits OR-ed in on inconsistent input
  * Returns OPR_INVALID_ARG for null pointers / negative sizes / n_seqs > n_convs
